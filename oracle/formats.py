@@ -105,7 +105,8 @@ def int4_quantize(w, group):
         lo = np.where(degenerate, np.float32(-1), lo).astype(np.float32)
         hi = np.where(degenerate, np.float32(1), hi).astype(np.float32)
         s = fp16_round(np.float32(hi - lo) / fifteen)
-    z = np.clip(np.rint((-lo) / s), 0, 15).astype(np.float32)
+    # the zero point is an integer code: stored as +0.0 .. 15.0 (never -0.0)
+    z = np.clip(np.rint((-lo) / s), 0, 15).astype(np.int32).astype(np.float32)
     q = np.rint(wg / s[:, :, None]) + z[:, :, None]
     q = np.clip(q, 0, 15).astype(np.uint8).reshape(n_rows, k)
     return q, s.astype(np.float16), z.astype(np.float16)

@@ -1,0 +1,278 @@
+"""ctypes binding of libwq.so: the C entry points under the same names.
+
+Argument marshalling only: each function checks that tensors are CUDA,
+contiguous and of the expected dtype, passes raw pointers and the current
+torch CUDA stream, and raises on a non-OK status. Every step of the product
+runs in the library's CUDA kernels; there is no CPU or library fallback, and
+importing this module fails loudly when libwq.so is missing.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwq.so")
+
+WQ_OK = 0
+WQ_ERR_INVALID_ARG = 1
+WQ_ERR_UNSUPPORTED = 2
+WQ_ERR_ALIGNMENT = 3
+WQ_ERR_CUDA = 4
+WQ_ERR_TIMEOUT = 5
+WQ_ERR_WORKSPACE = 6
+
+WQ_FMT_INT4_ASYM = 0
+WQ_FMT_NF4 = 1
+WQ_BF16 = 0
+WQ_FP16 = 1
+WQ_FP32 = 2
+WQ_OP_GEMV = 0
+WQ_OP_GEMM = 1
+WQ_OP_MSD_GEMM = 2
+
+# every symbol include/wq.h declares
+EXPORTED = [
+    "wq_status_string", "wq_version", "wq_nf4_codebook", "wq_packed_sizes",
+    "wq_quantize_pack", "wq_unpack", "wq_nf4_dequant", "wq_int4_dequant",
+    "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
+    "wq_workspace_bytes", "wq_device_error",
+]
+
+
+class WqError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libwq.so not built at %s; run "
+                          "`python -m bit_weight_quantized_weights_b200.build_lib`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, SZ, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, \
+        ctypes.c_uint32
+    sig = {
+        "wq_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "wq_version": ([], ctypes.c_char_p),
+        "wq_nf4_codebook": ([ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
+        "wq_packed_sizes": ([ctypes.c_int, I64, I64, I32, ctypes.POINTER(SZ),
+                             ctypes.POINTER(SZ), ctypes.POINTER(SZ)], ctypes.c_int),
+        "wq_quantize_pack": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P], ctypes.c_int),
+        "wq_unpack": ([ctypes.c_int, P, I64, I64, P, P], ctypes.c_int),
+        "wq_nf4_dequant": ([P, P, I64, I32, P, ctypes.c_int, P], ctypes.c_int),
+        "wq_int4_dequant": ([P, P, P, I64, I64, I32, P, ctypes.c_int, P], ctypes.c_int),
+        "wq_w4a16_gemv": ([P, I64, I64, I64, ctypes.c_int, I32, P, P, P, P, P, SZ, P],
+                          ctypes.c_int),
+        "wq_w4a16_gemm": ([P, I64, I64, I64, ctypes.c_int, I32, P, P, P, P, P, SZ, P],
+                          ctypes.c_int),
+        "wq_msd_decompose": ([P, I64, I64, I32, P, P, P], ctypes.c_int),
+        "wq_msd_gemm": ([P, I64, I64, I64, I32, I32, P, P, P, P, P, SZ, P], ctypes.c_int),
+        "wq_workspace_bytes": ([ctypes.c_int, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
+                               ctypes.c_int),
+        "wq_device_error": ([P, ctypes.c_int, ctypes.POINTER(U32)], ctypes.c_int),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status):
+    return lib.wq_status_string(int(status)).decode()
+
+
+def version():
+    return lib.wq_version().decode()
+
+
+def _check(status, where):
+    if status != WQ_OK:
+        raise WqError(status, where)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t, dtype, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+# ---------------------------------------------------------------------------
+# host-only queries
+# ---------------------------------------------------------------------------
+
+def wq_nf4_codebook():
+    """The 16 NF4 code values the kernels use (host computation)."""
+    buf = (ctypes.c_float * 16)()
+    _check(lib.wq_nf4_codebook(buf), "wq_nf4_codebook")
+    return [float(v) for v in buf]
+
+
+def wq_packed_sizes(fmt, n, k, group):
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.wq_packed_sizes(fmt, n, k, group, ctypes.byref(a), ctypes.byref(b),
+                               ctypes.byref(c)), "wq_packed_sizes")
+    return a.value, b.value, c.value
+
+
+def wq_workspace_bytes(op, m, n, k, group, n_components=2):
+    out = ctypes.c_size_t()
+    _check(lib.wq_workspace_bytes(op, m, n, k, group, n_components, ctypes.byref(out)),
+           "wq_workspace_bytes")
+    return out.value
+
+
+# ---------------------------------------------------------------------------
+# device entry points
+# ---------------------------------------------------------------------------
+
+def alloc_packed(fmt, n, k, group, device="cuda"):
+    """Allocate (qweight, scales, zeros) tensors of the canonical packed layout."""
+    qb, sb, zb = wq_packed_sizes(fmt, n, k, group)
+    if fmt == WQ_FMT_INT4_ASYM:
+        qw = torch.empty(n, k // 8, dtype=torch.int32, device=device)
+        sc = torch.empty(n, k // group, dtype=torch.float16, device=device)
+        zr = torch.empty(n, k // group, dtype=torch.float16, device=device)
+    else:
+        qw = torch.empty(n * k // 2, dtype=torch.uint8, device=device)
+        sc = torch.empty(n * k // 64, dtype=torch.float32, device=device)
+        zr = None
+    assert qw.numel() * qw.element_size() == qb and sc.numel() * sc.element_size() == sb
+    return qw, sc, zr
+
+
+def wq_quantize_pack(fmt, w, group, qweight=None, scales=None, zeros=None, stream=None):
+    """Quantize fp32 W [N, K] on the GPU; returns (qweight, scales, zeros)."""
+    _cuda(w, torch.float32, "W")
+    n, k = w.shape
+    if qweight is None:
+        qweight, scales, zeros = alloc_packed(fmt, n, k, group, w.device)
+    _check(lib.wq_quantize_pack(fmt, _ptr(w), n, k, group, _ptr(qweight), _ptr(scales),
+                                _ptr(zeros), _stream(stream)), "wq_quantize_pack")
+    return qweight, scales, zeros
+
+
+def wq_unpack(fmt, qweight, n, k, out=None, stream=None):
+    _cuda(qweight, None, "qweight")
+    if out is None:
+        out = torch.empty(n * k, dtype=torch.uint8, device=qweight.device)
+    _check(lib.wq_unpack(fmt, _ptr(qweight), n, k, _ptr(out), _stream(stream)), "wq_unpack")
+    return out
+
+
+def wq_nf4_dequant(codes, absmax, numel, out=None, out_dtype=torch.bfloat16, stream=None):
+    _cuda(codes, torch.uint8, "codes")
+    _cuda(absmax, torch.float32, "absmax")
+    if out is None:
+        out = torch.empty(numel, dtype=out_dtype, device=codes.device)
+    dt = WQ_BF16 if out.dtype == torch.bfloat16 else WQ_FP16
+    _check(lib.wq_nf4_dequant(_ptr(codes), _ptr(absmax), numel, 64, _ptr(out), dt,
+                              _stream(stream)), "wq_nf4_dequant")
+    return out
+
+
+def wq_int4_dequant(qweight, scales, zeros, n, k, group, out=None, out_dtype=torch.bfloat16,
+                    stream=None):
+    _cuda(qweight, torch.int32, "qweight")
+    _cuda(scales, torch.float16, "scales")
+    _cuda(zeros, torch.float16, "zeros")
+    if out is None:
+        out = torch.empty(n, k, dtype=out_dtype, device=qweight.device)
+    dt = WQ_BF16 if out.dtype == torch.bfloat16 else WQ_FP16
+    _check(lib.wq_int4_dequant(_ptr(qweight), _ptr(scales), _ptr(zeros), n, k, group, _ptr(out),
+                               dt, _stream(stream)), "wq_int4_dequant")
+    return out
+
+
+def _product(fn, name, x, n, fmt, group, qweight, scales, zeros, out, workspace, stream):
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _cuda(out, torch.bfloat16, "y")
+    ws = _ptr(workspace)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(fn(_ptr(x), m, n, k, fmt, group, _ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(out),
+              ws, wsb, _stream(stream)), name)
+    return out
+
+
+def wq_w4a16_gemv(x, n, fmt, group, qweight, scales, zeros, out=None, stream=None):
+    """Decode GEMV: x bf16 [M<=16, K] -> y bf16 [M, N]."""
+    return _product(lib.wq_w4a16_gemv, "wq_w4a16_gemv", x, n, fmt, group, qweight, scales, zeros,
+                    out, None, stream)
+
+
+def gemm_workspace(m, n, k, group, device="cuda"):
+    nbytes = wq_workspace_bytes(WQ_OP_GEMM, m, n, k, group)
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def wq_w4a16_gemm(x, n, fmt, group, qweight, scales, zeros, workspace=None, out=None,
+                  stream=None):
+    """Prefill GEMM with fused dequantization on tcgen05: y bf16 [M, N]."""
+    _cuda(x, torch.bfloat16, "x")
+    if workspace is None:
+        workspace = gemm_workspace(x.shape[0], n, x.shape[1], group, x.device)
+    return _product(lib.wq_w4a16_gemm, "wq_w4a16_gemm", x, n, fmt, group, qweight, scales, zeros,
+                    out, workspace, stream)
+
+
+def wq_msd_decompose(x, n_components=2, digits=None, comp_scales=None, stream=None):
+    """Digit planes int8 [C, M, K] and scales fp32 [C, M] of bf16 x [M, K]."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if digits is None:
+        digits = torch.empty(n_components, m, k, dtype=torch.int8, device=x.device)
+        comp_scales = torch.empty(n_components, m, dtype=torch.float32, device=x.device)
+    _check(lib.wq_msd_decompose(_ptr(x), m, k, n_components, _ptr(digits), _ptr(comp_scales),
+                                _stream(stream)), "wq_msd_decompose")
+    return digits, comp_scales
+
+
+def msd_workspace(m, n, k, group, n_components=2, device="cuda"):
+    nbytes = wq_workspace_bytes(WQ_OP_MSD_GEMM, m, n, k, group, n_components)
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def wq_msd_gemm(x, n, n_components, group, qweight, scales, zeros, workspace=None, out=None,
+                stream=None):
+    """Multi-Scale Dequant GEMM: y bf16 [M, N] from int8 digit planes of x."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if workspace is None:
+        workspace = msd_workspace(m, n, k, group, n_components, x.device)
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib.wq_msd_gemm(_ptr(x), m, n, k, n_components, group, _ptr(qweight), _ptr(scales),
+                           _ptr(zeros), _ptr(out), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream)),
+           "wq_msd_gemm")
+    return out
+
+
+def wq_device_error(clear=True, stream=None):
+    """Synchronise and read the sticky device error word: (status, detail)."""
+    d = ctypes.c_uint32()
+    st = lib.wq_device_error(_stream(stream), 1 if clear else 0, ctypes.byref(d))
+    return st, d.value

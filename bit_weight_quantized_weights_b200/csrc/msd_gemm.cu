@@ -1,0 +1,386 @@
+// Multi-Scale Dequant GEMM on the int8 tensor cores (tcgen05.mma kind::i8).
+//
+// Source: "Multi-Scale Dequant: Eliminating Dequantization Bottleneck via
+// Activation Decomposition for Efficient LLM Inference", Abstract: instead of
+// lifting the low-bit weights to bf16, the bf16 activations are decomposed
+// into low-precision components that multiply the quantized weights directly
+// on the native integer GEMM hardware. The group's scale is applied after the
+// group's integer sum ("MixPE: Quantization and Hardware Co-design for
+// Efficient LLM Inference", Abstract).
+//
+//   y[m, n] = s_C[m] * sum_g s[n, g] * sum_c 256^(C-c) * P_c[m, n, g]
+//   P_c[m, n, g] = sum_{k in g} a_c[m, k] * (q[n, k] - z[n, g])     (exact int32)
+//
+// (s_c = s_C * 256^(C-c) exactly, so the components combine as integers.)
+// The zero point is folded into the 8-bit weight operand: q - z lies in
+// [-15, 15], an exact signed byte; no weight is ever converted to floating
+// point. The group sums of the digits are therefore not needed.
+//
+// B200 design (one 128-token x 128-feature tile per CTA, BK = 128 = one group
+// of 128):
+//   warp 0       TMA producer: the C digit-plane tiles (int8, 128-byte
+//                swizzled) and the packed weight tile, STAGES-deep ring.
+//   warp 1       TMEM owner; one lane issues C x 4 tcgen05.mma.kind::i8
+//                (128 x 128 x 32, s8 x s8 -> s32) per k-tile into the group's
+//                TMEM accumulators (C x 128 columns, double-buffered when they
+//                fit), commits stages and finished groups.
+//   warps 2-5    unpack: nibbles -> bytes (two permutes per 8 codes), minus
+//                the group's zero point per byte, into the UMMA K-major
+//                128-byte-swizzled B tile.
+//   warps 6-13   drain each finished group from TMEM: combine the components
+//                in int32, convert, scale by the group's s[n, g], accumulate in
+//                fp32 registers; the last group writes bf16 y.
+#include "sm100.cuh"
+
+namespace wq {
+
+__device__ unsigned int g_msd_error;
+
+wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, int8_t*, float*,
+                               cudaStream_t);
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 128;
+constexpr int kStages = 3;
+constexpr int kThreads = 448;
+constexpr int kUnpackWarps = 4;
+constexpr int kEpiWarps = 8;
+constexpr int kPlaneBytes = BM * BK;      // 16 KB per digit plane tile
+constexpr int kBBytes = BN * BK;          // 16 KB
+constexpr int kWBytes = BN * BK / 2;      // 8 KB packed
+
+inline int64_t m_padded(int64_t M) { return (M + 127) / 128 * 128; }
+
+inline size_t planes_bytes(int64_t M, int64_t K, int C) {
+  size_t b = (size_t)C * m_padded(M) * K;
+  return (b + 255) / 256 * 256;
+}
+
+template <int C>
+struct MsdCfg {
+  static constexpr int kNB = (2 * C * BN <= 512) ? 2 : 1;  // TMEM accumulator buffers
+  static constexpr int kTmemCols = (C * BN * kNB <= 256) ? 256 : 512;
+  static constexpr int kStageBytes = C * kPlaneBytes + kBBytes + kWBytes;
+  static constexpr int kSmem = kStages * kStageBytes + 2 * 128 * 4 + 256 + 1024;
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// 8 INT4 codes of one packed word -> 8 signed bytes q - z, in k order.
+__device__ __forceinline__ uint2 unpack_word_minus_zero(uint32_t w, uint32_t zrep) {
+  const uint32_t v = w & 0x0F0F0F0Fu;
+  const uint32_t u = (w >> 4) & 0x0F0F0F0Fu;
+  const uint32_t lo = prmt(v, u, 0x5140u);  // codes 0..3
+  const uint32_t hi = prmt(v, u, 0x7362u);  // codes 4..7
+  // per byte: (128 + q - z) ^ 128 == (q - z) as a two's-complement byte; no
+  // borrow crosses bytes because 128 + q - z >= 113
+  return make_uint2(((lo | 0x80808080u) - zrep) ^ 0x80808080u,
+                    ((hi | 0x80808080u) - zrep) ^ 0x80808080u);
+}
+
+template <int C, bool kIntCombine>
+__global__ void __launch_bounds__(kThreads, 1)
+    msd_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                    const __grid_constant__ CUtensorMap tmap_w, const __half* __restrict__ scales,
+                    const __half* __restrict__ zeros, const float* __restrict__ comp_scales,
+                    uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad) {
+  using Cfg = MsdCfg<C>;
+  constexpr int NB = Cfg::kNB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sA = smem;                                  // [stage][plane] 16 KB
+  uint8_t* sB = sA + kStages * C * kPlaneBytes;        // [stage] 16 KB
+  uint8_t* sW = sB + kStages * kBBytes;                // [stage] 8 KB
+  float* sclE = reinterpret_cast<float*>(sW + kStages * kWBytes);  // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sclE + 256);
+  uint64_t* full = bars;
+  uint64_t* deq = bars + kStages;
+  uint64_t* empty = bars + 2 * kStages;
+  uint64_t* acc_full = bars + 3 * kStages;
+  uint64_t* acc_empty = acc_full + NB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NB);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * BM;
+  const int KT = K / BK;
+  const int TPG = G / BK;   // k-tiles per group
+  const int NG = K / G;
+
+  if (threadIdx.x == 0) {
+    sm100::tma_prefetch_desc(&tmap_a);
+    sm100::tma_prefetch_desc(&tmap_w);
+    for (int s = 0; s < kStages; ++s) {
+      sm100::mbar_init(&full[s], 1);
+      sm100::mbar_init(&deq[s], kUnpackWarps);
+      sm100::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < NB; ++b) {
+      sm100::mbar_init(&acc_full[b], 1);
+      sm100::mbar_init(&acc_empty[b], kEpiWarps);
+    }
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    sm100::tmem_relinquish();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % kStages;
+        const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+        if (kt >= kStages &&
+            !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_msd_error, 0x1101u, abort_flag))
+          break;
+        sm100::mbar_arrive_expect_tx(&full[s], C * kPlaneBytes + kWBytes);
+#pragma unroll
+        for (int c = 0; c < C; ++c)
+          sm100::tma_load_2d(sA + (s * C + c) * kPlaneBytes, &tmap_a, &full[s], kt * BK,
+                             c * m_pad + m0);
+        sm100::tma_load_2d(sW + s * kWBytes, &tmap_w, &full[s], kt * (BK / 8), n0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = sm100::idesc_s8_s32(BM, BN);
+      int kt = 0;
+      bool ok = true;
+      for (int gi = 0; gi < NG && ok; ++gi) {
+        const int b = gi % NB;
+        if (gi >= NB) {
+          if (!sm100::mbar_wait(&acc_empty[b], (uint32_t)((gi / NB) - 1) & 1u, &g_msd_error,
+                                0x1201u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+        }
+        for (int t = 0; t < TPG; ++t, ++kt) {
+          const int s = kt % kStages;
+          const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+          if (!sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1202u, abort_flag) ||
+              !sm100::mbar_wait(&deq[s], ph, &g_msd_error, 0x1203u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          sm100::tc_fence_after();
+          const uint32_t b_base = smem_u32(sB + s * kBBytes);
+#pragma unroll
+          for (int c = 0; c < C; ++c) {
+            const uint32_t a_base = smem_u32(sA + (s * C + c) * kPlaneBytes);
+            const uint32_t d = tmem + (uint32_t)((b * C + c) * BN);
+#pragma unroll
+            for (int kk = 0; kk < BK / 32; ++kk) {
+              sm100::mma_i8(d, sm100::sdesc_sw128_kmajor(a_base + kk * 32),
+                            sm100::sdesc_sw128_kmajor(b_base + kk * 32), idesc,
+                            (t | kk) != 0 ? 1u : 0u);
+            }
+          }
+          sm100::mma_commit(&empty[s]);
+        }
+        if (ok) sm100::mma_commit(&acc_full[b]);
+      }
+    }
+  } else if (warp < 2 + kUnpackWarps) {
+    // ---------------- unpack: B row r = feature n0 + r ----------------
+    const int r = threadIdx.x - 64;
+    const __half* zrow = zeros + (int64_t)(n0 + r) * NG;
+    uint32_t zrep = 0;
+    for (int kt = 0; kt < KT; ++kt) {
+      const int s = kt % kStages;
+      const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+      if (kt % TPG == 0) {
+        const uint32_t z = (uint32_t)__half2float(zrow[kt / TPG]);
+        zrep = z * 0x01010101u;
+      }
+      bool got = sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1301u, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;
+      const uint4* wsrc = reinterpret_cast<const uint4*>(sW + s * kWBytes + r * 64);
+      uint8_t* bdst = sB + s * kBBytes + r * 128;
+#pragma unroll
+      for (int j4 = 0; j4 < 4; ++j4) {
+        const uint4 wv = wsrc[j4];  // words 4*j4 .. 4*j4+3 -> chunks 2*j4, 2*j4+1
+        const uint2 b0 = unpack_word_minus_zero(wv.x, zrep);
+        const uint2 b1 = unpack_word_minus_zero(wv.y, zrep);
+        const uint2 b2 = unpack_word_minus_zero(wv.z, zrep);
+        const uint2 b3 = unpack_word_minus_zero(wv.w, zrep);
+        const int c0 = 2 * j4, c1 = 2 * j4 + 1;
+        *reinterpret_cast<uint4*>(bdst + ((c0 ^ (r & 7)) << 4)) = make_uint4(b0.x, b0.y, b1.x, b1.y);
+        *reinterpret_cast<uint4*>(bdst + ((c1 ^ (r & 7)) << 4)) = make_uint4(b2.x, b2.y, b3.x, b3.y);
+      }
+      sm100::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&deq[s]);
+    }
+  } else {
+    // ---------------- drain / epilogue ----------------
+    const int e = threadIdx.x - 64 - 32 * kUnpackWarps;  // 0..255
+    const int q = warp & 3;                              // TMEM lane quarter
+    const int half = (warp - 2 - kUnpackWarps) >> 2;     // 64-column half
+    const int row = 32 * q + lane;
+    float acc[64];
+#pragma unroll
+    for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+    float pref = 0.0f;
+    if (e < BN) pref = __half2float(scales[(int64_t)(n0 + e) * NG]);
+    bool ok = true;
+    for (int gi = 0; gi < NG; ++gi) {
+      const int b = gi % NB;
+      if (e < BN) sclE[(gi & 1) * 128 + e] = pref;
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (e < BN && gi + 1 < NG) pref = __half2float(scales[(int64_t)(n0 + e) * NG + gi + 1]);
+      // every epilogue warp runs all NG iterations (the named barrier above
+      // counts on it); after a failed wait the rest only keep that barrier
+      if (ok) {
+        bool got = sm100::mbar_wait(&acc_full[b], (uint32_t)(gi / NB) & 1u, &g_msd_error,
+                                    0x1401u, abort_flag);
+        ok = __all_sync(0xffffffffu, got);
+      }
+      if (!ok) continue;
+      sm100::tc_fence_after();
+      const float* scl = sclE + (gi & 1) * 128 + half * 64;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const int col = half * 64 + 16 * cc;
+        const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * C * BN + col);
+        uint32_t p[16];
+        tmem_ld16(base, p);
+        sm100::tmem_ld_wait();
+        int32_t ti[16];
+        float tf[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          ti[j] = (int32_t)p[j];
+          tf[j] = (float)(int32_t)p[j];
+        }
+#pragma unroll
+        for (int c = 1; c < C; ++c) {
+          tmem_ld16(base + (uint32_t)(c * BN), p);
+          sm100::tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (kIntCombine) ti[j] = ti[j] * 256 + (int32_t)p[j];
+            else tf[j] = fmaf(tf[j], 256.0f, (float)(int32_t)p[j]);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float t = kIntCombine ? (float)ti[j] : tf[j];
+          acc[16 * cc + j] = fmaf(scl[16 * cc + j], t, acc[16 * cc + j]);
+        }
+      }
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
+    }
+    const int m = m0 + row;
+    if (ok && m < M) {
+      const float sC = comp_scales[(int64_t)(C - 1) * M + m];
+      uint16_t* dst = y + (int64_t)m * N + n0 + half * 64;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint4 o;
+        o.x = pack_bf16x2(acc[8 * i + 0] * sC, acc[8 * i + 1] * sC);
+        o.y = pack_bf16x2(acc[8 * i + 2] * sC, acc[8 * i + 3] * sC);
+        o.z = pack_bf16x2(acc[8 * i + 4] * sC, acc[8 * i + 5] * sC);
+        o.w = pack_bf16x2(acc[8 * i + 6] * sC, acc[8 * i + 7] * sC);
+        *reinterpret_cast<uint4*>(dst + 8 * i) = o;
+      }
+    }
+  }
+
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, Cfg::kTmemCols);
+  }
+}
+
+template <int C, bool kInt>
+wq_status launch_c(const CUtensorMap& ta, const CUtensorMap& tw, const void* scales,
+                   const void* zeros, const float* cs, void* y, int64_t M, int64_t N, int64_t K,
+                   int32_t G, cudaStream_t st) {
+  using Cfg = MsdCfg<C>;
+  auto kern = msd_gemm_kernel<C, kInt>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+      cudaSuccess)
+    return WQ_ERR_CUDA;
+  const int64_t mp = m_padded(M);
+  dim3 grid((unsigned)(N / BN), (unsigned)(mp / BM));
+  kern<<<grid, kThreads, Cfg::kSmem, st>>>(ta, tw, static_cast<const __half*>(scales),
+                                           static_cast<const __half*>(zeros), cs,
+                                           static_cast<uint16_t*>(y), (int)M, (int)N, (int)K, G,
+                                           (int)mp);
+  return launch_status();
+}
+
+}  // namespace
+
+// Workspace: digit planes [C][M_pad][K] int8 (M_pad = M rounded up to 128),
+// then the component scales [C][M] fp32, 256-byte aligned.
+size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C) {
+  return planes_bytes(M, K, C) + (size_t)C * M * 4;
+}
+
+wq_status launch_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_t C, int32_t G,
+                          const void* qweight, const void* scales, const void* zeros, void* y,
+                          void* workspace, cudaStream_t st) {
+  int8_t* planes = static_cast<int8_t*>(workspace);
+  float* cs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + planes_bytes(M, K, C));
+  const int64_t mp = m_padded(M);
+  wq_status s = launch_msd_decompose(x, M, K, C, mp, planes, cs, st);
+  if (s != WQ_OK) return s;
+  CUtensorMap ta, tw;
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K, (uint64_t)(C * mp),
+                    (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return WQ_ERR_CUDA;
+  if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)K / 8, (uint64_t)N,
+                    (uint64_t)K / 2, BK / 8, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return WQ_ERR_CUDA;
+  // integer combination of the components while it cannot overflow int32:
+  // |P_1| <= 127 * 15 * G and 256 * |P_1| + |P_2| must stay below 2^31
+  const bool int_ok = (int64_t)G * 127 * 15 * 257 < ((int64_t)1 << 31);
+  switch (C) {
+    case 1: return launch_c<1, true>(ta, tw, scales, zeros, cs, y, M, N, K, G, st);
+    case 2:
+      return int_ok ? launch_c<2, true>(ta, tw, scales, zeros, cs, y, M, N, K, G, st)
+                    : launch_c<2, false>(ta, tw, scales, zeros, cs, y, M, N, K, G, st);
+    default: return launch_c<3, false>(ta, tw, scales, zeros, cs, y, M, N, K, G, st);
+  }
+}
+
+wq_status read_msd_error(bool clear, uint32_t* v) {
+  uint32_t h = 0;
+  if (cudaMemcpyFromSymbol(&h, g_msd_error, sizeof(h)) != cudaSuccess) return WQ_ERR_CUDA;
+  if (clear && h) {
+    const uint32_t z = 0;
+    if (cudaMemcpyToSymbol(g_msd_error, &z, sizeof(z)) != cudaSuccess) return WQ_ERR_CUDA;
+  }
+  *v = h;
+  return WQ_OK;
+}
+
+}  // namespace wq

@@ -1,0 +1,67 @@
+// Activations bf16 -> fp16 with a per-row power-of-two scale.
+//
+// The fused GEMM multiplies in fp16 (11 significant bits, so the dequantized
+// weight (q - z) * s rounds 16x more finely than in bf16). bf16 activations
+// have 8 significant bits, so x * 2^e is exact in fp16 as long as it lies in
+// fp16's normal range. Per row, e puts the row's largest magnitude in
+// [2^14, 2^15): every element down to amax * 2^-28 converts exactly, none can
+// overflow, and the GEMM epilogue multiplies by 2^-e (exact) before rounding
+// to bf16.
+#include "common.cuh"
+
+namespace wq {
+namespace {
+
+__global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restrict__ x, int K,
+                                                       uint16_t* __restrict__ x16,
+                                                       float* __restrict__ inv_scale) {
+  __shared__ float red[8];
+  const int m = blockIdx.x;
+  const uint16_t* row = x + (int64_t)m * K;
+  uint16_t* out = x16 + (int64_t)m * K;
+  const int chunks = K / 8;
+  float amax = 0.0f;
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + c * 8);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo_to_f32(w[i])), fabsf(bf16_hi_to_f32(w[i]))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  // exponent of amax (amax finite and > 0): amax in [2^ex, 2^(ex+1))
+  int e = 0;
+  if (amax > 0.0f && amax <= 3.0e38f) {
+    const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+    e = 14 - ex;
+    e = e > 100 ? 100 : (e < -100 ? -100 : e);
+  }
+  const float sc = __uint_as_float((uint32_t)(127 + e) << 23);       // 2^e
+  if (threadIdx.x == 0) inv_scale[m] = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + c * 8);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = pack_f16x2(bf16_lo_to_f32(w[i]) * sc, bf16_hi_to_f32(w[i]) * sc);
+    *reinterpret_cast<uint4*>(out + c * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace
+
+wq_status launch_x_to_f16(const void* x, int64_t M, int64_t K, void* x16, float* inv_scale,
+                          cudaStream_t st) {
+  x_to_f16_kernel<<<(unsigned)M, 256, 0, st>>>(static_cast<const uint16_t*>(x), (int)K,
+                                               static_cast<uint16_t*>(x16), inv_scale);
+  return launch_status();
+}
+
+}  // namespace wq

@@ -1,0 +1,62 @@
+"""Seeded synthetic inputs and the workload table (no quantization arithmetic).
+
+Both the CUDA path and the CPU oracle consume exactly the tensors produced
+here. The recipe: a CPU torch.Generator seeded per workload; weights
+W ~ N(0, 0.02) fp32 [N, K]; activations x ~ N(0, 1) fp32 [M, K] drawn after W,
+a set of outlier channels (round(frac * K) columns chosen by randperm on the
+same generator) multiplied by a constant, then x is rounded once to bf16.
+The shapes are the Llama / Qwen linear-layer shapes the quantized-kernel pages
+evaluate on (synthetic stand-ins: no trained weights are involved).
+"""
+
+import torch
+
+# (name, kind, shapes, extra) for each workload family.
+GEMV_TINY = dict(name="gemv_tiny_int4_g64", M=1, N=1024, K=1024, group=64)
+NF4_DEQUANT_SHAPES = [(28672, 8192), (8192, 8192), (5120, 25600)]
+DECODE_SHAPES = [(4096, 4096), (11008, 4096), (4096, 11008)]
+DECODE_M = [1, 4, 8, 16]
+PREFILL_SHAPES = [(4096, 4096), (14336, 4096), (4096, 14336)]
+PREFILL_M = [512, 2048, 8192]
+MSD_SHAPES = [(5120, 5120), (25600, 5120), (5120, 25600)]
+MSD_M = [1, 16, 128, 1024]
+
+DECODE_OUTLIERS = (0.01, 20.0)
+MSD_OUTLIERS = (0.005, 50.0)
+
+
+def generator(seed=0):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def weights(n, k, seed=0, gen=None):
+    """fp32 [N, K] ~ N(0, 0.02), CPU."""
+    g = gen if gen is not None else generator(seed)
+    return torch.randn(n, k, generator=g, dtype=torch.float32) * 0.02
+
+
+def activations(m, k, seed=0, gen=None, outliers=None):
+    """bf16 [M, K]: N(0, 1) with optional (fraction, scale) outlier channels, CPU."""
+    g = gen if gen is not None else generator(seed)
+    x = torch.randn(m, k, generator=g, dtype=torch.float32)
+    if outliers is not None:
+        frac, scale = outliers
+        cnt = max(1, round(frac * k))
+        idx = torch.randperm(k, generator=g)[:cnt]
+        x[:, idx] *= scale
+    return x.to(torch.bfloat16)
+
+
+def layer(m, n, k, seed=0, outliers=None):
+    """(W fp32 [N, K], x bf16 [M, K]) drawn in that order from one generator."""
+    g = generator(seed)
+    w = weights(n, k, gen=g)
+    x = activations(m, k, gen=g, outliers=outliers)
+    return w, x
+
+
+def flat_weights(n, k, seed=0):
+    """fp32 [N, K] weights for the standalone NF4 dequantization workload."""
+    return weights(n, k, seed=seed)

@@ -1,0 +1,242 @@
+/*
+ * wq.h -- C ABI of the 4-bit weight-only quantized product library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library computes y = x . dequant(W_q)^T for bf16 activations x [M, K]
+ * and 4-bit weights W [N, K] (N output features, K input features), with the
+ * dequantization fused into the product, plus the Multi-Scale Dequant path in
+ * which the activations are split into int8 digit planes that multiply the
+ * integer weight codes directly.
+ *
+ * Sources (each entry point names the passage that defines it):
+ *  [MSD]   "Multi-Scale Dequant: Eliminating Dequantization Bottleneck via
+ *          Activation Decomposition for Efficient LLM Inference", Abstract.
+ *  [MIXPE] "MixPE: Quantization and Hardware Co-design for Efficient LLM
+ *          Inference", Abstract.
+ *  [NF4]   "Fast NF4 Dequantization Kernels for Large Language Model
+ *          Inference", Abstract.
+ *  [QLORA] "QLoRA: Efficient Finetuning of Quantized LLMs" (cited by title on
+ *          "DecDEC: A Systems Approach to Advancing Low-Bit LLM Quantization"):
+ *          the NF4 codebook construction.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer owned by the caller unless the
+ *    comment says "host". The library never allocates, frees or retains
+ *    caller memory. Workspace, where an entry point takes one, is caller
+ *    provided and sized by wq_workspace_bytes().
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Every device call is asynchronous on that stream; the library
+ *    never synchronises, except wq_device_error(), which says so.
+ *  - Device pointers must be 16-byte aligned (WQ_ERR_ALIGNMENT otherwise).
+ *  - All arguments are validated before anything is launched; a failed
+ *    validation returns a status and launches nothing. No C++ exception
+ *    crosses this boundary. A launch failure returns WQ_ERR_CUDA (the CUDA
+ *    error is left for cudaGetLastError to report as usual).
+ *  - Rounding: every float -> integer rounding is round-half-to-even, every
+ *    division is an IEEE binary32 division, every narrowing is
+ *    round-to-nearest-even. No fast-math.
+ *  - The current CUDA device is the one every pointer must live on.
+ *
+ * Canonical packed layouts (the only layouts that cross this ABI)
+ * ---------------------------------------------------------------
+ *  INT4 asymmetric, group size G along K ([MIXPE]):
+ *    qweight  uint32 [N, K/8]  code of column k in bits 4*(k%8) .. +3
+ *    scales   fp16   [N, K/G]  s, row-major
+ *    zeros    fp16   [N, K/G]  z (an exact integer 0..15), row-major
+ *    dequant: w = (q - z) * s  (exact in fp32)
+ *    quantize (per row n, group g): lo = min(min w, 0), hi = max(max w, 0);
+ *    s = fp16(fp32(hi - lo) / 15), recomputed with lo=-1, hi=1 if that is 0;
+ *    z = clamp(rint(-lo / s), 0, 15); q = clamp(rint(w / s) + z, 0, 15).
+ *  NF4, block of 64 consecutive elements of the row-major [N, K] weight
+ *  ([NF4], [QLORA]):
+ *    codes    uint8  [N*K/2]   element 2j in the HIGH nibble of byte j,
+ *                              element 2j+1 in the low nibble
+ *    absmax   fp32   [N*K/64]
+ *    dequant: w = fp32(codebook[code] * absmax)
+ *    quantize: absmax = max|w|; code = index of the codebook value nearest to
+ *    fp32(w / absmax), ties to the lower index; an all-zero block stores
+ *    absmax 0 and code 7 (the exact zero).
+ */
+#ifndef WQ_H_
+#define WQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WQ_OK = 0,
+  WQ_ERR_INVALID_ARG = 1,   /* NULL pointer, negative or inconsistent size  */
+  WQ_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels cover */
+  WQ_ERR_ALIGNMENT = 3,     /* a device pointer is not 16-byte aligned      */
+  WQ_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed         */
+  WQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired           */
+  WQ_ERR_WORKSPACE = 6      /* workspace NULL or smaller than required      */
+} wq_status;
+
+typedef enum { WQ_FMT_INT4_ASYM = 0, WQ_FMT_NF4 = 1 } wq_format;
+typedef enum { WQ_BF16 = 0, WQ_FP16 = 1, WQ_FP32 = 2 } wq_dtype;
+typedef enum { WQ_OP_GEMV = 0, WQ_OP_GEMM = 1, WQ_OP_MSD_GEMM = 2 } wq_op;
+
+/* Human-readable name of a status. Never NULL. Host only. */
+const char* wq_status_string(wq_status status);
+
+/* Library version string, e.g. "wq 0.1 sm_100a". Host only. */
+const char* wq_version(void);
+
+/*
+ * The 16 NF4 code values (fp32, ascending) the device kernels use. Host only;
+ * `out` is a host array of 16 floats. The library computes them once from the
+ * QLoRA construction ([QLORA], used by [NF4]): quantiles of the standard
+ * normal at probabilities evenly spaced from delta = (1 - 1/30 + 1 - 1/32)/2
+ * towards 1/2 (8 positive, 7 negative), an exact 0, normalised by the largest,
+ * each rounded once to fp32.
+ */
+wq_status wq_nf4_codebook(float out[16]);
+
+/*
+ * Byte sizes of the caller-allocated packed buffers for `fmt` and an [N, K]
+ * weight. INT4: group G (G % 8 == 0, K % G == 0); qweight N*K/2, scales and
+ * zeros N*(K/G)*2 each. NF4: group must be 64 (the block size), N*K % 64 == 0;
+ * qweight N*K/2, scales = absmax N*K/64*4, zeros 0. This is the 4x memory
+ * reduction of [NF4]. Host only; output pointers are host pointers.
+ */
+wq_status wq_packed_sizes(wq_format fmt, int64_t N, int64_t K, int32_t group,
+                          size_t* qweight_bytes, size_t* scale_bytes,
+                          size_t* zero_bytes);
+
+/*
+ * Quantize and pack fp32 weights W [N, K] (device, row-major) into the
+ * canonical layout above ([MIXPE] group scale/zero; [NF4] codes + absmax).
+ * INT4: `scales`/`zeros` are fp16 [N, K/G]. NF4: group == 64, `scales` is the
+ * fp32 absmax [N*K/64] and `zeros` must be NULL. Requires K % 8 == 0.
+ * Bit-exact with the CPU oracle for finite weights whose group ranges fit
+ * fp16 (|hi - lo| / 15 <= 65504). Non-finite weights give unspecified codes.
+ */
+wq_status wq_quantize_pack(wq_format fmt, const float* W, int64_t N, int64_t K,
+                           int32_t group, void* qweight, void* scales,
+                           void* zeros, void* stream);
+
+/*
+ * Unpack codes to one byte per element: codes[n*K + k] in 0..15, for either
+ * format (NF4: numel = N*K, flattened). For checking packed data.
+ */
+wq_status wq_unpack(wq_format fmt, const void* qweight, int64_t N, int64_t K,
+                    uint8_t* codes, void* stream);
+
+/*
+ * Standalone NF4 dequantization ([NF4]: lifting NF4 back to 16-bit before the
+ * product, the kernel that page accelerates):
+ *   out[i] = RN_dtype( fp32(codebook[code_i] * absmax[i / 64]) )
+ * codes: packed NF4 [numel/2]; absmax fp32 [numel/64]; out bf16 or fp16
+ * [numel]. blocksize must be 64, numel % 64 == 0. Bit-exact with the oracle.
+ */
+wq_status wq_nf4_dequant(const uint8_t* codes, const float* absmax,
+                         int64_t numel, int32_t blocksize, void* out,
+                         wq_dtype out_dtype, void* stream);
+
+/*
+ * Standalone INT4 dequantization ([MSD]: lifting the low-bit weights to bf16,
+ * the step MSD removes; used by the dequantize-then-GEMM baseline):
+ *   out[n, k] = RN_dtype( (q - z) * s )   (the product is exact in fp32)
+ * out bf16 or fp16 [N, K]. K % 8 == 0, K % group == 0, group % 8 == 0.
+ */
+wq_status wq_int4_dequant(const uint32_t* qweight, const void* scales,
+                          const void* zeros, int64_t N, int64_t K,
+                          int32_t group, void* out, wq_dtype out_dtype,
+                          void* stream);
+
+/*
+ * Decode W4A16 GEMV ([MSD], [MIXPE], [NF4]): y[m, n] = sum_k x[m, k] w[n, k]
+ * for 1 <= M <= 16, fp32 accumulation, bf16 output.
+ *   x bf16 [M, K] row-major; y bf16 [M, N] row-major.
+ *   INT4: scales/zeros fp16 [N, K/G], G % 64 == 0, K % G == 0. The group's
+ *         scale and zero are applied after the group's sum ([MIXPE]).
+ *   NF4 : group == 64, scales = fp32 absmax [N*K/64], zeros NULL; the block's
+ *         absmax is applied after the block's sum.
+ * Requires K % 128 == 0 and N % 16 == 0. M == 0 or N == 0 is a no-op.
+ * Workspace: none needed (pass NULL, 0); split-K partials are reduced on chip
+ * through thread-block-cluster shared memory.
+ */
+wq_status wq_w4a16_gemv(const void* x, int64_t M, int64_t N, int64_t K,
+                        wq_format fmt, int32_t group, const void* qweight,
+                        const void* scales, const void* zeros, void* y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Prefill W4A16 GEMM with fused dequantization on the tensor cores ([MSD]:
+ * the dequantize-then-multiply product; here the dequantized tile never
+ * leaves shared memory). Same arguments and layouts as wq_w4a16_gemv, any
+ * M >= 1. INT4 only (WQ_ERR_UNSUPPORTED for NF4). Requires K % 128 == 0,
+ * N % 128 == 0, G % 64 == 0, K % G == 0, and group scales with 15 * s <= 65504.
+ * The product runs in fp16 with fp32 accumulation: x is first copied to fp16
+ * scaled per row by a power of two (exact for bf16 values down to 2^-28 of the
+ * row's largest), each weight is fp16_rn((q - z) * s), and the epilogue
+ * removes the power of two before rounding y to bf16.
+ * Workspace: at least wq_workspace_bytes(WQ_OP_GEMM, ...) bytes (the fp16
+ * copy of x and the per-row scales); contents on entry do not matter.
+ * May return WQ_ERR_TIMEOUT through wq_device_error if an internal bounded
+ * wait expires.
+ */
+wq_status wq_w4a16_gemm(const void* x, int64_t M, int64_t N, int64_t K,
+                        wq_format fmt, int32_t group, const void* qweight,
+                        const void* scales, const void* zeros, void* y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Multi-Scale Dequant activation decomposition ([MSD]): per row m of x
+ * (bf16 [M, K]), n_components (C, 1..3) int8 digit planes a [C, M, K] and
+ * fp32 scales s [C, M] with x ~= sum_c s[c, m] a[c, m, :]:
+ *   s[0] = fp32(amax / 127) (1 for an all-zero row), a[0] = clamp(rint(x /
+ *   s[0]), -127, 127); s[c] = s[c-1] / 256; the residual after c components is
+ *   r = RN32(r - s[c] a[c]) (one rounding); a[c] = rint(r / s[c]) in [-128,
+ *   128], a +128 written as -128 with +1 carried into a[c-1].
+ *   Two components give |x - x_hat| <= s[1] / 2: close to 16 effective bits.
+ * Bit-exact with the oracle. M == 0 is a no-op; K % 16 == 0.
+ */
+wq_status wq_msd_decompose(const void* x, int64_t M, int64_t K,
+                           int32_t n_components, int8_t* digits,
+                           float* comp_scales, void* stream);
+
+/*
+ * Multi-Scale Dequant GEMM ([MSD], with [MIXPE]'s post-group scaling):
+ *   y[m, n] = sum_c s_c[m] sum_g s[n, g] (sum_{k in g} a_c[m, k] (q[n, k] - z[n, g]))
+ * i.e. x_hat . dequant(W)^T, with x_hat the C-component decomposition of x
+ * (wq_msd_decompose). The integer weight codes enter int8 tensor-core MMAs
+ * directly; no weight is converted to a floating-point type.
+ * INT4 asymmetric weights only; group G % 128 == 0 (G == K is per-channel),
+ * K % G == 0, K % 128 == 0, N % 128 == 0, 1 <= n_components <= 3.
+ * Workspace: at least wq_workspace_bytes(WQ_OP_MSD_GEMM, ...) bytes (it holds
+ * the digit planes and scales); its contents on entry do not matter.
+ */
+wq_status wq_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K,
+                      int32_t n_components, int32_t group, const void* qweight,
+                      const void* scales, const void* zeros, void* y,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes an entry point needs for the given problem (0 if none).
+ * Host only; `bytes` is a host pointer.
+ */
+wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K,
+                             int32_t group, int32_t n_components,
+                             size_t* bytes);
+
+/*
+ * Read (and, if `clear` != 0, reset) the library's sticky device error word,
+ * which kernels with bounded waits set when a wait expires. SYNCHRONISES
+ * `stream` first. Returns WQ_ERR_TIMEOUT if the word was set, WQ_OK if not.
+ * `detail` (host, may be NULL) receives the raw word: the id of the kernel
+ * role and wait site that gave up.
+ */
+wq_status wq_device_error(void* stream, int clear, uint32_t* detail);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* WQ_H_ */

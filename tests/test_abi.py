@@ -1,0 +1,134 @@
+"""The C-ABI library loads, exports every declared symbol, and validates its
+arguments on the host (CPU only: no call here reaches a kernel launch)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def wq():
+    from bit_weight_quantized_weights_b200 import build_lib
+    build_lib.build()
+    from bit_weight_quantized_weights_b200 import binding
+    return binding
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "wq.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(wq_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = _declared_symbols()
+    for name in ["wq_quantize_pack", "wq_nf4_dequant", "wq_w4a16_gemv", "wq_w4a16_gemm",
+                 "wq_msd_gemm", "wq_msd_decompose", "wq_workspace_bytes"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(wq):
+    lib = ctypes.CDLL(wq.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert sorted(wq.EXPORTED) == _declared_symbols()
+
+
+def test_status_strings(wq):
+    for s in range(7):
+        assert wq.status_string(s) and wq.status_string(s) != "unknown status"
+    assert wq.status_string(99) == "unknown status"
+    assert "sm_100a" in wq.version()
+
+
+def test_codebook_matches_oracle_bit_exact(wq):
+    """The library computes the codebook on its own (bisection + Newton on
+    erfc); it must equal the oracle's SciPy construction bit for bit."""
+    from oracle import formats
+    cb = np.array(wq.wq_nf4_codebook(), dtype=np.float32)
+    assert np.array_equal(cb.view(np.uint32), formats.nf4_codebook().view(np.uint32))
+
+
+def test_packed_sizes(wq):
+    assert wq.wq_packed_sizes(wq.WQ_FMT_INT4_ASYM, 1024, 1024, 64) == (512 * 1024, 1024 * 16 * 2,
+                                                                        1024 * 16 * 2)
+    q, s, z = wq.wq_packed_sizes(wq.WQ_FMT_NF4, 28672, 8192, 64)
+    assert q == 28672 * 8192 // 2 and s == 28672 * 8192 // 64 * 4 and z == 0
+    with pytest.raises(wq.WqError):
+        wq.wq_packed_sizes(wq.WQ_FMT_INT4_ASYM, 16, 100, 64)   # K % G
+    with pytest.raises(wq.WqError):
+        wq.wq_packed_sizes(wq.WQ_FMT_NF4, 16, 128, 128)        # NF4 block must be 64
+
+
+def test_workspace_sizes(wq):
+    assert wq.wq_workspace_bytes(wq.WQ_OP_GEMV, 16, 4096, 4096, 128) == 0
+    assert wq.wq_workspace_bytes(wq.WQ_OP_GEMM, 8192, 4096, 4096, 128) >= 8192 * 4096 * 2 + 8192 * 4
+    assert wq.wq_workspace_bytes(wq.WQ_OP_GEMM, 0, 4096, 4096, 128) == 0
+    ws = wq.wq_workspace_bytes(wq.WQ_OP_MSD_GEMM, 1024, 5120, 5120, 128, 2)
+    assert ws >= 2 * 1024 * 5120 + 2 * 1024 * 4
+    assert wq.wq_workspace_bytes(wq.WQ_OP_MSD_GEMM, 0, 5120, 5120, 128, 2) == 0
+
+
+# Fake device addresses: validation must fail (or finish as a no-op) before
+# anything dereferences them or launches.
+A16 = 0x10000
+MIS = 0x10001
+
+
+def _gemv(wq, m, n, k, fmt=0, group=128, x=A16, q=A16, s=A16, z=A16, y=A16):
+    return wq.lib.wq_w4a16_gemv(x, m, n, k, fmt, group, q, s, z, y, None, 0, None)
+
+
+def test_gemv_validation(wq):
+    assert _gemv(wq, 17, 4096, 4096) == wq.WQ_ERR_UNSUPPORTED        # decode only
+    assert _gemv(wq, 1, 4096, 4000) == wq.WQ_ERR_INVALID_ARG          # K % G
+    assert _gemv(wq, 1, 4096, 4096, group=96) == wq.WQ_ERR_INVALID_ARG  # K % G (4096 % 96)
+    assert _gemv(wq, 1, 4096, 4096, group=32) == wq.WQ_ERR_UNSUPPORTED  # G % 64
+    assert _gemv(wq, 1, 4096, 4096, x=0) == wq.WQ_ERR_INVALID_ARG
+    assert _gemv(wq, 1, 4096, 4096, y=MIS) == wq.WQ_ERR_ALIGNMENT
+    assert _gemv(wq, 1, 4100, 4096) == wq.WQ_ERR_UNSUPPORTED          # N % 16
+    assert _gemv(wq, 1, 4096, 4096, fmt=1, group=64) == wq.WQ_ERR_INVALID_ARG  # NF4 w/ zeros
+    assert _gemv(wq, 1, 4096, 4096, fmt=7) == wq.WQ_ERR_INVALID_ARG
+    assert _gemv(wq, -1, 4096, 4096) == wq.WQ_ERR_INVALID_ARG
+    assert _gemv(wq, 0, 4096, 4096) == wq.WQ_OK                      # empty: no-op
+    assert _gemv(wq, 4, 0, 4096) == wq.WQ_OK
+
+
+def test_gemm_and_msd_validation(wq):
+    L = wq.lib
+    assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 1, 64, A16, A16, None, A16, None, 0,
+                           None) == wq.WQ_ERR_UNSUPPORTED               # NF4 GEMM
+    assert L.wq_w4a16_gemm(A16, 512, 4160, 4096, 0, 128, A16, A16, A16, A16, None, 0,
+                           None) == wq.WQ_ERR_UNSUPPORTED               # N % 128
+    assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 0, 128, A16, A16, A16, MIS, None, 0,
+                           None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_w4a16_gemm(A16, 0, 4096, 4096, 0, 128, A16, A16, A16, A16, None, 0,
+                           None) == wq.WQ_OK
+    assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 0, 128, A16, A16, A16, A16, None, 0,
+                           None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 1024,
+                           None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_msd_gemm(A16, 16, 5120, 5120, 2, 128, A16, A16, A16, A16, None, 0,
+                         None) == wq.WQ_ERR_WORKSPACE
+    assert L.wq_msd_gemm(A16, 16, 5120, 5120, 4, 128, A16, A16, A16, A16, A16, 1 << 30,
+                         None) == wq.WQ_ERR_INVALID_ARG                 # C in 1..3
+    assert L.wq_msd_gemm(A16, 16, 5120, 5120, 2, 64, A16, A16, A16, A16, A16, 1 << 30,
+                         None) == wq.WQ_ERR_UNSUPPORTED                 # G % 128
+    assert L.wq_msd_decompose(A16, 4, 100, 2, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_msd_decompose(A16, 0, 128, 2, A16, A16, None) == wq.WQ_OK
+
+
+def test_pack_and_dequant_validation(wq):
+    L = wq.lib
+    assert L.wq_quantize_pack(0, A16, 16, 100, 64, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(1, A16, 16, 128, 64, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_quantize_pack(0, MIS, 16, 128, 64, A16, A16, A16, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_nf4_dequant(A16, A16, 100, 64, A16, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_nf4_dequant(A16, A16, 128, 32, A16, 0, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_nf4_dequant(A16, A16, 128, 64, A16, 2, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_nf4_dequant(A16, A16, 0, 64, A16, 0, None) == wq.WQ_OK
+    assert L.wq_int4_dequant(A16, A16, A16, 16, 128, 12, A16, 0, None) == wq.WQ_ERR_INVALID_ARG

@@ -1,0 +1,88 @@
+"""GPU parity of the tcgen05 prefill GEMM (fused INT4 dequantization).
+
+Small cases (several tiles in M, N and K, ragged M, every group size the
+kernel supports) compare every output with the fp64 oracle; the full prefill
+workloads (M = 512, 2048, 8192 x Llama-3-8B shapes, INT4 g128) compare sampled
+rows x columns computed one by one by the oracle. The kernel multiplies in
+fp16 (x exact after a per-row power-of-two scaling, each weight rounded once
+to fp16), so besides the product tolerance every output must lie within one
+bf16 rounding of the exact product (plus 1e-3 of its RMS for the fp16 weight
+rounding and fp32 accumulation).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import products
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wq():
+    import bit_weight_quantized_weights_b200 as pkg
+    return pkg.binding
+
+
+def _x(m, k, seed):
+    from bit_weight_quantized_weights_b200 import workloads
+    return workloads.activations(m, k, gen=workloads.generator(seed + 2000))
+
+
+@pytest.mark.parametrize("m,n,k,group", [
+    (128, 256, 256, 128),     # one 128x128 tile column pair, 4 k-tiles
+    (300, 384, 640, 128),     # ragged M, N not a multiple of 256, ring wraps (10 k-tiles)
+    (1, 128, 128, 64),        # one row
+    (257, 512, 1024, 1024),   # per-channel groups
+    (64, 256, 512, 64),       # M below one tile
+])
+def test_gemm_small_every_element(wq, m, n, k, group):
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed=m)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, m)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_INT4_ASYM, group, qw, sc, zr)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    y_ref = products.w4a16_int4(helpers.x_f32(x), q, s, z, group)
+    helpers.check_product(y, y_ref, "gemm %dx%dx%d g%d" % (m, n, k, group))
+    helpers.check_within_bf16_rounding(y, y_ref, "gemm %dx%dx%d g%d" % (m, n, k, group),
+                                       slack=1e-3)
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (14336, 4096), (4096, 14336)])
+@pytest.mark.parametrize("m", [512, 2048, 8192])
+def test_gemm_prefill_full_size_sampled(wq, m, n, k):
+    q, s, z, qweight = helpers.int4_packed(n, k, 128, seed=0)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, 0)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    rng = np.random.default_rng(m + n + k)
+    rows = np.sort(rng.choice(m, 48, replace=False))
+    cols = np.sort(rng.choice(n, 192, replace=False))
+    ys = y.cpu()[rows][:, cols]
+    y_ref = products.w4a16_int4(helpers.x_f32(x)[rows], q[cols], s[cols], z[cols], 128)
+    helpers.check_product(ys, y_ref, "gemm %dx%dx%d sampled" % (m, n, k))
+    helpers.check_within_bf16_rounding(ys, y_ref, "gemm %dx%dx%d sampled" % (m, n, k),
+                                       slack=1e-3)
+
+
+def test_gemm_large_activation_range(wq):
+    """Rows whose magnitudes span many binades (and one beyond the fp16 range)
+    still multiply exactly: the per-row power-of-two scaling keeps them exact."""
+    m, n, k, group = 130, 256, 512, 128
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed=77)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, 77).float()
+    x[0] *= 1e5          # beyond fp16's range before scaling
+    x[1] *= 1e-6         # far below it
+    x[2, ::3] *= 1e-3
+    x = x.to(torch.bfloat16)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_INT4_ASYM, group, qw, sc, zr)
+    y_ref = products.w4a16_int4(helpers.x_f32(x), q, s, z, group)
+    for r in range(3):
+        helpers.check_within_bf16_rounding(y[r:r + 1], y_ref[r:r + 1], "row %d" % r, slack=1e-3)
+    helpers.check_within_bf16_rounding(y[3:], y_ref[3:], "rest", slack=1e-3)

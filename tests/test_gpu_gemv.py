@@ -1,0 +1,111 @@
+"""GPU parity of the decode GEMV against the fp64 oracle product.
+
+All decode workloads (Llama-2-7B linear shapes, M = 1, 4, 8, 16, INT4 g128 and
+NF4 b64, 1% outlier channels x20) and the tiny INT4 g64 case are run at full
+size, every output compared. INT4 dequantizes exactly inside the kernel and
+NF4 multiplies fp16 code values (11 significant bits) by exactly scaled fp16
+activations, so besides the product tolerance every output must lie within
+one bf16 rounding of the exact product.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import formats, products
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wq():
+    import bit_weight_quantized_weights_b200 as pkg
+    return pkg.binding
+
+
+def _x(m, k, seed, outliers):
+    from bit_weight_quantized_weights_b200 import workloads
+    g = workloads.generator(seed + 1000)
+    return workloads.activations(m, k, gen=g, outliers=outliers)
+
+
+def _run_int4(wq, m, n, k, group, outliers=(0.01, 20.0), seed=0, exact_check=True):
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, seed, outliers)
+    y = wq.wq_w4a16_gemv(x.cuda(), n, wq.WQ_FMT_INT4_ASYM, group, qw, sc, zr)
+    torch.cuda.synchronize()
+    y_ref = products.w4a16_int4(helpers.x_f32(x), q, s, z, group)
+    helpers.check_product(y, y_ref, "int4 gemv M=%d %dx%d" % (m, n, k))
+    if exact_check:
+        helpers.check_within_bf16_rounding(y, y_ref, "int4 gemv M=%d %dx%d" % (m, n, k))
+
+
+def _run_nf4(wq, m, n, k, outliers=(0.01, 20.0), seed=0):
+    codes, absmax, packed = helpers.nf4_packed(n, k, seed)
+    cw, am = helpers.to_dev_nf4(absmax, packed)
+    x = _x(m, k, seed, outliers)
+    y = wq.wq_w4a16_gemv(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None)
+    torch.cuda.synchronize()
+    y_ref = products.w4a16_nf4(helpers.x_f32(x), codes, absmax, k)
+    helpers.check_within_bf16_rounding(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k), slack=1e-3)
+    return helpers.check_product(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k))
+
+
+def test_gemv_tiny_int4_g64(wq):
+    """x [1 x 1024], W [1024 x 1024], INT4 with fp16 scale/zero per 64 inputs."""
+    _run_int4(wq, 1, 1024, 1024, 64, outliers=None)
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("m", [1, 4, 8, 16])
+def test_gemv_decode_int4_g128(wq, m, n, k):
+    _run_int4(wq, m, n, k, 128)
+
+
+@pytest.mark.parametrize("n,k", [(4096, 4096), (11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("m", [1, 4, 8, 16])
+def test_gemv_decode_nf4(wq, m, n, k):
+    _run_nf4(wq, m, n, k)
+
+
+@pytest.mark.parametrize("m,n,k,group", [(3, 1040, 384, 128), (9, 144, 256, 256),
+                                         (16, 16, 128, 128), (5, 2064, 1152, 64),
+                                         (2, 528, 640, 640)])
+def test_gemv_ragged_and_groups(wq, m, n, k, group):
+    """N not a multiple of the 128-row tile, odd M, groups larger than the
+    128-wide unit, per-channel groups (G = K)."""
+    _run_int4(wq, m, n, k, group, seed=m)
+
+
+@pytest.mark.parametrize("m,n,k", [(3, 1040, 384), (13, 272, 1280)])
+def test_gemv_ragged_nf4(wq, m, n, k):
+    _run_nf4(wq, m, n, k, seed=m)
+
+
+def test_gemv_empty_is_noop(wq):
+    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    y = torch.full((0, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    qw = torch.zeros(64, 32, dtype=torch.int32, device="cuda")
+    sc = torch.ones(64, 2, dtype=torch.float16, device="cuda")
+    wq.wq_w4a16_gemv(x, 64, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, sc, out=y)
+
+
+def test_gemv_rejects_m17(wq):
+    x = torch.zeros(17, 256, dtype=torch.bfloat16, device="cuda")
+    qw = torch.zeros(64, 32, dtype=torch.int32, device="cuda")
+    sc = torch.ones(64, 2, dtype=torch.float16, device="cuda")
+    with pytest.raises(wq.WqError) as e:
+        wq.wq_w4a16_gemv(x, 64, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, sc)
+    assert e.value.status == wq.WQ_ERR_UNSUPPORTED
+
+
+def test_gemv_nan_propagates(wq):
+    """A NaN activation makes that token's outputs NaN (documented behaviour)."""
+    q, s, z, qweight = helpers.int4_packed(128, 256, 128, 9)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = torch.ones(2, 256, dtype=torch.bfloat16)
+    x[1, 7] = float("nan")
+    y = wq.wq_w4a16_gemv(x.cuda(), 128, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr).cpu()
+    assert torch.isfinite(y[0].float()).all() and torch.isnan(y[1].float()).all()

@@ -1,0 +1,110 @@
+"""GPU parity of the Multi-Scale Dequant path: the activation decomposition is
+bit-exact with the oracle (digits and scales)."""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import msd
+from tests import helpers
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def wq():
+    import bit_weight_quantized_weights_b200 as pkg
+    return pkg.binding
+
+
+def _x(m, k, seed, outliers=(0.005, 50.0)):
+    from bit_weight_quantized_weights_b200 import workloads
+    return workloads.activations(m, k, gen=workloads.generator(seed + 3000), outliers=outliers)
+
+
+@pytest.mark.parametrize("m,k", [(1, 5120), (16, 5120), (128, 25600), (1024, 5120), (3, 4096)])
+@pytest.mark.parametrize("c", [1, 2, 3])
+def test_decompose_bit_exact(wq, m, k, c):
+    x = _x(m, k, m + c)
+    if m >= 3:
+        x[1] = 0.0                                         # all-zero row
+        x[2, :8] = torch.tensor([127.0, 1.0, 0.5, -0.5, 0.25, 63.5, -127.0, 0.75])
+        x[2, 8:] = 0.0                                     # the hand-derived row
+    a_ref, s_ref = msd.decompose(helpers.x_f32(x), c)
+    a, s = wq.wq_msd_decompose(x.cuda(), c)
+    torch.cuda.synchronize()
+    assert np.array_equal(a.cpu().numpy(), a_ref)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# ---------------------------------------------------------------------------
+# the decomposed integer GEMM
+# ---------------------------------------------------------------------------
+
+def _msd_case(wq, m, n, k, group, c, seed, rows=None, cols=None):
+    from oracle import products
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed=seed)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, seed)
+    y = wq.wq_msd_gemm(x.cuda(), n, c, group, qw, sc, zr)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    xf = helpers.x_f32(x)
+    a, sa = msd.decompose(xf, c)
+    if rows is None:
+        rows = np.arange(m)
+    if cols is None:
+        cols = np.arange(n)
+    y_dec = msd.msd_product(a[:, rows], sa[:, rows], q[cols], s[cols], z[cols], group)
+    y_exact = products.w4a16_int4(xf[rows], q[cols], s[cols], z[cols], group)
+    yg = y.cpu()[rows][:, cols]
+    what = "msd C=%d M=%d %dx%d g%d" % (c, m, n, k, group)
+    # (i) the decomposed product itself: only the final bf16 rounding remains
+    helpers.check_within_bf16_rounding(yg, y_dec, what + " vs decomposed", slack=1e-4)
+    # (ii) against the undecomposed product, under the product tolerance
+    if c >= 2:
+        helpers.check_product(yg, y_exact, what + " vs exact")
+    return yg, y_exact
+
+
+@pytest.mark.parametrize("m,n,k,group,c", [
+    (128, 256, 512, 128, 2),     # 2 tiles along N, 4 groups
+    (300, 384, 640, 128, 2),     # ragged M (3 M-tiles), 5 groups
+    (1, 128, 256, 128, 2),       # one token
+    (16, 256, 1024, 1024, 2),    # per-channel group (single drain)
+    (130, 128, 384, 128, 1),     # one component
+    (130, 256, 384, 128, 3),     # three components (single TMEM buffer)
+    (64, 128, 1152, 384, 2),     # group of 3 k-tiles
+])
+def test_msd_gemm_small_every_element(wq, m, n, k, group, c):
+    _msd_case(wq, m, n, k, group, c, seed=m + c)
+
+
+@pytest.mark.parametrize("n,k", [(5120, 5120), (25600, 5120), (5120, 25600)])
+@pytest.mark.parametrize("m", [1, 16, 128, 1024])
+@pytest.mark.parametrize("per_channel", [True, False])
+def test_msd_gemm_full_size_sampled(wq, m, n, k, per_channel):
+    """Qwen3-32B shapes, 0.5% outlier channels x50, INT4 per-channel and g128,
+    two components; sampled rows x columns against the oracle."""
+    group = k if per_channel else 128
+    rng = np.random.default_rng(m * 7 + n + k + group)
+    rows = np.sort(rng.choice(m, min(m, 48), replace=False))
+    cols = np.sort(rng.choice(n, 192, replace=False))
+    _msd_case(wq, m, n, k, group, 2, seed=0, rows=rows, cols=cols)
+
+
+def test_msd_accuracy_not_below_dequant_baseline(wq):
+    """The page reports that MSD does not lose accuracy against dequantize-then-
+    multiply baselines; here the measured L2 errors of both against the exact
+    product are reported (parity unpinned: the page prints no numbers). The
+    assertion is only the product tolerance for two components."""
+    from oracle import products, numerics
+    m, n, k, group = 64, 512, 5120, 128
+    yg, y_exact = _msd_case(wq, m, n, k, group, 2, seed=5)
+    q, s, z, _ = helpers.int4_packed(n, k, group, seed=5)
+    x = helpers.x_f32(_x(m, k, 5))
+    y_bf16w = products.dequant_then_bf16_matmul_int4(x, q, s, z, group)
+    rel_msd, _ = numerics.compare(yg.float().numpy(), y_exact)
+    rel_deq, _ = numerics.compare(numerics.bf16_round(y_bf16w.astype(np.float32)), y_exact)
+    print("relative L2 error: msd C=2 %.3e, bf16 dequantize-then-GEMM %.3e" % (rel_msd, rel_deq))
+    assert rel_msd <= helpers.REL_FRO_TOL

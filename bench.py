@@ -1,0 +1,540 @@
+"""Benchmark of the 4-bit weight-only quantized product hot path on B200.
+
+One *step* runs every hot-path operation once on synthetic Llama/Qwen-shaped
+layers (seeded, weights N(0, 0.02) quantized on the GPU, activations N(0, 1)
+with outlier channels):
+
+  nf4_dequant   NF4 -> bf16, W [28672 x 8192]                      (HBM-bound)
+  gemv_int4     decode GEMV, M = 16, W [11008 x 4096], INT4 g128    (HBM-bound)
+  gemv_nf4      decode GEMV, M = 16, W [11008 x 4096], NF4 b64      (HBM-bound)
+  gemm          prefill GEMM, M = 8192, W [14336 x 4096], INT4 g128 (tensor-bound)
+  msd_m16       MSD GEMM, C = 2, M = 16, W [25600 x 5120], g128     (HBM-bound)
+  msd_m1024     MSD GEMM, C = 2, M = 1024, W [25600 x 5120], g128   (tensor-bound)
+
+Metric: "% of B200 roofline" of the whole step, work-weighted: for every op
+its roofline time max(algorithmic bytes / HBM peak, algorithmic ops / tensor
+peak) is summed, and divided by the measured step time. With N GPUs each rank
+runs its own replica (no data-path collective) and the value is the sum over
+ranks (weak scaling; 100 per GPU is the ceiling).
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+synchronize on both sides, CUDA events on the launching stream, max over
+ranks. L2: every op's inputs were last touched one step earlier and the 600 MB
+NF4 dequantization stream (> 4x the 126 MB L2) runs in between, so every op
+starts L2-cold. `--impl reference` times the CPU oracle on a bounded sample of
+the same step instead (rank 0 only).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-GEMM GB/s (decode) & TFLOP/s (prefill) as % of B200 roofline"
+UNIT = "% of one B200 roofline (work-weighted over the step, summed over GPUs)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+GEMV_SHAPE = (11008, 4096)
+GEMM_SHAPE = (8192, 14336, 4096)
+MSD_SHAPE = (25600, 5120)
+NF4_SHAPE = (28672, 8192)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def op_table(peaks):
+    """Algorithmic bytes and ops of each op of the step, with its roofline time.
+
+    Bytes: packed weights (0.5 B/weight) + scales/zeros or absmax + activations
+    read + outputs written; ops: 2*M*N*K multiply-adds (x2 components for MSD).
+    The int8 peak is the measured bf16 peak x 2 (dense int8 runs at twice the
+    bf16 rate on B200)."""
+    bw = peaks["hbm_gbs"] * 1e9
+    tf16 = peaks["bf16_tflops"] * 1e12
+    ti8 = 2.0 * tf16
+    n, k = NF4_SHAPE
+    gn, gk = GEMV_SHAPE
+    m, pn, pk = GEMM_SHAPE
+    sn, sk = MSD_SHAPE
+    ops = {
+        "nf4_dequant": dict(bytes=n * k * (0.5 + 4 / 64 + 2), flops=0, peak_flops=tf16, bound="hbm"),
+        "gemv_int4": dict(bytes=gn * gk * (0.5 + 4 / 128) + 2 * 16 * gk + 2 * 16 * gn,
+                          flops=2 * 16 * gn * gk, peak_flops=tf16, bound="hbm"),
+        "gemv_nf4": dict(bytes=gn * gk * (0.5 + 4 / 64) + 2 * 16 * gk + 2 * 16 * gn,
+                         flops=2 * 16 * gn * gk, peak_flops=tf16, bound="hbm"),
+        "gemm": dict(bytes=pn * pk * (0.5 + 4 / 128) + 2 * m * pk + 2 * m * pn,
+                     flops=2 * m * pn * pk, peak_flops=tf16, bound="tensor"),
+        "msd_m16": dict(bytes=sn * sk * (0.5 + 4 / 128) + 2 * 16 * sk + 2 * 16 * sn,
+                        flops=2 * 2 * 16 * sn * sk, peak_flops=ti8, bound="hbm"),
+        "msd_m1024": dict(bytes=sn * sk * (0.5 + 4 / 128) + 2 * 1024 * sk + 2 * 1024 * sn,
+                          flops=2 * 2 * 1024 * sn * sk, peak_flops=ti8, bound="tensor"),
+    }
+    for v in ops.values():
+        v["t_roof"] = max(v["bytes"] / bw, v["flops"] / v["peak_flops"] if v["flops"] else 0.0)
+    return ops
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML every 50 ms."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.05)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons)}
+
+
+# ---------------------------------------------------------------------------
+# the GPU step
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Device-resident inputs, outputs and workspaces of one hot-path step."""
+
+    def __init__(self, wq, device, seed=0):
+        g = torch.Generator(device=device)
+        g.manual_seed(seed)
+        self.wq = wq
+        F = wq.WQ_FMT_INT4_ASYM
+
+        def normal(*shape, std=1.0):
+            return torch.randn(*shape, generator=g, device=device) * std
+
+        def acts(m, k, frac, scale):
+            x = normal(m, k)
+            idx = torch.randperm(k, generator=g, device=device)[:max(1, round(frac * k))]
+            x[:, idx] *= scale
+            return x.to(torch.bfloat16)
+
+        n, k = NF4_SHAPE
+        w = normal(n, k, std=0.02)
+        self.nf4_codes, self.nf4_absmax, _ = wq.wq_quantize_pack(wq.WQ_FMT_NF4, w, 64)
+        del w
+        self.nf4_out = torch.empty(n * k, dtype=torch.bfloat16, device=device)
+
+        gn, gk = GEMV_SHAPE
+        w = normal(gn, gk, std=0.02)
+        self.gi = wq.wq_quantize_pack(F, w, 128)
+        self.gn = wq.wq_quantize_pack(wq.WQ_FMT_NF4, w, 64)
+        del w
+        self.gx = acts(16, gk, 0.01, 20.0)
+        self.gy_i = torch.empty(16, gn, dtype=torch.bfloat16, device=device)
+        self.gy_n = torch.empty(16, gn, dtype=torch.bfloat16, device=device)
+
+        m, pn, pk = GEMM_SHAPE
+        w = normal(pn, pk, std=0.02)
+        self.pw = wq.wq_quantize_pack(F, w, 128)
+        del w
+        self.px = normal(m, pk).to(torch.bfloat16)
+        self.py = torch.empty(m, pn, dtype=torch.bfloat16, device=device)
+        self.pws = wq.gemm_workspace(m, pn, pk, 128, device)
+
+        sn, sk = MSD_SHAPE
+        w = normal(sn, sk, std=0.02)
+        self.sw = wq.wq_quantize_pack(F, w, 128)
+        del w
+        self.sx16 = acts(16, sk, 0.005, 50.0)
+        self.sx1024 = acts(1024, sk, 0.005, 50.0)
+        self.sy16 = torch.empty(16, sn, dtype=torch.bfloat16, device=device)
+        self.sy1024 = torch.empty(1024, sn, dtype=torch.bfloat16, device=device)
+        self.sws16 = wq.msd_workspace(16, sn, sk, 128, 2, device)
+        self.sws1024 = wq.msd_workspace(1024, sn, sk, 128, 2, device)
+        torch.cuda.synchronize()
+
+    LAUNCHES_PER_STEP = 9  # nf4 1, gemv 2, gemm 2 (x->fp16 + GEMM), msd 2 x 2 (decompose + GEMM)
+
+    def ops(self):
+        wq = self.wq
+        n, k = NF4_SHAPE
+        gn, _ = GEMV_SHAPE
+        _, pn, _ = GEMM_SHAPE
+        sn, _ = MSD_SHAPE
+        return [
+            ("nf4_dequant", lambda: wq.wq_nf4_dequant(self.nf4_codes, self.nf4_absmax, n * k,
+                                                      out=self.nf4_out)),
+            ("gemv_int4", lambda: wq.wq_w4a16_gemv(self.gx, gn, wq.WQ_FMT_INT4_ASYM, 128,
+                                                   *self.gi, out=self.gy_i)),
+            ("gemv_nf4", lambda: wq.wq_w4a16_gemv(self.gx, gn, wq.WQ_FMT_NF4, 64, *self.gn,
+                                                  out=self.gy_n)),
+            ("gemm", lambda: wq.wq_w4a16_gemm(self.px, pn, wq.WQ_FMT_INT4_ASYM, 128, *self.pw,
+                                              workspace=self.pws, out=self.py)),
+            ("msd_m16", lambda: wq.wq_msd_gemm(self.sx16, sn, 2, 128, *self.sw,
+                                               workspace=self.sws16, out=self.sy16)),
+            ("msd_m1024", lambda: wq.wq_msd_gemm(self.sx1024, sn, 2, 128, *self.sw,
+                                                 workspace=self.sws1024, out=self.sy1024)),
+        ]
+
+
+def captured_traffic(op):
+    """DRAM bytes (read + write) per launch of `op` from the committed ncu
+    summary, or None when that kernel's source changed since the capture."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(prof):
+        return None
+    with open(prof) as f:
+        entry = json.load(f).get(op)
+    if not entry:
+        return None
+    with open(os.path.join(ROOT, entry["source"]), "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != entry["source_sha"]:
+            return None
+    return entry["bytes_per_launch"]
+
+
+def run_gpu(args, rank, world, device):
+    from bit_weight_quantized_weights_b200 import binding as wq
+    peaks = load_peaks()
+    table = op_table(peaks)
+    step = Step(wq, device)
+    ops = step.ops()
+
+    for _ in range(args.warmup):
+        for _, fn in ops:
+            fn()
+    st, detail = wq.wq_device_error()
+    if st != wq.WQ_OK:
+        raise RuntimeError("device error word set during warm-up: 0x%x" % detail)
+
+    # per-op events inside the timed steps
+    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)] for name, _ in ops}
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0.record()
+        for i in range(args.steps):
+            for name, fn in ops:
+                a, b = ev[name][i]
+                a.record()
+                fn()
+                b.record()
+        t1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = max_over_ranks(elapsed_ms, world, device)
+    per_op_ms = {name: sum(a.elapsed_time(b) for a, b in ev[name]) / args.steps for name, _ in ops}
+    st, detail = wq.wq_device_error()
+    if st != wq.WQ_OK:
+        raise RuntimeError("device error word set during timing: 0x%x" % detail)
+
+    ms_per_step = elapsed_ms / args.steps
+    roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
+    value = 100.0 * roof_ms / ms_per_step * world
+
+    # dominant kernel: the op with the largest share of the step
+    dom = max(per_op_ms, key=per_op_ms.get)
+    d = table[dom]
+    dur_s = per_op_ms[dom] * 1e-3
+    if d["bound"] == "tensor":
+        achieved = d["flops"] / dur_s / 1e12
+        peak = d["peak_flops"] / 1e12
+        unit = "TFLOP/s" if dom == "gemm" else "TOP/s"
+    else:
+        achieved = d["bytes"] / dur_s / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    traffic = captured_traffic(dom)
+
+    e2e = measure_e2e(args, step, ops, table, world, device) if args.e2e else None
+
+    details = {name: dict(ms=per_op_ms[name], roof_ms=table[name]["t_roof"] * 1e3,
+                          frac=table[name]["t_roof"] * 1e3 / per_op_ms[name],
+                          gbs=table[name]["bytes"] / (per_op_ms[name] * 1e-3) / 1e9,
+                          tflops=table[name]["flops"] / (per_op_ms[name] * 1e-3) / 1e12)
+               for name in per_op_ms}
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4/nf4 weights, bf16 activations; fp16 and int8 tensor-core MMA, fp32 accumulate",
+        "data": "synthetic (seeded; W ~ N(0,0.02) quantized on the GPU, x ~ N(0,1) with outlier channels)",
+        "config": {"workload": "hot-path step: nf4_dequant 28672x8192; gemv int4-g128 and nf4-b64 "
+                               "M=16 11008x4096; gemm int4-g128 8192x14336x4096; msd C=2 g128 "
+                               "M=16 and M=1024 25600x5120",
+                   "l2": "cold: each op's inputs were last touched a step earlier, with the "
+                         "600 MB NF4 stream (>4x L2) in between",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": d["bound"], "kernel": dom, "achieved": round(achieved, 2),
+                     "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "peak_source": peaks["source"] + " (burst)"},
+        "per_op": {k: {a: round(b, 4) for a, b in v.items()} for k, v in details.items()},
+        "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(peaks)
+    return line
+
+
+def measure_e2e(args, step, ops, table, world, device):
+    """The same step through the same C-ABI calls, but with every op's inputs
+    in pinned host memory and its outputs read back to pinned host memory,
+    the copies inside the timed region."""
+    ins = {"nf4_dequant": [step.nf4_codes, step.nf4_absmax], "gemv_int4": [step.gx],
+           "gemv_nf4": [], "gemm": [step.px], "msd_m16": [step.sx16], "msd_m1024": [step.sx1024]}
+    outs = {"nf4_dequant": step.nf4_out, "gemv_int4": step.gy_i, "gemv_nf4": step.gy_n,
+            "gemm": step.py, "msd_m16": step.sy16, "msd_m1024": step.sy1024}
+    host_in = {n: [t.cpu().pin_memory() for t in ts] for n, ts in ins.items()}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in outs.items()}
+    h2d = sum(t.numel() * t.element_size() for ts in host_in.values() for t in ts)
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    steps = max(1, min(args.steps, 5))
+
+    def one():
+        for name, fn in ops:
+            for dev_t, h in zip(ins[name], host_in[name]):
+                dev_t.copy_(h, non_blocking=True)
+            fn()
+            host_out[name].copy_(outs[name], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world, device) / steps
+    roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
+    return {"value": round(100.0 * roof_ms / ms * world, 3), "unit": UNIT,
+            "ms_per_step": round(ms, 3), "steps": steps,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample of the step
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """The CPU oracle on a row sample of every op of the step.
+
+    prepare() draws and quantizes the sampled inputs (not timed); run() times
+    only the oracle's arithmetic and returns (cpu seconds, roofline seconds of
+    the sampled work). `scale` shrinks every sample proportionally."""
+
+    def __init__(self, peaks, scale=1.0):
+        self.table = op_table(peaks)
+        self.scale = scale
+        self.frac = {"nf4_dequant": scale / 256, "gemv_int4": scale / 16,
+                     "gemv_nf4": scale / 16, "gemm": max(1, round(16 * scale)) / 8192,
+                     "msd_m16": scale / 16, "msd_m1024": max(1, round(4 * scale)) / 1024}
+
+    def prepare(self):
+        from oracle import formats
+        from bit_weight_quantized_weights_b200 import workloads
+        f = self.frac
+        n, k = NF4_SHAPE
+        w = workloads.weights(max(1, int(n * f["nf4_dequant"])), k, seed=1).numpy()
+        self.nf4 = formats.nf4_quantize(w)
+        gn, gk = GEMV_SHAPE
+        w, x = workloads.layer(16, max(16, int(gn * f["gemv_int4"])), gk, seed=2,
+                               outliers=(0.01, 20.0))
+        self.gx = x.float().numpy()
+        self.gi = formats.int4_quantize(w.numpy(), 128)
+        self.gn = formats.nf4_quantize(w.numpy())
+        m, pn, pk = GEMM_SHAPE
+        w, x = workloads.layer(round(m * f["gemm"]), pn, pk, seed=3)
+        self.px = x.float().numpy()
+        self.pw = formats.int4_quantize(w.numpy(), 128)
+        sn, sk = MSD_SHAPE
+        w, x = workloads.layer(16, max(16, int(sn * f["msd_m16"])), sk, seed=4,
+                               outliers=(0.005, 50.0))
+        self.s16 = (x.float().numpy(), formats.int4_quantize(w.numpy(), 128))
+        w, x = workloads.layer(round(1024 * f["msd_m1024"]), sn, sk, seed=5,
+                               outliers=(0.005, 50.0))
+        self.s1024 = (x.float().numpy(), formats.int4_quantize(w.numpy(), 128))
+        return self
+
+    def run(self):
+        from oracle import formats, msd, products
+        t0 = time.perf_counter()
+        formats.nf4_dequant_bf16(*self.nf4)
+        products.w4a16_int4(self.gx, *self.gi, 128)
+        products.w4a16_nf4(self.gx, *self.gn, GEMV_SHAPE[1])
+        products.w4a16_int4(self.px, *self.pw, 128)
+        for xf, (q, s, z) in (self.s16, self.s1024):
+            a, sa = msd.decompose(xf, 2)
+            msd.msd_product(a, sa, q, s, z, 128)
+        t_cpu = time.perf_counter() - t0
+        roof = sum(self.table[name]["t_roof"] * fr for name, fr in self.frac.items())
+        return t_cpu, roof
+
+    def describe(self):
+        f = self.frac
+        return ("oracle (NumPy, fp64) on a sample of the step: %.4g of the NF4 rows, %.4g of the "
+                "GEMV rows, %d of 8192 GEMM tokens, %.4g of the MSD M=16 rows, %d of 1024 MSD "
+                "tokens; value = roofline time of that work / CPU time"
+                % (f["nf4_dequant"], f["gemv_int4"], round(f["gemm"] * 8192), f["msd_m16"],
+                   round(f["msd_m1024"] * 1024)))
+
+
+def oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([p.get("num_threads", 1) for p in threadpool_info()] + [1]))
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(peaks, scale=1.0):
+    """The oracle as it stands, timed once on a bounded sample of the step."""
+    sample = OracleSample(peaks, scale).prepare()
+    t_cpu, roof = sample.run()
+    return {"value": round(100.0 * roof / t_cpu, 6), "unit": UNIT, "cores": oracle_cores(),
+            "kind": "oracle", "sample": sample.describe(), "cpu_seconds": round(t_cpu, 2)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas: barrier + max of the timing only)
+# ---------------------------------------------------------------------------
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="wq", choices=["wq", "reference"])
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--detail", default=None, help="also write the JSON line to this file")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        peaks = load_peaks()
+        steps = max(1, args.steps)
+        sample = OracleSample(peaks, scale=0.25).prepare()
+        for _ in range(args.warmup):
+            sample.run()
+        t_tot, roof_tot = 0.0, 0.0
+        for _ in range(steps):
+            t, r = sample.run()
+            t_tot += t
+            roof_tot += r
+        value = round(100.0 * roof_tot / t_tot, 6)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1,
+                "steps": steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t_tot / steps, 1),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded)",
+                "config": {"workload": "same hot-path step as the GPU arm; each step is a bounded "
+                                       "row sample run by the CPU oracle on the host cores"},
+                "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle_cores(),
+                                 "kind": "oracle", "sample": sample.describe()},
+                "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        line = run_gpu(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        s = json.dumps(line)
+        print(s)
+        if args.detail:
+            with open(args.detail, "w") as f:
+                f.write(s + "\n")
+
+
+if __name__ == "__main__":
+    main()

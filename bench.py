@@ -473,6 +473,59 @@ def max_over_ranks(v, world, device):
     return float(t.item())
 
 
+PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd")
+
+
+def profile_case(case, device):
+    """One small case of one kernel, run twice (warm-up + the launch an ncu
+    capture selects with -s 1 -c 1). Inputs exceed L2 except the GEMV, whose
+    DRAM figures rely on ncu's cache flush between passes."""
+    from bit_weight_quantized_weights_b200 import binding as wq
+    g = torch.Generator(device=device)
+    g.manual_seed(0)
+
+    def normal(*shape, std=1.0):
+        return torch.randn(*shape, generator=g, device=device) * std
+
+    if case == "nf4":
+        n, k = 8192, 8192
+        cw, am, _ = wq.wq_quantize_pack(wq.WQ_FMT_NF4, normal(n, k, std=0.02), 64)
+        out = torch.empty(n * k, dtype=torch.bfloat16, device=device)
+        fn = lambda: wq.wq_nf4_dequant(cw, am, n * k, out=out)  # noqa: E731
+    elif case in ("gemv_int4", "gemv_nf4"):
+        (n, k), m = GEMV_SHAPE, 16
+        fmt = wq.WQ_FMT_INT4_ASYM if case == "gemv_int4" else wq.WQ_FMT_NF4
+        grp = 128 if fmt == wq.WQ_FMT_INT4_ASYM else 64
+        pw = wq.wq_quantize_pack(fmt, normal(n, k, std=0.02), grp)
+        x = normal(m, k).to(torch.bfloat16)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        fn = lambda: wq.wq_w4a16_gemv(x, n, fmt, grp, *pw, out=y)  # noqa: E731
+    elif case == "gemm":
+        m, n, k = 4096, GEMM_SHAPE[1], GEMM_SHAPE[2]
+        pw = wq.wq_quantize_pack(wq.WQ_FMT_INT4_ASYM, normal(n, k, std=0.02), 128)
+        x = normal(m, k).to(torch.bfloat16)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        ws = wq.gemm_workspace(m, n, k, 128, device)
+        fn = lambda: wq.wq_w4a16_gemm(x, n, wq.WQ_FMT_INT4_ASYM, 128, *pw, workspace=ws,  # noqa
+                                      out=y)
+    elif case == "msd":
+        m, (n, k) = 1024, MSD_SHAPE
+        pw = wq.wq_quantize_pack(wq.WQ_FMT_INT4_ASYM, normal(n, k, std=0.02), 128)
+        x = normal(m, k).to(torch.bfloat16)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        ws = wq.msd_workspace(m, n, k, 128, 2, device)
+        fn = lambda: wq.wq_msd_gemm(x, n, 2, 128, *pw, workspace=ws, out=y)  # noqa: E731
+    else:
+        raise SystemExit("unknown case %r (one of %s)" % (case, ", ".join(PROFILE_CASES)))
+    for _ in range(2):
+        fn()
+        torch.cuda.synchronize()
+    st, detail = wq.wq_device_error()
+    if st != wq.WQ_OK:
+        raise SystemExit("device error word 0x%x" % detail)
+    print("case %s ok" % case)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,6 +535,8 @@ def main():
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--detail", default=None, help="also write the JSON line to this file")
+    ap.add_argument("--case", default=None, choices=PROFILE_CASES,
+                    help="run one small profiling case of one kernel and exit")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -519,6 +574,9 @@ def main():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.case:
+        profile_case(args.case, device)
+        return
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),

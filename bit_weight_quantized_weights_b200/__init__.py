@@ -5,11 +5,19 @@ weights: quantize/pack, standalone dequantization, a decode GEMV, a tcgen05
 prefill GEMM with fused dequantization, and the Multi-Scale Dequant path
 (int8 activation digit planes times integer weight codes). The kernels live in
 libwq.so (C ABI: include/wq.h); ``binding`` is its thin ctypes layer.
+
+Importing the package does not load the library (so ``build_lib`` can run
+before it exists); the first use of ``binding`` or of any ``wq_*`` name loads
+it and raises ImportError if libwq.so has not been built.
 """
 
-from . import binding  # noqa: F401  (fails loudly if libwq.so is missing)
-from .binding import (  # noqa: F401
-    WQ_FMT_INT4_ASYM, WQ_FMT_NF4, wq_nf4_codebook, wq_packed_sizes, wq_quantize_pack, wq_unpack,
-    wq_nf4_dequant, wq_int4_dequant, wq_w4a16_gemv, wq_w4a16_gemm, wq_msd_decompose, wq_msd_gemm,
-    wq_workspace_bytes, wq_device_error,
-)
+import importlib
+
+
+def __getattr__(name):
+    if name == "binding" or name.startswith("wq_") or name.startswith("WQ_"):
+        binding = importlib.import_module(".binding", __name__)
+        if name == "binding":
+            return binding
+        return getattr(binding, name)
+    raise AttributeError(name)

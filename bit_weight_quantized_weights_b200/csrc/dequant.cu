@@ -8,11 +8,11 @@
 // Inference", Abstract, removes from the GEMM path; here it feeds the
 // dequantize-then-GEMM baseline.
 //
-// B200 design: a grid-stride stream over 16-byte chunks of packed codes; each
-// thread turns one chunk into 64 (NF4) or 32 (INT4) output elements and writes
-// them with 16-byte evict-first stores. The 16-entry codebook sits in shared
-// memory (all lanes reading one of 16 words never conflict: equal words
-// broadcast, distinct words sit in distinct banks).
+// B200 design: a grid-stride stream sized to fill every SM; loads and 16-byte
+// evict-first stores are laid out so each warp instruction covers contiguous
+// full sectors. The 16-entry codebook sits in shared memory (all lanes reading
+// one of 16 words never conflict: equal words broadcast, distinct words sit in
+// distinct banks).
 #include "common.cuh"
 
 namespace wq {
@@ -23,36 +23,71 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return kBf16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
 
-// Each thread: 16 code bytes (32 elements, half of one 64-element block).
+// One warp step covers 1024 elements (512 code bytes). Lane l takes 4 code
+// bytes (8 elements) from each of four 128-byte slices, so every load
+// instruction of the warp reads 128 contiguous bytes and every 16-byte store
+// instruction writes 512 contiguous bytes (full sectors). Two warp steps are
+// issued per loop trip to keep eight independent loads in flight per thread.
 template <bool kBf16>
 __global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint8_t* __restrict__ codes,
                                                           const float* __restrict__ absmax,
-                                                          int64_t n_chunks, Nf4Table tab,
+                                                          int64_t numel, Nf4Table tab,
                                                           uint16_t* __restrict__ out) {
   __shared__ float cb[16];
   if (threadIdx.x < 16) cb[threadIdx.x] = tab.v[threadIdx.x];
   __syncthreads();
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < n_chunks; c += stride) {
-    const uint4 v = ld_stream_u4(codes + c * 16);
-    const float a = __ldg(absmax + (c >> 1));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[16];
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t steps = numel / 1024;   // full warp steps
+  constexpr int U = 2;                  // warp steps per loop trip
+  for (int64_t s0 = warp * U; s0 < steps; s0 += nwarps * U) {
+    uint32_t w[U][4];
+    float a[U][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int u = 0; u < U; ++u) {
+      const int64_t st = s0 + u;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const uint32_t byte = (w[i] >> (8 * j)) & 0xFFu;
-        // element 2j of the byte pair is the high nibble
-        const float e0 = __fmul_rn(cb[byte >> 4], a);
-        const float e1 = __fmul_rn(cb[byte & 0xFu], a);
-        o[i * 4 + j] = pack2<kBf16>(e0, e1);
+        if (st < steps) {
+          const int64_t e0 = st * 1024 + 256 * j + 8 * lane;  // first element of this lane
+          w[u][j] = __ldcs(reinterpret_cast<const unsigned int*>(codes + (e0 >> 1)));
+          a[u][j] = __ldg(absmax + (e0 >> 6));
+        }
       }
     }
-    uint16_t* dst = out + c * 32;
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      st_stream_u4(dst + i * 8, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
+    for (int u = 0; u < U; ++u) {
+      const int64_t st = s0 + u;
+      if (st < steps) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t o[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t byte = (w[u][j] >> (8 * b)) & 0xFFu;
+            // element 2b of the pair is the high nibble
+            o[b] = pack2<kBf16>(__fmul_rn(cb[byte >> 4], a[u][j]),
+                                __fmul_rn(cb[byte & 0xFu], a[u][j]));
+          }
+          st_stream_u4(out + st * 1024 + 256 * j + 8 * lane, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+  }
+  // tail: elements past the last full 1024 (a multiple of 64), one lane per 8
+  const int64_t tail0 = steps * 1024;
+  for (int64_t e0 = tail0 + 8 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); e0 < numel;
+       e0 += 8 * (int64_t)gridDim.x * blockDim.x) {
+    const uint32_t wv = *reinterpret_cast<const uint32_t*>(codes + (e0 >> 1));
+    const float av = absmax[e0 >> 6];
+    uint32_t o[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t byte = (wv >> (8 * b)) & 0xFFu;
+      o[b] = pack2<kBf16>(__fmul_rn(cb[byte >> 4], av), __fmul_rn(cb[byte & 0xFu], av));
+    }
+    *reinterpret_cast<uint4*>(out + e0) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
@@ -94,13 +129,12 @@ inline unsigned stream_grid(int64_t items) {
 
 wq_status launch_nf4_dequant(const uint8_t* codes, const float* absmax, int64_t numel, void* out,
                              wq_dtype dt, cudaStream_t st) {
-  const int64_t chunks = numel / 32;
-  const unsigned grid = stream_grid(chunks);
+  const unsigned grid = stream_grid(numel / 32);
   if (dt == WQ_BF16)
-    nf4_dequant_kernel<true><<<grid, 256, 0, st>>>(codes, absmax, chunks, nf4_table(),
+    nf4_dequant_kernel<true><<<grid, 256, 0, st>>>(codes, absmax, numel, nf4_table(),
                                                    static_cast<uint16_t*>(out));
   else
-    nf4_dequant_kernel<false><<<grid, 256, 0, st>>>(codes, absmax, chunks, nf4_table(),
+    nf4_dequant_kernel<false><<<grid, 256, 0, st>>>(codes, absmax, numel, nf4_table(),
                                                     static_cast<uint16_t*>(out));
   return launch_status();
 }

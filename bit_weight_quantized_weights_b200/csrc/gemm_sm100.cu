@@ -12,7 +12,7 @@
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma.kind::f16
 //               (128 x BN x 16, fp16 operands, fp32 accumulator in TMEM) and
 //               commits each stage back to the producer.
-//   warps 2-9   dequantize the packed tile into the fp16 B operand, written
+//   warps 2-17  dequantize the packed tile into the fp16 B operand, written
 //               straight into the UMMA K-major 128-byte-swizzled layout, then
 //               serve as the epilogue (tcgen05.ld -> x 2^-e -> bf16 -> global).
 // Operands are fp16, not bf16: the activations arrive as fp16 copies scaled
@@ -33,8 +33,8 @@ __device__ unsigned int g_gemm_error;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
-constexpr int kThreads = 320;
-constexpr int kDeqWarps = 8;
+constexpr int kDeqWarps = 16;
+constexpr int kThreads = 64 + 32 * kDeqWarps;
 
 template <int BN>
 struct GemmCfg {
@@ -157,15 +157,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::mma_commit(accf);
     }
   } else {
-    // ---------------- dequantize (warps 2..9), then epilogue ----------------
-    const int dq = threadIdx.x - 64;  // 0..255
-    constexpr int kTPR = 256 / BN;    // threads per B row: 1 or 2
-    constexpr int kWords = 8 / kTPR;  // packed words per thread per k-tile
+    // ---------------- dequantize (warps 2..17), then epilogue ----------------
+    const int dq = threadIdx.x - 64;            // 0..511
+    constexpr int kTPR = 32 * kDeqWarps / BN;   // threads per B row: 2 or 4
+    constexpr int kWords = 8 / kTPR;            // packed words per thread per k-tile
     const int r = dq / kTPR;
     const int w0 = (dq % kTPR) * kWords;
     const int n = n0 + r;
     const int ng = K / G;
     const int tiles_per_group = G / BK;
+    // group parameters are loaded one group ahead of their use
+    const __half* srow = scales + (int64_t)n * ng;
+    const __half* zrow = zeros + (int64_t)n * ng;
+    __half s_next = srow[0], z_next = zrow[0];
     uint32_t zb2 = 0, s2 = 0;
     bool ok = true;
     for (int kt = 0; kt < KT && ok; ++kt) {
@@ -173,10 +177,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (uint32_t)(kt / ST) & 1u;
       if (kt % tiles_per_group == 0) {
         const int gi = kt / tiles_per_group;
-        const uint32_t sb = __half_as_ushort(scales[(int64_t)n * ng + gi]);
-        const uint32_t zq = (uint32_t)__half2float(zeros[(int64_t)n * ng + gi]);
+        const uint32_t sb = __half_as_ushort(s_next);
+        const uint32_t zq = (uint32_t)__half2float(z_next);
         s2 = sb | (sb << 16);
         zb2 = (0x6400u | zq) * 0x00010001u;  // fp16x2 (1024 + z, 1024 + z)
+        if (gi + 1 < ng) {
+          s_next = srow[gi + 1];
+          z_next = zrow[gi + 1];
+        }
       }
       const bool got = sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x301u, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
@@ -186,16 +194,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t* wsrc =
           reinterpret_cast<const uint32_t*>(sW + s * C::kWBytes) + r * 8 + w0;
       uint8_t* bdst = sB + s * C::kBBytes + r * 128;
+      uint32_t ws[kWords];
+      if (kWords == 4) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wsrc);
+        ws[0] = wv.x; ws[1] = wv.y; ws[2 % kWords] = wv.z; ws[3 % kWords] = wv.w;
+      } else {
+        const uint2 wv = *reinterpret_cast<const uint2*>(wsrc);
+        ws[0] = wv.x; ws[1] = wv.y;
+      }
 #pragma unroll
-      for (int j4 = 0; j4 < kWords; j4 += 4) {
-        const uint4 wv = *reinterpret_cast<const uint4*>(wsrc + j4);
-        const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = w0 + j4 + j;  // 16-byte chunk index within the 128-byte row
-          const uint4 o = dequant_word(ws[j], zb2, s2);
-          *reinterpret_cast<uint4*>(bdst + ((c ^ (r & 7)) << 4)) = o;
-        }
+      for (int j = 0; j < kWords; ++j) {
+        const int c = w0 + j;  // 16-byte chunk index within the 128-byte row
+        const uint4 o = dequant_word(ws[j], zb2, s2);
+        *reinterpret_cast<uint4*>(bdst + ((c ^ (r & 7)) << 4)) = o;
       }
       sm100::fence_proxy_async_smem();
       __syncwarp();
@@ -206,13 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__all_sync(0xffffffffu, ok)) {
       sm100::tc_fence_after();
       const int q = warp & 3;              // TMEM lane quarter this warp may read
-      const int half = (warp - 2) >> 2;    // which half of the columns
+      const int slice = (warp - 2) >> 2;   // which quarter of the columns
       const int row = 32 * q + lane;
       const int m = m0 + row;
       const float rs = m < M ? inv_scale[m] : 0.0f;  // 2^-e of this row
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        const int col0 = half * (BN / 2) + 32 * c;
+      for (int c = 0; c < BN / 128; ++c) {
+        const int col0 = slice * (BN / 4) + 32 * c;
         uint32_t v[32];
         sm100::tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col0, v);
         sm100::tmem_ld_wait();

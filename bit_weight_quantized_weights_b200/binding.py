@@ -37,7 +37,7 @@ EXPORTED = [
     "wq_status_string", "wq_version", "wq_nf4_codebook", "wq_packed_sizes",
     "wq_quantize_pack", "wq_unpack", "wq_nf4_dequant", "wq_int4_dequant",
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
-    "wq_workspace_bytes", "wq_device_error",
+    "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
 ]
 
 
@@ -73,6 +73,7 @@ def _load():
         "wq_workspace_bytes": ([ctypes.c_int, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
                                ctypes.c_int),
         "wq_device_error": ([P, ctypes.c_int, ctypes.POINTER(U32)], ctypes.c_int),
+        "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -268,6 +269,21 @@ def wq_msd_gemm(x, n, n_components, group, qweight, scales, zeros, workspace=Non
                            _ptr(zeros), _ptr(out), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)),
            "wq_msd_gemm")
+    return out
+
+
+def wq_msd_gemm_noalloc(x, n, n_components, group, qweight, scales, zeros, out=None,
+                        stream=None):
+    """wq_msd_gemm without a workspace: the library's fixed device scratch array
+    is used, so the call allocates nothing (problem size limited to 8 MiB of
+    scratch; calls overlapping on the GPU race on it)."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib.wq_msd_gemm_noalloc(_ptr(x), m, n, k, n_components, group, _ptr(qweight),
+                                   _ptr(scales), _ptr(zeros), _ptr(out), _stream(stream)),
+           "wq_msd_gemm_noalloc")
     return out
 
 

@@ -219,6 +219,34 @@ wq_status wq_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K,
                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * wq_msd_gemm for callers that cannot allocate device memory. The library's
+ * pages have no counterpart to this call; it exists for deployment. Some
+ * callers cannot hand the library a workspace: an engine that carves up all
+ * device memory once at start-up and must not grow, a plugin host whose fixed
+ * call signature has no workspace argument, or a latency-critical loop in
+ * which a device allocation (which may synchronise the GPU) is forbidden.
+ * This entry point takes the same arguments as wq_msd_gemm minus the
+ * workspace and computes the same result with the same kernels, using a
+ * fixed 8 MiB scratch array that the library reserves in device memory on
+ * every GPU that loads it (held until the process exits). It allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - Limit: wq_workspace_bytes(WQ_OP_MSD_GEMM, M, N, K, group, C) must not
+ *    exceed 8 MiB (C * roundup(M, 128) * K + C * M * 4 bytes, e.g. M <= 128
+ *    at K = 25600 with C = 2); larger problems return WQ_ERR_UNSUPPORTED and
+ *    launch nothing.
+ *  - The first call on a device looks up the scratch array's device address
+ *    (once per device, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array, and each call overwrites what it reads
+ *    before reading it (nothing has to start at zero). Calls that overlap on
+ *    the GPU (other streams, or other threads' streams) race on it: order
+ *    them on one stream.
+ */
+wq_status wq_msd_gemm_noalloc(const void* x, int64_t M, int64_t N, int64_t K,
+                              int32_t n_components, int32_t group, const void* qweight,
+                              const void* scales, const void* zeros, void* y, void* stream);
+
+/*
  * Workspace bytes an entry point needs for the given problem (0 if none).
  * Host only; `bytes` is a host pointer.
  */

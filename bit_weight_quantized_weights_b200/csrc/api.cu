@@ -24,6 +24,7 @@ wq_status launch_msd_gemm(const void*, int64_t, int64_t, int64_t, int32_t, int32
 size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C);
 wq_status read_gemm_error(bool clear, uint32_t* v);
 wq_status read_msd_error(bool clear, uint32_t* v);
+wq_status read_gemv_error(bool clear, uint32_t* v);
 }  // namespace wq
 
 using namespace wq;
@@ -255,13 +256,15 @@ wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K, int32_t 
 wq_status wq_device_error(void* stream, int clear, uint32_t* detail) {
   return guarded([&] {
     if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return WQ_ERR_CUDA;
-    uint32_t a = 0, b = 0;
+    uint32_t a = 0, b = 0, c = 0;
     wq_status s = read_gemm_error(clear != 0, &a);
     if (s != WQ_OK) return s;
     s = read_msd_error(clear != 0, &b);
     if (s != WQ_OK) return s;
-    if (detail) *detail = a ? a : b;
-    return (a || b) ? WQ_ERR_TIMEOUT : WQ_OK;
+    s = read_gemv_error(clear != 0, &c);
+    if (s != WQ_OK) return s;
+    if (detail) *detail = a ? a : (b ? b : c);
+    return (a || b || c) ? WQ_ERR_TIMEOUT : WQ_OK;
   });
 }
 

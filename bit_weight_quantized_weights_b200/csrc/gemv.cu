@@ -23,9 +23,11 @@
 //   far from busy; HBM is the bound.
 // * INT4 codes become bf16 in registers without arithmetic: OR-ing a nibble
 //   into the mantissa of 128.0 (bit pattern 0x4300) gives exactly 128 + q, two
-//   per 32-bit LOP3. The MMA sums (128 + q) x over a 64-wide sub-group, a
-//   second MMA with an all-ones A operand sums x itself, and the epilogue
-//   applies s * (P - (128 + z) * sum(x)), the MixPE post-group form.
+//   per 32-bit LOP3, paired as (k, k + 4). x is staged in that same pairing,
+//   so its fragments load straight from shared memory. The MMA sums
+//   (128 + q) x over the group's part of a 128-wide unit and the epilogue
+//   applies s * (P - (128 + z) * sum(x)), the MixPE post-group form, with the
+//   sums of x per 64-wide sub-group computed once per CTA while x is staged.
 // * NF4 codes go through a 256-entry table indexed by a whole packed byte that
 //   yields the two fp16 code values already paired as one A-operand register.
 //   The table is replicated per lane (lane l reads column l, so bank l): every
@@ -40,11 +42,18 @@
 //   bf16. No workspace, no atomics.
 //
 // Data placement per CTA (dynamic shared memory):
-//   xs   [8*NT tokens][Kc] bf16 (fp16 for NF4), the CTA's K-chunk of x
-//        (zero-padded tokens); odd tokens have bit 3 of k flipped (a 16-byte
-//        swizzle that keeps the fragment loads conflict-free)
+//   xs   [8*NT tokens][Kc] bf16 (fp16 for NF4), the CTA's K-chunk of x, in
+//        16-byte chunks. Only the M real tokens are written: a padding
+//        token's MMA column never reaches an output. Chunk c of token m sits
+//        at chunk c ^ (m & 1), and for the wide INT4 layout (groups that are
+//        multiples of 128) also ^ (bit 3 of c moved to bit 1), so that the
+//        fragment loads of a warp hit distinct banks. For INT4 each chunk
+//        holds the pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7), the nibble pairing.
+//   xsum [Kc/64 or Kc/128][8*NT tokens] fp32, sums of x per group part (INT4)
 //   lut  [256 entries][32 lanes] u32 (NF4 only)
 //   red  [128 rows][16 tokens] fp32, the partials the cluster reads
+#include <mutex>
+
 #include "common.cuh"
 
 namespace wq {
@@ -53,6 +62,8 @@ namespace {
 __device__ unsigned int g_gemv_error;  // this kernel has no waits; kept for the ABI
 
 constexpr int kRowsPerCta = 128;
+constexpr int kMaxSplit = 16;         // cluster size limit (non-portable above 8)
+constexpr int kMaxXChunkBytes = 64 * 1024;
 
 struct GemvArgs {
   const uint16_t* x;
@@ -68,8 +79,7 @@ struct GemvArgs {
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -77,15 +87,22 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                              uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Cluster barrier that publishes this CTA's shared-memory writes to the others.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// Cluster barrier with no ordering of this thread's memory operations: used
+// only to keep shared memory alive until every peer has read it (those reads
+// have already returned their values when a peer arrives).
+__device__ __forceinline__ void cluster_sync_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;"
                ::: "memory");
 }
 __device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
@@ -104,20 +121,33 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
   return lop3_and_or(w >> (4 * e), 0x000F000Fu, 0x43004300u);
 }
 
-// One 128-k unit of this lane's two weight rows, with its group parameters.
+// One 128-k unit of this lane's two weight rows (g and g + 8), with its
+// group parameters.
+//   wide  : w[0..3] = 16 bytes of row g at byte 16t, w[4..7] the same of row
+//           g + 8 (k = 32t .. 32t + 31); prm[0..1] = (scale, zero) of rows g,
+//           g + 8 (one group spans the unit).
+//   narrow: w[0..1] row g, half 0 (byte 8t), w[2..3] row g, half 1 (byte
+//           32 + 8t), w[4..7] the same of row g + 8; prm[2h + i] = the
+//           parameters of half h for row g (i = 0) or g + 8 (i = 1).
 struct Unit {
-  uint2 w[4];       // [row g h0, row g h1, row g+8 h0, row g+8 h1] (8 bytes each)
-  uint32_t prm[4];  // INT4: (scale, zero) fp16 pairs [h][row]; NF4: absmax [h][row]
+  uint32_t w[8];
+  uint32_t prm[4];
 };
 
-template <bool kNF4>
+template <bool kNF4, bool kWide>
 __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint8_t* wB, int u,
                                           int nA, int nB, const GemvArgs& p, int ng) {
   const int64_t off = (int64_t)u * 64;
-  U.w[0] = ld_stream_u2(wA + off);
-  U.w[1] = ld_stream_u2(wA + off + 32);
-  U.w[2] = ld_stream_u2(wB + off);
-  U.w[3] = ld_stream_u2(wB + off + 32);
+  if (kWide) {
+    const uint4 a = ld_stream_u4(wA + off), b = ld_stream_u4(wB + off);
+    U.w[0] = a.x; U.w[1] = a.y; U.w[2] = a.z; U.w[3] = a.w;
+    U.w[4] = b.x; U.w[5] = b.y; U.w[6] = b.z; U.w[7] = b.w;
+  } else {
+    const uint2 a0 = ld_stream_u2(wA + off), a1 = ld_stream_u2(wA + off + 32);
+    const uint2 b0 = ld_stream_u2(wB + off), b1 = ld_stream_u2(wB + off + 32);
+    U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
+    U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
+  }
   if (kNF4) {
     const float* am = static_cast<const float*>(p.scales);
     const float2 aA =
@@ -132,7 +162,7 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     const unsigned short* s16 = reinterpret_cast<const unsigned short*>(p.scales);
     const unsigned short* z16 = reinterpret_cast<const unsigned short*>(p.zeros);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < (kWide ? 1 : 2); ++h) {
       const int gi = (u * 128 + h * 64) / p.G;
       const int64_t iA = (int64_t)nA * ng + gi, iB = (int64_t)nB * ng + gi;
       U.prm[2 * h + 0] = (uint32_t)__ldg(s16 + iA) | ((uint32_t)__ldg(z16 + iA) << 16);
@@ -141,17 +171,149 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
   }
 }
 
-template <int NT, bool kNF4>
-__global__ void __launch_bounds__(256, 3) gemv_kernel(GemvArgs p, Nf4Table tab) {
+// acc += s * (P - (128 + z) * sum(x)) for the four accumulator slots of one
+// token tile; pv holds (s, z) as fp16 halves, sx the two tokens' sums of x.
+__device__ __forceinline__ void int4_post(float (&acc)[4], const float (&cp)[4], uint32_t pv_g,
+                                          uint32_t pv_g8, float2 sx) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t pv = (r >> 1) ? pv_g8 : pv_g;  // row g for r < 2, g + 8 else
+    const float s = __half2float(__ushort_as_half((unsigned short)(pv & 0xFFFFu)));
+    const float zb = 128.0f + __half2float(__ushort_as_half((unsigned short)(pv >> 16)));
+    acc[r] = fmaf(s, fmaf(-zb, (r & 1) ? sx.y : sx.x, cp[r]), acc[r]);
+  }
+}
+
+// The products of one 128-k unit, accumulated into acc (see the data
+// placement above for the shared-memory layouts read here).
+template <int NT, bool kNF4, bool kWide>
+__device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16_t* xs, int kc,
+                                             const float* xsum, const uint32_t* lut_lane, int g,
+                                             int t, float (&acc)[NT][4]) {
+  constexpr int kTok = 8 * NT;
+  if (kWide) {
+    // two accumulator chains (even and odd k-steps) halve the MMA dependency chain
+    float cp[2][NT][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cp[c][a][r] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint4 X[NT];
+#pragma unroll
+      for (int a = 0; a < NT; ++a) {
+        const int tok = g + 8 * a;
+        const int pc = (16 * lu + 4 * t + j) ^ (t & 2) ^ (tok & 1);
+        X[a] = *reinterpret_cast<const uint4*>(xs + (size_t)tok * kc + pc * 8);
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t a0 = int4_pair(U.w[j], 2 * hh), a1 = int4_pair(U.w[4 + j], 2 * hh);
+        const uint32_t a2 = int4_pair(U.w[j], 2 * hh + 1), a3 = int4_pair(U.w[4 + j], 2 * hh + 1);
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+          mma16816(cp[hh][a], a0, a1, a2, a3, hh ? X[a].z : X[a].x, hh ? X[a].w : X[a].y);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < NT; ++a) {
+      float cs[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) cs[r] = cp[0][a][r] + cp[1][a][r];
+      const float2 sx = *reinterpret_cast<const float2*>(xsum + lu * kTok + 8 * a + 2 * t);
+      int4_post(acc[a], cs, U.prm[0], U.prm[1], sx);
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float cp[2][NT][4];  // even and odd k-steps
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) cp[c][a][r] = 0.0f;
+      uint4 X[NT][2];
+#pragma unroll
+      for (int a = 0; a < NT; ++a) {
+        const int tok = g + 8 * a;
+        const int c0 = 16 * lu + 8 * h + 2 * t;
+        const uint16_t* base = xs + (size_t)tok * kc;
+        X[a][0] = *reinterpret_cast<const uint4*>(base + (c0 ^ (tok & 1)) * 8);
+        X[a][1] = *reinterpret_cast<const uint4*>(base + ((c0 + 1) ^ (tok & 1)) * 8);
+      }
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const int jw = ks >> 1, hh = ks & 1;
+        const uint32_t WA = U.w[2 * h + jw], WB = U.w[4 + 2 * h + jw];
+        uint32_t a0, a1, a2, a3;
+        if (!kNF4) {
+          a0 = int4_pair(WA, 2 * hh);
+          a1 = int4_pair(WB, 2 * hh);
+          a2 = int4_pair(WA, 2 * hh + 1);
+          a3 = int4_pair(WB, 2 * hh + 1);
+        } else {
+          // bytes 2hh and 2hh + 1 of the word: elements (2i, 2i + 1) per byte
+          const int sh0 = 16 * hh, sh1 = sh0 + 8;
+          a0 = lut_lane[((WA >> sh0) & 0xFFu) * 32];
+          a1 = lut_lane[((WB >> sh0) & 0xFFu) * 32];
+          a2 = lut_lane[((WA >> sh1) & 0xFFu) * 32];
+          a3 = lut_lane[((WB >> sh1) & 0xFFu) * 32];
+        }
+#pragma unroll
+        for (int a = 0; a < NT; ++a) {
+          const uint32_t b0 = hh ? X[a][jw].z : X[a][jw].x;
+          const uint32_t b1 = hh ? X[a][jw].w : X[a][jw].y;
+          if (!kNF4)
+            mma16816(cp[hh][a], a0, a1, a2, a3, b0, b1);
+          else
+            mma16816_f16(cp[hh][a], a0, a1, a2, a3, b0, b1);
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < NT; ++a) {
+        float cs[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cs[r] = cp[0][a][r] + cp[1][a][r];
+        if (kNF4) {
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            acc[a][r] = fmaf(__uint_as_float(U.prm[2 * h + (r >> 1)]), cs[r], acc[a][r]);
+        } else {
+          const float2 sx =
+              *reinterpret_cast<const float2*>(xsum + (2 * lu + h) * kTok + 8 * a + 2 * t);
+          int4_post(acc[a], cs, U.prm[2 * h], U.prm[2 * h + 1], sx);
+        }
+      }
+    }
+  }
+}
+
+// Units of weights each warp keeps in flight ahead of the one it computes.
+template <int NT>
+struct PrefetchDepth {
+  static constexpr int value = NT == 1 ? 4 : 3;
+};
+
+template <int NT, bool kNF4, bool kWide>
+__global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int kTok = 8 * NT;
+  constexpr int D = PrefetchDepth<NT>::value;
   const int kc = p.kc;
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   uint8_t* cursor = smem + (size_t)kTok * kc * 2;
   uint32_t* lut = nullptr;
+  float* xsum = nullptr;
   if (kNF4) {
     lut = reinterpret_cast<uint32_t*>(cursor);
     cursor += 256 * 32 * 4;
+  } else {
+    xsum = reinterpret_cast<float*>(cursor);
+    cursor += (size_t)kTok * (kc / 64) * 4;
   }
   float* red = reinterpret_cast<float*>(cursor);
   __shared__ float tok_inv[16];
@@ -169,23 +331,53 @@ __global__ void __launch_bounds__(256, 3) gemv_kernel(GemvArgs p, Nf4Table tab) 
   const int nA = n0 + g, nB = n0 + g + 8;
   const int ng = p.K / p.G;
 
-  // the first unit's loads go out before anything else
+  // the first D units' loads go out before anything else
   const int64_t row_bytes = (int64_t)p.K / 2;
-  const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + 8 * t;
+  const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + (kWide ? 16 : 8) * t;
   const uint8_t* wrowB = wrowA + 8 * row_bytes;
-  Unit cur, nxt;
-  if (active && u0 < u1) load_unit<kNF4>(cur, wrowA, wrowB, u0, nA, nB, p, ng);
+  Unit ring[D];
+  if (active) {
+#pragma unroll
+    for (int i = 0; i < D; ++i)
+      if (u0 + i < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng);
+  }
 
   // ---- stage x[:, k0 : k0+klen) into shared memory (16-byte chunks) -------
   {
-    const int chunks_per_row = kc / 8;
-    for (int c = tid; c < kTok * chunks_per_row; c += blockDim.x) {
-      const int gt = c / chunks_per_row;
-      const int kl = (c - gt * chunks_per_row) * 8;
+    // Only the M real tokens are staged: the MMA columns of padding tokens
+    // never reach an output. cpr is a multiple of 16, so the chunks of one
+    // 64- or 128-wide sub-group sit in 8 or 16 consecutive lanes; the loop
+    // runs whole warps (its bound is rounded up to 32) for the shuffles.
+    const int cpr = kc / 8;
+    const int nchunks = p.M * cpr;
+    for (int c = tid; c < ((nchunks + 31) & ~31); c += blockDim.x) {
+      const bool real = c < nchunks;
+      const int gt = c / cpr;
+      const int cl = c - gt * cpr;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (gt < p.M && kl < klen)
-        v = *reinterpret_cast<const uint4*>(p.x + (size_t)gt * p.K + k0 + kl);
-      *reinterpret_cast<uint4*>(xs + (size_t)gt * kc + (kl ^ ((gt & 1) << 3))) = v;
+      if (real && cl * 8 < klen)
+        v = *reinterpret_cast<const uint4*>(p.x + (size_t)gt * p.K + k0 + cl * 8);
+      int pc = cl ^ (gt & 1);
+      if (!kNF4) {
+        float sm = 0.0f;
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sm += bf16_lo_to_f32(w[q]) + bf16_hi_to_f32(w[q]);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+        sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+        if (kWide) {
+          sm += __shfl_xor_sync(0xffffffffu, sm, 8);
+          if (real && (cl & 15) == 0) xsum[(cl >> 4) * kTok + gt] = sm;
+          pc ^= (cl >> 2) & 2;
+        } else {
+          if (real && (cl & 7) == 0) xsum[(cl >> 3) * kTok + gt] = sm;
+        }
+        // pair (k, k + 4) as one bf16x2 word, the INT4 nibble pairing
+        v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
+                       prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
+      }
+      if (real) *reinterpret_cast<uint4*>(xs + (size_t)gt * kc + pc * 8) = v;
     }
   }
   if (kNF4) {
@@ -239,89 +431,16 @@ __global__ void __launch_bounds__(256, 3) gemv_kernel(GemvArgs p, Nf4Table tab) 
     for (int r = 0; r < 4; ++r) acc[a][r] = 0.0f;
 
   if (active) {
-    const uint32_t lut_lane = kNF4 ? smem_u32(lut) + 4u * lane : 0u;
-    constexpr uint32_t kOnes = 0x3F803F80u;  // bf16x2 (1, 1)
-    for (int u = u0; u < u1; ++u) {
-      if (u + 1 < u1) load_unit<kNF4>(nxt, wrowA, wrowB, u + 1, nA, nB, p, ng);
-      const int lu = u - u0;
+    const uint32_t* lut_lane = kNF4 ? lut + lane : nullptr;
+    for (int ub = u0; ub < u1; ub += D) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint2 wa = cur.w[h], wb = cur.w[2 + h];
-        uint32_t X[NT][8];
-#pragma unroll
-        for (int a = 0; a < NT; ++a) {
-          const int tok = g + 8 * a;
-          const uint16_t* base = xs + (size_t)tok * kc;
-          const int kk = lu * 128 + h * 64 + 16 * t;
-          const uint4 c0 = *reinterpret_cast<const uint4*>(base + (kk ^ ((tok & 1) << 3)));
-          const uint4 c1 = *reinterpret_cast<const uint4*>(base + ((kk + 8) ^ ((tok & 1) << 3)));
-          X[a][0] = c0.x; X[a][1] = c0.y; X[a][2] = c0.z; X[a][3] = c0.w;
-          X[a][4] = c1.x; X[a][5] = c1.y; X[a][6] = c1.z; X[a][7] = c1.w;
-        }
-        float cp[NT][4], cs[NT][4];
-#pragma unroll
-        for (int a = 0; a < NT; ++a)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            cp[a][r] = 0.0f;
-            cs[a][r] = 0.0f;
-          }
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          uint32_t a0, a1, a2, a3, bs0, bs1;
-          if (!kNF4) {
-            const int jw = ks >> 1, hh = ks & 1;
-            const uint32_t WA = jw ? wa.y : wa.x, WB = jw ? wb.y : wb.x;
-            a0 = int4_pair(WA, 2 * hh);
-            a1 = int4_pair(WB, 2 * hh);
-            a2 = int4_pair(WA, 2 * hh + 1);
-            a3 = int4_pair(WB, 2 * hh + 1);
-            bs0 = 4 * jw + hh;
-            bs1 = 4 * jw + hh + 2;
-          } else {
-            // bytes 2ks and 2ks+1 of this lane's 8-byte slice
-            const uint32_t WA = (ks >> 1) ? wa.y : wa.x, WB = (ks >> 1) ? wb.y : wb.x;
-            const int sh0 = 16 * (ks & 1), sh1 = sh0 + 8;
-            const uint32_t eA0 = (WA >> sh0) & 0xFFu, eA1 = (WA >> sh1) & 0xFFu;
-            const uint32_t eB0 = (WB >> sh0) & 0xFFu, eB1 = (WB >> sh1) & 0xFFu;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a0) : "r"(lut_lane + eA0 * 128u));
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a1) : "r"(lut_lane + eB0 * 128u));
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a2) : "r"(lut_lane + eA1 * 128u));
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(a3) : "r"(lut_lane + eB1 * 128u));
-            bs0 = 2 * ks;
-            bs1 = 2 * ks + 1;
-          }
-#pragma unroll
-          for (int a = 0; a < NT; ++a) {
-            if (!kNF4) {
-              // (x[2i], x[2i+4]) and (x[2i+1], x[2i+5]) from consecutive pairs
-              const uint32_t b0 = prmt(X[a][bs0], X[a][bs1], 0x5410u);
-              const uint32_t b1 = prmt(X[a][bs0], X[a][bs1], 0x7632u);
-              mma16816(cp[a], a0, a1, a2, a3, b0, b1);
-              mma16816(cs[a], kOnes, kOnes, kOnes, kOnes, b0, b1);  // sum of x
-            } else {
-              mma16816_f16(cp[a], a0, a1, a2, a3, X[a][bs0], X[a][bs1]);
-            }
-          }
-        }
-        // post-group (INT4) / post-block (NF4) scaling
-#pragma unroll
-        for (int a = 0; a < NT; ++a) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const uint32_t pv = cur.prm[2 * h + (r >> 1)];  // row g for r < 2, g+8 else
-            if (kNF4) {
-              acc[a][r] = fmaf(__uint_as_float(pv), cp[a][r], acc[a][r]);
-            } else {
-              const float s = __half2float(__ushort_as_half((unsigned short)(pv & 0xFFFFu)));
-              const float zb =
-                  128.0f + __half2float(__ushort_as_half((unsigned short)(pv >> 16)));
-              acc[a][r] = fmaf(s, fmaf(-zb, cs[a][r], cp[a][r]), acc[a][r]);
-            }
-          }
+      for (int i = 0; i < D; ++i) {
+        const int u = ub + i;
+        if (u < u1) {
+          compute_unit<NT, kNF4, kWide>(ring[i], u - u0, xs, kc, xsum, lut_lane, g, t, acc);
+          if (u + D < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u + D, nA, nB, p, ng);
         }
       }
-      cur = nxt;
     }
   }
 
@@ -340,56 +459,70 @@ __global__ void __launch_bounds__(256, 3) gemv_kernel(GemvArgs p, Nf4Table tab) 
     __syncthreads();
   }
   {
-    const int rows_per_rank = kRowsPerCta / p.S;  // S divides 128 (S is 1, 2, 4 or 8)
-    const int r_begin = rank * rows_per_rank;
-    const int items = rows_per_rank * p.M;
+    const int r_begin = rank * kRowsPerCta / p.S;
+    const int nrows = (rank + 1) * kRowsPerCta / p.S - r_begin;
+    const int items = nrows * p.M;
     for (int i = tid; i < items; i += blockDim.x) {
-      const int tok = i / rows_per_rank;
-      const int row = r_begin + (i - tok * rows_per_rank);
+      const int tok = i / nrows;
+      const int row = r_begin + (i - tok * nrows);
       const int n = row_tile + row;
       const float* src = &red[row * 16 + tok];
-      float parts[8];
+      float parts[kMaxSplit];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)  // all remote loads in flight before the sum
+      for (int q = 0; q < kMaxSplit; ++q)  // all remote loads in flight before the sum
         parts[q] =
             (q < p.S) ? (p.S > 1 ? ld_cluster_f32(map_rank(src, (uint32_t)q)) : *src) : 0.0f;
       float v = 0.0f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) v += parts[q];
+      for (int q = 0; q < kMaxSplit; ++q) v += parts[q];
       if (n < p.N) p.y[(int64_t)tok * p.N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
     }
   }
-  if (p.S > 1) cluster_sync_all();  // keep shared memory alive until all ranks have read it
+  if (p.S > 1) cluster_sync_relaxed();  // keep shared memory alive until all ranks have read it
 }
 
 template <int NT, bool kNF4>
 size_t gemv_smem(int kc) {
-  return (size_t)8 * NT * kc * 2 + (size_t)kRowsPerCta * 16 * 4 + (kNF4 ? 256 * 32 * 4 : 0);
+  return (size_t)8 * NT * kc * 2 + (size_t)kRowsPerCta * 16 * 4 +
+         (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
 }
 
+struct Plan {
+  int S = 0;
+  int kc = 0;
+  size_t smem = 0;
+};
+
 // Cluster size S (K split): every CTA holds one 128-row tile over one K-chunk.
-// S is chosen among {1, 2, 4, 8} (S <= 128-wide units, x chunk <= 48 KB) to
-// fill the resident CTA slots of the GPU with the fewest partial waves.
-template <int NT, bool kNF4>
-int gemv_split(int64_t N, int64_t K) {
+// S (1..16, at most one unit per CTA, x chunk <= 64 KB) is chosen to fill the
+// resident CTA slots of the GPU with the fewest waves: the whole weight
+// stream should be in flight from the first microseconds.
+template <int NT, bool kNF4, bool kWide>
+Plan make_plan(int64_t N, int64_t K) {
   const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
   const int64_t units = K / 128;
+  auto kern = gemv_kernel<NT, kNF4, kWide>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaGetLastError();
   double best = -1.0;
-  int bS = 0;
-  for (int S = 1; S <= 8; S *= 2) {
+  Plan bp;
+  for (int S = 1; S <= kMaxSplit; ++S) {
     if (S > units) break;
     const int kc = (int)((units + S - 1) / S) * 128;
-    if ((int64_t)8 * NT * kc * 2 > 48 * 1024) continue;
+    if ((int64_t)8 * NT * kc * 2 > kMaxXChunkBytes) continue;
     const size_t smem = gemv_smem<NT, kNF4>(kc);
-    auto kern = gemv_kernel<NT, kNF4>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
+        cudaSuccess) {
+      cudaGetLastError();
       continue;
+    }
     int slots = 0;
     if (S == 1) {
       int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess)
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess) {
+        cudaGetLastError();
         continue;
+      }
       slots = per_sm * num_sms();
     } else {
       cudaLaunchConfig_t cfg = {};
@@ -417,26 +550,53 @@ int gemv_split(int64_t N, int64_t K) {
     const double score = (double)grid / ((double)waves * slots) - 0.02 * (double)(waves - 1);
     if (score > best + 1e-9) {
       best = score;
-      bS = S;
+      bp.S = S;
+      bp.kc = kc;
+      bp.smem = smem;
     }
   }
-  return bS;
+  return bp;
 }
 
-template <int NT, bool kNF4>
+// Plans are cached per (device, N, K): the occupancy queries cost far more
+// host time than the launch itself.
+template <int NT, bool kNF4, bool kWide>
+Plan plan_for(int64_t N, int64_t K) {
+  struct Entry {
+    int dev;
+    int64_t N, K;
+    Plan plan;
+  };
+  constexpr int kEntries = 64;
+  static Entry cache[kEntries];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return Plan{};
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].N == N && cache[i].K == K) return cache[i].plan;
+  const Plan pl = make_plan<NT, kNF4, kWide>(N, K);
+  if (pl.S > 0 && used < kEntries) cache[used++] = Entry{dev, N, K, pl};
+  return pl;
+}
+
+template <int NT, bool kNF4, bool kWide>
 wq_status launch_t(GemvArgs a, cudaStream_t st) {
-  a.S = gemv_split<NT, kNF4>(a.N, a.K);
-  if (a.S < 1) return WQ_ERR_UNSUPPORTED;
-  a.kc = ((a.units + a.S - 1) / a.S) * 128;
-  const size_t smem = gemv_smem<NT, kNF4>(a.kc);
-  auto kern = gemv_kernel<NT, kNF4>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  const Plan pl = plan_for<NT, kNF4, kWide>(a.N, a.K);
+  if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
+  a.S = pl.S;
+  a.kc = pl.kc;
+  auto kern = gemv_kernel<NT, kNF4, kWide>;
+  // the attribute is a per-function maximum; plans of other shapes may have
+  // set a smaller one since
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)a.S, (unsigned)((a.N + kRowsPerCta - 1) / kRowsPerCta), 1);
   cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -468,8 +628,11 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   a.units = (int)(K / 128);
   a.S = 1;
   a.kc = 0;
-  if (fmt == WQ_FMT_NF4) return NT == 1 ? launch_t<1, true>(a, st) : launch_t<2, true>(a, st);
-  return NT == 1 ? launch_t<1, false>(a, st) : launch_t<2, false>(a, st);
+  if (fmt == WQ_FMT_NF4)
+    return NT == 1 ? launch_t<1, true, false>(a, st) : launch_t<2, true, false>(a, st);
+  if (group % 128 == 0)
+    return NT == 1 ? launch_t<1, false, true>(a, st) : launch_t<2, false, true>(a, st);
+  return NT == 1 ? launch_t<1, false, false>(a, st) : launch_t<2, false, false>(a, st);
 }
 
 wq_status read_gemv_error(bool clear, uint32_t* v) {

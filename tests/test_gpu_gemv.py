@@ -72,10 +72,11 @@ def test_gemv_decode_nf4(wq, m, n, k):
 
 @pytest.mark.parametrize("m,n,k,group", [(3, 1040, 384, 128), (9, 144, 256, 256),
                                          (16, 16, 128, 128), (5, 2064, 1152, 64),
-                                         (2, 528, 640, 640)])
+                                         (2, 528, 640, 640), (7, 1040, 768, 192)])
 def test_gemv_ragged_and_groups(wq, m, n, k, group):
     """N not a multiple of the 128-row tile, odd M, groups larger than the
-    128-wide unit, per-channel groups (G = K)."""
+    128-wide unit, groups that straddle two units (G = 192), per-channel
+    groups (G = K)."""
     _run_int4(wq, m, n, k, group, seed=m)
 
 

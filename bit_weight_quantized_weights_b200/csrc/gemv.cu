@@ -11,16 +11,18 @@
 // B200 design
 // -----------
 // * The weight stream is the whole cost (0.53 byte per weight against 2*M
-//   flops). Weights are read with plain 8-byte loads that do not allocate in
-//   L1, by many small CTAs (up to three per SM), each warp keeping the next
-//   128-k unit of its 16 rows (and that unit's group parameters) in flight
-//   while it computes the current one. Measured on B200, plain coalesced loads
-//   stream HBM far better than a TMA ring of small boxes for this work.
+//   flops). Weights are read with plain 16-byte (8-byte for 64-wide groups
+//   and NF4) loads that do not allocate in L1, by two 256-thread CTAs per SM,
+//   each warp keeping three or four 128-k units of its 16 rows (with their
+//   group parameters) in flight while it computes the oldest. Measured on
+//   B200, plain coalesced loads stream HBM far better than a TMA ring of
+//   small boxes for this work.
 // * At M = 16 the multiply-adds alone (2*16 flops per weight at ~12 Tweights/s)
 //   exceed what the CUDA cores can issue, so the product runs on the tensor
 //   cores with warp-level mma.m16n8k16 (fp32 accumulate): weight rows form
-//   the 16-row A operand, tokens the 8-column B operand. The tensor pipe stays
-//   far from busy; HBM is the bound.
+//   the 16-row A operand, tokens the 8-column B operand. Measured on B200,
+//   one such MMA issues every ~8.3 cycles per SM sub-partition, so even at
+//   M = 16 (16 MMAs per KB of weights) the pipe keeps up with ~8 TB/s.
 // * INT4 codes become bf16 in registers without arithmetic: OR-ing a nibble
 //   into the mantissa of 128.0 (bit pattern 0x4300) gives exactly 128 + q, two
 //   per 32-bit LOP3, paired as (k, k + 4). x is staged in that same pairing,
@@ -37,9 +39,12 @@
 //   of two that puts its largest magnitude in [2^14, 2^15) (exact for bf16
 //   values down to 2^-28 of it); the power is divided back out of the partial.
 // * Split-K across a thread-block cluster: the S CTAs of a cluster share one
-//   128-row tile and split K; their fp32 partials are summed through
-//   distributed shared memory, in a fixed rank order, and written once as
-//   bf16. No workspace, no atomics.
+//   128-row tile and split K. Each CTA pushes its fp32 partials into the
+//   shared memory of the rank that owns those rows (remote stores, no round
+//   trip); after one cluster barrier each owner sums its rows in rank order
+//   and writes them once as bf16. No workspace, no atomics.
+// * x reaches shared memory by 16-byte asynchronous copies issued before the
+//   first weight loads, so the whole CTA waits on one round trip for it.
 //
 // Data placement per CTA (dynamic shared memory):
 //   xs   [8*NT tokens][Kc] bf16 (fp16 for NF4), the CTA's K-chunk of x, in
@@ -51,7 +56,8 @@
 //        holds the pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7), the nibble pairing.
 //   xsum [Kc/64 or Kc/128][8*NT tokens] fp32, sums of x per group part (INT4)
 //   lut  [256 entries][32 lanes] u32 (NF4 only)
-//   red  [128 rows][16 tokens] fp32, the partials the cluster reads
+//   red  [S ranks][ceil(128/S) rows][16 tokens] fp32, the partials of the
+//        rows this rank owns, as pushed by every rank of the cluster
 #include <mutex>
 
 #include "common.cuh"
@@ -75,7 +81,17 @@ struct GemvArgs {
   int units;              // K / 128
   int S;                  // cluster size along K
   int kc;                 // shared-memory K-chunk length (max over ranks)
+  uint32_t gmagic;        // h / (G / 64) == umulhi(h, gmagic) for 64-wide part h; 0 if G == 64
 };
+
+// n / d without a divide: umulhi(n, floor(2^32 / d) + 1) is exact whenever
+// n * d < 2^32 (d >= 2).
+__host__ __device__ __forceinline__ uint32_t div_magic(uint32_t d) {
+  return d < 2 ? 0u : (uint32_t)(0xFFFFFFFFu / d) + 1u;
+}
+__device__ __forceinline__ int div_by_magic(int n, uint32_t magic) {
+  return magic ? (int)__umulhi((uint32_t)n, magic) : n;
+}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -98,23 +114,29 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
                ::: "memory");
 }
-// Cluster barrier with no ordering of this thread's memory operations: used
-// only to keep shared memory alive until every peer has read it (those reads
-// have already returned their values when a peer arrives).
-__device__ __forceinline__ void cluster_sync_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;"
-               ::: "memory");
-}
 __device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
 }
+
+// 16-byte asynchronous global -> shared copy (L2 only), and its completion.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Rows of a 128-row tile are split over the S ranks of a cluster as
+// [b(r), b(r + 1)) with b(r) = floor(128 r / S); the owner of row is the r
+// with b(r) <= row < b(r + 1).
+__host__ __device__ __forceinline__ int rank_row_begin(int r, int S) { return r * 128 / S; }
+__device__ __forceinline__ int row_owner(int row, int S) { return ((row + 1) * S + 127) / 128 - 1; }
 
 // (128 + nibble) as bf16 for nibbles e and e + 4 of w -> one bf16x2 register.
 __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
@@ -163,7 +185,7 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     const unsigned short* z16 = reinterpret_cast<const unsigned short*>(p.zeros);
 #pragma unroll
     for (int h = 0; h < (kWide ? 1 : 2); ++h) {
-      const int gi = (u * 128 + h * 64) / p.G;
+      const int gi = div_by_magic(2 * u + h, p.gmagic);
       const int64_t iA = (int64_t)nA * ng + gi, iB = (int64_t)nB * ng + gi;
       U.prm[2 * h + 0] = (uint32_t)__ldg(s16 + iA) | ((uint32_t)__ldg(z16 + iA) << 16);
       U.prm[2 * h + 1] = (uint32_t)__ldg(s16 + iB) | ((uint32_t)__ldg(z16 + iB) << 16);
@@ -331,7 +353,19 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   const int nA = n0 + g, nB = n0 + g + 8;
   const int ng = p.K / p.G;
 
-  // the first D units' loads go out before anything else
+  // ---- x[:, k0 : k0+klen) -> shared memory, as 16-byte asynchronous copies
+  // issued before the weight loads (every MMA waits on x). Only the M real
+  // tokens are copied: a padding token's MMA column never reaches an output.
+  const int kchunks = klen / 8;  // a multiple of 16
+  const uint32_t cmagic = div_magic((uint32_t)kchunks);
+  for (int c = tid; c < p.M * kchunks; c += blockDim.x) {
+    const int gt = div_by_magic(c, cmagic), cl = c - gt * kchunks;
+    int pc = cl ^ (gt & 1);
+    if (!kNF4 && kWide) pc ^= (cl >> 2) & 2;
+    cp_async16(xs + (size_t)gt * kc + pc * 8, p.x + (size_t)gt * p.K + k0 + cl * 8);
+  }
+
+  // then the first D units of weights of this warp
   const int64_t row_bytes = (int64_t)p.K / 2;
   const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + (kWide ? 16 : 8) * t;
   const uint8_t* wrowB = wrowA + 8 * row_bytes;
@@ -341,43 +375,38 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     for (int i = 0; i < D; ++i)
       if (u0 + i < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng);
   }
+  cp_async_wait_all();
+  __syncthreads();
 
-  // ---- stage x[:, k0 : k0+klen) into shared memory (16-byte chunks) -------
-  {
-    // Only the M real tokens are staged: the MMA columns of padding tokens
-    // never reach an output. cpr is a multiple of 16, so the chunks of one
-    // 64- or 128-wide sub-group sit in 8 or 16 consecutive lanes; the loop
-    // runs whole warps (its bound is rounded up to 32) for the shuffles.
-    const int cpr = kc / 8;
-    const int nchunks = p.M * cpr;
+  if (!kNF4) {
+    // In place, chunk by chunk: sums of x per 64- (narrow) or 128-wide (wide)
+    // sub-group, and the (k, k + 4) pairing of the INT4 nibbles. The chunks of
+    // one sub-group sit in 8 or 16 consecutive lanes; the loop runs whole
+    // warps (bound rounded up to 32) for the shuffles.
+    const int nchunks = p.M * kchunks;
     for (int c = tid; c < ((nchunks + 31) & ~31); c += blockDim.x) {
       const bool real = c < nchunks;
-      const int gt = c / cpr;
-      const int cl = c - gt * cpr;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (real && cl * 8 < klen)
-        v = *reinterpret_cast<const uint4*>(p.x + (size_t)gt * p.K + k0 + cl * 8);
+      const int gt = div_by_magic(c, cmagic), cl = c - gt * kchunks;
       int pc = cl ^ (gt & 1);
-      if (!kNF4) {
-        float sm = 0.0f;
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      if (kWide) pc ^= (cl >> 2) & 2;
+      uint4* slot = reinterpret_cast<uint4*>(xs + (size_t)gt * kc + pc * 8);
+      uint4 v = real ? *slot : make_uint4(0, 0, 0, 0);
+      float sm = 0.0f;
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) sm += bf16_lo_to_f32(w[q]) + bf16_hi_to_f32(w[q]);
-        sm += __shfl_xor_sync(0xffffffffu, sm, 1);
-        sm += __shfl_xor_sync(0xffffffffu, sm, 2);
-        sm += __shfl_xor_sync(0xffffffffu, sm, 4);
-        if (kWide) {
-          sm += __shfl_xor_sync(0xffffffffu, sm, 8);
-          if (real && (cl & 15) == 0) xsum[(cl >> 4) * kTok + gt] = sm;
-          pc ^= (cl >> 2) & 2;
-        } else {
-          if (real && (cl & 7) == 0) xsum[(cl >> 3) * kTok + gt] = sm;
-        }
-        // pair (k, k + 4) as one bf16x2 word, the INT4 nibble pairing
-        v = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
-                       prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
+      for (int q = 0; q < 4; ++q) sm += bf16_lo_to_f32(w[q]) + bf16_hi_to_f32(w[q]);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 1);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 2);
+      sm += __shfl_xor_sync(0xffffffffu, sm, 4);
+      if (kWide) {
+        sm += __shfl_xor_sync(0xffffffffu, sm, 8);
+        if (real && (cl & 15) == 0) xsum[(cl >> 4) * kTok + gt] = sm;
+      } else {
+        if (real && (cl & 7) == 0) xsum[(cl >> 3) * kTok + gt] = sm;
       }
-      if (real) *reinterpret_cast<uint4*>(xs + (size_t)gt * kc + pc * 8) = v;
+      if (real)
+        *slot = make_uint4(prmt(v.x, v.z, 0x5410u), prmt(v.x, v.z, 0x7632u),
+                           prmt(v.y, v.w, 0x5410u), prmt(v.y, v.w, 0x7632u));
     }
   }
   if (kNF4) {
@@ -396,7 +425,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     const int gt = tid / tpt, j = tid % tpt;
     uint16_t* row = xs + (size_t)gt * kc;
     float mx = 0.0f;
-    for (int c = j; c < kc / 8; c += tpt) {
+    for (int c = j; c < kchunks; c += tpt) {
       const uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -412,7 +441,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     }
     const float sc = __uint_as_float((uint32_t)(127 + e) << 23);
     if (j == 0) tok_inv[gt] = __uint_as_float((uint32_t)(127 - e) << 23);
-    for (int c = j; c < kc / 8; c += tpt) {
+    for (int c = j; c < kchunks; c += tpt) {
       uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
       uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -444,14 +473,32 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     }
   }
 
-  // ---- cluster split-K reduction through distributed shared memory --------
+  // ---- cluster split-K reduction: each CTA pushes its partials into the
+  // shared memory of the rank that owns the rows (red[src rank][local row]
+  // [token] there), one cluster barrier, then each owner sums its rows in
+  // rank order and writes them once as bf16. Remote stores need no round
+  // trip, and no CTA touches another's shared memory after the barrier.
+  const int rows_max = (kRowsPerCta + p.S - 1) / p.S;
 #pragma unroll
   for (int a = 0; a < NT; ++a)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int row = warp * 16 + g + 8 * (r >> 1);
-      const int tok = 8 * a + 2 * t + (r & 1);
-      red[row * 16 + tok] = kNF4 ? acc[a][r] * tok_inv[tok] : acc[a][r];
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = warp * 16 + g + 8 * hr;
+      const int owner = row_owner(row, p.S);
+      const int lr = row - rank_row_begin(owner, p.S);
+      const int tok = 8 * a + 2 * t;
+      float v0 = acc[a][2 * hr], v1 = acc[a][2 * hr + 1];
+      if (kNF4) {
+        v0 *= tok_inv[tok];
+        v1 *= tok_inv[tok + 1];
+      }
+      float* dst = red + ((size_t)rank * rows_max + lr) * 16 + tok;
+      if (p.S > 1) {
+        st_cluster_f32x2(map_rank(dst, (uint32_t)owner), v0, v1);
+      } else {
+        dst[0] = v0;
+        dst[1] = v1;
+      }
     }
   if (p.S > 1) {
     cluster_sync_all();
@@ -459,32 +506,24 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     __syncthreads();
   }
   {
-    const int r_begin = rank * kRowsPerCta / p.S;
-    const int nrows = (rank + 1) * kRowsPerCta / p.S - r_begin;
+    const int r_begin = rank_row_begin(rank, p.S);
+    const int nrows = rank_row_begin(rank + 1, p.S) - r_begin;
     const int items = nrows * p.M;
     for (int i = tid; i < items; i += blockDim.x) {
       const int tok = i / nrows;
-      const int row = r_begin + (i - tok * nrows);
-      const int n = row_tile + row;
-      const float* src = &red[row * 16 + tok];
-      float parts[kMaxSplit];
-#pragma unroll
-      for (int q = 0; q < kMaxSplit; ++q)  // all remote loads in flight before the sum
-        parts[q] =
-            (q < p.S) ? (p.S > 1 ? ld_cluster_f32(map_rank(src, (uint32_t)q)) : *src) : 0.0f;
+      const int lr = i - tok * nrows;
+      const int n = row_tile + r_begin + lr;
       float v = 0.0f;
-#pragma unroll
-      for (int q = 0; q < kMaxSplit; ++q) v += parts[q];
+      for (int q = 0; q < p.S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
       if (n < p.N) p.y[(int64_t)tok * p.N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
     }
   }
-  if (p.S > 1) cluster_sync_relaxed();  // keep shared memory alive until all ranks have read it
 }
 
 template <int NT, bool kNF4>
-size_t gemv_smem(int kc) {
-  return (size_t)8 * NT * kc * 2 + (size_t)kRowsPerCta * 16 * 4 +
-         (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
+size_t gemv_smem(int kc, int S) {
+  const size_t red = (size_t)S * ((kRowsPerCta + S - 1) / S) * 16 * 4;
+  return (size_t)8 * NT * kc * 2 + red + (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
 }
 
 struct Plan {
@@ -510,7 +549,7 @@ Plan make_plan(int64_t N, int64_t K) {
     if (S > units) break;
     const int kc = (int)((units + S - 1) / S) * 128;
     if ((int64_t)8 * NT * kc * 2 > kMaxXChunkBytes) continue;
-    const size_t smem = gemv_smem<NT, kNF4>(kc);
+    const size_t smem = gemv_smem<NT, kNF4>(kc, S);
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess) {
       cudaGetLastError();
@@ -546,8 +585,9 @@ Plan make_plan(int64_t N, int64_t K) {
     if (slots < 1) continue;
     const int64_t grid = tiles * S;
     const int64_t waves = (grid + slots - 1) / slots;
-    // share of the resident slots kept busy, discounted per extra wave
-    const double score = (double)grid / ((double)waves * slots) - 0.02 * (double)(waves - 1);
+    // fewest waves first (a second wave repeats the whole load ramp), then
+    // the largest share of the resident slots kept busy
+    const double score = (double)grid / ((double)waves * slots) - (double)waves;
     if (score > best + 1e-9) {
       best = score;
       bp.S = S;
@@ -628,6 +668,7 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   a.units = (int)(K / 128);
   a.S = 1;
   a.kc = 0;
+  a.gmagic = div_magic((uint32_t)(group / 64));
   if (fmt == WQ_FMT_NF4)
     return NT == 1 ? launch_t<1, true, false>(a, st) : launch_t<2, true, false>(a, st);
   if (group % 128 == 0)

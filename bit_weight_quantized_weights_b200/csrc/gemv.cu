@@ -543,7 +543,7 @@ Plan make_plan(int64_t N, int64_t K) {
   auto kern = gemv_kernel<NT, kNF4, kWide>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaGetLastError();
-  double best = -1.0;
+  double best = -1e30;
   Plan bp;
   for (int S = 1; S <= kMaxSplit; ++S) {
     if (S > units) break;

@@ -80,6 +80,12 @@ def test_gemv_ragged_and_groups(wq, m, n, k, group):
     _run_int4(wq, m, n, k, group, seed=m)
 
 
+def test_gemv_more_tiles_than_resident_ctas(wq):
+    """512 row tiles over a short K: more CTAs than fit on the GPU at once,
+    so the launch needs several waves."""
+    _run_int4(wq, 3, 65536, 256, 128, seed=5)
+
+
 @pytest.mark.parametrize("m,n,k", [(3, 1040, 384), (13, 272, 1280)])
 def test_gemv_ragged_nf4(wq, m, n, k):
     _run_nf4(wq, m, n, k, seed=m)

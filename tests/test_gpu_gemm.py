@@ -37,6 +37,8 @@ def _x(m, k, seed):
     (1, 128, 128, 64),        # one row
     (257, 512, 1024, 1024),   # per-channel groups
     (64, 256, 512, 64),       # M below one tile
+    (600, 12800, 256, 128),   # 192-token tiles, several per CTA (both accumulators reused)
+    (384, 9344, 256, 64),     # 128-token tiles, up to two per CTA
 ])
 def test_gemm_small_every_element(wq, m, n, k, group):
     q, s, z, qweight = helpers.int4_packed(n, k, group, seed=m)

@@ -246,6 +246,38 @@ def captured_traffic(op):
     return entry["bytes_per_launch"]
 
 
+def dequant_then_cublas(wq, step, fused_ms, warmup):
+    """The dequantize-then-bf16-GEMM baseline on the step's GEMM workload: the
+    library's INT4 dequantization to a bf16 [N, K] weight, then torch.matmul
+    (cuBLAS). Timed after the step's timed region, outside ms_per_step."""
+    m, n, k = GEMM_SHAPE
+    qw, sc, zr = step.pw
+    wd = torch.empty(n, k, dtype=torch.bfloat16, device=step.px.device)
+    y = torch.empty(m, n, dtype=torch.bfloat16, device=step.px.device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    reps = 5
+    t_deq = t_mm = 0.0
+    for i in range(max(warmup, 1) + reps):
+        ev[0].record()
+        wq.wq_int4_dequant(qw, sc, zr, n, k, 128, out=wd)
+        ev[1].record()
+        torch.matmul(step.px, wd.t(), out=y)
+        ev[2].record()
+        torch.cuda.synchronize()
+        if i >= max(warmup, 1):
+            t_deq += ev[0].elapsed_time(ev[1]) / reps
+            t_mm += ev[1].elapsed_time(ev[2]) / reps
+    del wd, y
+    flops = 2.0 * m * n * k
+    return {"workload": "gemm int4-g128 %dx%dx%d" % (m, n, k),
+            "dequant_then_cublas_ms": round(t_deq + t_mm, 4), "dequant_ms": round(t_deq, 4),
+            "cublas_bf16_ms": round(t_mm, 4),
+            "dequant_then_cublas_tflops": round(flops / ((t_deq + t_mm) * 1e-3) / 1e12, 1),
+            "fused_gemm_ms": round(fused_ms, 4),
+            "fused_tflops": round(flops / (fused_ms * 1e-3) / 1e12, 1),
+            "fused_speedup": round((t_deq + t_mm) / fused_ms, 3)}
+
+
 def run_gpu(args, rank, world, device):
     from bit_weight_quantized_weights_b200 import binding as wq
     peaks = load_peaks()
@@ -283,6 +315,8 @@ def run_gpu(args, rank, world, device):
     st, detail = wq.wq_device_error()
     if st != wq.WQ_OK:
         raise RuntimeError("device error word set during timing: 0x%x" % detail)
+
+    comparator = dequant_then_cublas(wq, step, per_op_ms["gemm"], args.warmup) if rank == 0 else None
 
     ms_per_step = elapsed_ms / args.steps
     roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
@@ -325,6 +359,7 @@ def run_gpu(args, rank, world, device):
                      "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_source": peaks["source"] + " (burst)"},
         "per_op": {k: {a: round(b, 4) for a, b in v.items()} for k, v in details.items()},
+        "comparator": comparator,
         "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks.summary(),
     }

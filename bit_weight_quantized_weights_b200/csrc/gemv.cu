@@ -58,17 +58,15 @@
 //   lut  [256 entries][32 lanes] u32 (NF4 only)
 //   red  [S ranks][ceil(128/S) rows][16 tokens] fp32, the partials of the
 //        rows this rank owns, as pushed by every rank of the cluster
-#include <mutex>
-
-#include "common.cuh"
+#include "splitk_common.cuh"
 
 namespace wq {
 namespace {
 
 __device__ unsigned int g_gemv_error;  // this kernel has no waits; kept for the ABI
 
-constexpr int kRowsPerCta = 128;
-constexpr int kMaxSplit = 16;         // cluster size limit (non-portable above 8)
+using namespace splitk;
+
 constexpr int kMaxXChunkBytes = 64 * 1024;
 
 struct GemvArgs {
@@ -83,15 +81,6 @@ struct GemvArgs {
   int kc;                 // shared-memory K-chunk length (max over ranks)
   uint32_t gmagic;        // h / (G / 64) == umulhi(h, gmagic) for 64-wide part h; 0 if G == 64
 };
-
-// n / d without a divide: umulhi(n, floor(2^32 / d) + 1) is exact whenever
-// n * d < 2^32 (d >= 2).
-__host__ __device__ __forceinline__ uint32_t div_magic(uint32_t d) {
-  return d < 2 ? 0u : (uint32_t)(0xFFFFFFFFu / d) + 1u;
-}
-__device__ __forceinline__ int div_by_magic(int n, uint32_t magic) {
-  return magic ? (int)__umulhi((uint32_t)n, magic) : n;
-}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -108,35 +97,6 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-
-// Cluster barrier that publishes this CTA's shared-memory writes to the others.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
-               ::: "memory");
-}
-__device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
-}
-
-// 16-byte asynchronous global -> shared copy (L2 only), and its completion.
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-// Rows of a 128-row tile are split over the S ranks of a cluster as
-// [b(r), b(r + 1)) with b(r) = floor(128 r / S); the owner of row is the r
-// with b(r) <= row < b(r + 1).
-__host__ __device__ __forceinline__ int rank_row_begin(int r, int S) { return r * 128 / S; }
-__device__ __forceinline__ int row_owner(int row, int S) { return ((row + 1) * S + 127) / 128 - 1; }
 
 // (128 + nibble) as bf16 for nibbles e and e + 4 of w -> one bf16x2 register.
 __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
@@ -473,180 +433,29 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     }
   }
 
-  // ---- cluster split-K reduction: each CTA pushes its partials into the
-  // shared memory of the rank that owns the rows (red[src rank][local row]
-  // [token] there), one cluster barrier, then each owner sums its rows in
-  // rank order and writes them once as bf16. Remote stores need no round
-  // trip, and no CTA touches another's shared memory after the barrier.
-  const int rows_max = (kRowsPerCta + p.S - 1) / p.S;
-#pragma unroll
-  for (int a = 0; a < NT; ++a)
-#pragma unroll
-    for (int hr = 0; hr < 2; ++hr) {
-      const int row = warp * 16 + g + 8 * hr;
-      const int owner = row_owner(row, p.S);
-      const int lr = row - rank_row_begin(owner, p.S);
-      const int tok = 8 * a + 2 * t;
-      float v0 = acc[a][2 * hr], v1 = acc[a][2 * hr + 1];
-      if (kNF4) {
-        v0 *= tok_inv[tok];
-        v1 *= tok_inv[tok + 1];
-      }
-      float* dst = red + ((size_t)rank * rows_max + lr) * 16 + tok;
-      if (p.S > 1) {
-        st_cluster_f32x2(map_rank(dst, (uint32_t)owner), v0, v1);
-      } else {
-        dst[0] = v0;
-        dst[1] = v1;
-      }
-    }
-  if (p.S > 1) {
-    cluster_sync_all();
-  } else {
-    __syncthreads();
-  }
-  {
-    const int r_begin = rank_row_begin(rank, p.S);
-    const int nrows = rank_row_begin(rank + 1, p.S) - r_begin;
-    const int items = nrows * p.M;
-    for (int i = tid; i < items; i += blockDim.x) {
-      const int tok = i / nrows;
-      const int lr = i - tok * nrows;
-      const int n = row_tile + r_begin + lr;
-      float v = 0.0f;
-      for (int q = 0; q < p.S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
-      if (n < p.N) p.y[(int64_t)tok * p.N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
-    }
-  }
+  // ---- cluster split-K reduction (through distributed shared memory) -----
+  reduce_and_store<NT>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N, p.y);
 }
 
 template <int NT, bool kNF4>
 size_t gemv_smem(int kc, int S) {
-  const size_t red = (size_t)S * ((kRowsPerCta + S - 1) / S) * 16 * 4;
-  return (size_t)8 * NT * kc * 2 + red + (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
-}
-
-struct Plan {
-  int S = 0;
-  int kc = 0;
-  size_t smem = 0;
-};
-
-// Cluster size S (K split): every CTA holds one 128-row tile over one K-chunk.
-// S (1..16, at most one unit per CTA, x chunk <= 64 KB) is chosen to fill the
-// resident CTA slots of the GPU with the fewest waves: the whole weight
-// stream should be in flight from the first microseconds.
-template <int NT, bool kNF4, bool kWide>
-Plan make_plan(int64_t N, int64_t K) {
-  const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
-  const int64_t units = K / 128;
-  auto kern = gemv_kernel<NT, kNF4, kWide>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  cudaGetLastError();
-  double best = -1e30;
-  Plan bp;
-  for (int S = 1; S <= kMaxSplit; ++S) {
-    if (S > units) break;
-    const int kc = (int)((units + S - 1) / S) * 128;
-    if ((int64_t)8 * NT * kc * 2 > kMaxXChunkBytes) continue;
-    const size_t smem = gemv_smem<NT, kNF4>(kc, S);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    int slots = 0;
-    if (S == 1) {
-      int per_sm = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem) != cudaSuccess) {
-        cudaGetLastError();
-        continue;
-      }
-      slots = per_sm * num_sms();
-    } else {
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
-      cfg.blockDim = dim3(256, 1, 1);
-      cfg.dynamicSmemBytes = smem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = (unsigned)S;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
-        cudaGetLastError();
-        continue;
-      }
-      slots = clusters * S;
-    }
-    if (slots < 1) continue;
-    const int64_t grid = tiles * S;
-    const int64_t waves = (grid + slots - 1) / slots;
-    // fewest waves first (a second wave repeats the whole load ramp), then
-    // the largest share of the resident slots kept busy
-    const double score = (double)grid / ((double)waves * slots) - (double)waves;
-    if (score > best + 1e-9) {
-      best = score;
-      bp.S = S;
-      bp.kc = kc;
-      bp.smem = smem;
-    }
-  }
-  return bp;
-}
-
-// Plans are cached per (device, N, K): the occupancy queries cost far more
-// host time than the launch itself.
-template <int NT, bool kNF4, bool kWide>
-Plan plan_for(int64_t N, int64_t K) {
-  struct Entry {
-    int dev;
-    int64_t N, K;
-    Plan plan;
-  };
-  constexpr int kEntries = 64;
-  static Entry cache[kEntries];
-  static int used = 0;
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return Plan{};
-  std::lock_guard<std::mutex> lock(mu);
-  for (int i = 0; i < used; ++i)
-    if (cache[i].dev == dev && cache[i].N == N && cache[i].K == K) return cache[i].plan;
-  const Plan pl = make_plan<NT, kNF4, kWide>(N, K);
-  if (pl.S > 0 && used < kEntries) cache[used++] = Entry{dev, N, K, pl};
-  return pl;
+  return (size_t)8 * NT * kc * 2 + red_bytes(S) +
+         (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
 }
 
 template <int NT, bool kNF4, bool kWide>
 wq_status launch_t(GemvArgs a, cudaStream_t st) {
-  const Plan pl = plan_for<NT, kNF4, kWide>(a.N, a.K);
+  auto kern = gemv_kernel<NT, kNF4, kWide>;
+  const int M = a.M;
+  const Plan pl = cached_plan(reinterpret_cast<const void*>(kern), M, a.N, a.K, 0, [&] {
+    return make_plan(
+        kern, 256, a.N, a.K, [&](int kc) { return (int64_t)8 * NT * kc * 2 <= kMaxXChunkBytes; },
+        [&](int kc, int S) { return gemv_smem<NT, kNF4>(kc, S); });
+  });
   if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
   a.S = pl.S;
   a.kc = pl.kc;
-  auto kern = gemv_kernel<NT, kNF4, kWide>;
-  // the attribute is a per-function maximum; plans of other shapes may have
-  // set a smaller one since
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
-      cudaSuccess)
-    return WQ_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)a.S, (unsigned)((a.N + kRowsPerCta - 1) / kRowsPerCta), 1);
-  cfg.blockDim = dim3(256, 1, 1);
-  cfg.dynamicSmemBytes = pl.smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)a.S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, a, nf4_table()) != cudaSuccess) return WQ_ERR_CUDA;
-  return launch_status();
+  return launch_split(kern, pl, 256, a.N, st, a, nf4_table());
 }
 
 }  // namespace

@@ -345,6 +345,11 @@ size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C) {
   return planes_bytes(M, K, C) + (size_t)C * M * 4;
 }
 
+wq_status launch_msd_gemv(const int8_t* planes, int64_t plane_rows, const float* comp_scales,
+                          int64_t M, int64_t N, int64_t K, int32_t C, int32_t G,
+                          const void* qweight, const void* scales, const void* zeros, void* y,
+                          cudaStream_t st);
+
 wq_status launch_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_t C, int32_t G,
                           const void* qweight, const void* scales, const void* zeros, void* y,
                           void* workspace, cudaStream_t st) {
@@ -353,6 +358,10 @@ wq_status launch_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_
   const int64_t mp = m_padded(M);
   wq_status s = launch_msd_decompose(x, M, K, C, mp, planes, cs, st);
   if (s != WQ_OK) return s;
+  // decode sizes: the weight stream is the cost, so the split-K GEMV with
+  // integer warp MMAs replaces the 128-token tcgen05 tiles
+  if (M <= 16 && G % 128 == 0)
+    return launch_msd_gemv(planes, mp, cs, M, N, K, C, G, qweight, scales, zeros, y, st);
   CUtensorMap ta, tw;
   if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K, (uint64_t)(C * mp),
                     (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))

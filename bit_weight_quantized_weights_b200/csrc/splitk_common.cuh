@@ -1,0 +1,239 @@
+// Shared pieces of the decode (M <= 16) kernels: the W4A16 GEMV and the
+// Multi-Scale Dequant GEMV. Both give every CTA one 128-row weight tile over
+// one K-chunk, split K across a thread-block cluster, and reduce the fp32
+// partials through distributed shared memory.
+#pragma once
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace wq {
+namespace splitk {
+
+constexpr int kRowsPerCta = 128;
+constexpr int kMaxSplit = 16;  // cluster size limit (non-portable above 8)
+
+// n / d without a divide: umulhi(n, floor(2^32 / d) + 1) is exact whenever
+// n * d < 2^32 (d >= 2).
+__host__ __device__ __forceinline__ uint32_t div_magic(uint32_t d) {
+  return d < 2 ? 0u : (uint32_t)(0xFFFFFFFFu / d) + 1u;
+}
+__device__ __forceinline__ int div_by_magic(int n, uint32_t magic) {
+  return magic ? (int)__umulhi((uint32_t)n, magic) : n;
+}
+
+// Cluster barrier that publishes this CTA's shared-memory writes to the others.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float a, float b) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only), and its completion.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// Rows of a 128-row tile are split over the S ranks of a cluster as
+// [b(r), b(r + 1)) with b(r) = floor(128 r / S); the owner of row is the r
+// with b(r) <= row < b(r + 1).
+__host__ __device__ __forceinline__ int rank_row_begin(int r, int S) { return r * 128 / S; }
+__device__ __forceinline__ int row_owner(int row, int S) { return ((row + 1) * S + 127) / 128 - 1; }
+
+// Shared-memory bytes of the reduction buffer red[S ranks][ceil(128/S)][16].
+__host__ __device__ __forceinline__ size_t red_bytes(int S) {
+  return (size_t)S * ((kRowsPerCta + S - 1) / S) * 16 * 4;
+}
+
+// The cluster split-K reduction. acc[a][r] of this lane holds rows
+// warp*16 + g + 8 (r >> 1), tokens 8a + 2t + (r & 1) (the m16n8 accumulator
+// layout); tok_scale (optional, per token) multiplies it first. Each CTA
+// pushes its partials into the shared memory of the rank that owns the rows
+// (red[src rank][local row][token] there), one cluster barrier, then each
+// owner sums its rows in rank order and writes them once as bf16. Remote
+// stores need no round trip, and no CTA touches another's shared memory after
+// the barrier. All threads of the CTA must call this.
+template <int NT>
+__device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], const float* tok_scale,
+                                                 float* red, int S, int rank, int row_tile, int M,
+                                                 int N, uint16_t* y) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int rows_max = (kRowsPerCta + S - 1) / S;
+#pragma unroll
+  for (int a = 0; a < NT; ++a)
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int row = warp * 16 + g + 8 * hr;
+      const int owner = row_owner(row, S);
+      const int lr = row - rank_row_begin(owner, S);
+      const int tok = 8 * a + 2 * t;
+      float v0 = acc[a][2 * hr], v1 = acc[a][2 * hr + 1];
+      if (tok_scale) {
+        v0 *= tok_scale[tok];
+        v1 *= tok_scale[tok + 1];
+      }
+      float* dst = red + ((size_t)rank * rows_max + lr) * 16 + tok;
+      if (S > 1) {
+        st_cluster_f32x2(map_rank(dst, (uint32_t)owner), v0, v1);
+      } else {
+        dst[0] = v0;
+        dst[1] = v1;
+      }
+    }
+  if (S > 1) {
+    cluster_sync_all();
+  } else {
+    __syncthreads();
+  }
+  const int r_begin = rank_row_begin(rank, S);
+  const int nrows = rank_row_begin(rank + 1, S) - r_begin;
+  const int items = nrows * M;
+  for (int i = tid; i < items; i += blockDim.x) {
+    const int tok = i / nrows;
+    const int lr = i - tok * nrows;
+    const int n = row_tile + r_begin + lr;
+    float v = 0.0f;
+    for (int q = 0; q < S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
+    if (n < N) y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+  }
+}
+
+struct Plan {
+  int S = 0;
+  int kc = 0;
+  size_t smem = 0;
+};
+
+// Cluster size S (K split): every CTA holds one 128-row tile over one K-chunk
+// of kc = ceil(units / S) * 128. S (1..16, at most one 128-k unit per CTA,
+// fits(kc) true) is chosen to fill the resident CTA slots of the GPU with the
+// fewest waves: the whole weight stream should be in flight from the first
+// microseconds. smem_of(kc, S) gives the CTA's dynamic shared memory.
+template <class Kern, class Fits, class SmemOf>
+Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf smem_of) {
+  const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t units = K / 128;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaGetLastError();
+  double best = -1e30;
+  Plan bp;
+  for (int S = 1; S <= kMaxSplit; ++S) {
+    if (S > units) break;
+    const int kc = (int)((units + S - 1) / S) * 128;
+    if (!fits(kc)) continue;
+    const size_t smem = smem_of(kc, S);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    int slots = 0;
+    if (S == 1) {
+      int per_sm = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      slots = per_sm * num_sms();
+    } else {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
+      cfg.blockDim = dim3((unsigned)threads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)S;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        continue;
+      }
+      slots = clusters * S;
+    }
+    if (slots < 1) continue;
+    const int64_t grid = tiles * S;
+    const int64_t waves = (grid + slots - 1) / slots;
+    // fewest waves first (a second wave repeats the whole load ramp), then
+    // the largest share of the resident slots kept busy
+    const double score = (double)grid / ((double)waves * slots) - (double)waves;
+    if (score > best + 1e-9) {
+      best = score;
+      bp.S = S;
+      bp.kc = kc;
+      bp.smem = smem;
+    }
+  }
+  return bp;
+}
+
+// Plans are cached per (kernel, device, M, N, K, extra): the occupancy
+// queries cost far more host time than the launch itself.
+template <class MakeFn>
+Plan cached_plan(const void* kern, int M, int64_t N, int64_t K, int extra, MakeFn make) {
+  struct Entry {
+    const void* kern;
+    int dev, M, extra;
+    int64_t N, K;
+    Plan plan;
+  };
+  constexpr int kEntries = 128;
+  static Entry cache[kEntries];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return Plan{};
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].kern == kern && cache[i].dev == dev && cache[i].M == M && cache[i].N == N &&
+        cache[i].K == K && cache[i].extra == extra)
+      return cache[i].plan;
+  const Plan pl = make();
+  if (pl.S > 0 && used < kEntries) cache[used++] = Entry{kern, dev, M, extra, N, K, pl};
+  return pl;
+}
+
+// Launch `kern` on the plan's (S x row tiles) grid with S-CTA clusters.
+template <class Kern, class Args>
+wq_status launch_split(Kern kern, const Plan& pl, int threads, int64_t N, cudaStream_t st,
+                       const Args& args, const Nf4Table& tab) {
+  // the attribute is a per-function maximum; plans of other shapes may have
+  // set a smaller one since
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
+      cudaSuccess)
+    return WQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.S, (unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)pl.S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, args, tab) != cudaSuccess) return WQ_ERR_CUDA;
+  return launch_status();
+}
+
+}  // namespace splitk
+}  // namespace wq

@@ -88,3 +88,21 @@ def test_gemm_large_activation_range(wq):
     for r in range(3):
         helpers.check_within_bf16_rounding(y[r:r + 1], y_ref[r:r + 1], "row %d" % r, slack=1e-3)
     helpers.check_within_bf16_rounding(y[3:], y_ref[3:], "rest", slack=1e-3)
+
+
+def test_dequant_then_cublas_comparator(wq):
+    """The dequantize-then-bf16-GEMM comparator: the library's INT4 dequant to
+    bf16, then torch.matmul (cuBLAS). Its result matches the oracle's model of
+    that baseline (bf16-rounded weights, exact product) within one output
+    rounding plus the fp32 accumulation, and the exact product within the
+    product tolerance."""
+    m, n, k, group = 256, 512, 1024, 128
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed=11)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, 11)
+    wd = wq.wq_int4_dequant(qw, sc, zr, n, k, group)
+    y = torch.matmul(x.cuda(), wd.t()).cpu()
+    xf = helpers.x_f32(x)
+    y_model = products.dequant_then_bf16_matmul_int4(xf, q, s, z, group)
+    helpers.check_within_bf16_rounding(y, y_model, "dequant-then-cuBLAS vs its model", slack=1e-3)
+    helpers.check_product(y, products.w4a16_int4(xf, q, s, z, group), "dequant-then-cuBLAS")

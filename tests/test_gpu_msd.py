@@ -75,6 +75,12 @@ def _msd_case(wq, m, n, k, group, c, seed, rows=None, cols=None):
     (130, 128, 384, 128, 1),     # one component
     (130, 256, 384, 128, 3),     # three components (single TMEM buffer)
     (64, 128, 1152, 384, 2),     # group of 3 k-tiles
+    # decode sizes (M <= 16, groups of 128 or more): the split-K integer GEMV
+    (5, 384, 640, 128, 1),       # one component, ragged K split
+    (9, 256, 768, 256, 3),       # two token tiles, three components
+    (16, 1024, 2048, 128, 2),    # full token tile pair, several row tiles
+    (13, 512, 1280, 640, 2),     # groups of five units
+    (17, 256, 512, 128, 2),      # first size past the decode path: tcgen05 tiles
 ])
 def test_msd_gemm_small_every_element(wq, m, n, k, group, c):
     _msd_case(wq, m, n, k, group, c, seed=m + c)

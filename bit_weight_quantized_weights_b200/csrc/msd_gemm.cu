@@ -31,6 +31,7 @@
 //                in int32, convert, scale by the group's s[n, g], accumulate in
 //                fp32 registers; the last group writes bf16 y.
 #include "sm100.cuh"
+#include "splitk_common.cuh"
 
 namespace wq {
 
@@ -91,12 +92,12 @@ __device__ __forceinline__ uint2 unpack_word_minus_zero(uint32_t w, uint32_t zre
                     ((hi | 0x80808080u) - zrep) ^ 0x80808080u);
 }
 
-template <int C, bool kIntCombine>
+template <int C, bool kIntCombine, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     msd_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w, const __half* __restrict__ scales,
                     const __half* __restrict__ zeros, const float* __restrict__ comp_scales,
-                    uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad) {
+                    uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad, int S) {
   using Cfg = MsdCfg<C>;
   constexpr int NB = Cfg::kNB;
   extern __shared__ uint8_t smem_raw[];
@@ -116,11 +117,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
-  const int KT = K / BK;
-  const int TPG = G / BK;   // k-tiles per group
+  // split-K: cluster rank `rank` (of S along grid x) owns k-tiles [kt0, kt1)
+  // (without kSplit the launch has S == 1; the constants let the compiler
+  // keep the single-rank loops as simple as a kernel without the split)
+  const int rank = kSplit ? (int)blockIdx.x : 0;
+  // grid: (S, feature tiles, token tiles) with kSplit, else (feature tiles,
+  // token tiles)
+  const int n0 = (kSplit ? blockIdx.y : blockIdx.x) * BN;
+  const int m0 = (kSplit ? blockIdx.z : blockIdx.y) * BM;
+  const int KTA = K / BK;
+  const int kt0 = kSplit ? (int)((int64_t)rank * KTA / S) : 0;
+  const int kt1 = kSplit ? (int)((int64_t)(rank + 1) * KTA / S) : KTA;
+  const int KT = kt1 - kt0;  // k-tiles of this rank
+  const int TPG = G / BK;    // k-tiles per group
   const int NG = K / G;
+  // the rank's k-tiles cut its groups into sub-groups g_first .. g_last
+  const int g_first = kSplit ? kt0 / TPG : 0;
+  const int NSG = kSplit ? (kt1 - 1) / TPG - g_first + 1 : NG;
 
   if (threadIdx.x == 0) {
     sm100::tma_prefetch_desc(&tmap_a);
@@ -148,10 +161,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % kStages;
-        const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
-        if (kt >= kStages &&
+      for (int i = 0; i < KT; ++i) {
+        const int kt = kt0 + i;
+        const int s = i % kStages;
+        const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+        if (i >= kStages &&
             !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_msd_error, 0x1101u, abort_flag))
           break;
         sm100::mbar_arrive_expect_tx(&full[s], C * kPlaneBytes + kWBytes);
@@ -165,9 +179,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = sm100::idesc_s8_s32(BM, BN);
-      int kt = 0;
+      int i = 0;  // k-tiles consumed by this rank
       bool ok = true;
-      for (int gi = 0; gi < NG && ok; ++gi) {
+      for (int gi = 0; gi < NSG && ok; ++gi) {
         const int b = gi % NB;
         if (gi >= NB) {
           if (!sm100::mbar_wait(&acc_empty[b], (uint32_t)((gi / NB) - 1) & 1u, &g_msd_error,
@@ -177,9 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           sm100::tc_fence_after();
         }
-        for (int t = 0; t < TPG; ++t, ++kt) {
-          const int s = kt % kStages;
-          const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+        const int g = g_first + gi;
+        const int sg0 = kSplit ? max(kt0, g * TPG) : g * TPG;
+        const int sg1 = kSplit ? min(kt1, (g + 1) * TPG) : (g + 1) * TPG;
+        for (int t = 0; t < sg1 - sg0; ++t, ++i) {
+          const int s = i % kStages;
+          const uint32_t ph = (uint32_t)(i / kStages) & 1u;
           if (!sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1202u, abort_flag) ||
               !sm100::mbar_wait(&deq[s], ph, &g_msd_error, 0x1203u, abort_flag)) {
             ok = false;
@@ -207,10 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- unpack: B row r = feature n0 + r ----------------
     const int r = threadIdx.x - 64;
     const __half* zrow = zeros + (int64_t)(n0 + r) * NG;
-    uint32_t zrep = 0;
-    for (int kt = 0; kt < KT; ++kt) {
-      const int s = kt % kStages;
-      const uint32_t ph = (uint32_t)(kt / kStages) & 1u;
+    // the zero point of the rank's first group (its k-tiles may start inside it)
+    uint32_t zrep = (uint32_t)__half2float(zrow[kt0 / TPG]) * 0x01010101u;
+    for (int i = 0; i < KT; ++i) {
+      const int kt = kt0 + i;
+      const int s = i % kStages;
+      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
       if (kt % TPG == 0) {
         const uint32_t z = (uint32_t)__half2float(zrow[kt / TPG]);
         zrep = z * 0x01010101u;
@@ -244,14 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
     float pref = 0.0f;
-    if (e < BN) pref = __half2float(scales[(int64_t)(n0 + e) * NG]);
+    if (e < BN) pref = __half2float(scales[(int64_t)(n0 + e) * NG + g_first]);
     bool ok = true;
-    for (int gi = 0; gi < NG; ++gi) {
+    for (int gi = 0; gi < NSG; ++gi) {
       const int b = gi % NB;
       if (e < BN) sclE[(gi & 1) * 128 + e] = pref;
       named_bar_sync(1, 32 * kEpiWarps);
-      if (e < BN && gi + 1 < NG) pref = __half2float(scales[(int64_t)(n0 + e) * NG + gi + 1]);
-      // every epilogue warp runs all NG iterations (the named barrier above
+      if (e < BN && gi + 1 < NSG)
+        pref = __half2float(scales[(int64_t)(n0 + e) * NG + g_first + gi + 1]);
+      // every epilogue warp runs all NSG iterations (the named barrier above
       // counts on it); after a failed wait the rest only keep that barrier
       if (ok) {
         bool got = sm100::mbar_wait(&acc_full[b], (uint32_t)(gi / NB) & 1u, &g_msd_error,
@@ -295,19 +315,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
     }
-    const int m = m0 + row;
-    if (ok && m < M) {
-      const float sC = comp_scales[(int64_t)(C - 1) * M + m];
-      uint16_t* dst = y + (int64_t)m * N + n0 + half * 64;
+    if (!kSplit) {
+      const int m = m0 + row;
+      if (ok && m < M) {
+        const float sC = comp_scales[(int64_t)(C - 1) * M + m];
+        uint16_t* dst = y + (int64_t)m * N + n0 + half * 64;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint4 o;
-        o.x = pack_bf16x2(acc[8 * i + 0] * sC, acc[8 * i + 1] * sC);
-        o.y = pack_bf16x2(acc[8 * i + 2] * sC, acc[8 * i + 3] * sC);
-        o.z = pack_bf16x2(acc[8 * i + 4] * sC, acc[8 * i + 5] * sC);
-        o.w = pack_bf16x2(acc[8 * i + 6] * sC, acc[8 * i + 7] * sC);
-        *reinterpret_cast<uint4*>(dst + 8 * i) = o;
+        for (int i = 0; i < 8; ++i) {
+          uint4 o;
+          o.x = pack_bf16x2(acc[8 * i + 0] * sC, acc[8 * i + 1] * sC);
+          o.y = pack_bf16x2(acc[8 * i + 2] * sC, acc[8 * i + 3] * sC);
+          o.z = pack_bf16x2(acc[8 * i + 4] * sC, acc[8 * i + 5] * sC);
+          o.w = pack_bf16x2(acc[8 * i + 6] * sC, acc[8 * i + 7] * sC);
+          *reinterpret_cast<uint4*>(dst + 8 * i) = o;
+        }
       }
+    } else {
+      // push this rank's partials to the rank that owns the token rows
+      splitk::cluster_sync_all();  // every rank is past its main loop
+      const int rows_max = (BM + S - 1) / S;
+      const int owner = splitk::row_owner(row, S);
+      const int lr = row - splitk::rank_row_begin(owner, S);
+      float* dst = reinterpret_cast<float*>(smem) + ((size_t)rank * rows_max + lr) * BN + half * 64;
+      const uint32_t rdst = splitk::map_rank(dst, (uint32_t)owner);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(rdst + 16u * i),
+                     "f"(acc[4 * i]), "f"(acc[4 * i + 1]), "f"(acc[4 * i + 2]),
+                     "f"(acc[4 * i + 3])
+                     : "memory");
+      splitk::cluster_sync_all();  // all partials have landed
+    }
+  }
+  if (kSplit) {
+    // Split-K over the cluster: once every rank has finished its main loop
+    // (first cluster barrier; the stage ring is then free everywhere), the
+    // drain warps pushed their partials into the ring of the rank that owns
+    // those token rows (red[src rank][local row][128 features] there, remote
+    // stores); after the second barrier each owner sums its rows in rank
+    // order and writes them once as bf16. Every thread of every rank passes
+    // both barriers, also after an abort.
+    if (warp < 2 + kUnpackWarps) {
+      __syncwarp();
+      splitk::cluster_sync_all();
+      splitk::cluster_sync_all();
+    }
+    const float* red = reinterpret_cast<const float*>(smem);
+    const int rows_max = (BM + S - 1) / S;
+    const int r_begin = splitk::rank_row_begin(rank, S);
+    const int nrows = splitk::rank_row_begin(rank + 1, S) - r_begin;
+    for (int it = threadIdx.x; it < nrows * (BN / 2); it += blockDim.x) {
+      const int lr = it / (BN / 2), cp = it - lr * (BN / 2);
+      const int m = m0 + r_begin + lr;
+      if (m >= M) continue;
+      float v0 = 0.0f, v1 = 0.0f;
+      for (int qq = 0; qq < S; ++qq) {
+        const float2 pv =
+            *reinterpret_cast<const float2*>(red + ((size_t)qq * rows_max + lr) * BN + 2 * cp);
+        v0 += pv.x;
+        v1 += pv.y;
+      }
+      const float sC = comp_scales[(int64_t)(C - 1) * M + m];
+      *reinterpret_cast<uint32_t*>(y + (int64_t)m * N + n0 + 2 * cp) =
+          pack_bf16x2(v0 * sC, v1 * sC);
     }
   }
 
@@ -319,21 +389,70 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// K split (cluster size) for problems with fewer output tiles than SMs: each
+// rank of an S-CTA cluster takes a contiguous run of k-tiles (at least one)
+// and the partials meet through distributed shared memory. S is the largest
+// value up to 8 whose clusters all fit on the GPU at once.
+template <class Kern>
+int msd_split(Kern kern, int smem, int64_t tiles, int64_t ktiles) {
+  if (tiles >= num_sms()) return 1;
+  int S = (int)(num_sms() / tiles);
+  S = S > 8 ? 8 : S;
+  S = S > ktiles ? (int)ktiles : S;
+  for (; S > 1; --S) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      continue;
+    }
+    if (clusters >= tiles) break;
+  }
+  return S < 1 ? 1 : S;
+}
+
 template <int C, bool kInt>
 wq_status launch_c(const CUtensorMap& ta, const CUtensorMap& tw, const void* scales,
                    const void* zeros, const float* cs, void* y, int64_t M, int64_t N, int64_t K,
                    int32_t G, cudaStream_t st) {
   using Cfg = MsdCfg<C>;
-  auto kern = msd_gemm_kernel<C, kInt>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
-      cudaSuccess)
-    return WQ_ERR_CUDA;
   const int64_t mp = m_padded(M);
-  dim3 grid((unsigned)(N / BN), (unsigned)(mp / BM));
-  kern<<<grid, kThreads, Cfg::kSmem, st>>>(ta, tw, static_cast<const __half*>(scales),
-                                           static_cast<const __half*>(zeros), cs,
-                                           static_cast<uint16_t*>(y), (int)M, (int)N, (int)K, G,
-                                           (int)mp);
+  const int64_t tiles = (N / BN) * (mp / BM);
+  auto kern_split = msd_gemm_kernel<C, kInt, true>;
+  auto kern_one = msd_gemm_kernel<C, kInt, false>;
+  for (auto kf : {kern_split, kern_one})
+    if (cudaFuncSetAttribute(kf, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) !=
+        cudaSuccess)
+      return WQ_ERR_CUDA;
+  const int S = msd_split(kern_split, Cfg::kSmem, tiles, K / BK);
+  auto kern = S > 1 ? kern_split : kern_one;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = S > 1 ? dim3((unsigned)S, (unsigned)(N / BN), (unsigned)(mp / BM))
+                      : dim3((unsigned)(N / BN), (unsigned)(mp / BM), 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S > 1 ? 1 : 0;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tw, static_cast<const __half*>(scales),
+                         static_cast<const __half*>(zeros), cs, static_cast<uint16_t*>(y), (int)M,
+                         (int)N, (int)K, G, (int)mp, S) != cudaSuccess)
+    return WQ_ERR_CUDA;
   return launch_status();
 }
 

@@ -511,7 +511,7 @@ def max_over_ranks(v, world, device):
     return float(t.item())
 
 
-PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd")
+PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd", "msd_m16")
 
 
 def profile_case(case, device):
@@ -546,8 +546,8 @@ def profile_case(case, device):
         ws = wq.gemm_workspace(m, n, k, 128, device)
         fn = lambda: wq.wq_w4a16_gemm(x, n, wq.WQ_FMT_INT4_ASYM, 128, *pw, workspace=ws,  # noqa
                                       out=y)
-    elif case == "msd":
-        m, (n, k) = 1024, MSD_SHAPE
+    elif case in ("msd", "msd_m16"):
+        m, (n, k) = (1024 if case == "msd" else 16), MSD_SHAPE
         pw = wq.wq_quantize_pack(wq.WQ_FMT_INT4_ASYM, normal(n, k, std=0.02), 128)
         x = normal(m, k).to(torch.bfloat16)
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)

@@ -249,6 +249,14 @@ def captured_traffic(op):
     return entry["bytes_per_launch"]
 
 
+def job_value(table, ms_per_step, world):
+    """Whole-job value: 100 x (roofline time of one GPU's step) / (the slowest
+    rank's step time) x ranks. Each replica runs the full step (weak
+    scaling), so the work grows with the number of GPUs."""
+    roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
+    return 100.0 * roof_ms / ms_per_step * world
+
+
 def dequant_then_cublas(wq, step, fused_ms, warmup):
     """The dequantize-then-bf16-GEMM baseline on the step's GEMM workload: the
     library's INT4 dequantization to a bf16 [N, K] weight, then torch.matmul
@@ -322,8 +330,7 @@ def run_gpu(args, rank, world, device):
     comparator = dequant_then_cublas(wq, step, per_op_ms["gemm"], args.warmup) if rank == 0 else None
 
     ms_per_step = elapsed_ms / args.steps
-    roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
-    value = 100.0 * roof_ms / ms_per_step * world
+    value = job_value(table, ms_per_step, world)
 
     # dominant kernel: the op with the largest share of the step
     dom = max(per_op_ms, key=per_op_ms.get)
@@ -405,8 +412,7 @@ def measure_e2e(args, step, ops, table, world, device):
     b.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b), world, device) / steps
-    roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
-    return {"value": round(100.0 * roof_ms / ms * world, 3), "unit": UNIT,
+    return {"value": round(job_value(table, ms, world), 3), "unit": UNIT,
             "ms_per_step": round(ms, 3), "steps": steps,
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 

@@ -14,8 +14,8 @@ wq_status launch_int4_dequant(const uint32_t*, const void*, const void*, int64_t
                               void*, wq_dtype, cudaStream_t);
 wq_status launch_gemv(const void*, int64_t, int64_t, int64_t, wq_format, int32_t, const void*,
                       const void*, const void*, void*, cudaStream_t);
-wq_status launch_gemm(const void*, int64_t, int64_t, int64_t, int32_t, const void*, const void*,
-                      const void*, void*, void*, cudaStream_t);
+wq_status launch_gemm(const void*, int64_t, int64_t, int64_t, wq_format, int32_t, const void*,
+                      const void*, const void*, void*, void*, cudaStream_t);
 size_t gemm_workspace_bytes(int64_t M, int64_t K);
 wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, int8_t*, float*,
                                cudaStream_t);
@@ -192,13 +192,12 @@ wq_status wq_w4a16_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_forma
                         void* y, void* workspace, size_t ws_bytes, void* stream) {
   wq_status s = check_product(x, M, N, K, fmt, group, qweight, scales, zeros, y);
   if (s != WQ_OK) return s;
-  if (fmt != WQ_FMT_INT4_ASYM) return WQ_ERR_UNSUPPORTED;
   if (N % 128 != 0) return WQ_ERR_UNSUPPORTED;
   if (M == 0 || N == 0) return WQ_OK;
   if (!workspace || ws_bytes < gemm_workspace_bytes(M, K)) return WQ_ERR_WORKSPACE;
   if (!aligned16(workspace)) return WQ_ERR_ALIGNMENT;
   return guarded([&] {
-    return launch_gemm(x, M, N, K, group, qweight, scales, zeros, y, workspace,
+    return launch_gemm(x, M, N, K, fmt, group, qweight, scales, zeros, y, workspace,
                        as_stream(stream));
   });
 }

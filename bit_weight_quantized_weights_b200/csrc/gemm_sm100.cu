@@ -27,6 +27,9 @@
 //               main loop they are the epilogue: TMEM -> x 2^-e per token ->
 //               bf16 -> shared staging tile [BT tokens][128 rows] -> one TMA
 //               store into y.
+// NF4 weights (block 64 = one k-tile) take the same path: a 256-entry
+// per-lane table turns each code byte into the fp16 pair of its two codebook
+// values, and one fp16 multiply applies the block's absmax.
 // Operands are fp16, not bf16: the activations arrive as fp16 copies scaled
 // by a power of two per row (exact), and the dequantized weight is
 // fp16_rn((q - z) * s): the nibble becomes fp16 1024 + q or 64 + q by one
@@ -39,7 +42,7 @@
 namespace wq {
 
 wq_status launch_x_to_f16(const void* x, int64_t M, int64_t K, void* x16, float* inv_scale,
-                          cudaStream_t st);
+                          bool permute, cudaStream_t st);
 
 namespace {
 
@@ -60,7 +63,11 @@ struct GemmCfg {
   static constexpr int kOutBytes = BT * BW * 2;   // epilogue staging (reuses the ring)
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kRingOrOut = kRing > kOutBytes ? kRing : kOutBytes;
-  static constexpr int kSmem = kRingOrOut + BT * 4 /*2^-e per token*/ + 1024 /*align*/ + 512;
+  static constexpr int kLutBytes = 256 * 32 * 4;  // NF4: byte -> fp16 pair, one copy per lane
+  // ring or staging, 2^-e per token, barriers (512 B), alignment slack; NF4
+  // adds the lookup table after the barriers
+  static constexpr int kSmem = kRingOrOut + BT * 4 + 512 + 1024;
+  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
   static constexpr uint32_t kTmemCols = (BT + SA * 32 <= 256) ? 256 : 512;
 };
@@ -91,13 +98,13 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb_hi, uint32_
   out[3] = f16x2_mul(f16x2_sub(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), zb_lo), s2);
 }
 
-template <int BT>
+template <int BT, bool kNF4>
 __global__ void __launch_bounds__(kThreads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_w,
-                      const __grid_constant__ CUtensorMap tmap_y, const __half* __restrict__ scales,
+                      const __grid_constant__ CUtensorMap tmap_y, const void* __restrict__ scales,
                       const __half* __restrict__ zeros, const float* __restrict__ inv_scale, int M,
-                      int N, int K, int G) {
+                      int N, int K, int G, Nf4Table tab) {
   using C = GemmCfg<BT>;
   constexpr int ST = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -114,6 +121,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* accf = afree + SA;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // NF4 only: lut[byte][lane] = fp16 pair (codebook[high nibble], codebook[low
+  // nibble]) = elements (2j, 2j + 1); lane l reads column l, so bank l
+  uint32_t* lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 512);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BW;
@@ -138,6 +148,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int j = (int)threadIdx.x - 64; j >= 0 && j < BT; j += kThreads - 64)
     s_inv[j] = (m0 + j < M) ? inv_scale[m0 + j] : 0.0f;
+  if (kNF4) {
+    // four lanes' copies of one entry per 16-byte store
+    for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
+      const int e = i >> 3;
+      const uint32_t v = pack_f16x2(tab.v[e >> 4], tab.v[e & 15]);
+      reinterpret_cast<uint4*>(lut)[i] = make_uint4(v, v, v, v);
+    }
+  }
   if (warp == 1) {
     sm100::tmem_alloc(tmem_slot, C::kTmemCols);
     sm100::tmem_relinquish();
@@ -158,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* st = ring + s * C::kStageBytes;
         sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         sm100::tma_load_2d(st, &tmap_x, &full[s], kt * BK, m0);
-        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &full[s], kt * (BK / 8), n0);
+        // packed tile: 8 uint32 words (INT4) or 32 code bytes (NF4) per row
+        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &full[s], kt * (kNF4 ? BK / 2 : BK / 8), n0);
       }
     }
   } else if (warp == 1) {
@@ -194,16 +213,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ng = K / G;
     const int tiles_per_group = G / BK;
     // group parameters are loaded one group ahead of their use
-    const __half* srow = scales + (int64_t)n * ng;
-    const __half* zrow = zeros + (int64_t)n * ng;
-    __half s_next = srow[0], z_next = zrow[0];
+    const __half* srow = static_cast<const __half*>(scales) + (int64_t)n * ng;
+    const __half* zrow = kNF4 ? nullptr : zeros + (int64_t)n * ng;
+    __half s_next = kNF4 ? __ushort_as_half(0) : srow[0];
+    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[0];
     uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
+    // NF4: the absmax of (row n, 64-element block kt) is one per k-tile
+    const float* arow = static_cast<const float*>(scales) + (int64_t)n * (K / 64);
+    float am_next = kNF4 ? arow[0] : 0.0f;
+    const uint32_t* lut_lane = lut + lane;
     int gi = 0, left = 0;  // current group, k-tiles left in it
     bool ok = true;
     for (int kt = 0; kt < KT && ok; ++kt) {
       const int s = kt % ST, a = kt % SA;
       const uint32_t ph = (uint32_t)(kt / ST) & 1u, pa = (uint32_t)(kt / SA) & 1u;
-      if (left == 0) {
+      uint32_t am2 = 0;
+      if (kNF4) {
+        // fp16x2 (absmax, absmax), rounded once; the next one is loaded now
+        am2 = pack_f16x2(am_next, am_next);
+        if (kt + 1 < KT) am_next = arow[kt + 1];
+      } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
         const uint32_t zq = (uint32_t)__half2float(z_next);
         s2 = sb | (sb << 16);
@@ -227,10 +256,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint4 wv = *reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
                                                        r * 32 + hk * 16);
       uint32_t cols[16];
-      dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
-      dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
-      dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
-      dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+      if (kNF4) {
+        // 16 code bytes = elements (2j, 2j + 1) in k order: one table read
+        // gives the fp16 code pair, one multiply applies the block's absmax
+        const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
+      } else {
+        dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
+        dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
+        dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
+        dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+      }
       sm100::tmem_st16(tmem + lane_base + C::kAccCols + (uint32_t)(a * 32 + hk * 16), cols);
       sm100::tmem_st_wait();
       sm100::tc_fence_before();
@@ -272,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BT>
+template <int BT, bool kNF4>
 wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t N, int64_t K,
                     int32_t G, const void* qweight, const void* scales, const void* zeros, void* y,
                     cudaStream_t st) {
@@ -280,21 +318,26 @@ wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t 
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M,
                     (uint64_t)K * 2, BK, BT, CU_TENSOR_MAP_SWIZZLE_128B))
     return WQ_ERR_CUDA;
-  if (!make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)K / 8, (uint64_t)N,
-                    (uint64_t)K / 2, BK / 8, BW, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return WQ_ERR_CUDA;
+  // the packed tile is 32 bytes of each of 128 rows in both formats
+  const bool wmap = kNF4 ? make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qweight,
+                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, BK / 2, BW,
+                                        CU_TENSOR_MAP_SWIZZLE_NONE)
+                         : make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight,
+                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, BK / 8, BW,
+                                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!wmap) return WQ_ERR_CUDA;
   if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, BW, BT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WQ_ERR_CUDA;
   using C = GemmCfg<BT>;
-  auto kern = w4a16_gemm_kernel<BT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+  auto kern = w4a16_gemm_kernel<BT, kNF4>;
+  const int smem = C::smem(kNF4);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
   dim3 grid((unsigned)(N / BW), (unsigned)((M + BT - 1) / BT));
-  kern<<<grid, kThreads, C::kSmem, st>>>(tx, tw, ty, static_cast<const __half*>(scales),
-                                         static_cast<const __half*>(zeros), inv_scale, (int)M,
-                                         (int)N, (int)K, G);
+  kern<<<grid, kThreads, smem, st>>>(tx, tw, ty, scales, static_cast<const __half*>(zeros),
+                                     inv_scale, (int)M, (int)N, (int)K, G, nf4_table());
   return launch_status();
 }
 
@@ -305,19 +348,23 @@ size_t gemm_workspace_bytes(int64_t M, int64_t K) {
   return ((size_t)M * K * 2 + 255) / 256 * 256 + (size_t)M * 4;
 }
 
-wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_t G,
+wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_format fmt, int32_t G,
                       const void* qweight, const void* scales, const void* zeros, void* y,
                       void* workspace, cudaStream_t st) {
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* x16 = ws;
   float* inv_scale = reinterpret_cast<float*>(ws + ((size_t)M * K * 2 + 255) / 256 * 256);
-  wq_status s = launch_x_to_f16(x, M, K, x16, inv_scale, st);
+  const bool nf4 = fmt == WQ_FMT_NF4;
+  wq_status s = launch_x_to_f16(x, M, K, x16, inv_scale, /*permute=*/!nf4, st);
   if (s != WQ_OK) return s;
   // 256-token tiles when they alone fill the machine, else 128-token ones.
   const int64_t tiles256 = (N / BW) * ((M + 255) / 256);
-  return tiles256 >= (int64_t)num_sms()
-             ? launch_bt<256>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
-             : launch_bt<128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  const bool wide = tiles256 >= (int64_t)num_sms();
+  if (nf4)
+    return wide ? launch_bt<256, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+                : launch_bt<128, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  return wide ? launch_bt<256, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+              : launch_bt<128, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
 }
 
 wq_status read_gemm_error(bool clear, uint32_t* v) {

@@ -8,16 +8,18 @@
 // overflow, and the GEMM epilogue multiplies by 2^-e (exact) before rounding
 // to bf16.
 //
-// Within every 8-element chunk the copy stores x in the order
+// For INT4 weights the copy stores every 8-element chunk in the order
 // x0 x4 x1 x5 x2 x6 x3 x7: the order in which the GEMM's dequantization
 // produces the weights of one packed INT4 word (nibbles e and e + 4 share a
 // 32-bit register). A product over k is the same under any permutation of k
-// applied to both operands.
+// applied to both operands. For NF4 weights (codes already in k order) the
+// copy keeps the natural order.
 #include "common.cuh"
 
 namespace wq {
 namespace {
 
+template <bool kPermute>
 __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restrict__ x, int K,
                                                        uint16_t* __restrict__ x16,
                                                        float* __restrict__ inv_scale) {
@@ -53,12 +55,17 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
   for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
     const uint4 a = *reinterpret_cast<const uint4*>(row + c * 8);
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-    // stored in the order x0 x4 x1 x5 x2 x6 x3 x7 (see the header)
     uint32_t o[4];
-    o[0] = pack_f16x2(bf16_lo_to_f32(w[0]) * sc, bf16_lo_to_f32(w[2]) * sc);
-    o[1] = pack_f16x2(bf16_hi_to_f32(w[0]) * sc, bf16_hi_to_f32(w[2]) * sc);
-    o[2] = pack_f16x2(bf16_lo_to_f32(w[1]) * sc, bf16_lo_to_f32(w[3]) * sc);
-    o[3] = pack_f16x2(bf16_hi_to_f32(w[1]) * sc, bf16_hi_to_f32(w[3]) * sc);
+    if (kPermute) {  // x0 x4 x1 x5 x2 x6 x3 x7 (see the header)
+      o[0] = pack_f16x2(bf16_lo_to_f32(w[0]) * sc, bf16_lo_to_f32(w[2]) * sc);
+      o[1] = pack_f16x2(bf16_hi_to_f32(w[0]) * sc, bf16_hi_to_f32(w[2]) * sc);
+      o[2] = pack_f16x2(bf16_lo_to_f32(w[1]) * sc, bf16_lo_to_f32(w[3]) * sc);
+      o[3] = pack_f16x2(bf16_hi_to_f32(w[1]) * sc, bf16_hi_to_f32(w[3]) * sc);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = pack_f16x2(bf16_lo_to_f32(w[i]) * sc, bf16_hi_to_f32(w[i]) * sc);
+    }
     *reinterpret_cast<uint4*>(out + c * 8) = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
@@ -66,9 +73,10 @@ __global__ void __launch_bounds__(256) x_to_f16_kernel(const uint16_t* __restric
 }  // namespace
 
 wq_status launch_x_to_f16(const void* x, int64_t M, int64_t K, void* x16, float* inv_scale,
-                          cudaStream_t st) {
-  x_to_f16_kernel<<<(unsigned)M, 256, 0, st>>>(static_cast<const uint16_t*>(x), (int)K,
-                                               static_cast<uint16_t*>(x16), inv_scale);
+                          bool permute, cudaStream_t st) {
+  auto kern = permute ? x_to_f16_kernel<true> : x_to_f16_kernel<false>;
+  kern<<<(unsigned)M, 256, 0, st>>>(static_cast<const uint16_t*>(x), (int)K,
+                                    static_cast<uint16_t*>(x16), inv_scale);
   return launch_status();
 }
 

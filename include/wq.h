@@ -169,10 +169,13 @@ wq_status wq_w4a16_gemv(const void* x, int64_t M, int64_t N, int64_t K,
 
 /*
  * Prefill W4A16 GEMM with fused dequantization on the tensor cores ([MSD]:
- * the dequantize-then-multiply product; here the dequantized tile never
- * leaves shared memory). Same arguments and layouts as wq_w4a16_gemv, any
- * M >= 1. INT4 only (WQ_ERR_UNSUPPORTED for NF4). Requires K % 128 == 0,
- * N % 128 == 0, G % 64 == 0, K % G == 0, and group scales with 15 * s <= 65504.
+ * the dequantize-then-multiply product; here the dequantized tile is written
+ * straight into tensor memory and never leaves the SM). Same arguments and
+ * layouts as wq_w4a16_gemv, any
+ * M >= 1, INT4 or NF4 ([NF4]: codebook value x block absmax, both rounded to
+ * fp16 and multiplied in fp16). Requires K % 128 == 0, N % 128 == 0,
+ * G % 64 == 0, K % G == 0, and INT4 group scales with 15 * s <= 65504 (NF4
+ * absmax <= 65504).
  * The product runs in fp16 with fp32 accumulation: x is first copied to fp16
  * scaled per row by a power of two (exact for bf16 values down to 2^-28 of the
  * row's largest), each weight is fp16_rn((q - z) * s), and the epilogue

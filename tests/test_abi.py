@@ -101,7 +101,9 @@ def test_gemv_validation(wq):
 def test_gemm_and_msd_validation(wq):
     L = wq.lib
     assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 1, 64, A16, A16, None, A16, None, 0,
-                           None) == wq.WQ_ERR_UNSUPPORTED               # NF4 GEMM
+                           None) == wq.WQ_ERR_WORKSPACE                 # NF4 GEMM needs one
+    assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 1, 128, A16, A16, None, A16, None, 0,
+                           None) == wq.WQ_ERR_INVALID_ARG               # NF4 block is 64
     assert L.wq_w4a16_gemm(A16, 512, 4160, 4096, 0, 128, A16, A16, A16, A16, None, 0,
                            None) == wq.WQ_ERR_UNSUPPORTED               # N % 128
     assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 0, 128, A16, A16, A16, MIS, None, 0,

@@ -106,3 +106,41 @@ def test_dequant_then_cublas_comparator(wq):
     y_model = products.dequant_then_bf16_matmul_int4(xf, q, s, z, group)
     helpers.check_within_bf16_rounding(y, y_model, "dequant-then-cuBLAS vs its model", slack=1e-3)
     helpers.check_product(y, products.w4a16_int4(xf, q, s, z, group), "dequant-then-cuBLAS")
+
+
+def _run_nf4_gemm(wq, m, n, k, seed, rows=None, cols=None):
+    codes, absmax, packed = helpers.nf4_packed(n, k, seed)
+    cw, am = helpers.to_dev_nf4(absmax, packed)
+    x = _x(m, k, seed)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    xf = helpers.x_f32(x)
+    if rows is None:
+        rows = np.arange(m)
+    if cols is None:
+        cols = np.arange(n)
+    codes2 = codes.reshape(n, k)
+    y_ref = products.w4a16_nf4(xf[rows], codes2[cols], absmax.reshape(n, k // 64)[cols], k)
+    ys = y.cpu()[rows][:, cols]
+    what = "nf4 gemm %dx%dx%d" % (m, n, k)
+    helpers.check_product(ys, y_ref, what)
+    # codebook value, absmax and their product each round once to fp16
+    # (2^-11 relative): about 2^-10.2 per weight, which spreads over the sum
+    helpers.check_within_bf16_rounding(ys, y_ref, what, slack=3e-3)
+
+
+@pytest.mark.parametrize("m,n,k", [(128, 256, 256), (300, 384, 640), (1, 128, 128),
+                                   (600, 12800, 256)])
+def test_gemm_nf4_small_every_element(wq, m, n, k):
+    """NF4 weights on the fused GEMM: ragged M, several k-tiles, one token,
+    and enough tiles for both tile widths."""
+    _run_nf4_gemm(wq, m, n, k, seed=m)
+
+
+@pytest.mark.parametrize("m,n,k", [(2048, 14336, 4096), (8192, 4096, 14336)])
+def test_gemm_nf4_full_size_sampled(wq, m, n, k):
+    rng = np.random.default_rng(m + n + k + 64)
+    rows = np.sort(rng.choice(m, 48, replace=False))
+    cols = np.sort(rng.choice(n, 192, replace=False))
+    _run_nf4_gemm(wq, m, n, k, seed=1, rows=rows, cols=cols)

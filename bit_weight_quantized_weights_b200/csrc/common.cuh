@@ -76,6 +76,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// fp32 -> bf16 bits, round to nearest even.
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  uint16_t r;
+  asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(v));
+  return r;
+}
+
 // Two fp32 -> packed fp16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;

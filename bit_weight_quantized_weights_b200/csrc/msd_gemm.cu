@@ -23,13 +23,18 @@
 //   warp 1       TMEM owner; one lane issues C x 4 tcgen05.mma.kind::i8
 //                (128 x 128 x 32, s8 x s8 -> s32) per k-tile into the group's
 //                TMEM accumulators (C x 128 columns, double-buffered when they
-//                fit), commits stages and finished groups.
+//                fit), commits stages and finished groups. The unpacked
+//                weights are the MMA's A operand (M = 128 features) and a
+//                digit plane its B operand (N = 128 tokens), so a TMEM lane is
+//                one feature and a column one token.
 //   warps 2-5    unpack: nibbles -> bytes (two permutes per 8 codes), minus
 //                the group's zero point per byte, into the UMMA K-major
-//                128-byte-swizzled B tile.
+//                128-byte-swizzled weight tile.
 //   warps 6-13   drain each finished group from TMEM: combine the components
-//                in int32, convert, scale by the group's s[n, g], accumulate in
-//                fp32 registers; the last group writes bf16 y.
+//                in int32, convert, scale by the group's s[n, g] (one value
+//                per thread: its feature), accumulate in fp32 registers; the
+//                last group scales by the tokens' s_C[m] and writes bf16 y
+//                through a shared-memory transpose.
 #include "sm100.cuh"
 #include "splitk_common.cuh"
 
@@ -43,13 +48,14 @@ wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, 
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 128;
-constexpr int kStages = 3;
 constexpr int kThreads = 448;
 constexpr int kUnpackWarps = 4;
 constexpr int kEpiWarps = 8;
 constexpr int kPlaneBytes = BM * BK;      // 16 KB per digit plane tile
 constexpr int kBBytes = BN * BK;          // 16 KB
 constexpr int kWBytes = BN * BK / 2;      // 8 KB packed
+constexpr int kOutPitch = BN + 8;         // bf16 transpose tile row (16-byte rows, banks shifted)
+constexpr int kRedPitch = BM + 4;         // fp32 split-K partial row (16-byte aligned)
 
 inline int64_t m_padded(int64_t M) { return (M + 127) / 128 * 128; }
 
@@ -63,7 +69,13 @@ struct MsdCfg {
   static constexpr int kNB = (2 * C * BN <= 512) ? 2 : 1;  // TMEM accumulator buffers
   static constexpr int kTmemCols = (C * BN * kNB <= 256) ? 256 : 512;
   static constexpr int kStageBytes = C * kPlaneBytes + kBBytes + kWBytes;
-  static constexpr int kSmem = kStages * kStageBytes + 2 * 128 * 4 + 256 + 1024;
+  static constexpr int kStages = 3;
+  static constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
+  // the transpose tile and the split-K partials reuse the stage ring
+  static_assert(kStages >= 2 && 3 * kStages + 2 * kNB <= 31, "stages and barriers");
+  static_assert(kStages * kStageBytes >= BM * kOutPitch * 2, "transpose tile");
+  // S ranks of ceil(128 / S) rows, S <= 8
+  static_assert(kStages * kStageBytes >= (BN + 7) * kRedPitch * 4, "split-K partials");
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
@@ -100,14 +112,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad, int S) {
   using Cfg = MsdCfg<C>;
   constexpr int NB = Cfg::kNB;
+  constexpr int kStages = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* sA = smem;                                  // [stage][plane] 16 KB
   uint8_t* sB = sA + kStages * C * kPlaneBytes;        // [stage] 16 KB
   uint8_t* sW = sB + kStages * kBBytes;                // [stage] 8 KB
-  float* sclE = reinterpret_cast<float*>(sW + kStages * kWBytes);  // [2][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sclE + 256);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sW + kStages * kWBytes);
   uint64_t* full = bars;
   uint64_t* deq = bars + kStages;
   uint64_t* empty = bars + 2 * kStages;
@@ -178,7 +190,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = sm100::idesc_s8_s32(BM, BN);
+      // the C plane tiles of a stage are adjacent 128-row K-major tiles, so
+      // up to two planes form one N = 256 B operand: one MMA then reads the
+      // weight tile for both (a 128-wide MMA costs ~85 % of a 256-wide one)
+      constexpr int kPair = C >= 2 ? 2 : 1;
+      constexpr uint32_t idesc_pair = sm100::idesc_s8_s32(BN, kPair * BM);
+      constexpr uint32_t idesc_one = sm100::idesc_s8_s32(BN, BM);
       int i = 0;  // k-tiles consumed by this rank
       bool ok = true;
       for (int gi = 0; gi < NSG && ok; ++gi) {
@@ -205,15 +222,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           sm100::tc_fence_after();
           const uint32_t b_base = smem_u32(sB + s * kBBytes);
 #pragma unroll
-          for (int c = 0; c < C; ++c) {
-            const uint32_t a_base = smem_u32(sA + (s * C + c) * kPlaneBytes);
-            const uint32_t d = tmem + (uint32_t)((b * C + c) * BN);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // A = weights (features x k), B = digit planes (tokens x k);
+            // accumulator columns c * 128 + token hold plane c
+            const uint32_t acc_in = (t | kk) != 0 ? 1u : 0u;
+            const uint64_t adesc = sm100::sdesc_sw128_kmajor(b_base + kk * 32);
+            sm100::mma_i8(tmem + (uint32_t)(b * C * BN),
+                          adesc,
+                          sm100::sdesc_sw128_kmajor(smem_u32(sA + s * C * kPlaneBytes) + kk * 32),
+                          idesc_pair, acc_in);
 #pragma unroll
-            for (int kk = 0; kk < BK / 32; ++kk) {
-              sm100::mma_i8(d, sm100::sdesc_sw128_kmajor(a_base + kk * 32),
-                            sm100::sdesc_sw128_kmajor(b_base + kk * 32), idesc,
-                            (t | kk) != 0 ? 1u : 0u);
-            }
+            for (int c = kPair; c < C; ++c)
+              sm100::mma_i8(tmem + (uint32_t)((b * C + c) * BN), adesc,
+                            sm100::sdesc_sw128_kmajor(smem_u32(sA + (s * C + c) * kPlaneBytes) +
+                                                      kk * 32),
+                            idesc_one, acc_in);
           }
           sm100::mma_commit(&empty[s]);
         }
@@ -239,7 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint4* wsrc = reinterpret_cast<const uint4*>(sW + s * kWBytes + r * 64);
       uint8_t* bdst = sB + s * kBBytes + r * 128;
 #pragma unroll
-      for (int j4 = 0; j4 < 4; ++j4) {
+      for (int jj = 0; jj < 4; ++jj) {
+        // rows are 64 bytes apart: rotating the chunk order by r / 2 puts
+        // the 16-byte reads of a warp on distinct banks
+        const int j4 = (jj + (r >> 1)) & 3;
         const uint4 wv = wsrc[j4];  // words 4*j4 .. 4*j4+3 -> chunks 2*j4, 2*j4+1
         const uint2 b0 = unpack_word_minus_zero(wv.x, zrep);
         const uint2 b1 = unpack_word_minus_zero(wv.y, zrep);
@@ -255,32 +281,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- drain / epilogue ----------------
-    const int e = threadIdx.x - 64 - 32 * kUnpackWarps;  // 0..255
+    // thread = TMEM lane = feature n0 + row; its 64 columns are the tokens
+    // m0 + 64 * half + j
     const int q = warp & 3;                              // TMEM lane quarter
-    const int half = (warp - 2 - kUnpackWarps) >> 2;     // 64-column half
+    const int half = (warp - 2 - kUnpackWarps) >> 2;     // 64-token half
     const int row = 32 * q + lane;
     float acc[64];
 #pragma unroll
     for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
-    float pref = 0.0f;
-    if (e < BN) pref = __half2float(scales[(int64_t)(n0 + e) * NG + g_first]);
+    const __half* srow = scales + (int64_t)(n0 + row) * NG + g_first;
+    float scl = __half2float(srow[0]);
     bool ok = true;
     for (int gi = 0; gi < NSG; ++gi) {
       const int b = gi % NB;
-      if (e < BN) sclE[(gi & 1) * 128 + e] = pref;
-      named_bar_sync(1, 32 * kEpiWarps);
-      if (e < BN && gi + 1 < NSG)
-        pref = __half2float(scales[(int64_t)(n0 + e) * NG + g_first + gi + 1]);
-      // every epilogue warp runs all NSG iterations (the named barrier above
-      // counts on it); after a failed wait the rest only keep that barrier
+      const float scl_next = gi + 1 < NSG ? __half2float(srow[gi + 1]) : 0.0f;
       if (ok) {
         bool got = sm100::mbar_wait(&acc_full[b], (uint32_t)(gi / NB) & 1u, &g_msd_error,
                                     0x1401u, abort_flag);
         ok = __all_sync(0xffffffffu, got);
       }
-      if (!ok) continue;
+      if (!ok) break;
       sm100::tc_fence_after();
-      const float* scl = sclE + (gi & 1) * 128 + half * 64;
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int col = half * 64 + 16 * cc;
@@ -308,35 +329,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float t = kIntCombine ? (float)ti[j] : tf[j];
-          acc[16 * cc + j] = fmaf(scl[16 * cc + j], t, acc[16 * cc + j]);
+          acc[16 * cc + j] = fmaf(scl, t, acc[16 * cc + j]);
         }
       }
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
+      scl = scl_next;
     }
     if (!kSplit) {
-      const int m = m0 + row;
-      if (ok && m < M) {
-        const float sC = comp_scales[(int64_t)(C - 1) * M + m];
-        uint16_t* dst = y + (int64_t)m * N + n0 + half * 64;
+      // transpose through shared memory (the stage ring is idle once the
+      // last group is drained: every TMA load has been consumed), then write
+      // whole 256-byte rows of y
+      uint16_t* out_s = reinterpret_cast<uint16_t*>(smem);  // [128 tokens][kOutPitch]
+      if (ok) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint4 o;
-          o.x = pack_bf16x2(acc[8 * i + 0] * sC, acc[8 * i + 1] * sC);
-          o.y = pack_bf16x2(acc[8 * i + 2] * sC, acc[8 * i + 3] * sC);
-          o.z = pack_bf16x2(acc[8 * i + 4] * sC, acc[8 * i + 5] * sC);
-          o.w = pack_bf16x2(acc[8 * i + 6] * sC, acc[8 * i + 7] * sC);
-          *reinterpret_cast<uint4*>(dst + 8 * i) = o;
+        for (int j = 0; j < 64; ++j) {
+          const int m = m0 + half * 64 + j;
+          const float sC = m < M ? comp_scales[(int64_t)(C - 1) * M + m] : 0.0f;
+          out_s[(half * 64 + j) * kOutPitch + row] = bf16_bits(acc[j] * sC);
+        }
+      }
+      named_bar_sync(1, 32 * kEpiWarps);
+      if (ok) {
+        const int e = threadIdx.x - 64 - 32 * kUnpackWarps;  // 0..255
+        for (int it = e; it < BM * (BN / 8); it += 32 * kEpiWarps) {
+          const int t = it / (BN / 8), ch = it % (BN / 8);
+          const int m = m0 + t;
+          if (m < M)
+            *reinterpret_cast<uint4*>(y + (int64_t)m * N + n0 + 8 * ch) =
+                *reinterpret_cast<const uint4*>(out_s + t * kOutPitch + 8 * ch);
         }
       }
     } else {
-      // push this rank's partials to the rank that owns the token rows
+      // push this rank's partials to the rank that owns the feature row
       splitk::cluster_sync_all();  // every rank is past its main loop
-      const int rows_max = (BM + S - 1) / S;
+      const int rows_max = (BN + S - 1) / S;
       const int owner = splitk::row_owner(row, S);
       const int lr = row - splitk::rank_row_begin(owner, S);
-      float* dst = reinterpret_cast<float*>(smem) + ((size_t)rank * rows_max + lr) * BN + half * 64;
+      float* dst = reinterpret_cast<float*>(smem) + ((size_t)rank * rows_max + lr) * kRedPitch +
+                   half * 64;
       const uint32_t rdst = splitk::map_rank(dst, (uint32_t)owner);
 #pragma unroll
       for (int i = 0; i < 16; ++i)
@@ -360,24 +392,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       splitk::cluster_sync_all();
       splitk::cluster_sync_all();
     }
+    // red[src rank][local feature row][token]; the owner of feature rows
+    // [r_begin, r_begin + nrows) sums them in rank order and writes y, each
+    // thread one (token, feature) with consecutive threads on consecutive
+    // features
     const float* red = reinterpret_cast<const float*>(smem);
-    const int rows_max = (BM + S - 1) / S;
+    const int rows_max = (BN + S - 1) / S;
     const int r_begin = splitk::rank_row_begin(rank, S);
     const int nrows = splitk::rank_row_begin(rank + 1, S) - r_begin;
-    for (int it = threadIdx.x; it < nrows * (BN / 2); it += blockDim.x) {
-      const int lr = it / (BN / 2), cp = it - lr * (BN / 2);
-      const int m = m0 + r_begin + lr;
+    for (int it = threadIdx.x; it < nrows * BM; it += blockDim.x) {
+      const int t = it / nrows, lr = it - t * nrows;
+      const int m = m0 + t;
       if (m >= M) continue;
-      float v0 = 0.0f, v1 = 0.0f;
-      for (int qq = 0; qq < S; ++qq) {
-        const float2 pv =
-            *reinterpret_cast<const float2*>(red + ((size_t)qq * rows_max + lr) * BN + 2 * cp);
-        v0 += pv.x;
-        v1 += pv.y;
-      }
+      float v = 0.0f;
+      for (int qq = 0; qq < S; ++qq) v += red[((size_t)qq * rows_max + lr) * kRedPitch + t];
       const float sC = comp_scales[(int64_t)(C - 1) * M + m];
-      *reinterpret_cast<uint32_t*>(y + (int64_t)m * N + n0 + 2 * cp) =
-          pack_bf16x2(v0 * sC, v1 * sC);
+      y[(int64_t)m * N + n0 + r_begin + lr] = bf16_bits(v * sC);
     }
   }
 

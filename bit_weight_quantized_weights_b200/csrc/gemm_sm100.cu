@@ -22,11 +22,12 @@
 //               (128 x BT x 16, A from TMEM, B = x from shared memory, fp32
 //               accumulator in TMEM).
 //   warps 2-9   dequantize one k-tile per TMEM A stage (SA stages of 32
-//               columns): warp w owns TMEM lanes 32 (w % 4) .. +31, i.e. one
-//               weight row per thread, and half of the tile's 64 k. After the
-//               main loop they are the epilogue: TMEM -> x 2^-e per token ->
-//               bf16 -> shared staging tile [BT tokens][128 rows] -> one TMA
-//               store into y.
+//   (2-17 NF4)  columns); NF4 has two groups of 8 taking alternate k-tiles. Warp w
+//               owns TMEM lanes 32 (w % 4) .. +31, i.e. one weight row per
+//               thread, and half of its k-tile's 64 k. After the main loop
+//               they are the epilogue: TMEM -> x 2^-e per token -> bf16 ->
+//               shared staging tile [BT tokens][128 rows] -> one TMA store
+//               into y.
 // NF4 weights (block 64 = one k-tile) take the same path: a 256-entry
 // per-lane table turns each code byte into the fp16 pair of its two codebook
 // values, and one fp16 multiply applies the block's absmax.
@@ -50,13 +51,26 @@ __device__ unsigned int g_gemm_error;
 
 constexpr int BW = 128;          // weight rows per CTA (MMA M)
 constexpr int BK = 64;           // k per stage
-constexpr int kDeqWarps = 8;     // two per TMEM lane quarter
-constexpr int kThreads = 64 + 32 * kDeqWarps;
+constexpr int kDeqWarps = 8;     // per k-tile: two per TMEM lane quarter
+// Dequantization warp groups, each taking every kGroups-th k-tile: a warp
+// handles one k-tile at a time through a chain of dependent steps (wait, load,
+// convert, TMEM store, wait for it, arrive). NF4's table lookups make that
+// chain long enough that two groups overlapping two k-tiles pay (+6 to +19 %
+// measured); for INT4 a second group measured 3-5 % slower.
+template <bool kNF4>
+struct Deq {
+  static constexpr int kGroups = kNF4 ? 2 : 1;
+  static constexpr int kThreads = 64 + 32 * kDeqWarps * kGroups;
+};
 constexpr int SA = 4;            // TMEM A stages (32 columns each)
 
-template <int BT>
+template <int BT, bool kNF4>
 struct GemmCfg {
-  static constexpr int kStages = (BT == 256) ? 5 : 8;
+  // A multiple of the dequantization groups, so that every ring stage and A
+  // stage is always waited on by the same group, one phase at a time (a
+  // parity wait must never run two phases ahead of its barrier). NF4 needs
+  // room for its lookup table.
+  static constexpr int kStages = (BT == 256) ? (kNF4 ? 4 : 5) : 8;
   static constexpr int kXBytes = BT * BK * 2;     // 32 / 16 KB
   static constexpr int kWBytes = BW * BK / 2;     // 4 KB
   static constexpr int kStageBytes = kXBytes + kWBytes;
@@ -70,6 +84,8 @@ struct GemmCfg {
   static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
   static constexpr uint32_t kTmemCols = (BT + SA * 32 <= 256) ? 256 : 512;
+  static_assert(kStages % Deq<kNF4>::kGroups == 0 && SA % Deq<kNF4>::kGroups == 0,
+                "stages per group");
 };
 
 __device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
@@ -99,14 +115,16 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb_hi, uint32_
 }
 
 template <int BT, bool kNF4>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_y, const void* __restrict__ scales,
                       const __half* __restrict__ zeros, const float* __restrict__ inv_scale, int M,
                       int N, int K, int G, Nf4Table tab) {
-  using C = GemmCfg<BT>;
+  using C = GemmCfg<BT, kNF4>;
   constexpr int ST = C::kStages;
+  constexpr int kDeqGroups = Deq<kNF4>::kGroups;
+  constexpr int kThreads = Deq<kNF4>::kThreads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -204,34 +222,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- dequantize (warps 2..9), then epilogue ----------------
-    const int dq = warp - 2;            // 0..7
+    const int dq = warp - 2;            // 0 .. 8 * kDeqGroups - 1
+    const int grp = dq / kDeqWarps;     // this warp's k-tiles: kt = grp (mod kDeqGroups)
     const int q = warp & 3;             // TMEM lane quarter this warp may access
-    const int hk = dq >> 2;             // which half of the k-tile (32 k, 4 words)
+    const int hk = (dq % kDeqWarps) >> 2;  // which half of the k-tile (32 k, 4 words)
     const int r = 32 * q + lane;        // weight row within the tile = TMEM lane
     const int n = n0 + r;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int ng = K / G;
     const int tiles_per_group = G / BK;
-    // group parameters are loaded one group ahead of their use
     const __half* srow = static_cast<const __half*>(scales) + (int64_t)n * ng;
     const __half* zrow = kNF4 ? nullptr : zeros + (int64_t)n * ng;
+    // INT4 runs one dequantization group: the group parameters are loaded
+    // one group ahead of their use and converted once per group
+    static_assert(kNF4 || kDeqGroups == 1, "INT4 parameter stepping assumes one group");
     __half s_next = kNF4 ? __ushort_as_half(0) : srow[0];
     __half z_next = kNF4 ? __ushort_as_half(0) : zrow[0];
     uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
+    int gi = 0, left = 0;  // current group, k-tiles left in it
+    const bool any = grp < KT;
     // NF4: the absmax of (row n, 64-element block kt) is one per k-tile
     const float* arow = static_cast<const float*>(scales) + (int64_t)n * (K / 64);
-    float am_next = kNF4 ? arow[0] : 0.0f;
+    float am_next = (kNF4 && any) ? arow[grp] : 0.0f;
     const uint32_t* lut_lane = lut + lane;
-    int gi = 0, left = 0;  // current group, k-tiles left in it
     bool ok = true;
-    for (int kt = 0; kt < KT && ok; ++kt) {
+    for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
       const int s = kt % ST, a = kt % SA;
       const uint32_t ph = (uint32_t)(kt / ST) & 1u, pa = (uint32_t)(kt / SA) & 1u;
+      const bool more = kt + kDeqGroups < KT;
       uint32_t am2 = 0;
       if (kNF4) {
-        // fp16x2 (absmax, absmax), rounded once; the next one is loaded now
+        // fp16x2 (absmax, absmax), rounded once; this warp's next one is
+        // loaded now
         am2 = pack_f16x2(am_next, am_next);
-        if (kt + 1 < KT) am_next = arow[kt + 1];
+        if (more) am_next = arow[kt + kDeqGroups];
       } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
         const uint32_t zq = (uint32_t)__half2float(z_next);
@@ -245,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++gi;
         left = tiles_per_group;
       }
-      --left;
+      if (!kNF4) --left;
       bool got = sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x301u, abort_flag);
       if (got && kt >= SA)
         got = sm100::mbar_wait(&afree[a], pa ^ 1u, &g_gemm_error, 0x302u, abort_flag);
@@ -280,9 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (all_ok) {
       sm100::tc_fence_after();
-      // this warp: TMEM lanes of quarter q, token columns [hk * BT/2, (hk+1) * BT/2)
+      // this warp: TMEM lanes of quarter q, token columns
+      // [(dq / 4) * kEpiCols, (dq / 4 + 1) * kEpiCols)
+      constexpr int kEpiCols = BT / (2 * kDeqGroups);
 #pragma unroll 1
-      for (int c0 = hk * (BT / 2); c0 < (hk + 1) * (BT / 2); c0 += 32) {
+      for (int c0 = (dq / 4) * kEpiCols; c0 < (dq / 4 + 1) * kEpiCols; c0 += 32) {
         uint32_t v[32];
         sm100::tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
         sm100::tmem_ld_wait();
@@ -294,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sm100::fence_proxy_async_smem();
     }
-    sm100::named_barrier(1, 32 * kDeqWarps);
+    sm100::named_barrier(1, 32 * kDeqWarps * kDeqGroups);
     if (threadIdx.x == 64 && *abort_flag == 0) {
       sm100::tma_store_2d(&tmap_y, out_s, n0, m0);
       sm100::bulk_commit();
@@ -308,6 +334,329 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair version (cta_group::2). A 2-CTA cluster computes 256 weight rows
+// by 256 tokens with one 256 x 256 x 16 MMA per k step, issued by the even
+// CTA. Each CTA dequantizes its own 128 weight rows into its own TMEM (the
+// A rows it contributes) and loads only its 128-token half of the x tile (the
+// B columns it contributes); its TMEM accumulator holds its 128 rows by all
+// 256 tokens. Per SM the x bytes per k-tile halve (16 KB instead of 32 KB).
+// Measured on B200 (per-role clock stamps and A/B builds):
+//   * the ring's round trip (MMA done -> slot free -> next load -> landed ->
+//     dequantized -> MMA issued) over the slots in flight sets the pace, with
+//     the loads themselves far from any bandwidth limit;
+//   * the stage ring and the TMEM A stages have the same depth (8), so one
+//     MMA commit per k-tile frees both (each commit costs the issuing thread
+//     time; two per k-tile were 7 % slower);
+//   * the odd CTA's dequantization warps arrive on the even CTA's barrier
+//     with the default CTA-scope release (a cluster-scope release costs about
+//     a microsecond per arrive and halved the kernel's speed);
+//   * a separate, deeper ring for the packed weights, loaded 8 k-tiles ahead,
+//     measured no faster.
+// Synchronisation (stage s = kt % 8 holds this CTA's x half and its packed
+// weight tile):
+//   xfull[s]   (even CTA's) both CTAs' x halves landed (their TMA loads count
+//              bytes on it; the even CTA's producer sets the expected total)
+//   wfull[s]   (each CTA's) its packed weight tile landed
+//   done[s]    the MMAs of k-tile kt completed: stage s and A stage s are
+//              free (the even CTA's commit arrives on both CTAs)
+//   aready[s]  (even CTA's) all 16 dequantization warps of the pair wrote A
+//              stage s (the odd CTA's arrive remotely)
+//   accf       all MMAs done (the even CTA's commit arrives on both CTAs)
+// All waits are bounded; every thread of both CTAs reaches the final cluster
+// barriers on every path.
+struct Gemm2Cfg {
+  static constexpr int BT = 256;                  // tokens per pair tile (MMA N)
+  static constexpr int kStages = 8;               // stages = TMEM A stages
+  static constexpr int kXBytes = 128 * BK * 2;    // this CTA's x half: 16 KB
+  static constexpr int kWBytes = BW * BK / 2;     // 4 KB
+  static constexpr int kStageBytes = kXBytes + kWBytes;
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kOutBytes = BT * BW * 2;   // epilogue staging (reuses the ring)
+  static constexpr int kLutBytes = 256 * 32 * 4;
+  static constexpr int kSmem = kRing + BT * 4 + 512 + 1024;
+  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
+  static constexpr uint32_t kAccCols = BT;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kAccCols + kStages * 32 <= kTmemCols, "A stages fit in TMEM");
+  static_assert(kOutBytes <= kRing, "the staging tile fits in the ring");
+  static_assert(kStages % 2 == 0, "every stage is waited on by one group (up to two)");
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
+  // xfull, wfull, done, aready, accf, then the TMEM slot and the abort flag
+  static_assert(8 * (4 * kStages + 1) + 8 <= 512, "barriers fit their 512 bytes");
+};
+
+template <bool kNF4>
+__global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
+    w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                           const __grid_constant__ CUtensorMap tmap_w,
+                           const __grid_constant__ CUtensorMap tmap_y,
+                           const void* __restrict__ scales, const __half* __restrict__ zeros,
+                           const float* __restrict__ inv_scale, int M, int N, int K, int G,
+                           Nf4Table tab) {
+  using C = Gemm2Cfg;
+  constexpr int BT = C::BT;
+  constexpr int ST = C::kStages;
+  constexpr int kDeqGroups = Deq<kNF4>::kGroups;
+  constexpr int kThreads = Deq<kNF4>::kThreads;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;                                    // ST x (x half, packed W tile)
+  uint16_t* out_s = reinterpret_cast<uint16_t*>(smem);     // epilogue: [BT][BW] bf16
+  float* s_inv = reinterpret_cast<float*>(smem + C::kRing);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_inv + BT);
+  uint64_t* xfull = bars;
+  uint64_t* wfull = bars + ST;
+  uint64_t* done = bars + 2 * ST;
+  uint64_t* aready = bars + 3 * ST;
+  uint64_t* accf = aready + ST;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 512);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = sm100::cluster_ctarank();  // 0: issues the MMAs
+  const bool leader = rank == 0;
+  const int n0 = (int)(blockIdx.x >> 1) * (2 * BW) + BW * (int)rank;
+  const int m0 = blockIdx.y * BT;                  // the pair's first token
+  const int KT = K / BK;
+
+  if (threadIdx.x == 0) {
+    sm100::tma_prefetch_desc(&tmap_x);
+    sm100::tma_prefetch_desc(&tmap_w);
+    sm100::tma_prefetch_desc(&tmap_y);
+    for (int s = 0; s < ST; ++s) {
+      sm100::mbar_init(&xfull[s], 1);
+      sm100::mbar_init(&wfull[s], 1);
+      sm100::mbar_init(&done[s], 1);
+      sm100::mbar_init(&aready[s], 2 * kDeqWarps);
+    }
+    sm100::mbar_init(accf, 1);
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  for (int j = (int)threadIdx.x - 64; j >= 0 && j < BT; j += kThreads - 64)
+    s_inv[j] = (m0 + j < M) ? inv_scale[m0 + j] : 0.0f;
+  if (kNF4) {
+    for (int i = threadIdx.x; i < 256 * 8; i += kThreads) {
+      const int e = i >> 3;
+      const uint32_t v = pack_f16x2(tab.v[e >> 4], tab.v[e & 15]);
+      reinterpret_cast<uint4*>(lut)[i] = make_uint4(v, v, v, v);
+    }
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    sm100::tmem_relinquish_pair();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  // both CTAs' barriers are initialised before any load or remote arrive
+  // can target them
+  sm100::cluster_sync();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % ST;
+        const uint32_t ph = (uint32_t)(kt / ST) & 1u;
+        if (kt >= ST && !sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x111u, abort_flag))
+          break;
+        uint8_t* st = ring + s * C::kStageBytes;
+        sm100::mbar_arrive_expect_tx(&wfull[s], C::kWBytes);
+        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &wfull[s], kt * (kNF4 ? BK / 2 : BK / 8),
+                           n0);
+        if (leader) sm100::mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
+        sm100::tma_load_2d_pair(st, &tmap_x, sm100::cluster_addr(&xfull[s], 0), kt * BK,
+                                m0 + 128 * (int)rank);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- pair MMA issuer (even CTA) ----------------
+      constexpr uint32_t idesc = sm100::idesc_f16_f32(2 * BW, BT);
+      for (int kt = 0; kt < KT; ++kt) {
+        const int s = kt % ST;
+        const uint32_t ph = (uint32_t)(kt / ST) & 1u;
+        if (!sm100::mbar_wait(&xfull[s], ph, &g_gemm_error, 0x211u, abort_flag)) break;
+        if (!sm100::mbar_wait(&aready[s], ph, &g_gemm_error, 0x212u, abort_flag)) break;
+        sm100::tc_fence_after();
+        const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t bd = sm100::sdesc_sw128_kmajor(x_base + kk * 32);
+          const uint32_t at = tmem + C::kAccCols + (uint32_t)(s * 32 + kk * 8);
+          sm100::mma_f16_tmem_a_pair(tmem, at, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
+        }
+        sm100::mma_commit_pair(&done[s], 0x3);
+      }
+      sm100::mma_commit_pair(accf, 0x3);
+    }
+  } else {
+    // ---------------- dequantize (warps 2..9), then epilogue ----------------
+    const int dq = warp - 2;
+    const int grp = dq / kDeqWarps;
+    const int q = warp & 3;
+    const int hk = (dq % kDeqWarps) >> 2;
+    const int r = 32 * q + lane;
+    const int n = n0 + r;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int ng = K / G;
+    const int tiles_per_group = G / BK;
+    const __half* srow = static_cast<const __half*>(scales) + (int64_t)n * ng;
+    const __half* zrow = kNF4 ? nullptr : zeros + (int64_t)n * ng;
+    // INT4 runs one dequantization group: the group parameters are loaded
+    // one group ahead of their use and converted once per group
+    static_assert(kNF4 || kDeqGroups == 1, "INT4 parameter stepping assumes one group");
+    __half s_next = kNF4 ? __ushort_as_half(0) : srow[0];
+    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[0];
+    uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
+    int gi = 0, left = 0;  // current group, k-tiles left in it
+    const bool any = grp < KT;
+    const float* arow = static_cast<const float*>(scales) + (int64_t)n * (K / 64);
+    float am_next = (kNF4 && any) ? arow[grp] : 0.0f;
+    const uint32_t* lut_lane = lut + lane;
+    bool ok = true;
+    for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
+      const int s = kt % ST;
+      const uint32_t ph = (uint32_t)(kt / ST) & 1u;
+      const bool more = kt + kDeqGroups < KT;
+      uint32_t am2 = 0;
+      if (kNF4) {
+        am2 = pack_f16x2(am_next, am_next);
+        if (more) am_next = arow[kt + kDeqGroups];
+      } else if (left == 0) {
+        const uint32_t sb = __half_as_ushort(s_next);
+        const uint32_t zq = (uint32_t)__half2float(z_next);
+        s2 = sb | (sb << 16);
+        zb_hi = (0x6400u | zq) * 0x00010001u;
+        zb_lo = (0x5400u | (zq << 4)) * 0x00010001u;
+        if (gi + 1 < ng) {
+          s_next = srow[gi + 1];
+          z_next = zrow[gi + 1];
+        }
+        ++gi;
+        left = tiles_per_group;
+      }
+      if (!kNF4) --left;
+      // the weight tile landed; A stage s is free once the MMAs of k-tile
+      // kt - ST completed (they also freed the stage this tile landed in)
+      bool got = sm100::mbar_wait(&wfull[s], ph, &g_gemm_error, 0x311u, abort_flag);
+      if (got && kt >= ST)
+        got = sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x312u, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      const uint4 wv = *reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
+                                                       r * 32 + hk * 16);
+      uint32_t cols[16];
+      if (kNF4) {
+        const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
+      } else {
+        dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
+        dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
+        dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
+        dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+      }
+      sm100::tmem_st16(tmem + lane_base + C::kAccCols + (uint32_t)(s * 32 + hk * 16), cols);
+      sm100::tmem_st_wait();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          sm100::mbar_arrive(&aready[s]);
+        else
+          sm100::mbar_arrive_cluster(sm100::cluster_addr(&aready[s], 0));
+      }
+    }
+    // ---------------- epilogue: this CTA's 128 rows x 256 tokens ----------------
+    if (ok) ok = sm100::mbar_wait(accf, 0, &g_gemm_error, 0x411u, abort_flag);
+    const bool all_ok = __all_sync(0xffffffffu, ok);
+    if (all_ok) {
+      sm100::tc_fence_after();
+      constexpr int kEpiCols = BT / (2 * kDeqGroups);
+#pragma unroll 1
+      for (int c0 = (dq / 4) * kEpiCols; c0 < (dq / 4 + 1) * kEpiCols; c0 += 32) {
+        uint32_t v[32];
+        sm100::tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
+        sm100::tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float val = __uint_as_float(v[j]) * s_inv[c0 + j];
+          out_s[(c0 + j) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
+        }
+      }
+      sm100::fence_proxy_async_smem();
+    }
+    sm100::named_barrier(1, 32 * kDeqWarps * kDeqGroups);
+    if (threadIdx.x == 64 && *abort_flag == 0) {
+      sm100::tma_store_2d(&tmap_y, out_s, n0, m0);
+      sm100::bulk_commit();
+      sm100::bulk_wait_read_all();
+    }
+  }
+
+  // neither CTA frees its TMEM or exits while the pair may still use it
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc_pair(tmem, C::kTmemCols);
+  }
+  sm100::cluster_sync();
+}
+
+template <bool kNF4>
+wq_status launch_pair(const void* x16, const float* inv_scale, int64_t M, int64_t N, int64_t K,
+                      int32_t G, const void* qweight, const void* scales, const void* zeros,
+                      void* y, cudaStream_t st) {
+  using C = Gemm2Cfg;
+  CUtensorMap tx, tw, ty;
+  // x: this CTA's 128-token half of the pair's tile
+  if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M,
+                    (uint64_t)K * 2, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return WQ_ERR_CUDA;
+  const bool wmap = kNF4 ? make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qweight,
+                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, BK / 2, BW,
+                                        CU_TENSOR_MAP_SWIZZLE_NONE)
+                         : make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight,
+                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, BK / 8, BW,
+                                        CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!wmap) return WQ_ERR_CUDA;
+  if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                    (uint64_t)N * 2, BW, C::BT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return WQ_ERR_CUDA;
+  auto kern = w4a16_gemm_pair_kernel<kNF4>;
+  const int smem = C::smem(kNF4);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return WQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(N / BW), (unsigned)((M + C::BT - 1) / C::BT), 1);
+  cfg.blockDim = dim3(Deq<kNF4>::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, scales, static_cast<const __half*>(zeros),
+                         inv_scale, (int)M, (int)N, (int)K, G, nf4_table()) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  return launch_status();
 }
 
 template <int BT, bool kNF4>
@@ -329,19 +678,30 @@ wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t 
   if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, BW, BT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WQ_ERR_CUDA;
-  using C = GemmCfg<BT>;
+  using C = GemmCfg<BT, kNF4>;
   auto kern = w4a16_gemm_kernel<BT, kNF4>;
   const int smem = C::smem(kNF4);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
   dim3 grid((unsigned)(N / BW), (unsigned)((M + BT - 1) / BT));
-  kern<<<grid, kThreads, smem, st>>>(tx, tw, ty, scales, static_cast<const __half*>(zeros),
+  kern<<<grid, Deq<kNF4>::kThreads, smem, st>>>(tx, tw, ty, scales, static_cast<const __half*>(zeros),
                                      inv_scale, (int)M, (int)N, (int)K, G, nf4_table());
   return launch_status();
 }
 
 }  // namespace
+
+// The CTA-pair kernel is the default for wide tiles; WQ_GEMM_PAIRS=0 in the
+// environment selects the single-CTA kernel (kept as the reference design
+// and for comparison).
+bool gemm_pairs_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("WQ_GEMM_PAIRS");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 // Workspace: the fp16 copy of x [M, K] (256-byte aligned), then 2^-e per row.
 size_t gemm_workspace_bytes(int64_t M, int64_t K) {
@@ -360,9 +720,15 @@ wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   // 256-token tiles when they alone fill the machine, else 128-token ones.
   const int64_t tiles256 = (N / BW) * ((M + 255) / 256);
   const bool wide = tiles256 >= (int64_t)num_sms();
-  if (nf4)
+  // CTA pairs (256 weight rows x 256 tokens per pair) where the rows pair up
+  const bool pair = wide && N % (2 * BW) == 0 && gemm_pairs_enabled();
+  if (nf4) {
+    if (pair)
+      return launch_pair<true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
     return wide ? launch_bt<256, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
                 : launch_bt<128, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  }
+  if (pair) return launch_pair<false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   return wide ? launch_bt<256, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
               : launch_bt<128, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
 }

@@ -92,6 +92,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+// Packed fp32 pair arithmetic (sm_100 f32x2: each lane rounds as the scalar
+// operation would).
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 // 8 INT4 codes of one packed word -> 8 signed bytes q - z, in k order.
 __device__ __forceinline__ uint2 unpack_word_minus_zero(uint32_t w, uint32_t zrep) {
   const uint32_t v = w & 0x0F0F0F0Fu;
@@ -286,9 +304,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                              // TMEM lane quarter
     const int half = (warp - 2 - kUnpackWarps) >> 2;     // 64-token half
     const int row = 32 * q + lane;
-    float acc[64];
+    // acc2[i] holds the tokens 2i, 2i + 1 of this thread's 64 (packed pairs)
+    uint64_t acc2[32];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+    for (int j = 0; j < 32; ++j) acc2[j] = 0ull;
     const __half* srow = scales + (int64_t)(n0 + row) * NG + g_first;
     float scl = __half2float(srow[0]);
     bool ok = true;
@@ -302,40 +321,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       sm100::tc_fence_after();
+      const uint64_t scl2 = f2_pack(scl, scl);
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         const int col = half * 64 + 16 * cc;
         const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * C * BN + col);
-        uint32_t p[16];
-        tmem_ld16(base, p);
+        uint32_t p[C][16];
+#pragma unroll
+        for (int c = 0; c < C; ++c) tmem_ld16(base + (uint32_t)(c * BN), p[c]);
         sm100::tmem_ld_wait();
-        int32_t ti[16];
-        float tf[16];
+        float t[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          ti[j] = (int32_t)p[j];
-          tf[j] = (float)(int32_t)p[j];
-        }
+          if (kIntCombine) {
+            int32_t v = (int32_t)p[0][j];
 #pragma unroll
-        for (int c = 1; c < C; ++c) {
-          tmem_ld16(base + (uint32_t)(c * BN), p);
-          sm100::tmem_ld_wait();
+            for (int c = 1; c < C; ++c) v = v * 256 + (int32_t)p[c][j];
+            t[j] = (float)v;
+          } else {
+            t[j] = (float)(int32_t)p[0][j];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (kIntCombine) ti[j] = ti[j] * 256 + (int32_t)p[j];
-            else tf[j] = fmaf(tf[j], 256.0f, (float)(int32_t)p[j]);
+            for (int c = 1; c < C; ++c) t[j] = fmaf(t[j], 256.0f, (float)(int32_t)p[c][j]);
           }
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float t = kIntCombine ? (float)ti[j] : tf[j];
-          acc[16 * cc + j] = fmaf(scl, t, acc[16 * cc + j]);
-        }
+        for (int j = 0; j < 8; ++j)
+          acc2[8 * cc + j] = f2_fma(scl2, f2_pack(t[2 * j], t[2 * j + 1]), acc2[8 * cc + j]);
       }
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
       scl = scl_next;
+    }
+    float acc[64];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float2 v = f2_unpack(acc2[j]);
+      acc[2 * j] = v.x;
+      acc[2 * j + 1] = v.y;
     }
     if (!kSplit) {
       // transpose through shared memory (the stage ring is idle once the
@@ -419,36 +442,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// K split (cluster size) for problems with fewer output tiles than SMs: each
-// rank of an S-CTA cluster takes a contiguous run of k-tiles (at least one)
-// and the partials meet through distributed shared memory. S is the largest
-// value up to 8 whose clusters all fit on the GPU at once.
+// K split (cluster size). Each rank of an S-CTA cluster takes a contiguous
+// run of k-tiles (at least one) and the partials meet through distributed
+// shared memory. S minimises (waves of clusters) x (k-tiles per rank + a
+// reduction cost of two k-tiles when split): it fills the GPU when there are
+// fewer output tiles than SMs and evens out a last wave that would run
+// mostly empty (320 tiles = 2.2 waves of 148 take 3 full-K waves unsplit).
+// Clusters per wave come from the occupancy API; the choice is cached per
+// shape.
 template <class Kern>
 int msd_split(Kern kern, int smem, int64_t tiles, int64_t ktiles) {
-  if (tiles >= num_sms()) return 1;
-  int S = (int)(num_sms() / tiles);
-  S = S > 8 ? 8 : S;
-  S = S > ktiles ? (int)ktiles : S;
-  for (; S > 1; --S) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
-      cudaGetLastError();
-      continue;
-    }
-    if (clusters >= tiles) break;
-  }
-  return S < 1 ? 1 : S;
+  const splitk::Plan pl = splitk::cached_plan(
+      reinterpret_cast<const void*>(kern), (int)tiles, 0, ktiles, smem, [&] {
+        int best_s = 1;
+        double best = -1.0;
+        for (int S = 1; S <= 8 && S <= ktiles; ++S) {
+          int per_wave = 0;
+          if (S == 1) {
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem) !=
+                cudaSuccess) {
+              cudaGetLastError();
+              continue;
+            }
+            per_wave = per_sm * num_sms();
+          } else {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)S;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&per_wave, kern, &cfg) != cudaSuccess) {
+              cudaGetLastError();
+              continue;
+            }
+          }
+          if (per_wave < 1) continue;
+          const int64_t waves = (tiles + per_wave - 1) / per_wave;
+          const double cost = (double)waves * (double)((ktiles + S - 1) / S + (S > 1 ? 2 : 0));
+          if (best < 0.0 || cost < best) {
+            best = cost;
+            best_s = S;
+          }
+        }
+        return splitk::Plan{best_s, 0, (size_t)smem};
+      });
+  return pl.S < 1 ? 1 : pl.S;
 }
 
 template <int C, bool kInt>

@@ -444,12 +444,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // K split (cluster size). Each rank of an S-CTA cluster takes a contiguous
 // run of k-tiles (at least one) and the partials meet through distributed
-// shared memory. S minimises (waves of clusters) x (k-tiles per rank + a
-// reduction cost of two k-tiles when split): it fills the GPU when there are
-// fewer output tiles than SMs and evens out a last wave that would run
-// mostly empty (320 tiles = 2.2 waves of 148 take 3 full-K waves unsplit).
-// Clusters per wave come from the occupancy API; the choice is cached per
-// shape.
+// shared memory. S minimises (waves of clusters) x (k-tiles per rank + the
+// fixed cost of a CTA + the cost of the reduction when split), both costs in
+// k-tile times as measured on B200 (about 6 each): it fills the GPU when
+// there are fewer output tiles than SMs and evens out a last wave that would
+// run mostly empty when K is long (1024 x 5120 x 25600: 3 unsplit waves of
+// 200 k-tiles take 652 us, 4-way split 595 us). Clusters per wave come from
+// the occupancy API; the choice is cached per shape.
 template <class Kern>
 int msd_split(Kern kern, int smem, int64_t tiles, int64_t ktiles) {
   const splitk::Plan pl = splitk::cached_plan(
@@ -485,7 +486,9 @@ int msd_split(Kern kern, int smem, int64_t tiles, int64_t ktiles) {
           }
           if (per_wave < 1) continue;
           const int64_t waves = (tiles + per_wave - 1) / per_wave;
-          const double cost = (double)waves * (double)((ktiles + S - 1) / S + (S > 1 ? 2 : 0));
+          constexpr int kCtaCost = 6, kReduceCost = 6;  // in k-tile times
+          const double cost =
+              (double)waves * (double)((ktiles + S - 1) / S + kCtaCost + (S > 1 ? kReduceCost : 0));
           if (best < 0.0 || cost < best) {
             best = cost;
             best_s = S;

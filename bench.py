@@ -303,20 +303,39 @@ def run_gpu(args, rank, world, device):
     if st != wq.WQ_OK:
         raise RuntimeError("device error word set during warm-up: 0x%x" % detail)
 
-    # per-op events inside the timed steps
-    ev = {name: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    # per-op events inside the timed steps. By default the K timed steps
+    # (with their per-op events, recorded as graph nodes) are captured once as
+    # a CUDA graph and replayed as the timed region: the same launches in the
+    # same order on fresh inputs, without the host's per-launch cost between
+    # them. --eager launches them one by one instead.
+    graph = None
+    ev = {name: [(torch.cuda.Event(enable_timing=True, external=not args.eager),
+                  torch.cuda.Event(enable_timing=True, external=not args.eager))
                  for _ in range(args.steps)] for name, _ in ops}
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clocks:
-        t0.record()
+
+    def timed_steps():
         for i in range(args.steps):
             for name, fn in ops:
                 a, b = ev[name][i]
                 a.record()
                 fn()
                 b.record()
+
+    if not args.eager:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            timed_steps()
+        graph.replay()  # untimed: uploads the graph
+        torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0.record()
+        if graph is not None:
+            graph.replay()
+        else:
+            timed_steps()
         t1.record()
         torch.cuda.synchronize()
     barrier(world)
@@ -364,7 +383,10 @@ def run_gpu(args, rank, world, device):
                                "M=16 and M=1024 25600x5120",
                    "l2": "cold: each op's inputs were last touched a step earlier, with the "
                          "600 MB NF4 stream (>4x L2) in between",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "timing": ("eager launches" if args.eager else
+                              "the K timed steps replayed as one captured CUDA graph") +
+                             ", per-op CUDA events inside, device time"},
         "roofline": {"bound": d["bound"], "kernel": dom, "achieved": round(achieved, 2),
                      "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
                      "traffic": traffic, "peak_source": peaks["source"] + (" (HBM copy)" if d["bound"] == "hbm" else " (sustained bf16" + (")" if dom == "gemm" else " x 2 for int8)"))},
@@ -578,6 +600,9 @@ def main():
     ap.add_argument("--impl", default="wq", choices=["wq", "reference"])
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps one by one instead of replaying them as a "
+                         "captured CUDA graph")
     ap.add_argument("--detail", default=None, help="also write the JSON line to this file")
     ap.add_argument("--case", default=None, choices=PROFILE_CASES,
                     help="run one small profiling case of one kernel and exit")

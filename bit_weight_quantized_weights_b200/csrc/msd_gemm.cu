@@ -69,7 +69,8 @@ struct MsdCfg {
   static constexpr int kNB = (2 * C * BN <= 512) ? 2 : 1;  // TMEM accumulator buffers
   static constexpr int kTmemCols = (C * BN * kNB <= 256) ? 256 : 512;
   static constexpr int kStageBytes = C * kPlaneBytes + kBBytes + kWBytes;
-  static constexpr int kStages = 3;
+  // 4 stages where they fit (C <= 2: 224 KB), else 3
+  static constexpr int kStages = (4 * kStageBytes + 256 + 1024 <= 232448) ? 4 : 3;
   static constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
   // the transpose tile and the split-K partials reuse the stage ring
   static_assert(kStages >= 2 && 3 * kStages + 2 * kNB <= 31, "stages and barriers");
@@ -266,14 +267,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = threadIdx.x - 64;
     const __half* zrow = zeros + (int64_t)(n0 + r) * NG;
     // the zero point of the rank's first group (its k-tiles may start inside it)
-    uint32_t zrep = (uint32_t)__half2float(zrow[kt0 / TPG]) * 0x01010101u;
+    // and the next group's, loaded one group ahead (at 128-wide groups a
+    // zero-point load at the top of each k-tile sat on the critical path)
+    const int g0 = kt0 / TPG;
+    uint32_t zrep = (uint32_t)__half2float(zrow[g0]) * 0x01010101u;
+    __half z_next = zrow[(kt0 % TPG == 0) ? g0 : min(g0 + 1, NG - 1)];
     for (int i = 0; i < KT; ++i) {
       const int kt = kt0 + i;
       const int s = i % kStages;
       const uint32_t ph = (uint32_t)(i / kStages) & 1u;
       if (kt % TPG == 0) {
-        const uint32_t z = (uint32_t)__half2float(zrow[kt / TPG]);
-        zrep = z * 0x01010101u;
+        zrep = (uint32_t)__half2float(z_next) * 0x01010101u;
+        z_next = zrow[min(kt / TPG + 1, NG - 1)];
       }
       bool got = sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1301u, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;

@@ -48,9 +48,17 @@ wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, 
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 128;
-constexpr int kThreads = 448;
+#ifndef MSD_DRAIN_WARPS
+#define MSD_DRAIN_WARPS 8
+#endif
 constexpr int kUnpackWarps = 4;
-constexpr int kEpiWarps = 8;
+// group-drain warps: kEpiWarps / 4 per TMEM lane quarter, each with an
+// equal share of the 128 token columns. 8 (64 columns each) measured 4-6 %
+// faster than 16 on B200: the drain is bound by issue slots it shares with
+// the unpack warps, not by each warp's chain of TMEM loads.
+constexpr int kEpiWarps = MSD_DRAIN_WARPS;
+constexpr int kThreads = 64 + 32 * kUnpackWarps + 32 * kEpiWarps;
+constexpr int kDrainCols = BM / (kEpiWarps / 4);  // token columns per drain warp
 constexpr int kPlaneBytes = BM * BK;      // 16 KB per digit plane tile
 constexpr int kBBytes = BN * BK;          // 16 KB
 constexpr int kWBytes = BN * BK / 2;      // 8 KB packed
@@ -304,15 +312,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- drain / epilogue ----------------
-    // thread = TMEM lane = feature n0 + row; its 64 columns are the tokens
-    // m0 + 64 * half + j
+    // thread = TMEM lane = feature n0 + row; its kDrainCols columns are the
+    // tokens m0 + c0 + j
     const int q = warp & 3;                              // TMEM lane quarter
-    const int half = (warp - 2 - kUnpackWarps) >> 2;     // 64-token half
+    const int c0 = ((warp - 2 - kUnpackWarps) >> 2) * kDrainCols;
     const int row = 32 * q + lane;
-    // acc2[i] holds the tokens 2i, 2i + 1 of this thread's 64 (packed pairs)
-    uint64_t acc2[32];
+    // acc2[i] holds the tokens c0 + 2i, c0 + 2i + 1 (packed pairs)
+    uint64_t acc2[kDrainCols / 2];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) acc2[j] = 0ull;
+    for (int j = 0; j < kDrainCols / 2; ++j) acc2[j] = 0ull;
     const __half* srow = scales + (int64_t)(n0 + row) * NG + g_first;
     float scl = __half2float(srow[0]);
     bool ok = true;
@@ -328,8 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::tc_fence_after();
       const uint64_t scl2 = f2_pack(scl, scl);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int col = half * 64 + 16 * cc;
+      for (int cc = 0; cc < kDrainCols / 16; ++cc) {
+        const int col = c0 + 16 * cc;
         const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * C * BN + col);
         uint32_t p[C][16];
 #pragma unroll
@@ -358,9 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) sm100::mbar_arrive(&acc_empty[b]);
       scl = scl_next;
     }
-    float acc[64];
+    float acc[kDrainCols];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < kDrainCols / 2; ++j) {
       const float2 v = f2_unpack(acc2[j]);
       acc[2 * j] = v.x;
       acc[2 * j + 1] = v.y;
@@ -372,15 +380,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint16_t* out_s = reinterpret_cast<uint16_t*>(smem);  // [128 tokens][kOutPitch]
       if (ok) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int m = m0 + half * 64 + j;
+        for (int j = 0; j < kDrainCols; ++j) {
+          const int m = m0 + c0 + j;
           const float sC = m < M ? comp_scales[(int64_t)(C - 1) * M + m] : 0.0f;
-          out_s[(half * 64 + j) * kOutPitch + row] = bf16_bits(acc[j] * sC);
+          out_s[(c0 + j) * kOutPitch + row] = bf16_bits(acc[j] * sC);
         }
       }
       named_bar_sync(1, 32 * kEpiWarps);
       if (ok) {
-        const int e = threadIdx.x - 64 - 32 * kUnpackWarps;  // 0..255
+        const int e = threadIdx.x - 64 - 32 * kUnpackWarps;  // 0 .. 32 * kEpiWarps - 1
         for (int it = e; it < BM * (BN / 8); it += 32 * kEpiWarps) {
           const int t = it / (BN / 8), ch = it % (BN / 8);
           const int m = m0 + t;
@@ -396,10 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int owner = splitk::row_owner(row, S);
       const int lr = row - splitk::rank_row_begin(owner, S);
       float* dst = reinterpret_cast<float*>(smem) + ((size_t)rank * rows_max + lr) * kRedPitch +
-                   half * 64;
+                   c0;
       const uint32_t rdst = splitk::map_rank(dst, (uint32_t)owner);
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < kDrainCols / 4; ++i)
         asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(rdst + 16u * i),
                      "f"(acc[4 * i]), "f"(acc[4 * i + 1]), "f"(acc[4 * i + 2]),
                      "f"(acc[4 * i + 3])

@@ -367,11 +367,16 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
 //   accf       all MMAs done (the even CTA's commit arrives on both CTAs)
 // All waits are bounded; every thread of both CTAs reaches the final cluster
 // barriers on every path.
+// KB: k per stage, 64 or 128 (two 64-wide 128-byte-swizzled x blocks). The
+// wider stage halves the barrier round trips per MMA.
+template <int KB>
 struct Gemm2Cfg {
   static constexpr int BT = 256;                  // tokens per pair tile (MMA N)
-  static constexpr int kStages = 8;               // stages = TMEM A stages
-  static constexpr int kXBytes = 128 * BK * 2;    // this CTA's x half: 16 KB
-  static constexpr int kWBytes = BW * BK / 2;     // 4 KB
+  static constexpr int kXBlocks = KB / 64;        // 64-wide swizzled x blocks per stage
+  static constexpr int kACols = KB / 2;           // TMEM columns of one A stage (fp16 pairs)
+  static constexpr int kStages = KB == 64 ? 8 : 4;  // stages = TMEM A stages
+  static constexpr int kXBytes = 128 * KB * 2;    // this CTA's x half: 16 or 32 KB
+  static constexpr int kWBytes = BW * KB / 2;     // 4 or 8 KB
   static constexpr int kStageBytes = kXBytes + kWBytes;
   static constexpr int kRing = kStages * kStageBytes;
   static constexpr int kOutBytes = BT * BW * 2;   // epilogue staging (reuses the ring)
@@ -380,7 +385,7 @@ struct Gemm2Cfg {
   static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
   static constexpr uint32_t kTmemCols = 512;
-  static_assert(kAccCols + kStages * 32 <= kTmemCols, "A stages fit in TMEM");
+  static_assert(kAccCols + kStages * kACols <= kTmemCols, "A stages fit in TMEM");
   static_assert(kOutBytes <= kRing, "the staging tile fits in the ring");
   static_assert(kStages % 2 == 0, "every stage is waited on by one group (up to two)");
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
@@ -388,7 +393,7 @@ struct Gemm2Cfg {
   static_assert(8 * (4 * kStages + 1) + 8 <= 512, "barriers fit their 512 bytes");
 };
 
-template <bool kNF4>
+template <bool kNF4, int KB>
 __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     w4a16_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmap_x,
                            const __grid_constant__ CUtensorMap tmap_w,
@@ -396,7 +401,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
                            const void* __restrict__ scales, const __half* __restrict__ zeros,
                            const float* __restrict__ inv_scale, int M, int N, int K, int G,
                            Nf4Table tab) {
-  using C = Gemm2Cfg;
+  using C = Gemm2Cfg<KB>;
   constexpr int BT = C::BT;
   constexpr int ST = C::kStages;
   constexpr int kDeqGroups = Deq<kNF4>::kGroups;
@@ -422,7 +427,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   const bool leader = rank == 0;
   const int n0 = (int)(blockIdx.x >> 1) * (2 * BW) + BW * (int)rank;
   const int m0 = blockIdx.y * BT;                  // the pair's first token
-  const int KT = K / BK;
+  const int KT = K / KB;
 
   if (threadIdx.x == 0) {
     sm100::tma_prefetch_desc(&tmap_x);
@@ -469,11 +474,14 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
           break;
         uint8_t* st = ring + s * C::kStageBytes;
         sm100::mbar_arrive_expect_tx(&wfull[s], C::kWBytes);
-        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &wfull[s], kt * (kNF4 ? BK / 2 : BK / 8),
+        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &wfull[s], kt * (kNF4 ? KB / 2 : KB / 8),
                            n0);
         if (leader) sm100::mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
-        sm100::tma_load_2d_pair(st, &tmap_x, sm100::cluster_addr(&xfull[s], 0), kt * BK,
-                                m0 + 128 * (int)rank);
+#pragma unroll
+        for (int blk = 0; blk < C::kXBlocks; ++blk)
+          sm100::tma_load_2d_pair(st + blk * (128 * 64 * 2), &tmap_x,
+                                  sm100::cluster_addr(&xfull[s], 0), kt * KB + 64 * blk,
+                                  m0 + 128 * (int)rank);
       }
     }
   } else if (warp == 1) {
@@ -488,9 +496,10 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         sm100::tc_fence_after();
         const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bd = sm100::sdesc_sw128_kmajor(x_base + kk * 32);
-          const uint32_t at = tmem + C::kAccCols + (uint32_t)(s * 32 + kk * 8);
+        for (int kk = 0; kk < KB / 16; ++kk) {
+          const uint64_t bd =
+              sm100::sdesc_sw128_kmajor(x_base + (kk / 4) * (128 * 64 * 2) + (kk % 4) * 32);
+          const uint32_t at = tmem + C::kAccCols + (uint32_t)(s * C::kACols + kk * 8);
           sm100::mma_f16_tmem_a_pair(tmem, at, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
         }
         sm100::mma_commit_pair(&done[s], 0x3);
@@ -507,19 +516,26 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     const int n = n0 + r;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int ng = K / G;
-    const int tiles_per_group = G / BK;
+    // this thread's half of each k-tile is KB / 2 wide and lies in one group
+    // (G a multiple of KB, or G == KB / 2); its groups advance by gstep every
+    // tiles_per_group of its k-tiles
+    const int tiles_per_group = G >= KB ? G / KB : 1;
+    const int gstep = G >= KB ? 1 : KB / G;
     const __half* srow = static_cast<const __half*>(scales) + (int64_t)n * ng;
     const __half* zrow = kNF4 ? nullptr : zeros + (int64_t)n * ng;
     // INT4 runs one dequantization group: the group parameters are loaded
     // one group ahead of their use and converted once per group
     static_assert(kNF4 || kDeqGroups == 1, "INT4 parameter stepping assumes one group");
-    __half s_next = kNF4 ? __ushort_as_half(0) : srow[0];
-    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[0];
+    const int g_start = G >= KB ? 0 : hk;
+    __half s_next = kNF4 ? __ushort_as_half(0) : srow[g_start];
+    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[g_start];
     uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
-    int gi = 0, left = 0;  // current group, k-tiles left in it
+    int gi = g_start, left = 0;  // group whose parameters are loaded, k-tiles left
     const bool any = grp < KT;
     const float* arow = static_cast<const float*>(scales) + (int64_t)n * (K / 64);
-    float am_next = (kNF4 && any) ? arow[grp] : 0.0f;
+    // NF4: the absmax block of this thread's half of k-tile kt
+    auto am_block = [&](int kt) { return (kt * KB + hk * (KB / 2)) / 64; };
+    float am_next = (kNF4 && any) ? arow[am_block(grp)] : 0.0f;
     const uint32_t* lut_lane = lut + lane;
     bool ok = true;
     for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
@@ -529,18 +545,18 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       uint32_t am2 = 0;
       if (kNF4) {
         am2 = pack_f16x2(am_next, am_next);
-        if (more) am_next = arow[kt + kDeqGroups];
+        if (more) am_next = arow[am_block(kt + kDeqGroups)];
       } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
         const uint32_t zq = (uint32_t)__half2float(z_next);
         s2 = sb | (sb << 16);
         zb_hi = (0x6400u | zq) * 0x00010001u;
         zb_lo = (0x5400u | (zq << 4)) * 0x00010001u;
-        if (gi + 1 < ng) {
-          s_next = srow[gi + 1];
-          z_next = zrow[gi + 1];
+        if (gi + gstep < ng) {
+          s_next = srow[gi + gstep];
+          z_next = zrow[gi + gstep];
         }
-        ++gi;
+        gi += gstep;
         left = tiles_per_group;
       }
       if (!kNF4) --left;
@@ -553,21 +569,28 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         ok = false;
         break;
       }
-      const uint4 wv = *reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
-                                                       r * 32 + hk * 16);
-      uint32_t cols[16];
-      if (kNF4) {
-        const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+      // this thread's KB / 4 packed bytes: its row r, half hk of the k-tile
+      const uint4* wsrc = reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
+                                                         r * (KB / 2) + hk * (KB / 4));
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
-      } else {
-        dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
-        dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
-        dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
-        dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+      for (int h16 = 0; h16 < KB / 64; ++h16) {
+        const uint4 wv = wsrc[h16];
+        uint32_t cols[16];
+        if (kNF4) {
+          const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
+        } else {
+          dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
+          dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
+          dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
+          dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+        }
+        sm100::tmem_st16(tmem + lane_base + C::kAccCols +
+                             (uint32_t)(s * C::kACols + hk * (KB / 4) + h16 * 16),
+                         cols);
       }
-      sm100::tmem_st16(tmem + lane_base + C::kAccCols + (uint32_t)(s * 32 + hk * 16), cols);
       sm100::tmem_st_wait();
       sm100::tc_fence_before();
       __syncwarp();
@@ -616,27 +639,27 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   sm100::cluster_sync();
 }
 
-template <bool kNF4>
+template <bool kNF4, int KB>
 wq_status launch_pair(const void* x16, const float* inv_scale, int64_t M, int64_t N, int64_t K,
                       int32_t G, const void* qweight, const void* scales, const void* zeros,
                       void* y, cudaStream_t st) {
-  using C = Gemm2Cfg;
+  using C = Gemm2Cfg<KB>;
   CUtensorMap tx, tw, ty;
   // x: this CTA's 128-token half of the pair's tile
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M,
                     (uint64_t)K * 2, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return WQ_ERR_CUDA;
   const bool wmap = kNF4 ? make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qweight,
-                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, BK / 2, BW,
+                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, KB / 2, BW,
                                         CU_TENSOR_MAP_SWIZZLE_NONE)
                          : make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight,
-                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, BK / 8, BW,
+                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, KB / 8, BW,
                                         CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!wmap) return WQ_ERR_CUDA;
   if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, BW, C::BT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WQ_ERR_CUDA;
-  auto kern = w4a16_gemm_pair_kernel<kNF4>;
+  auto kern = w4a16_gemm_pair_kernel<kNF4, KB>;
   const int smem = C::smem(kNF4);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
@@ -703,6 +726,14 @@ bool gemm_pairs_enabled() {
   return on;
 }
 
+bool gemm_kb128_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("WQ_GEMM_KB");
+    return !(e && e[0] == '6');
+  }();
+  return on;
+}
+
 // Workspace: the fp16 copy of x [M, K] (256-byte aligned), then 2^-e per row.
 size_t gemm_workspace_bytes(int64_t M, int64_t K) {
   return ((size_t)M * K * 2 + 255) / 256 * 256 + (size_t)M * 4;
@@ -722,13 +753,20 @@ wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   const bool wide = tiles256 >= (int64_t)num_sms();
   // CTA pairs (256 weight rows x 256 tokens per pair) where the rows pair up
   const bool pair = wide && N % (2 * BW) == 0 && gemm_pairs_enabled();
+  // 128-wide k stages where every thread's half stage lies in one group
+  const bool wide_k = K % 128 == 0 && (G % 128 == 0 || G == 64) && gemm_kb128_enabled();
   if (nf4) {
     if (pair)
-      return launch_pair<true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+      return wide_k
+                 ? launch_pair<true, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+                 : launch_pair<true, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
     return wide ? launch_bt<256, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
                 : launch_bt<128, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   }
-  if (pair) return launch_pair<false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  if (pair)
+    return wide_k
+               ? launch_pair<false, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+               : launch_pair<false, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   return wide ? launch_bt<256, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
               : launch_bt<128, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
 }

@@ -64,15 +64,20 @@ struct Deq {
 };
 constexpr int SA = 4;            // TMEM A stages (32 columns each)
 
-template <int BT, bool kNF4>
+// KB: k per stage, 64 or 128 (two 64-wide swizzled x blocks; half the
+// barrier round trips per MMA).
+template <int BT, bool kNF4, int KB>
 struct GemmCfg {
+  static constexpr int kXBlocks = KB / 64;
+  static constexpr int kACols = KB / 2;           // TMEM columns of one A stage
   // A multiple of the dequantization groups, so that every ring stage and A
   // stage is always waited on by the same group, one phase at a time (a
   // parity wait must never run two phases ahead of its barrier). NF4 needs
   // room for its lookup table.
-  static constexpr int kStages = (BT == 256) ? (kNF4 ? 4 : 5) : 8;
-  static constexpr int kXBytes = BT * BK * 2;     // 32 / 16 KB
-  static constexpr int kWBytes = BW * BK / 2;     // 4 KB
+  static constexpr int kStages =
+      KB == 64 ? ((BT == 256) ? (kNF4 ? 4 : 5) : 8) : ((BT == 256) ? 3 : 4);
+  static constexpr int kXBytes = BT * KB * 2;     // 16-64 KB
+  static constexpr int kWBytes = BW * KB / 2;     // 4 or 8 KB
   static constexpr int kStageBytes = kXBytes + kWBytes;
   static constexpr int kOutBytes = BT * BW * 2;   // epilogue staging (reuses the ring)
   static constexpr int kRing = kStages * kStageBytes;
@@ -83,9 +88,11 @@ struct GemmCfg {
   static constexpr int kSmem = kRingOrOut + BT * 4 + 512 + 1024;
   static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
-  static constexpr uint32_t kTmemCols = (BT + SA * 32 <= 256) ? 256 : 512;
+  static constexpr uint32_t kTmemCols = (BT + SA * kACols <= 256) ? 256 : 512;
+  static_assert(BT + SA * kACols <= 512, "A stages fit in TMEM");
   static_assert(kStages % Deq<kNF4>::kGroups == 0 && SA % Deq<kNF4>::kGroups == 0,
                 "stages per group");
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
 };
 
 __device__ __forceinline__ uint32_t f16x2_sub(uint32_t a, uint32_t b) {
@@ -114,14 +121,14 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb_hi, uint32_
   out[3] = f16x2_mul(f16x2_sub(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), zb_lo), s2);
 }
 
-template <int BT, bool kNF4>
+template <int BT, bool kNF4, int KB>
 __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_y, const void* __restrict__ scales,
                       const __half* __restrict__ zeros, const float* __restrict__ inv_scale, int M,
                       int N, int K, int G, Nf4Table tab) {
-  using C = GemmCfg<BT, kNF4>;
+  using C = GemmCfg<BT, kNF4, KB>;
   constexpr int ST = C::kStages;
   constexpr int kDeqGroups = Deq<kNF4>::kGroups;
   constexpr int kThreads = Deq<kNF4>::kThreads;
@@ -146,7 +153,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BW;
   const int m0 = blockIdx.y * BT;
-  const int KT = K / BK;
+  const int KT = K / KB;
 
   if (threadIdx.x == 0) {
     sm100::tma_prefetch_desc(&tmap_x);
@@ -193,9 +200,11 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
           break;
         uint8_t* st = ring + s * C::kStageBytes;
         sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        sm100::tma_load_2d(st, &tmap_x, &full[s], kt * BK, m0);
-        // packed tile: 8 uint32 words (INT4) or 32 code bytes (NF4) per row
-        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &full[s], kt * (kNF4 ? BK / 2 : BK / 8), n0);
+#pragma unroll
+        for (int blk = 0; blk < C::kXBlocks; ++blk)
+          sm100::tma_load_2d(st + blk * (BT * 64 * 2), &tmap_x, &full[s], kt * KB + 64 * blk, m0);
+        // packed tile: KB / 8 uint32 words (INT4) or KB / 2 code bytes (NF4) per row
+        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &full[s], kt * (kNF4 ? KB / 2 : KB / 8), n0);
       }
     }
   } else if (warp == 1) {
@@ -210,9 +219,10 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         sm100::tc_fence_after();
         const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t bd = sm100::sdesc_sw128_kmajor(x_base + kk * 32);
-          const uint32_t at = tmem + C::kAccCols + (uint32_t)(a * 32 + kk * 8);
+        for (int kk = 0; kk < KB / 16; ++kk) {
+          const uint64_t bd =
+              sm100::sdesc_sw128_kmajor(x_base + (kk / 4) * (BT * 64 * 2) + (kk % 4) * 32);
+          const uint32_t at = tmem + C::kAccCols + (uint32_t)(a * C::kACols + kk * 8);
           sm100::mma_f16_tmem_a(tmem, at, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
         }
         sm100::mma_commit(&empty[s]);
@@ -230,20 +240,27 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     const int n = n0 + r;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int ng = K / G;
-    const int tiles_per_group = G / BK;
+    // this thread's half of each k-tile is KB / 2 wide and lies in one group
+    // (G a multiple of KB, or G == KB / 2); its groups advance by gstep every
+    // tiles_per_group of its k-tiles
+    const int tiles_per_group = G >= KB ? G / KB : 1;
+    const int gstep = G >= KB ? 1 : KB / G;
+    const int g_start = G >= KB ? 0 : hk;
     const __half* srow = static_cast<const __half*>(scales) + (int64_t)n * ng;
     const __half* zrow = kNF4 ? nullptr : zeros + (int64_t)n * ng;
     // INT4 runs one dequantization group: the group parameters are loaded
     // one group ahead of their use and converted once per group
     static_assert(kNF4 || kDeqGroups == 1, "INT4 parameter stepping assumes one group");
-    __half s_next = kNF4 ? __ushort_as_half(0) : srow[0];
-    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[0];
+    __half s_next = kNF4 ? __ushort_as_half(0) : srow[g_start];
+    __half z_next = kNF4 ? __ushort_as_half(0) : zrow[g_start];
     uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
-    int gi = 0, left = 0;  // current group, k-tiles left in it
+    int gi = g_start, left = 0;  // group whose parameters are loaded, k-tiles left
     const bool any = grp < KT;
     // NF4: the absmax of (row n, 64-element block kt) is one per k-tile
     const float* arow = static_cast<const float*>(scales) + (int64_t)n * (K / 64);
-    float am_next = (kNF4 && any) ? arow[grp] : 0.0f;
+    // NF4: the absmax block of this thread's half of k-tile kt
+    auto am_block = [&](int kt) { return (kt * KB + hk * (KB / 2)) / 64; };
+    float am_next = (kNF4 && any) ? arow[am_block(grp)] : 0.0f;
     const uint32_t* lut_lane = lut + lane;
     bool ok = true;
     for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
@@ -255,18 +272,18 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         // fp16x2 (absmax, absmax), rounded once; this warp's next one is
         // loaded now
         am2 = pack_f16x2(am_next, am_next);
-        if (more) am_next = arow[kt + kDeqGroups];
+        if (more) am_next = arow[am_block(kt + kDeqGroups)];
       } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
         const uint32_t zq = (uint32_t)__half2float(z_next);
         s2 = sb | (sb << 16);
         zb_hi = (0x6400u | zq) * 0x00010001u;         // fp16x2 (1024 + z, 1024 + z)
         zb_lo = (0x5400u | (zq << 4)) * 0x00010001u;  // fp16x2 (64 + z, 64 + z)
-        if (gi + 1 < ng) {
-          s_next = srow[gi + 1];
-          z_next = zrow[gi + 1];
+        if (gi + gstep < ng) {
+          s_next = srow[gi + gstep];
+          z_next = zrow[gi + gstep];
         }
-        ++gi;
+        gi += gstep;
         left = tiles_per_group;
       }
       if (!kNF4) --left;
@@ -277,23 +294,30 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         ok = false;
         break;
       }
-      const uint4 wv = *reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
-                                                       r * 32 + hk * 16);
-      uint32_t cols[16];
-      if (kNF4) {
-        // 16 code bytes = elements (2j, 2j + 1) in k order: one table read
-        // gives the fp16 code pair, one multiply applies the block's absmax
-        const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+      // this thread's KB / 4 packed bytes: its row r, half hk of the k-tile
+      const uint4* wsrc = reinterpret_cast<const uint4*>(ring + s * C::kStageBytes + C::kXBytes +
+                                                         r * (KB / 2) + hk * (KB / 4));
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
-      } else {
-        dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
-        dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
-        dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
-        dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+      for (int h16 = 0; h16 < KB / 64; ++h16) {
+        const uint4 wv = wsrc[h16];
+        uint32_t cols[16];
+        if (kNF4) {
+          // 16 code bytes = elements (2j, 2j + 1) in k order: one table read
+          // gives the fp16 code pair, one multiply applies the block's absmax
+          const uint32_t wb[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            cols[j] = f16x2_mul(lut_lane[((wb[j >> 2] >> (8 * (j & 3))) & 0xFFu) * 32], am2);
+        } else {
+          dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
+          dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
+          dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
+          dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+        }
+        sm100::tmem_st16(tmem + lane_base + C::kAccCols +
+                             (uint32_t)(a * C::kACols + hk * (KB / 4) + h16 * 16),
+                         cols);
       }
-      sm100::tmem_st16(tmem + lane_base + C::kAccCols + (uint32_t)(a * 32 + hk * 16), cols);
       sm100::tmem_st_wait();
       sm100::tc_fence_before();
       __syncwarp();
@@ -682,7 +706,7 @@ wq_status launch_pair(const void* x16, const float* inv_scale, int64_t M, int64_
   return launch_status();
 }
 
-template <int BT, bool kNF4>
+template <int BT, bool kNF4, int KB>
 wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t N, int64_t K,
                     int32_t G, const void* qweight, const void* scales, const void* zeros, void* y,
                     cudaStream_t st) {
@@ -692,17 +716,17 @@ wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t 
     return WQ_ERR_CUDA;
   // the packed tile is 32 bytes of each of 128 rows in both formats
   const bool wmap = kNF4 ? make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qweight,
-                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, BK / 2, BW,
+                                        (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, KB / 2, BW,
                                         CU_TENSOR_MAP_SWIZZLE_NONE)
                          : make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight,
-                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, BK / 8, BW,
+                                        (uint64_t)K / 8, (uint64_t)N, (uint64_t)K / 2, KB / 8, BW,
                                         CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!wmap) return WQ_ERR_CUDA;
   if (!make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
                     (uint64_t)N * 2, BW, BT, CU_TENSOR_MAP_SWIZZLE_NONE))
     return WQ_ERR_CUDA;
-  using C = GemmCfg<BT, kNF4>;
-  auto kern = w4a16_gemm_kernel<BT, kNF4>;
+  using C = GemmCfg<BT, kNF4, KB>;
+  auto kern = w4a16_gemm_kernel<BT, kNF4, KB>;
   const int smem = C::smem(kNF4);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
       cudaSuccess)
@@ -760,15 +784,24 @@ wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
       return wide_k
                  ? launch_pair<true, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
                  : launch_pair<true, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
-    return wide ? launch_bt<256, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
-                : launch_bt<128, true>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+    // 256-token NF4 tiles keep 64-k stages: with the lookup table only two
+    // 128-k stages would fit
+    if (wide) return launch_bt<256, true, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+    return wide_k
+               ? launch_bt<128, true, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+               : launch_bt<128, true, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   }
   if (pair)
     return wide_k
                ? launch_pair<false, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
                : launch_pair<false, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
-  return wide ? launch_bt<256, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
-              : launch_bt<128, false>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  if (wide)
+    return wide_k
+               ? launch_bt<256, false, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+               : launch_bt<256, false, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
+  return wide_k
+             ? launch_bt<128, false, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
+             : launch_bt<128, false, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
 }
 
 wq_status read_gemm_error(bool clear, uint32_t* v) {

@@ -106,14 +106,21 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
 // One 128-k unit of this lane's two weight rows (g and g + 8), with its
 // group parameters.
 //   wide  : w[0..3] = 16 bytes of row g at byte 16t, w[4..7] the same of row
-//           g + 8 (k = 32t .. 32t + 31); prm[0..1] = (scale, zero) of rows g,
-//           g + 8 (one group spans the unit).
+//           g + 8 (k = 32t .. 32t + 31); INT4: prm[0..1] = the scale bits of
+//           rows g, g + 8 and prm[2..3] their zero bits (one group spans the
+//           unit).
 //   narrow: w[0..1] row g, half 0 (byte 8t), w[2..3] row g, half 1 (byte
-//           32 + 8t), w[4..7] the same of row g + 8; prm[2h + i] = the
-//           parameters of half h for row g (i = 0) or g + 8 (i = 1).
+//           32 + 8t), w[4..7] the same of row g + 8; prm[2h + i] = the scale
+//           bits of half h for row g (i = 0) or g + 8 (i = 1), zz[2h + i] the
+//           zero bits.
+// NF4: prm[2h + i] = the absmax of block h of row g or g + 8.
+// The fp16 parameters stay as loaded (zero-extended 16-bit loads, no
+// arithmetic on them) until the unit is computed, so the loads never stall a
+// warp that is still issuing its first units and staging x.
 struct Unit {
   uint32_t w[8];
   uint32_t prm[4];
+  uint32_t zz[4];  // narrow INT4 only
 };
 
 template <bool kNF4, bool kWide>
@@ -147,21 +154,30 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     for (int h = 0; h < (kWide ? 1 : 2); ++h) {
       const int gi = div_by_magic(2 * u + h, p.gmagic);
       const int64_t iA = (int64_t)nA * ng + gi, iB = (int64_t)nB * ng + gi;
-      U.prm[2 * h + 0] = (uint32_t)__ldg(s16 + iA) | ((uint32_t)__ldg(z16 + iA) << 16);
-      U.prm[2 * h + 1] = (uint32_t)__ldg(s16 + iB) | ((uint32_t)__ldg(z16 + iB) << 16);
+      U.prm[2 * h + 0] = __ldg(s16 + iA);
+      U.prm[2 * h + 1] = __ldg(s16 + iB);
+      if (kWide) {
+        U.prm[2] = __ldg(z16 + iA);
+        U.prm[3] = __ldg(z16 + iB);
+      } else {
+        U.zz[2 * h + 0] = __ldg(z16 + iA);
+        U.zz[2 * h + 1] = __ldg(z16 + iB);
+      }
     }
   }
 }
 
 // acc += s * (P - (128 + z) * sum(x)) for the four accumulator slots of one
-// token tile; pv holds (s, z) as fp16 halves, sx the two tokens' sums of x.
-__device__ __forceinline__ void int4_post(float (&acc)[4], const float (&cp)[4], uint32_t pv_g,
-                                          uint32_t pv_g8, float2 sx) {
+// token tile; s_*, z_* hold the fp16 bits of rows g and g + 8, sx the two
+// tokens' sums of x.
+__device__ __forceinline__ void int4_post(float (&acc)[4], const float (&cp)[4], uint32_t s_g,
+                                          uint32_t s_g8, uint32_t z_g, uint32_t z_g8,
+                                          float2 sx) {
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const uint32_t pv = (r >> 1) ? pv_g8 : pv_g;  // row g for r < 2, g + 8 else
-    const float s = __half2float(__ushort_as_half((unsigned short)(pv & 0xFFFFu)));
-    const float zb = 128.0f + __half2float(__ushort_as_half((unsigned short)(pv >> 16)));
+    const bool hi = (r >> 1) != 0;  // row g for r < 2, g + 8 else
+    const float s = __half2float(__ushort_as_half((unsigned short)(hi ? s_g8 : s_g)));
+    const float zb = 128.0f + __half2float(__ushort_as_half((unsigned short)(hi ? z_g8 : z_g)));
     acc[r] = fmaf(s, fmaf(-zb, (r & 1) ? sx.y : sx.x, cp[r]), acc[r]);
   }
 }
@@ -206,7 +222,7 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
 #pragma unroll
       for (int r = 0; r < 4; ++r) cs[r] = cp[0][a][r] + cp[1][a][r];
       const float2 sx = *reinterpret_cast<const float2*>(xsum + lu * kTok + 8 * a + 2 * t);
-      int4_post(acc[a], cs, U.prm[0], U.prm[1], sx);
+      int4_post(acc[a], cs, U.prm[0], U.prm[1], U.prm[2], U.prm[3], sx);
     }
   } else {
 #pragma unroll
@@ -267,7 +283,8 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
         } else {
           const float2 sx =
               *reinterpret_cast<const float2*>(xsum + (2 * lu + h) * kTok + 8 * a + 2 * t);
-          int4_post(acc[a], cs, U.prm[2 * h], U.prm[2 * h + 1], sx);
+          int4_post(acc[a], cs, U.prm[2 * h], U.prm[2 * h + 1], U.zz[2 * h], U.zz[2 * h + 1],
+                    sx);
         }
       }
     }

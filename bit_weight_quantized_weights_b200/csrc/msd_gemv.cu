@@ -64,10 +64,13 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
 }
 
 // One 128-k unit of this lane's rows g and g + 8: w[0..3] = 16 bytes of row g
-// at byte 16t, w[4..7] the same of row g + 8; prm = (scale, zero) fp16 pairs.
+// at byte 16t, w[4..7] the same of row g + 8; prm[0..1] = the fp16 scale bits
+// of rows g, g + 8 and prm[2..3] their zero bits, kept as loaded (no
+// arithmetic on them before the unit is computed, so their loads never stall
+// a warp still issuing its first units).
 struct MsdUnit {
   uint32_t w[8];
-  uint32_t prm[2];
+  uint32_t prm[4];
 };
 
 __device__ __forceinline__ void msd_load_unit(MsdUnit& U, const uint8_t* wA, const uint8_t* wB,
@@ -80,8 +83,10 @@ __device__ __forceinline__ void msd_load_unit(MsdUnit& U, const uint8_t* wA, con
   const unsigned short* s16 = reinterpret_cast<const unsigned short*>(p.scales);
   const unsigned short* z16 = reinterpret_cast<const unsigned short*>(p.zeros);
   const int64_t iA = (int64_t)nA * ng + gi, iB = (int64_t)nB * ng + gi;
-  U.prm[0] = (uint32_t)__ldg(s16 + iA) | ((uint32_t)__ldg(z16 + iA) << 16);
-  U.prm[1] = (uint32_t)__ldg(s16 + iB) | ((uint32_t)__ldg(z16 + iB) << 16);
+  U.prm[0] = __ldg(s16 + iA);
+  U.prm[1] = __ldg(s16 + iB);
+  U.prm[2] = __ldg(z16 + iA);
+  U.prm[3] = __ldg(z16 + iB);
 }
 
 template <int NT>
@@ -236,9 +241,8 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
         // post-group scaling of this unit
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-          const uint32_t pv = U.prm[hr];
-          const float s = __half2float(__ushort_as_half((unsigned short)(pv & 0xFFFFu)));
-          const int z = (int)__half2float(__ushort_as_half((unsigned short)(pv >> 16)));
+          const float s = __half2float(__ushort_as_half((unsigned short)U.prm[hr]));
+          const int z = (int)__half2float(__ushort_as_half((unsigned short)U.prm[2 + hr]));
 #pragma unroll
           for (int a = 0; a < NT; ++a) {
             int2 R[C];

@@ -119,9 +119,11 @@ struct Plan {
 
 // Cluster size S (K split): every CTA holds one 128-row tile over one K-chunk
 // of kc = ceil(units / S) * 128. S (1..16, at most one 128-k unit per CTA,
-// fits(kc) true) is chosen to fill the resident CTA slots of the GPU with the
-// fewest waves: the whole weight stream should be in flight from the first
-// microseconds. smem_of(kc, S) gives the CTA's dynamic shared memory.
+// fits(kc) true) minimises waves x (kc + a fixed cost of 512 k per CTA for
+// staging x and the reduction): a wave lasts as long as its CTAs' K-chunks,
+// so two waves of half-K CTAs beat two waves of full-K ones (a large x chunk
+// can leave one CTA per SM). Ties go to the fuller GPU. smem_of(kc, S) gives
+// the CTA's dynamic shared memory.
 template <class Kern, class Fits, class SmemOf>
 Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf smem_of) {
   const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
@@ -171,9 +173,9 @@ Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf s
     if (slots < 1) continue;
     const int64_t grid = tiles * S;
     const int64_t waves = (grid + slots - 1) / slots;
-    // fewest waves first (a second wave repeats the whole load ramp), then
-    // the largest share of the resident slots kept busy
-    const double score = (double)grid / ((double)waves * slots) - (double)waves;
+    constexpr double kFixedK = 512.0;
+    const double fill = (double)grid / ((double)waves * slots);
+    const double score = -(double)waves * ((double)kc + kFixedK) + 1e-3 * fill;
     if (score > best + 1e-9) {
       best = score;
       bp.S = S;

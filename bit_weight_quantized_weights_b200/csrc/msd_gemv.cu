@@ -96,7 +96,8 @@ struct MsdTraits {
 
 template <int NT>
 size_t msd_smem(int kc, int S, int M, int C) {
-  return (size_t)C * M * kc + (size_t)C * (kc / 128) * 8 * NT * 4 + red_bytes(S);
+  // planes, digit sums, two partial buffers (alternating row tiles)
+  return (size_t)C * M * kc + (size_t)C * (kc / 128) * 8 * NT * 4 + 2 * red_bytes(S);
 }
 
 template <int NT, int C>
@@ -116,12 +117,17 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
   const int u1 = (int)((int64_t)(rank + 1) * p.units / p.S);
   const int k0 = u0 * 128;
   const int klen = (u1 - u0) * 128;
-  const int row_tile = (int)blockIdx.y * kRowsPerCta;
   const int g = lane >> 2, t = lane & 3;
-  const int n0 = row_tile + warp * 16;
-  const bool active = n0 < p.N;
-  const int nA = n0 + g, nB = n0 + g + 8;
   const int ng = p.K / p.G;
+  const int tiles = (p.N + kRowsPerCta - 1) / kRowsPerCta;
+  // Persistent over row tiles: this cluster takes tiles blockIdx.y,
+  // blockIdx.y + gridDim.y, ...; the digit planes of its K-chunk are staged
+  // and prepared once. Per tile: the warp's 16 rows and their weight rows.
+  int tile = (int)blockIdx.y;
+  int row_tile = tile * kRowsPerCta;
+  int n0 = row_tile + warp * 16;
+  bool active = n0 < p.N;
+  int nA = n0 + g, nB = n0 + g + 8;
 
   // ---- digit planes [C][M][k0 : k0+klen) -> shared memory (16-byte copies),
   // issued before the weight loads
@@ -139,6 +145,7 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
   const int64_t row_bytes = (int64_t)p.K / 2;
   const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + 16 * t;
   const uint8_t* wrowB = wrowA + 8 * row_bytes;
+  const float* red_buf[2] = {red, red + red_bytes(p.S) / 4};
   MsdUnit ring[D];
   if (active) {
 #pragma unroll
@@ -176,6 +183,28 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
   }
   __syncthreads();
 
+  // plane rows of this lane's B tokens (padding tokens read token 0's row:
+  // their MMA columns never reach an output) and the component scales of its
+  // accumulator tokens 8a + 2t + {0, 1}
+  const int8_t* prow[C][NT];
+  int psw[NT];
+  float scl[C][NT][2];
+#pragma unroll
+  for (int a = 0; a < NT; ++a) {
+    const int tr = (g + 8 * a < M) ? g + 8 * a : 0;
+    psw[a] = tr & 1;
+#pragma unroll
+    for (int c = 0; c < C; ++c) {
+      prow[c][a] = pl + ((size_t)c * M + tr) * kc;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tok = 8 * a + 2 * t + e;
+        scl[c][a][e] = tok < M ? p.cs[c * M + tok] : 0.0f;
+      }
+    }
+  }
+
+  for (int it = 0; tile < tiles; ++it) {
   // ---- main loop: warp owns 16 weight rows over this CTA's K-chunk --------
   float acc[NT][4];
 #pragma unroll
@@ -184,26 +213,6 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
     for (int r = 0; r < 4; ++r) acc[a][r] = 0.0f;
 
   if (active) {
-    // plane rows of this lane's B tokens (padding tokens read token 0's row:
-    // their MMA columns never reach an output) and the component scales of
-    // its accumulator tokens 8a + 2t + {0, 1}
-    const int8_t* prow[C][NT];
-    int psw[NT];
-    float scl[C][NT][2];
-#pragma unroll
-    for (int a = 0; a < NT; ++a) {
-      const int tr = (g + 8 * a < M) ? g + 8 * a : 0;
-      psw[a] = tr & 1;
-#pragma unroll
-      for (int c = 0; c < C; ++c) {
-        prow[c][a] = pl + ((size_t)c * M + tr) * kc;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tok = 8 * a + 2 * t + e;
-          scl[c][a][e] = tok < M ? p.cs[c * M + tok] : 0.0f;
-        }
-      }
-    }
     for (int ub = u0; ub < u1; ub += D) {
 #pragma unroll
       for (int i = 0; i < D; ++i) {
@@ -275,8 +284,31 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
     }
   }
 
+  // every slot of the ring is consumed: start the next tile's weight stream
+  // before this tile's reduction
+  const int cur_row_tile = row_tile;
+  tile += (int)gridDim.y;
+  if (tile < tiles) {
+    row_tile = tile * kRowsPerCta;
+    n0 = row_tile + warp * 16;
+    active = n0 < p.N;
+    nA = n0 + g;
+    nB = n0 + g + 8;
+    wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + 16 * t;
+    wrowB = wrowA + 8 * row_bytes;
+    if (active) {
+#pragma unroll
+      for (int i = 0; i < D; ++i)
+        if (u0 + i < u1) msd_load_unit(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng);
+    }
+  }
+
   // ---- cluster split-K reduction (through distributed shared memory) -----
-  reduce_and_store<NT>(acc, nullptr, red, p.S, rank, row_tile, M, p.N, p.y);
+  // (the partial buffers alternate between tiles: the next tile's pushes
+  // follow this tile's barrier, which the owner passes only after reading)
+  reduce_and_store<NT>(acc, nullptr, const_cast<float*>(red_buf[it & 1]), p.S, rank,
+                       cur_row_tile, M, p.N, p.y);
+  }
 }
 
 template <int NT, int C>
@@ -286,12 +318,12 @@ wq_status launch_msd_t(MsdArgs a, cudaStream_t st) {
     return make_plan(
         kern, 256, a.N, a.K,
         [&](int kc) { return (int64_t)C * a.M * kc <= kMaxPlaneChunkBytes; },
-        [&](int kc, int S) { return msd_smem<NT>(kc, S, a.M, C); });
+        [&](int kc, int S) { return msd_smem<NT>(kc, S, a.M, C); }, /*persistent=*/true);
   });
   if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
   a.S = pl.S;
   a.kc = pl.kc;
-  return launch_split(kern, pl, 256, a.N, st, a, nf4_table());
+  return launch_split(kern, pl, 256, a.N, st, a, nf4_table(), /*persistent=*/true);
 }
 
 template <int NT>

@@ -115,17 +115,21 @@ struct Plan {
   int S = 0;
   int kc = 0;
   size_t smem = 0;
+  int resident = 0;  // S-CTA clusters resident at once (persistent launches)
 };
 
 // Cluster size S (K split): every CTA holds one 128-row tile over one K-chunk
 // of kc = ceil(units / S) * 128. S (1..16, at most one 128-k unit per CTA,
-// fits(kc) true) minimises waves x (kc + a fixed cost of 512 k per CTA for
-// staging x and the reduction): a wave lasts as long as its CTAs' K-chunks,
-// so two waves of half-K CTAs beat two waves of full-K ones (a large x chunk
-// can leave one CTA per SM). Ties go to the fuller GPU. smem_of(kc, S) gives
-// the CTA's dynamic shared memory.
+// fits(kc) true) minimises the K streamed per CTA slot plus fixed costs, in
+// k: waves x (kc + 512 for staging x and the reduction), since a wave lasts
+// as long as its CTAs' K-chunks (two waves of half-K CTAs beat two waves of
+// full-K ones). A persistent kernel (each resident cluster loops over row
+// tiles and stages its x chunk once) pays the staging once: 512 once plus
+// waves x (kc + 256). Ties go to the fuller GPU. smem_of(kc, S) gives the
+// CTA's dynamic shared memory.
 template <class Kern, class Fits, class SmemOf>
-Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf smem_of) {
+Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf smem_of,
+               bool persistent = false) {
   const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
   const int64_t units = K / 128;
   cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -173,14 +177,15 @@ Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf s
     if (slots < 1) continue;
     const int64_t grid = tiles * S;
     const int64_t waves = (grid + slots - 1) / slots;
-    constexpr double kFixedK = 512.0;
+    const double per_wave = persistent ? 256.0 : 512.0, once = persistent ? 512.0 : 0.0;
     const double fill = (double)grid / ((double)waves * slots);
-    const double score = -(double)waves * ((double)kc + kFixedK) + 1e-3 * fill;
+    const double score = -((double)waves * ((double)kc + per_wave) + once) + 1e-3 * fill;
     if (score > best + 1e-9) {
       best = score;
       bp.S = S;
       bp.kc = kc;
       bp.smem = smem;
+      bp.resident = slots / S;
     }
   }
   return bp;
@@ -213,16 +218,20 @@ Plan cached_plan(const void* kern, int M, int64_t N, int64_t K, int extra, MakeF
 }
 
 // Launch `kern` on the plan's (S x row tiles) grid with S-CTA clusters.
+// persistent: the grid has at most pl.resident clusters along y, each looping
+// over the row tiles y, y + gridDim.y, ...
 template <class Kern, class Args>
 wq_status launch_split(Kern kern, const Plan& pl, int threads, int64_t N, cudaStream_t st,
-                       const Args& args, const Nf4Table& tab) {
+                       const Args& args, const Nf4Table& tab, bool persistent = false) {
   // the attribute is a per-function maximum; plans of other shapes may have
   // set a smaller one since
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)pl.S, (unsigned)((N + kRowsPerCta - 1) / kRowsPerCta), 1);
+  const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t gy = persistent && pl.resident > 0 && pl.resident < tiles ? pl.resident : tiles;
+  cfg.gridDim = dim3((unsigned)pl.S, (unsigned)gy, 1);
   cfg.blockDim = dim3((unsigned)threads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;

@@ -80,6 +80,8 @@ def _msd_case(wq, m, n, k, group, c, seed, rows=None, cols=None):
     (9, 256, 768, 256, 3),       # two token tiles, three components
     (16, 1024, 2048, 128, 2),    # full token tile pair, several row tiles
     (13, 512, 1280, 640, 2),     # groups of five units
+    (16, 38016, 512, 128, 2),    # 297 row tiles: more than the resident clusters, so each
+                                 # persistent cluster loops over several tiles
     (17, 256, 512, 128, 2),      # first size past the decode path: tcgen05 tiles
 ])
 def test_msd_gemm_small_every_element(wq, m, n, k, group, c):

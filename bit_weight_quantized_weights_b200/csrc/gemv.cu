@@ -11,8 +11,8 @@
 // B200 design
 // -----------
 // * The weight stream is the whole cost (0.53 byte per weight against 2*M
-//   flops). Weights are read with plain 16-byte (8-byte for 64-wide groups
-//   and NF4) loads that do not allocate in L1, by two 256-thread CTAs per SM,
+//   flops). Weights are read with plain 16-byte (8-byte for INT4 groups of
+//   64) loads that do not allocate in L1, by two 256-thread CTAs per SM,
 //   each warp keeping three or four 128-k units of its 16 rows (with their
 //   group parameters) in flight while it computes the oldest. Measured on
 //   B200, plain coalesced loads stream HBM far better than a TMA ring of
@@ -33,9 +33,11 @@
 // * NF4 codes go through a 256-entry table indexed by a whole packed byte that
 //   yields the two fp16 code values already paired as one A-operand register.
 //   The table is replicated per lane (lane l reads column l, so bank l): every
-//   lookup is conflict-free. The block's absmax is applied after the block's
-//   sum. The NF4 product runs in fp16 (the code values keep 11 significant
-//   bits): the staged x chunk is converted to fp16 scaled per token by a power
+//   lookup is conflict-free. Each lane's 16 bytes (32 codes) lie inside one
+//   64-element absmax block, so one fp16x2 multiply per register applies the
+//   block's absmax to the A operand before the MMA (code, absmax and product
+//   each rounded once to fp16, as in the fused GEMM), which lets NF4 use the
+//   16-byte layout. The NF4 product runs in fp16: the staged x chunk is converted to fp16 scaled per token by a power
 //   of two that puts its largest magnitude in [2^14, 2^15) (exact for bf16
 //   values down to 2^-28 of it); the power is divided back out of the partial.
 // * Split-K across a thread-block cluster: the S CTAs of a cluster share one
@@ -50,8 +52,8 @@
 //   xs   [8*NT tokens][Kc] bf16 (fp16 for NF4), the CTA's K-chunk of x, in
 //        16-byte chunks. Only the M real tokens are written: a padding
 //        token's MMA column never reaches an output. Chunk c of token m sits
-//        at chunk c ^ (m & 1), and for the wide INT4 layout (groups that are
-//        multiples of 128) also ^ (bit 3 of c moved to bit 1), so that the
+//        at chunk c ^ (m & 1), and for the 16-byte layout (NF4, INT4 groups
+//        that are multiples of 128) also ^ (bit 3 of c moved to bit 1), so that the
 //        fragment loads of a warp hit distinct banks. For INT4 each chunk
 //        holds the pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7), the nibble pairing.
 //   xsum [Kc/64 or Kc/128][8*NT tokens] fp32, sums of x per group part (INT4)
@@ -98,6 +100,12 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // (128 + nibble) as bf16 for nibbles e and e + 4 of w -> one bf16x2 register.
 __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
   return lop3_and_or(w >> (4 * e), 0x000F000Fu, 0x43004300u);
@@ -113,7 +121,8 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
 //           32 + 8t), w[4..7] the same of row g + 8; prm[2h + i] = the scale
 //           bits of half h for row g (i = 0) or g + 8 (i = 1), zz[2h + i] the
 //           zero bits.
-// NF4: prm[2h + i] = the absmax of block h of row g or g + 8.
+// NF4 (wide): prm[i] = the fp32 absmax bits of the lane's block (2u + t / 2)
+// of row g (i = 0) or g + 8 (i = 1).
 // The fp16 parameters stay as loaded (zero-extended 16-bit loads, no
 // arithmetic on them) until the unit is computed, so the loads never stall a
 // warp that is still issuing its first units and staging x.
@@ -125,7 +134,7 @@ struct Unit {
 
 template <bool kNF4, bool kWide>
 __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint8_t* wB, int u,
-                                          int nA, int nB, const GemvArgs& p, int ng) {
+                                          int nA, int nB, const GemvArgs& p, int ng, int t) {
   const int64_t off = (int64_t)u * 64;
   if (kWide) {
     const uint4 a = ld_stream_u4(wA + off), b = ld_stream_u4(wB + off);
@@ -137,7 +146,14 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
     U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
   }
-  if (kNF4) {
+  if (kNF4 && kWide) {
+    // the lane's 32 codes (bytes 16t .. 16t + 15 of the unit) lie in block
+    // 2u + t / 2 of rows g and g + 8
+    const float* am = static_cast<const float*>(p.scales);
+    const int blk = 2 * u + (t >> 1);
+    U.prm[0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + blk));
+    U.prm[1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + blk));
+  } else if (kNF4) {
     const float* am = static_cast<const float*>(p.scales);
     const float2 aA =
         __ldg(reinterpret_cast<const float2*>(am + (int64_t)nA * (p.K / 64) + 2 * u));
@@ -189,7 +205,48 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
                                              const float* xsum, const uint32_t* lut_lane, int g,
                                              int t, float (&acc)[NT][4]) {
   constexpr int kTok = 8 * NT;
-  if (kWide) {
+  if (kNF4 && kWide) {
+    // The lane's 16 bytes of rows g and g + 8 hold codes k = 32t .. 32t + 31,
+    // all in one absmax block, applied to the A operand before the MMA (one
+    // fp16 multiply per code pair). Step (w, hh) uses bytes 4w + 2hh and
+    // 4w + 2hh + 1: codes 32t + 8w + 4hh + {0..3}; x is staged in natural
+    // order, so that chunk 4t + w of each token holds exactly those x.
+    const uint32_t amA = pack_f16x2(__uint_as_float(U.prm[0]), __uint_as_float(U.prm[0]));
+    const uint32_t amB = pack_f16x2(__uint_as_float(U.prm[1]), __uint_as_float(U.prm[1]));
+    float cp[2][NT][4];
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+      for (int a = 0; a < NT; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) cp[c][a][r] = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      uint4 X[NT];
+#pragma unroll
+      for (int a = 0; a < NT; ++a) {
+        const int tok = g + 8 * a;
+        const int pc = (16 * lu + 4 * t + w) ^ (t & 2) ^ (tok & 1);
+        X[a] = *reinterpret_cast<const uint4*>(xs + (size_t)tok * kc + pc * 8);
+      }
+      const uint32_t WA = U.w[w], WB = U.w[4 + w];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int sh0 = 16 * hh, sh1 = sh0 + 8;
+        const uint32_t a0 = f16x2_mul(lut_lane[((WA >> sh0) & 0xFFu) * 32], amA);
+        const uint32_t a1 = f16x2_mul(lut_lane[((WB >> sh0) & 0xFFu) * 32], amB);
+        const uint32_t a2 = f16x2_mul(lut_lane[((WA >> sh1) & 0xFFu) * 32], amA);
+        const uint32_t a3 = f16x2_mul(lut_lane[((WB >> sh1) & 0xFFu) * 32], amB);
+#pragma unroll
+        for (int a = 0; a < NT; ++a)
+          mma16816_f16(cp[hh][a], a0, a1, a2, a3, hh ? X[a].z : X[a].x, hh ? X[a].w : X[a].y);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < NT; ++a)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) acc[a][r] += cp[0][a][r] + cp[1][a][r];
+  } else if (kWide) {
     // two accumulator chains (even and odd k-steps) halve the MMA dependency chain
     float cp[2][NT][4];
 #pragma unroll
@@ -338,7 +395,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   for (int c = tid; c < p.M * kchunks; c += blockDim.x) {
     const int gt = div_by_magic(c, cmagic), cl = c - gt * kchunks;
     int pc = cl ^ (gt & 1);
-    if (!kNF4 && kWide) pc ^= (cl >> 2) & 2;
+    if (kWide) pc ^= (cl >> 2) & 2;
     cp_async16(xs + (size_t)gt * kc + pc * 8, p.x + (size_t)gt * p.K + k0 + cl * 8);
   }
 
@@ -350,7 +407,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   if (active) {
 #pragma unroll
     for (int i = 0; i < D; ++i)
-      if (u0 + i < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng);
+      if (u0 + i < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng, t);
   }
   cp_async_wait_all();
   __syncthreads();
@@ -444,7 +501,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
         const int u = ub + i;
         if (u < u1) {
           compute_unit<NT, kNF4, kWide>(ring[i], u - u0, xs, kc, xsum, lut_lane, g, t, acc);
-          if (u + D < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u + D, nA, nB, p, ng);
+          if (u + D < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u + D, nA, nB, p, ng, t);
         }
       }
     }
@@ -496,7 +553,7 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   a.kc = 0;
   a.gmagic = div_magic((uint32_t)(group / 64));
   if (fmt == WQ_FMT_NF4)
-    return NT == 1 ? launch_t<1, true, false>(a, st) : launch_t<2, true, false>(a, st);
+    return NT == 1 ? launch_t<1, true, true>(a, st) : launch_t<2, true, true>(a, st);
   if (group % 128 == 0)
     return NT == 1 ? launch_t<1, false, true>(a, st) : launch_t<2, false, true>(a, st);
   return NT == 1 ? launch_t<1, false, false>(a, st) : launch_t<2, false, false>(a, st);

@@ -2,10 +2,12 @@
 
 All decode workloads (Llama-2-7B linear shapes, M = 1, 4, 8, 16, INT4 g128 and
 NF4 b64, 1% outlier channels x20) and the tiny INT4 g64 case are run at full
-size, every output compared. INT4 dequantizes exactly inside the kernel and
-NF4 multiplies fp16 code values (11 significant bits) by exactly scaled fp16
-activations, so besides the product tolerance every output must lie within
-one bf16 rounding of the exact product.
+size, every output compared. INT4 dequantizes exactly inside the kernel, so
+besides the product tolerance every INT4 output must lie within one bf16
+rounding of the exact product. NF4 multiplies exactly scaled fp16 activations
+by fp16 weights: the code value, the block's absmax and their product each
+round once to fp16, as in the fused GEMM, so its element bound carries the
+same 3e-3 RMS slack as the GEMM's NF4 cases.
 """
 
 import numpy as np
@@ -49,7 +51,9 @@ def _run_nf4(wq, m, n, k, outliers=(0.01, 20.0), seed=0):
     y = wq.wq_w4a16_gemv(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None)
     torch.cuda.synchronize()
     y_ref = products.w4a16_nf4(helpers.x_f32(x), codes, absmax, k)
-    helpers.check_within_bf16_rounding(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k), slack=1e-3)
+    # three fp16 roundings per weight (code, absmax, product; 2^-11 relative
+    # each, about 2^-10.2 together) spread over the K-term sum
+    helpers.check_within_bf16_rounding(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k), slack=3e-3)
     return helpers.check_product(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k))
 
 

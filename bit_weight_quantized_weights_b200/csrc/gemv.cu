@@ -200,10 +200,12 @@ __device__ __forceinline__ void int4_post(float (&acc)[4], const float (&cp)[4],
 
 // The products of one 128-k unit, accumulated into acc (see the data
 // placement above for the shared-memory layouts read here).
+// Token rows of xs above `mlast` are not staged; their lanes read row mlast
+// instead (those MMA columns never reach an output).
 template <int NT, bool kNF4, bool kWide>
 __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16_t* xs, int kc,
                                              const float* xsum, const uint32_t* lut_lane, int g,
-                                             int t, float (&acc)[NT][4]) {
+                                             int t, float (&acc)[NT][4], int mlast = 15) {
   constexpr int kTok = 8 * NT;
   if (kNF4 && kWide) {
     // The lane's 16 bytes of rows g and g + 8 hold codes k = 32t .. 32t + 31,
@@ -225,7 +227,7 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
       uint4 X[NT];
 #pragma unroll
       for (int a = 0; a < NT; ++a) {
-        const int tok = g + 8 * a;
+        const int tok = min(g + 8 * a, mlast);
         const int pc = (16 * lu + 4 * t + w) ^ (t & 2) ^ (tok & 1);
         X[a] = *reinterpret_cast<const uint4*>(xs + (size_t)tok * kc + pc * 8);
       }
@@ -260,7 +262,7 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
       uint4 X[NT];
 #pragma unroll
       for (int a = 0; a < NT; ++a) {
-        const int tok = g + 8 * a;
+        const int tok = min(g + 8 * a, mlast);
         const int pc = (16 * lu + 4 * t + j) ^ (t & 2) ^ (tok & 1);
         X[a] = *reinterpret_cast<const uint4*>(xs + (size_t)tok * kc + pc * 8);
       }

@@ -135,6 +135,7 @@ struct Unit {
 template <bool kNF4, bool kWide>
 __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint8_t* wB, int u,
                                           int nA, int nB, const GemvArgs& p, int ng, int t) {
+  static_assert(kWide || !kNF4, "NF4 uses the 16-byte layout");
   const int64_t off = (int64_t)u * 64;
   if (kWide) {
     const uint4 a = ld_stream_u4(wA + off), b = ld_stream_u4(wB + off);
@@ -146,23 +147,13 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
     U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
   }
-  if (kNF4 && kWide) {
+  if (kNF4) {
     // the lane's 32 codes (bytes 16t .. 16t + 15 of the unit) lie in block
     // 2u + t / 2 of rows g and g + 8
     const float* am = static_cast<const float*>(p.scales);
     const int blk = 2 * u + (t >> 1);
     U.prm[0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + blk));
     U.prm[1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + blk));
-  } else if (kNF4) {
-    const float* am = static_cast<const float*>(p.scales);
-    const float2 aA =
-        __ldg(reinterpret_cast<const float2*>(am + (int64_t)nA * (p.K / 64) + 2 * u));
-    const float2 aB =
-        __ldg(reinterpret_cast<const float2*>(am + (int64_t)nB * (p.K / 64) + 2 * u));
-    U.prm[0] = __float_as_uint(aA.x);
-    U.prm[1] = __float_as_uint(aB.x);
-    U.prm[2] = __float_as_uint(aA.y);
-    U.prm[3] = __float_as_uint(aB.y);
   } else {
     const unsigned short* s16 = reinterpret_cast<const unsigned short*>(p.scales);
     const unsigned short* z16 = reinterpret_cast<const unsigned short*>(p.zeros);
@@ -306,28 +297,13 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
       for (int ks = 0; ks < 4; ++ks) {
         const int jw = ks >> 1, hh = ks & 1;
         const uint32_t WA = U.w[2 * h + jw], WB = U.w[4 + 2 * h + jw];
-        uint32_t a0, a1, a2, a3;
-        if (!kNF4) {
-          a0 = int4_pair(WA, 2 * hh);
-          a1 = int4_pair(WB, 2 * hh);
-          a2 = int4_pair(WA, 2 * hh + 1);
-          a3 = int4_pair(WB, 2 * hh + 1);
-        } else {
-          // bytes 2hh and 2hh + 1 of the word: elements (2i, 2i + 1) per byte
-          const int sh0 = 16 * hh, sh1 = sh0 + 8;
-          a0 = lut_lane[((WA >> sh0) & 0xFFu) * 32];
-          a1 = lut_lane[((WB >> sh0) & 0xFFu) * 32];
-          a2 = lut_lane[((WA >> sh1) & 0xFFu) * 32];
-          a3 = lut_lane[((WB >> sh1) & 0xFFu) * 32];
-        }
+        const uint32_t a0 = int4_pair(WA, 2 * hh), a1 = int4_pair(WB, 2 * hh);
+        const uint32_t a2 = int4_pair(WA, 2 * hh + 1), a3 = int4_pair(WB, 2 * hh + 1);
 #pragma unroll
         for (int a = 0; a < NT; ++a) {
           const uint32_t b0 = hh ? X[a][jw].z : X[a][jw].x;
           const uint32_t b1 = hh ? X[a][jw].w : X[a][jw].y;
-          if (!kNF4)
-            mma16816(cp[hh][a], a0, a1, a2, a3, b0, b1);
-          else
-            mma16816_f16(cp[hh][a], a0, a1, a2, a3, b0, b1);
+          mma16816(cp[hh][a], a0, a1, a2, a3, b0, b1);
         }
       }
 #pragma unroll
@@ -335,16 +311,9 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
         float cs[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) cs[r] = cp[0][a][r] + cp[1][a][r];
-        if (kNF4) {
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-            acc[a][r] = fmaf(__uint_as_float(U.prm[2 * h + (r >> 1)]), cs[r], acc[a][r]);
-        } else {
-          const float2 sx =
-              *reinterpret_cast<const float2*>(xsum + (2 * lu + h) * kTok + 8 * a + 2 * t);
-          int4_post(acc[a], cs, U.prm[2 * h], U.prm[2 * h + 1], U.zz[2 * h], U.zz[2 * h + 1],
-                    sx);
-        }
+        const float2 sx =
+            *reinterpret_cast<const float2*>(xsum + (2 * lu + h) * kTok + 8 * a + 2 * t);
+        int4_post(acc[a], cs, U.prm[2 * h], U.prm[2 * h + 1], U.zz[2 * h], U.zz[2 * h + 1], sx);
       }
     }
   }

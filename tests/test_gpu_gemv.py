@@ -95,6 +95,47 @@ def test_gemv_ragged_nf4(wq, m, n, k):
     _run_nf4(wq, m, n, k, seed=m)
 
 
+def _at_16_bytes(t):
+    """A copy of t whose data starts 16 bytes past a 256-byte boundary: aligned
+    as the ABI requires, but not to 32 or 64 bytes."""
+    flat = t.contiguous().view(-1).view(torch.uint8)
+    buf = torch.empty(flat.numel() + 256, dtype=torch.uint8, device=t.device)
+    off = (16 - buf.data_ptr()) % 256
+    out = buf[off:off + flat.numel()]
+    out.copy_(flat)
+    return out.view(t.dtype).view(t.shape)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "nf4"])
+def test_gemv_operands_only_16_byte_aligned(wq, fmt):
+    """Every operand 16 bytes past a 256-byte boundary: the kernel must not
+    derive a lane's position (or its NF4 absmax block) from address bits
+    above the ABI's 16-byte alignment."""
+    m, n, k = 5, 1040, 640
+    x = _x(m, k, 3, None)
+    xd = _at_16_bytes(x.cuda())
+    y = _at_16_bytes(torch.zeros(m, n, dtype=torch.bfloat16, device="cuda"))
+    assert xd.data_ptr() % 32 == 16 and y.data_ptr() % 32 == 16
+    if fmt == "int4":
+        q, s, z, qweight = helpers.int4_packed(n, k, 128, seed=4)
+        qw, sc, zr = (_at_16_bytes(t) for t in helpers.to_dev_int4(s, z, qweight))
+        assert qw.data_ptr() % 32 == 16
+        wq.wq_w4a16_gemv(xd, n, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr, out=y)
+        y_ref = products.w4a16_int4(helpers.x_f32(x), q, s, z, 128)
+        slack = 1e-4
+    else:
+        codes, absmax, packed = helpers.nf4_packed(n, k, seed=4)
+        cw, am = (_at_16_bytes(t) for t in helpers.to_dev_nf4(absmax, packed))
+        assert cw.data_ptr() % 32 == 16 and am.data_ptr() % 32 == 16
+        wq.wq_w4a16_gemv(xd, n, wq.WQ_FMT_NF4, 64, cw, am, None, out=y)
+        y_ref = products.w4a16_nf4(helpers.x_f32(x), codes, absmax, k)
+        slack = 3e-3
+    torch.cuda.synchronize()
+    helpers.check_product(y, y_ref, "%s gemv, 16-byte aligned operands" % fmt)
+    helpers.check_within_bf16_rounding(y, y_ref, "%s gemv, 16-byte aligned operands" % fmt,
+                                       slack=slack)
+
+
 def test_gemv_empty_is_noop(wq):
     x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
     y = torch.full((0, 64), 7.0, dtype=torch.bfloat16, device="cuda")

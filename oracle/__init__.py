@@ -22,6 +22,8 @@ Modules
 ``products``   the W4A16 product y = x . dequant(W_q)^T in fp64.
 ``msd``        Multi-Scale Dequant activation decomposition and the
                decomposed integer product.
+``decdec``     salient-channel residual correction: the residual matrix,
+               the per-step channel selection and the corrected product.
 
 Parity pins: every function is pinned by ``tests/test_oracle_*.py`` against
 facts that do not come from the oracle itself (hand-computed golden groups,
@@ -32,4 +34,4 @@ dequantize-then-multiply baseline prints no numbers; it is measured and
 reported, never asserted.
 """
 
-from . import numerics, formats, products, msd  # noqa: F401
+from . import numerics, formats, products, msd, decdec  # noqa: F401

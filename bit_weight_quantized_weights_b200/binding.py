@@ -38,6 +38,7 @@ EXPORTED = [
     "wq_quantize_pack", "wq_unpack", "wq_nf4_dequant", "wq_int4_dequant",
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
+    "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected",
 ]
 
 
@@ -74,6 +75,10 @@ def _load():
                                ctypes.c_int),
         "wq_device_error": ([P, ctypes.c_int, ctypes.POINTER(U32)], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
+        "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
+        "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
+        "wq_w4a16_gemv_corrected": ([P, I64, I64, I64, ctypes.c_int, I32, P, P, P, P, P, I32, P,
+                                     P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -222,6 +227,45 @@ def wq_w4a16_gemv(x, n, fmt, group, qweight, scales, zeros, out=None, stream=Non
     """Decode GEMV: x bf16 [M<=16, K] -> y bf16 [M, N]."""
     return _product(lib.wq_w4a16_gemv, "wq_w4a16_gemv", x, n, fmt, group, qweight, scales, zeros,
                     out, None, stream)
+
+
+def wq_residual(fmt, w, group, qweight, scales, zeros, out=None, stream=None):
+    """R^T = fp16(W - dequant(W_q)) as fp16 [K, N] from fp32 W [N, K]."""
+    _cuda(w, torch.float32, "W")
+    n, k = w.shape
+    if out is None:
+        out = torch.empty(k, n, dtype=torch.float16, device=w.device)
+    _cuda(out, torch.float16, "residual_t")
+    _check(lib.wq_residual(fmt, _ptr(w), n, k, group, _ptr(qweight), _ptr(scales), _ptr(zeros),
+                           _ptr(out), _stream(stream)), "wq_residual")
+    return out
+
+
+def wq_select_salient(x, k, out=None, stream=None):
+    """The k salient channels of bf16 x [M, K] as int32 [k], increasing."""
+    _cuda(x, torch.bfloat16, "x")
+    m, kk = x.shape
+    if out is None:
+        out = torch.empty(max(k, 0), dtype=torch.int32, device=x.device)
+    _cuda(out, torch.int32, "idx")
+    _check(lib.wq_select_salient(_ptr(x), m, kk, k, _ptr(out), _stream(stream)),
+           "wq_select_salient")
+    return out
+
+
+def wq_w4a16_gemv_corrected(x, n, fmt, group, qweight, scales, zeros, residual_t, idx, out=None,
+                            stream=None):
+    """Decode GEMV plus the residuals of the channels idx (int32 [k])."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _cuda(out, torch.bfloat16, "y")
+    nsel = 0 if idx is None else idx.numel()
+    _check(lib.wq_w4a16_gemv_corrected(_ptr(x), m, n, k, fmt, group, _ptr(qweight), _ptr(scales),
+                                       _ptr(zeros), _ptr(residual_t), _ptr(idx), nsel, _ptr(out),
+                                       _stream(stream)), "wq_w4a16_gemv_corrected")
+    return out
 
 
 def gemm_workspace(m, n, k, group, device="cuda"):

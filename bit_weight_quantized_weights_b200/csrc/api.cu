@@ -13,7 +13,12 @@ wq_status launch_nf4_dequant(const uint8_t*, const float*, int64_t, void*, wq_dt
 wq_status launch_int4_dequant(const uint32_t*, const void*, const void*, int64_t, int64_t, int32_t,
                               void*, wq_dtype, cudaStream_t);
 wq_status launch_gemv(const void*, int64_t, int64_t, int64_t, wq_format, int32_t, const void*,
-                      const void*, const void*, void*, cudaStream_t);
+                      const void*, const void*, void*, cudaStream_t,
+                      const void* residual_t = nullptr, const int32_t* idx = nullptr,
+                      int32_t k = 0);
+wq_status launch_residual(wq_format, const float*, int64_t, int64_t, int32_t, const void*,
+                          const void*, const void*, void*, cudaStream_t);
+wq_status launch_select_salient(const void*, int64_t, int64_t, int32_t, int32_t*, cudaStream_t);
 wq_status launch_gemm(const void*, int64_t, int64_t, int64_t, wq_format, int32_t, const void*,
                       const void*, const void*, void*, void*, cudaStream_t);
 size_t gemm_workspace_bytes(int64_t M, int64_t K);
@@ -184,6 +189,53 @@ wq_status wq_w4a16_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_forma
   if (M == 0 || N == 0) return WQ_OK;
   return guarded([&] {
     return launch_gemv(x, M, N, K, fmt, group, qweight, scales, zeros, y, as_stream(stream));
+  });
+}
+
+wq_status wq_residual(wq_format fmt, const float* W, int64_t N, int64_t K, int32_t group,
+                      const void* qweight, const void* scales, const void* zeros,
+                      void* residual_t, void* stream) {
+  wq_status s = check_format(fmt, N, K, group);
+  if (s != WQ_OK) return s;
+  if (N == 0) return WQ_OK;
+  if (!W || !qweight || !scales || !residual_t) return WQ_ERR_INVALID_ARG;
+  if (fmt == WQ_FMT_INT4_ASYM && !zeros) return WQ_ERR_INVALID_ARG;
+  if (fmt == WQ_FMT_NF4 && zeros) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({W, qweight, scales, zeros, residual_t})) return WQ_ERR_ALIGNMENT;
+  if (N > INT32_MAX || K > INT32_MAX || (N + 31) / 32 > 65535) return WQ_ERR_UNSUPPORTED;
+  return guarded([&] {
+    return launch_residual(fmt, W, N, K, group, qweight, scales, zeros, residual_t,
+                           as_stream(stream));
+  });
+}
+
+wq_status wq_select_salient(const void* x, int64_t M, int64_t K, int32_t k, int32_t* idx,
+                            void* stream) {
+  if (M <= 0 || K <= 0 || k < 0 || k > K) return WQ_ERR_INVALID_ARG;
+  if (k == 0) return WQ_OK;
+  if (!x || !idx) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({x, idx})) return WQ_ERR_ALIGNMENT;
+  if (K > 65536 || M > INT32_MAX) return WQ_ERR_UNSUPPORTED;
+  return guarded([&] { return launch_select_salient(x, M, K, k, idx, as_stream(stream)); });
+}
+
+wq_status wq_w4a16_gemv_corrected(const void* x, int64_t M, int64_t N, int64_t K, wq_format fmt,
+                                  int32_t group, const void* qweight, const void* scales,
+                                  const void* zeros, const void* residual_t, const int32_t* idx,
+                                  int32_t k, void* y, void* stream) {
+  wq_status s = check_product(x, M, N, K, fmt, group, qweight, scales, zeros, y);
+  if (s != WQ_OK) return s;
+  if (k < 0 || k > K) return WQ_ERR_INVALID_ARG;
+  if (M > 16) return WQ_ERR_UNSUPPORTED;
+  if (N % 16 != 0) return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (k > 0) {
+    if (!residual_t || !idx) return WQ_ERR_INVALID_ARG;
+    if (!all_aligned({residual_t, idx})) return WQ_ERR_ALIGNMENT;
+  }
+  return guarded([&] {
+    return launch_gemv(x, M, N, K, fmt, group, qweight, scales, zeros, y, as_stream(stream),
+                       residual_t, idx, k);
   });
 }
 

@@ -1,0 +1,198 @@
+// Salient-channel residual correction for the decode GEMV: the residual
+// matrix and the per-step selection of salient channels. The correction itself
+// is added inside the GEMV's epilogue (gemv.cu, splitk_common.cuh).
+//
+// Source: "DecDEC: A Systems Approach to Advancing Low-Bit LLM Quantization",
+// Abstract. The residual is the difference between the full-precision and the
+// quantized weights. At every decoding step the salient channels, which the
+// activation outliers mark, are found from the step's activations, and only
+// their residuals are fetched to correct the quantization error.
+//
+// Readings, the same in the CPU oracle:
+// * R = fp16(W - W_hat): W_hat is (q - z) * s (exact in fp32) for INT4 and
+//   fp32(codebook[q] * absmax) for NF4, the subtraction is one fp32 rounding
+//   and the result one fp16 rounding. It is stored channel-major, R^T [K, N],
+//   so that a channel's residuals are one contiguous row.
+// * Salient channels: the k largest max_m |x[m, c]|, compared as the bf16 bit
+//   pattern with the sign cleared (NaN ranks above +inf), ties to the lower
+//   channel; the k indices are written in increasing order.
+// The host-memory placement of the residuals on the page's laptop GPU is not
+// reproduced: R^T lives in device memory and only the k selected rows are read.
+#include "common.cuh"
+
+namespace wq {
+namespace {
+
+// One 32 x 32 tile of R^T per CTA (32 x 8 threads): computed in [n][k] order
+// from the row-major weights, written transposed through shared memory.
+template <bool kNF4>
+__global__ void __launch_bounds__(256) residual_kernel(
+    const float* __restrict__ W, int N, int K, int G, const uint32_t* __restrict__ qw,
+    const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
+    const __half* __restrict__ zeros, const float* __restrict__ absmax, Nf4Table tab,
+    __half* __restrict__ rt) {
+  __shared__ __half tile[32][33];
+  const int k0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int i = ty; i < 32; i += 8) {
+    const int n = n0 + i, k = k0 + tx;
+    float r = 0.0f;
+    if (n < N && k < K) {
+      const int64_t e = (int64_t)n * K + k;
+      float wh;
+      if (kNF4) {
+        const uint8_t b = codes[e >> 1];
+        const int q = (e & 1) ? (b & 0xF) : (b >> 4);  // element 2j: high nibble
+        wh = __fmul_rn(tab.v[q], absmax[e >> 6]);      // one fp32 rounding
+      } else {
+        const uint32_t word = qw[(int64_t)n * (K / 8) + (k >> 3)];
+        const int q = (int)((word >> (4 * (k & 7))) & 0xFu);
+        const int64_t gi = (int64_t)n * (K / G) + k / G;
+        wh = __fmul_rn((float)q - __half2float(zeros[gi]), __half2float(scales[gi]));  // exact
+      }
+      r = __fsub_rn(W[e], wh);
+    }
+    tile[i][tx] = __float2half_rn(r);
+  }
+  __syncthreads();
+  for (int i = ty; i < 32; i += 8) {
+    const int k = k0 + i, n = n0 + tx;
+    if (n < N && k < K) rt[(int64_t)k * N + n] = tile[tx][i];
+  }
+}
+
+constexpr int kSelThreads = 1024;
+
+// Exclusive prefix sum over the CTA's threads; *total gets the sum.
+__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* warp_sums,
+                                                         unsigned* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += t;
+  }
+  if (lane == 31) warp_sums[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned w = warp_sums[lane];
+    unsigned wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned t = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += t;
+    }
+    warp_sums[lane] = wi - w;  // exclusive over warps
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const unsigned r = warp_sums[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+// Bin b of a histogram scanned from the top: the bin holding the want-th
+// largest key, and how many keys lie in higher bins.
+__device__ __forceinline__ void find_bin(const unsigned* hist, int nbins, unsigned want,
+                                         unsigned* bin, unsigned* above) {
+  unsigned acc = 0;
+  for (int b = nbins - 1; b >= 0; --b) {
+    if (acc + hist[b] >= want) {
+      *bin = (unsigned)b;
+      *above = acc;
+      return;
+    }
+    acc += hist[b];
+  }
+  *bin = 0;
+  *above = acc;
+}
+
+// The k salient channels of x [M, K] (1 <= k <= K), one CTA: 15-bit keys in
+// shared memory, a two-pass radix select of the k-th largest key T (high 8
+// bits, then low 7), then an order-preserving compaction that takes every key
+// above T and the lowest-index keys equal to T.
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __restrict__ x, int M,
+                                                             int K, int k, int* __restrict__ idx) {
+  extern __shared__ uint16_t keys[];
+  __shared__ unsigned hist[256];
+  __shared__ unsigned warp_sums[32];
+  __shared__ unsigned s_bin, s_above, s_T, s_need, s_total;
+  const int tid = threadIdx.x;
+  for (int c = tid; c < K; c += kSelThreads) {
+    unsigned best = 0;
+    for (int m = 0; m < M; ++m) best = max(best, (unsigned)(x[(size_t)m * K + c] & 0x7FFFu));
+    keys[c] = (uint16_t)best;
+  }
+  if (tid < 256) hist[tid] = 0;
+  __syncthreads();
+  for (int c = tid; c < K; c += kSelThreads) atomicAdd(&hist[keys[c] >> 7], 1u);
+  __syncthreads();
+  if (tid == 0) find_bin(hist, 256, (unsigned)k, &s_bin, &s_above);
+  __syncthreads();
+  const unsigned hi = s_bin, above_hi = s_above;
+  if (tid < 256) hist[tid] = 0;
+  __syncthreads();
+  for (int c = tid; c < K; c += kSelThreads)
+    if ((unsigned)(keys[c] >> 7) == hi) atomicAdd(&hist[keys[c] & 0x7F], 1u);
+  __syncthreads();
+  if (tid == 0) {
+    unsigned lo, above_lo;
+    find_bin(hist, 128, (unsigned)k - above_hi, &lo, &above_lo);
+    s_T = (hi << 7) | lo;
+    s_need = (unsigned)k - above_hi - above_lo;  // keys equal to T to take, >= 1
+  }
+  __syncthreads();
+  const unsigned T = s_T, need = s_need;
+  // this thread's contiguous range of channels
+  const int per = (K + kSelThreads - 1) / kSelThreads;
+  const int c0 = min(K, tid * per), c1 = min(K, c0 + per);
+  unsigned n_gt = 0, n_eq = 0;
+  for (int c = c0; c < c1; ++c) {
+    n_gt += keys[c] > T;
+    n_eq += keys[c] == T;
+  }
+  const unsigned eq_before = block_exclusive_scan(n_eq, warp_sums, &s_total);
+  const unsigned take_eq = eq_before >= need ? 0u : min(n_eq, need - eq_before);
+  unsigned pos = block_exclusive_scan(n_gt + take_eq, warp_sums, &s_total);
+  unsigned taken = 0;
+  for (int c = c0; c < c1; ++c) {
+    const unsigned key = keys[c];
+    if (key > T || (key == T && taken < take_eq)) {
+      idx[pos++] = c;
+      if (key == T) ++taken;
+    }
+  }
+}
+
+}  // namespace
+
+wq_status launch_residual(wq_format fmt, const float* W, int64_t N, int64_t K, int32_t G,
+                          const void* qweight, const void* scales, const void* zeros, void* rt,
+                          cudaStream_t st) {
+  const dim3 grid((unsigned)((K + 31) / 32), (unsigned)((N + 31) / 32));
+  if (fmt == WQ_FMT_NF4)
+    residual_kernel<true><<<grid, 256, 0, st>>>(
+        W, (int)N, (int)K, G, nullptr, static_cast<const uint8_t*>(qweight), nullptr, nullptr,
+        static_cast<const float*>(scales), nf4_table(), static_cast<__half*>(rt));
+  else
+    residual_kernel<false><<<grid, 256, 0, st>>>(
+        W, (int)N, (int)K, G, static_cast<const uint32_t*>(qweight), nullptr,
+        static_cast<const __half*>(scales), static_cast<const __half*>(zeros), nullptr,
+        nf4_table(), static_cast<__half*>(rt));
+  return launch_status();
+}
+
+wq_status launch_select_salient(const void* x, int64_t M, int64_t K, int32_t k, int32_t* idx,
+                                cudaStream_t st) {
+  const size_t smem = (size_t)K * 2;
+  if (cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  select_kernel<<<1, kSelThreads, smem, st>>>(static_cast<const uint16_t*>(x), (int)M, (int)K, k,
+                                              idx);
+  return launch_status();
+}
+
+}  // namespace wq

@@ -82,6 +82,7 @@ struct GemvArgs {
   int S;                  // cluster size along K
   int kc;                 // shared-memory K-chunk length (max over ranks)
   uint32_t gmagic;        // h / (G / 64) == umulhi(h, gmagic) for 64-wide part h; 0 if G == 64
+  Residual rc;            // salient-channel correction (k == 0: none)
 };
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -479,7 +480,8 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   }
 
   // ---- cluster split-K reduction (through distributed shared memory) -----
-  reduce_and_store<NT>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N, p.y);
+  reduce_and_store<NT>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N, p.y,
+                       p.rc);
 }
 
 template <int NT, bool kNF4>
@@ -507,7 +509,7 @@ wq_status launch_t(GemvArgs a, cudaStream_t st) {
 
 wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format fmt, int32_t group,
                       const void* qweight, const void* scales, const void* zeros, void* y,
-                      cudaStream_t st) {
+                      cudaStream_t st, const void* residual_t, const int32_t* idx, int32_t k) {
   const int NT = M <= 8 ? 1 : 2;
   GemvArgs a;
   a.x = static_cast<const uint16_t*>(x);
@@ -523,6 +525,13 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   a.S = 1;
   a.kc = 0;
   a.gmagic = div_magic((uint32_t)(group / 64));
+  if (k > 0) {
+    a.rc.rt = static_cast<const uint16_t*>(residual_t);
+    a.rc.idx = idx;
+    a.rc.x = a.x;
+    a.rc.k = k;
+    a.rc.K = (int)K;
+  }
   if (fmt == WQ_FMT_NF4)
     return NT == 1 ? launch_t<1, true, true>(a, st) : launch_t<2, true, true>(a, st);
   if (group % 128 == 0)

@@ -57,6 +57,32 @@ __host__ __device__ __forceinline__ size_t red_bytes(int S) {
   return (size_t)S * ((kRowsPerCta + S - 1) / S) * 16 * 4;
 }
 
+// Optional salient-channel residual correction ("DecDEC: A Systems Approach
+// to Advancing Low-Bit LLM Quantization", Abstract), added to an output in
+// fp32 before its bf16 rounding: y[m, n] += sum_j x[m, idx[j]] * R^T[idx[j], n]
+// with R^T fp16 [K, N] (a selected channel's residuals are one contiguous
+// row, so the owners' loads of consecutive n coalesce). k == 0 adds nothing.
+struct Residual {
+  const uint16_t* rt = nullptr;  // fp16 bits of R^T [K, N]
+  const int* idx = nullptr;      // k channel indices
+  const uint16_t* x = nullptr;   // bf16 bits of x [M, K]
+  int k = 0;
+  int K = 0;
+};
+
+__device__ __forceinline__ float residual_term(const Residual& rc, int tok, int n, int N) {
+  float v = 0.0f;
+  const uint16_t* xr = rc.x + (size_t)tok * rc.K;
+#pragma unroll 4
+  for (int j = 0; j < rc.k; ++j) {
+    const int c = __ldg(rc.idx + j);
+    const float xv = __uint_as_float((uint32_t)__ldg(xr + c) << 16);
+    const float r = __half2float(__ushort_as_half(__ldg(rc.rt + (size_t)c * N + n)));
+    v = fmaf(xv, r, v);
+  }
+  return v;
+}
+
 // The cluster split-K reduction. acc[a][r] of this lane holds rows
 // warp*16 + g + 8 (r >> 1), tokens 8a + 2t + (r & 1) (the m16n8 accumulator
 // layout); tok_scale (optional, per token) multiplies it first. Each CTA
@@ -64,11 +90,13 @@ __host__ __device__ __forceinline__ size_t red_bytes(int S) {
 // (red[src rank][local row][token] there), one cluster barrier, then each
 // owner sums its rows in rank order and writes them once as bf16. Remote
 // stores need no round trip, and no CTA touches another's shared memory after
-// the barrier. All threads of the CTA must call this.
+// the barrier. The owners add the residual correction rc, if any, before the
+// rounding. All threads of the CTA must call this.
 template <int NT>
 __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], const float* tok_scale,
                                                  float* red, int S, int rank, int row_tile, int M,
-                                                 int N, uint16_t* y) {
+                                                 int N, uint16_t* y,
+                                                 const Residual& rc = Residual()) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int rows_max = (kRowsPerCta + S - 1) / S;
@@ -107,7 +135,10 @@ __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], cons
     const int n = row_tile + r_begin + lr;
     float v = 0.0f;
     for (int q = 0; q < S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
-    if (n < N) y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+    if (n < N) {
+      if (rc.k > 0) v += residual_term(rc, tok, n, N);
+      y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+    }
   }
 }
 

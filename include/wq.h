@@ -18,6 +18,8 @@
  *  [QLORA] "QLoRA: Efficient Finetuning of Quantized LLMs" (cited by title on
  *          "DecDEC: A Systems Approach to Advancing Low-Bit LLM Quantization"):
  *          the NF4 codebook construction.
+ *  [DECDEC] "DecDEC: A Systems Approach to Advancing Low-Bit LLM
+ *          Quantization", Abstract: salient-channel residual correction.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -156,8 +158,9 @@ wq_status wq_int4_dequant(const uint32_t* qweight, const void* scales,
  *   x bf16 [M, K] row-major; y bf16 [M, N] row-major.
  *   INT4: scales/zeros fp16 [N, K/G], G % 64 == 0, K % G == 0. The group's
  *         scale and zero are applied after the group's sum ([MIXPE]).
- *   NF4 : group == 64, scales = fp32 absmax [N*K/64], zeros NULL; the block's
- *         absmax is applied after the block's sum.
+ *   NF4 : group == 64, scales = fp32 absmax [N*K/64], zeros NULL; the code
+ *         value, the block's absmax and their product are each rounded once
+ *         to fp16 (absmax <= 65504), as in wq_w4a16_gemm.
  * Requires K % 128 == 0 and N % 16 == 0. M == 0 or N == 0 is a no-op.
  * Workspace: none needed (pass NULL, 0); split-K partials are reduced on chip
  * through thread-block-cluster shared memory.
@@ -166,6 +169,43 @@ wq_status wq_w4a16_gemv(const void* x, int64_t M, int64_t N, int64_t K,
                         wq_format fmt, int32_t group, const void* qweight,
                         const void* scales, const void* zeros, void* y,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Salient-channel residual correction ([DECDEC]: the residual matrix is the
+ * full-precision weights minus the quantized ones; the residuals of the
+ * channels that the current activations mark as outliers are added back).
+ *
+ * wq_residual: R^T = fp16(W - W_hat) as fp16 [K, N] (channel-major: one
+ *   channel's residuals are contiguous). W fp32 [N, K] row-major; the packed
+ *   weights and parameters as for wq_w4a16_gemv. W_hat is (q - z) * s (exact
+ *   in fp32) for INT4 and fp32(codebook[q] * absmax) for NF4; the subtraction
+ *   rounds once in fp32, the result once to fp16. Bit-exact with the oracle.
+ *   N == 0 is a no-op.
+ *
+ * wq_select_salient: the k salient channels of x bf16 [M, K] (M >= 1,
+ *   0 <= k <= K <= 65536): the k largest max_m |x[m, c]|, ranked by the bf16
+ *   bit pattern with the sign cleared (NaN above +inf), ties to the lower
+ *   channel. idx int32 [k] receives them in increasing order. k == 0 is a
+ *   no-op. One CTA.
+ *
+ * wq_w4a16_gemv_corrected: wq_w4a16_gemv plus, for every output,
+ *   sum_j x[m, idx[j]] * R^T[idx[j], n], added in fp32 before the bf16
+ *   rounding. idx holds k channels (0 <= k <= K; k == 0 is wq_w4a16_gemv);
+ *   residual_t is fp16 [K, N] as written by wq_residual. Only the k selected
+ *   rows of R^T are read.
+ * All three are asynchronous on `stream`; buffers are caller-owned.
+ */
+wq_status wq_residual(wq_format fmt, const float* W, int64_t N, int64_t K,
+                      int32_t group, const void* qweight, const void* scales,
+                      const void* zeros, void* residual_t, void* stream);
+wq_status wq_select_salient(const void* x, int64_t M, int64_t K, int32_t k,
+                            int32_t* idx, void* stream);
+wq_status wq_w4a16_gemv_corrected(const void* x, int64_t M, int64_t N, int64_t K,
+                                  wq_format fmt, int32_t group,
+                                  const void* qweight, const void* scales,
+                                  const void* zeros, const void* residual_t,
+                                  const int32_t* idx, int32_t k, void* y,
+                                  void* stream);
 
 /*
  * Prefill W4A16 GEMM with fused dequantization on the tensor cores ([MSD]:

@@ -98,6 +98,34 @@ def test_gemv_validation(wq):
     assert _gemv(wq, 4, 0, 4096) == wq.WQ_OK
 
 
+def test_residual_correction_validation(wq):
+    L = wq.lib
+    # wq_residual(fmt, W, N, K, group, qweight, scales, zeros, residual_t, stream)
+    assert L.wq_residual(0, A16, 64, 100, 64, A16, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_residual(1, A16, 64, 128, 64, A16, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_residual(0, A16, 64, 128, 64, A16, A16, None, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_residual(0, MIS, 64, 128, 64, A16, A16, A16, A16, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_residual(0, A16, 0, 128, 64, A16, A16, A16, A16, None) == wq.WQ_OK
+    # wq_select_salient(x, M, K, k, idx, stream)
+    assert L.wq_select_salient(A16, 1, 4096, 4097, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_select_salient(A16, 0, 4096, 8, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_select_salient(A16, 1, 4096, -1, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_select_salient(A16, 1, 4096, 0, A16, None) == wq.WQ_OK
+    assert L.wq_select_salient(A16, 1, 4096, 8, MIS, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_select_salient(A16, 1, 65552, 8, A16, None) == wq.WQ_ERR_UNSUPPORTED
+    # wq_w4a16_gemv_corrected(x, M, N, K, fmt, G, q, s, z, residual_t, idx, k, y, stream)
+    cg = L.wq_w4a16_gemv_corrected
+    assert cg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 4097, A16,
+              None) == wq.WQ_ERR_INVALID_ARG
+    assert cg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, None, A16, 8, A16,
+              None) == wq.WQ_ERR_INVALID_ARG
+    assert cg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, A16, MIS, 8, A16,
+              None) == wq.WQ_ERR_ALIGNMENT
+    assert cg(A16, 17, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 8, A16,
+              None) == wq.WQ_ERR_UNSUPPORTED
+    assert cg(A16, 0, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 8, A16, None) == wq.WQ_OK
+
+
 def test_gemm_and_msd_validation(wq):
     L = wq.lib
     assert L.wq_w4a16_gemm(A16, 512, 4096, 4096, 1, 64, A16, A16, None, A16, None, 0,

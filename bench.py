@@ -294,6 +294,88 @@ def dequant_then_cublas(wq, step, fused_ms, warmup):
             "fused_speedup": round((t_deq + t_mm) / fused_ms, 3)}
 
 
+DECDEC_SHAPE = (11008, 4096)   # decode layer (N, K), INT4 g128
+DECDEC_K = 64                   # salient channels corrected per step (1.6 % of K)
+
+
+def _graph_us(fns, reps):
+    """Median over 5 replays of a CUDA graph of `reps` launches cycling over
+    fns, in microseconds per launch (device time, CUDA events)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for f in fns:
+            f()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            fns[i % len(fns)]()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(5):
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3 / reps)
+    del g
+    return statistics.median(ts)
+
+
+def measure_decdec(wq, peaks, device, with_oracle):
+    """Salient-channel residual correction ("DecDEC: A Systems Approach to
+    Advancing Low-Bit LLM Quantization", Abstract), a widening beyond the step:
+    the decode GEMV at 11008x4096 INT4 g128 plain and with the residuals of the
+    64 most salient channels added, graph-timed over 8 rotating copies of the
+    weights and residuals (their touched bytes exceed L2). Timed outside the
+    step and not part of its value."""
+    n, k = DECDEC_SHAPE
+    copies = 8
+    sets = []
+    for c in range(copies):
+        w = torch.randn(n, k, device=device, generator=torch.Generator(device=device).manual_seed(
+            900 + c)) * 0.02
+        qw, sc, zr = wq.wq_quantize_pack(wq.WQ_FMT_INT4_ASYM, w, 128)
+        sets.append((w, qw, sc, zr, torch.empty(k, n, dtype=torch.float16, device=device)))
+    res_us = _graph_us([lambda t=t: wq.wq_residual(wq.WQ_FMT_INT4_ASYM, t[0], 128, t[1], t[2],
+                                                   t[3], out=t[4]) for t in sets], 16)
+    res_bytes = n * k * (4 + 0.5 + 2) + n * (k // 128) * 4
+    out = {"workload": "decode gemv int4-g128 %dx%d, residuals of %d salient channels"
+                       % (n, k, DECDEC_K),
+           "residual_us": round(res_us, 2),
+           "residual_gbs": round(res_bytes / (res_us * 1e-6) / 1e9, 1),
+           "residual_frac": round(res_bytes / (res_us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4)}
+    for m in (1, 16):
+        x = (torch.randn(m, k, device=device, generator=torch.Generator(device=device).manual_seed(
+            950 + m))).to(torch.bfloat16)
+        x[:, ::64] *= 20.0  # outlier channels, 1.6 % of K
+        idx = torch.empty(DECDEC_K, dtype=torch.int32, device=device)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        plain = _graph_us([lambda t=t: wq.wq_w4a16_gemv(x, n, wq.WQ_FMT_INT4_ASYM, 128, t[1], t[2],
+                                                        t[3], out=y) for t in sets], 32)
+        sel = _graph_us([lambda: wq.wq_select_salient(x, DECDEC_K, out=idx)], 32)
+        corr = _graph_us([lambda t=t: wq.wq_w4a16_gemv_corrected(
+            x, n, wq.WQ_FMT_INT4_ASYM, 128, t[1], t[2], t[3], t[4], idx, out=y)
+            for t in sets], 32)
+        gemv_bytes = n * k * 0.5 + n * (k // 128) * 4 + 2 * m * k + 2 * m * n
+        corr_bytes = DECDEC_K * n * 2
+        out["m%d" % m] = {
+            "gemv_us": round(plain, 2), "select_us": round(sel, 2),
+            "corrected_gemv_us": round(corr, 2),
+            "overhead_pct": round(100.0 * (corr + sel - plain) / plain, 1),
+            "correction_bytes": corr_bytes,
+            "corrected_gemv_gbs": round((gemv_bytes + corr_bytes) / (corr * 1e-6) / 1e9, 1)}
+    if with_oracle:
+        out["cpu_baseline"] = decdec_cpu_baseline()
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, rank, world, device):
     from bit_weight_quantized_weights_b200 import binding as wq
     peaks = load_peaks()
@@ -352,6 +434,10 @@ def run_gpu(args, rank, world, device):
         raise RuntimeError("device error word set during timing: 0x%x" % detail)
 
     comparator = dequant_then_cublas(wq, step, per_op_ms["gemm"], args.warmup) if rank == 0 else None
+    next_rows = None
+    if rank == 0 and args.next_rows:
+        next_rows = {"decdec": measure_decdec(
+            wq, peaks, device, with_oracle=world == 1 and not args.no_cpu_baseline)}
 
     ms_per_step = elapsed_ms / args.steps
     value = job_value(table, ms_per_step, world)
@@ -398,6 +484,7 @@ def run_gpu(args, rank, world, device):
                      "traffic": traffic, "peak_source": peaks["source"] + (" (HBM copy)" if d["bound"] == "hbm" else " (sustained bf16" + (")" if dom == "gemm" else " x 2 for int8)"))},
         "per_op": {k: {a: round(b, 4) for a, b in v.items()} for k, v in details.items()},
         "comparator": comparator,
+        "next_rows": next_rows,
         "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
         "clocks": clocks.summary(),
     }
@@ -543,6 +630,28 @@ class OracleSample:
                    round(f["msd_m1024"] * 1024)))
 
 
+def decdec_cpu_baseline():
+    """The oracle's salient-channel correction for one decode step on the host
+    cores: channel selection plus the k-column correction over all 11008 rows
+    (the residual matrix built once beforehand, untimed)."""
+    import numpy as np
+    from oracle import decdec
+    n, k = DECDEC_SHAPE
+    rng = np.random.default_rng(0)
+    rt = (rng.standard_normal((k, n)) * 1e-3).astype(np.float16)
+    x = rng.standard_normal((1, k)).astype(np.float32)
+    x[:, ::64] *= 20.0
+    t0 = time.perf_counter()
+    reps = 20
+    for _ in range(reps):
+        idx = decdec.select_salient(x, DECDEC_K)
+        decdec.correction(x, rt, idx)
+    t = (time.perf_counter() - t0) / reps
+    return {"kind": "oracle", "cores": oracle_cores(),
+            "sample": "select + correction of one M=1 step (%d channels x %d rows)" % (DECDEC_K, n),
+            "select_and_correction_us": round(t * 1e6, 1)}
+
+
 def oracle_cores():
     try:
         from threadpoolctl import threadpool_info
@@ -576,7 +685,7 @@ def max_over_ranks(v, world, device):
     return float(t.item())
 
 
-PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd", "msd_m16")
+PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd", "msd_m16", "decdec")
 
 
 def profile_case(case, device):
@@ -618,6 +727,19 @@ def profile_case(case, device):
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
         ws = wq.msd_workspace(m, n, k, 128, 2, device)
         fn = lambda: wq.wq_msd_gemm(x, n, 2, 128, *pw, workspace=ws, out=y)  # noqa: E731
+    elif case == "decdec":
+        # select, then the corrected GEMV (ncu -k regex:gemv_kernel captures it)
+        (n, k), m = DECDEC_SHAPE, 1
+        w = normal(n, k, std=0.02)
+        pw = wq.wq_quantize_pack(wq.WQ_FMT_INT4_ASYM, w, 128)
+        rt = wq.wq_residual(wq.WQ_FMT_INT4_ASYM, w, 128, *pw)
+        x = normal(m, k).to(torch.bfloat16)
+        idx = torch.empty(DECDEC_K, dtype=torch.int32, device=device)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+
+        def fn():
+            wq.wq_select_salient(x, DECDEC_K, out=idx)
+            wq.wq_w4a16_gemv_corrected(x, n, wq.WQ_FMT_INT4_ASYM, 128, *pw, rt, idx, out=y)
     else:
         raise SystemExit("unknown case %r (one of %s)" % (case, ", ".join(PROFILE_CASES)))
     for _ in range(2):
@@ -637,6 +759,8 @@ def main():
     ap.add_argument("--impl", default="wq", choices=["wq", "reference"])
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
+                    help="skip the widening measurements timed after the step")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as a "
                          "captured CUDA graph")

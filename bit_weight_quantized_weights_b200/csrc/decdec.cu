@@ -92,21 +92,28 @@ __device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* w
   return r;
 }
 
-// Bin b of a histogram scanned from the top: the bin holding the want-th
-// largest key, and how many keys lie in higher bins.
+// The histogram bin holding the want-th largest key, and how many keys lie in
+// higher bins: thread t takes bin nbins - 1 - t, an exclusive scan over the
+// threads counts the keys above it, and the one thread whose bin contains
+// the want-th key writes the answer. All threads call it.
 __device__ __forceinline__ void find_bin(const unsigned* hist, int nbins, unsigned want,
-                                         unsigned* bin, unsigned* above) {
-  unsigned acc = 0;
-  for (int b = nbins - 1; b >= 0; --b) {
-    if (acc + hist[b] >= want) {
-      *bin = (unsigned)b;
-      *above = acc;
-      return;
-    }
-    acc += hist[b];
+                                         unsigned* warp_sums, unsigned* total, unsigned* bin,
+                                         unsigned* above) {
+  const int t = threadIdx.x;
+  const unsigned h = t < nbins ? hist[nbins - 1 - t] : 0u;
+  const unsigned before = block_exclusive_scan(h, warp_sums, total);
+  if (t < nbins && h > 0 && before < want && want <= before + h) {
+    *bin = (unsigned)(nbins - 1 - t);
+    *above = before;
   }
-  *bin = 0;
-  *above = acc;
+  __syncthreads();
+}
+
+// hist[bin] += 1 for every calling lane, one shared-memory atomic per
+// distinct bin among the warp's active lanes.
+__device__ __forceinline__ void hist_add(unsigned* hist, unsigned bin) {
+  const unsigned peers = __match_any_sync(__activemask(), bin);
+  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], __popc(peers));
 }
 
 // The k salient channels of x [M, K] (1 <= k <= K), one CTA: 15-bit keys in
@@ -127,21 +134,19 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
   }
   if (tid < 256) hist[tid] = 0;
   __syncthreads();
-  for (int c = tid; c < K; c += kSelThreads) atomicAdd(&hist[keys[c] >> 7], 1u);
+  for (int c = tid; c < K; c += kSelThreads) hist_add(hist, keys[c] >> 7);
   __syncthreads();
-  if (tid == 0) find_bin(hist, 256, (unsigned)k, &s_bin, &s_above);
-  __syncthreads();
+  find_bin(hist, 256, (unsigned)k, warp_sums, &s_total, &s_bin, &s_above);
   const unsigned hi = s_bin, above_hi = s_above;
   if (tid < 256) hist[tid] = 0;
   __syncthreads();
   for (int c = tid; c < K; c += kSelThreads)
-    if ((unsigned)(keys[c] >> 7) == hi) atomicAdd(&hist[keys[c] & 0x7F], 1u);
+    if ((unsigned)(keys[c] >> 7) == hi) hist_add(hist, keys[c] & 0x7Fu);
   __syncthreads();
+  find_bin(hist, 128, (unsigned)k - above_hi, warp_sums, &s_total, &s_bin, &s_above);
   if (tid == 0) {
-    unsigned lo, above_lo;
-    find_bin(hist, 128, (unsigned)k - above_hi, &lo, &above_lo);
-    s_T = (hi << 7) | lo;
-    s_need = (unsigned)k - above_hi - above_lo;  // keys equal to T to take, >= 1
+    s_T = (hi << 7) | s_bin;
+    s_need = (unsigned)k - above_hi - s_above;  // keys equal to T to take, >= 1
   }
   __syncthreads();
   const unsigned T = s_T, need = s_need;

@@ -326,7 +326,7 @@ struct PrefetchDepth {
   static constexpr int value = NT == 1 ? 4 : 3;
 };
 
-template <int NT, bool kNF4, bool kWide>
+template <int NT, bool kNF4, bool kWide, bool kRes>
 __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int kTok = 8 * NT;
@@ -480,8 +480,8 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   }
 
   // ---- cluster split-K reduction (through distributed shared memory) -----
-  reduce_and_store<NT>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N, p.y,
-                       p.rc);
+  reduce_and_store<NT, kRes>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N,
+                             p.y, p.rc);
 }
 
 template <int NT, bool kNF4>
@@ -490,9 +490,9 @@ size_t gemv_smem(int kc, int S) {
          (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
 }
 
-template <int NT, bool kNF4, bool kWide>
+template <int NT, bool kNF4, bool kWide, bool kRes>
 wq_status launch_t(GemvArgs a, cudaStream_t st) {
-  auto kern = gemv_kernel<NT, kNF4, kWide>;
+  auto kern = gemv_kernel<NT, kNF4, kWide, kRes>;
   const int M = a.M;
   const Plan pl = cached_plan(reinterpret_cast<const void*>(kern), M, a.N, a.K, 0, [&] {
     return make_plan(
@@ -532,11 +532,19 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
     a.rc.k = k;
     a.rc.K = (int)K;
   }
-  if (fmt == WQ_FMT_NF4)
-    return NT == 1 ? launch_t<1, true, true>(a, st) : launch_t<2, true, true>(a, st);
-  if (group % 128 == 0)
-    return NT == 1 ? launch_t<1, false, true>(a, st) : launch_t<2, false, true>(a, st);
-  return NT == 1 ? launch_t<1, false, false>(a, st) : launch_t<2, false, false>(a, st);
+  const bool res = k > 0;
+  if (fmt == WQ_FMT_NF4) {
+    if (res) return NT == 1 ? launch_t<1, true, true, true>(a, st) : launch_t<2, true, true, true>(a, st);
+    return NT == 1 ? launch_t<1, true, true, false>(a, st) : launch_t<2, true, true, false>(a, st);
+  }
+  if (group % 128 == 0) {
+    if (res)
+      return NT == 1 ? launch_t<1, false, true, true>(a, st) : launch_t<2, false, true, true>(a, st);
+    return NT == 1 ? launch_t<1, false, true, false>(a, st) : launch_t<2, false, true, false>(a, st);
+  }
+  if (res)
+    return NT == 1 ? launch_t<1, false, false, true>(a, st) : launch_t<2, false, false, true>(a, st);
+  return NT == 1 ? launch_t<1, false, false, false>(a, st) : launch_t<2, false, false, false>(a, st);
 }
 
 wq_status read_gemv_error(bool clear, uint32_t* v) {

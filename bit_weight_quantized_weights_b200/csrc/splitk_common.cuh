@@ -70,18 +70,51 @@ struct Residual {
   int K = 0;
 };
 
-__device__ __forceinline__ float residual_term(const Residual& rc, int tok, int n, int N) {
-  float v = 0.0f;
-  const uint16_t* xr = rc.x + (size_t)tok * rc.K;
-#pragma unroll 4
-  for (int j = 0; j < rc.k; ++j) {
-    const int c = __ldg(rc.idx + j);
-    const float xv = __uint_as_float((uint32_t)__ldg(xr + c) << 16);
-    const float r = __half2float(__ushort_as_half(__ldg(rc.rt + (size_t)c * N + n)));
-    v = fmaf(xv, r, v);
+// Items (token, owned row) per thread in the owners' epilogue: nrows * M is
+// at most 128 * 16 = 2048 over 256 threads.
+constexpr int kMaxItemsPerThread = 8;
+static_assert(kRowsPerCta * 16 <= 256 * kMaxItemsPerThread, "items of a 256-thread CTA");
+
+// This thread's part of the correction of its items (token tok[it], row
+// n[it]; n < 0 for none): channels j = j0, j0 + L, j0 + 2L, ... in batches
+// of 8, the 8 indices loaded once per batch for all items, then every item's
+// x and residual loads, all independent.
+__device__ __forceinline__ void residual_parts(const Residual& rc, const int (&tok)[kMaxItemsPerThread],
+                                               const int (&n)[kMaxItemsPerThread], int N, int j0,
+                                               int L, float (&out)[kMaxItemsPerThread]) {
+  int j = j0;
+  for (; j + 7 * L < rc.k; j += 8 * L) {
+    int c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = __ldg(rc.idx + j + i * L);
+#pragma unroll
+    for (int it = 0; it < kMaxItemsPerThread; ++it) {
+      if (n[it] < 0) continue;
+      const uint16_t* xr = rc.x + (size_t)tok[it] * rc.K;
+      float xv[8], r[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        xv[i] = __uint_as_float((uint32_t)__ldg(xr + c[i]) << 16);
+        r[i] = __half2float(__ushort_as_half(__ldg(rc.rt + (size_t)c[i] * N + n[it])));
+      }
+      float v = out[it];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v = fmaf(xv[i], r[i], v);
+      out[it] = v;
+    }
   }
-  return v;
+  for (; j < rc.k; j += L) {
+    const int c = __ldg(rc.idx + j);
+#pragma unroll
+    for (int it = 0; it < kMaxItemsPerThread; ++it) {
+      if (n[it] < 0) continue;
+      out[it] = fmaf(__uint_as_float((uint32_t)__ldg(rc.x + (size_t)tok[it] * rc.K + c) << 16),
+                     __half2float(__ushort_as_half(__ldg(rc.rt + (size_t)c * N + n[it]))),
+                     out[it]);
+    }
+  }
 }
+
 
 // The cluster split-K reduction. acc[a][r] of this lane holds rows
 // warp*16 + g + 8 (r >> 1), tokens 8a + 2t + (r & 1) (the m16n8 accumulator
@@ -90,9 +123,9 @@ __device__ __forceinline__ float residual_term(const Residual& rc, int tok, int 
 // (red[src rank][local row][token] there), one cluster barrier, then each
 // owner sums its rows in rank order and writes them once as bf16. Remote
 // stores need no round trip, and no CTA touches another's shared memory after
-// the barrier. The owners add the residual correction rc, if any, before the
-// rounding. All threads of the CTA must call this.
-template <int NT>
+// the barrier. With kRes the owners add the residual correction rc (k >= 1)
+// before the rounding. All threads of the CTA must call this.
+template <int NT, bool kRes = false>
 __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], const float* tok_scale,
                                                  float* red, int S, int rank, int row_tile, int M,
                                                  int N, uint16_t* y,
@@ -121,23 +154,70 @@ __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], cons
         dst[1] = v1;
       }
     }
-  if (S > 1) {
-    cluster_sync_all();
-  } else {
-    __syncthreads();
-  }
   const int r_begin = rank_row_begin(rank, S);
   const int nrows = rank_row_begin(rank + 1, S) - r_begin;
   const int items = nrows * M;
-  for (int i = tid; i < items; i += blockDim.x) {
-    const int tok = i / nrows;
-    const int lr = i - tok * nrows;
-    const int n = row_tile + r_begin + lr;
-    float v = 0.0f;
-    for (int q = 0; q < S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
-    if (n < N) {
-      if (rc.k > 0) v += residual_term(rc, tok, n, N);
-      y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+  if constexpr (!kRes) {
+    if (S > 1) {
+      cluster_sync_all();
+    } else {
+      __syncthreads();
+    }
+    for (int i = tid; i < items; i += blockDim.x) {
+      const int tok = i / nrows;
+      const int lr = i - tok * nrows;
+      const int n = row_tile + r_begin + lr;
+      float v = 0.0f;
+      for (int q = 0; q < S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
+      if (n < N) y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
+    }
+  } else {
+    // Item (token, owned row) i is handled by the L consecutive lanes of slot
+    // i mod slots: with fewer items than threads, each item's k channels are
+    // split over L lanes (a power of two up to 32) and summed by shuffles.
+    // The correction is computed before the cluster barrier, while the other
+    // ranks may still be pushing their partials.
+    int L = 1;
+    while (L < 32 && items * (2 * L) <= (int)blockDim.x) L *= 2;
+    const int slots = (int)blockDim.x / L, slot = tid / L, sub = tid % L;
+    float corr[kMaxItemsPerThread];
+    int c_tok[kMaxItemsPerThread], c_n[kMaxItemsPerThread];
+#pragma unroll
+    for (int it = 0; it < kMaxItemsPerThread; ++it) {
+      corr[it] = 0.0f;
+      const int i = slot + it * slots;
+      c_tok[it] = 0;
+      c_n[it] = -1;
+      if (i < items) {
+        const int tok = i / nrows;
+        const int n = row_tile + r_begin + (i - tok * nrows);
+        if (n < N) {
+          c_tok[it] = tok;
+          c_n[it] = n;
+        }
+      }
+    }
+    residual_parts(rc, c_tok, c_n, N, sub, L, corr);
+    if (L > 1) {
+#pragma unroll
+      for (int it = 0; it < kMaxItemsPerThread; ++it)
+        for (int o = L / 2; o > 0; o >>= 1) corr[it] += __shfl_xor_sync(0xffffffffu, corr[it], o);
+    }
+    if (S > 1) {
+      cluster_sync_all();
+    } else {
+      __syncthreads();
+    }
+#pragma unroll
+    for (int it = 0; it < kMaxItemsPerThread; ++it) {
+      const int i = slot + it * slots;
+      if (sub != 0 || i >= items) break;
+      const int tok = i / nrows;
+      const int lr = i - tok * nrows;
+      const int n = row_tile + r_begin + lr;
+      float v = corr[it];
+      for (int q = 0; q < S; ++q) v += red[((size_t)q * rows_max + lr) * 16 + tok];
+      if (n < N) y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
     }
   }
 }

@@ -202,7 +202,8 @@ wq_status wq_residual(wq_format fmt, const float* W, int64_t N, int64_t K, int32
   if (fmt == WQ_FMT_INT4_ASYM && !zeros) return WQ_ERR_INVALID_ARG;
   if (fmt == WQ_FMT_NF4 && zeros) return WQ_ERR_INVALID_ARG;
   if (!all_aligned({W, qweight, scales, zeros, residual_t})) return WQ_ERR_ALIGNMENT;
-  if (N > INT32_MAX || K > INT32_MAX || (N + 31) / 32 > 65535) return WQ_ERR_UNSUPPORTED;
+  if (K % 64 != 0 || N % 8 != 0) return WQ_ERR_UNSUPPORTED;
+  if (N > INT32_MAX || K > INT32_MAX || (N + 63) / 64 > 65535) return WQ_ERR_UNSUPPORTED;
   return guarded([&] {
     return launch_residual(fmt, W, N, K, group, qweight, scales, zeros, residual_t,
                            as_stream(stream));

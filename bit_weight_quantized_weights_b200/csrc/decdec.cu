@@ -23,41 +23,60 @@
 namespace wq {
 namespace {
 
-// One 32 x 32 tile of R^T per CTA (32 x 8 threads): computed in [n][k] order
-// from the row-major weights, written transposed through shared memory.
+// One 64 (k) x 64 (n) tile of R^T per 256-thread CTA. Each thread reads 4
+// consecutive weights of a row as one float4 (16 threads per 256-byte row
+// segment) and stores their residuals transposed into shared memory; the tile
+// then leaves as 16-byte rows of 8 consecutive n (8 threads per 128-byte k row).
+// K % 64 == 0; rows beyond N are skipped.
 template <bool kNF4>
 __global__ void __launch_bounds__(256) residual_kernel(
     const float* __restrict__ W, int N, int K, int G, const uint32_t* __restrict__ qw,
     const uint8_t* __restrict__ codes, const __half* __restrict__ scales,
     const __half* __restrict__ zeros, const float* __restrict__ absmax, Nf4Table tab,
     __half* __restrict__ rt) {
-  __shared__ __half tile[32][33];
-  const int k0 = blockIdx.x * 32, n0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int i = ty; i < 32; i += 8) {
-    const int n = n0 + i, k = k0 + tx;
-    float r = 0.0f;
-    if (n < N && k < K) {
-      const int64_t e = (int64_t)n * K + k;
-      float wh;
+  constexpr int kPitch = 64 + 8;  // halves per k row of the tile (16-byte rows stay aligned)
+  __shared__ __align__(16) __half tile[64 * kPitch];
+  const int k0 = blockIdx.x * 64, n0 = blockIdx.y * 64;
+  const int tid = threadIdx.x;
+  const int kq = (tid & 15) * 4;  // this thread's 4 consecutive k of the segment
+  for (int r = tid >> 4; r < 64; r += 16) {
+    const int n = n0 + r;
+    float4 w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float wh[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (n < N) {
+      const int64_t e = (int64_t)n * K + k0 + kq;  // multiple of 4
+      w4 = __ldg(reinterpret_cast<const float4*>(W + e));
       if (kNF4) {
-        const uint8_t b = codes[e >> 1];
-        const int q = (e & 1) ? (b & 0xF) : (b >> 4);  // element 2j: high nibble
-        wh = __fmul_rn(tab.v[q], absmax[e >> 6]);      // one fp32 rounding
+        const uint16_t b2 = __ldg(reinterpret_cast<const uint16_t*>(codes + (e >> 1)));
+        const float am = __ldg(absmax + (e >> 6));
+        // bytes j, j + 1 = elements (e, e+1), (e+2, e+3); element 2j: high nibble
+        const int q[4] = {(b2 >> 4) & 0xF, b2 & 0xF, (b2 >> 12) & 0xF, (b2 >> 8) & 0xF};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wh[i] = __fmul_rn(tab.v[q[i]], am);  // one fp32 rounding
       } else {
-        const uint32_t word = qw[(int64_t)n * (K / 8) + (k >> 3)];
-        const int q = (int)((word >> (4 * (k & 7))) & 0xFu);
-        const int64_t gi = (int64_t)n * (K / G) + k / G;
-        wh = __fmul_rn((float)q - __half2float(zeros[gi]), __half2float(scales[gi]));  // exact
+        const uint32_t word = __ldg(qw + (e >> 3));
+        const int sh = (int)(e & 7) * 4;  // 0 or 16: the word's low or high four codes
+        const int64_t gi = (int64_t)n * (K / G) + (k0 + kq) / G;
+        const float sc = __half2float(scales[gi]), z = __half2float(zeros[gi]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          wh[i] = __fmul_rn((float)((word >> (sh + 4 * i)) & 0xFu) - z, sc);  // exact
       }
-      r = __fsub_rn(W[e], wh);
     }
-    tile[i][tx] = __float2half_rn(r);
+    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tile[(kq + i) * kPitch + r] = __float2half_rn(__fsub_rn(wv[i], wh[i]));
   }
   __syncthreads();
-  for (int i = ty; i < 32; i += 8) {
-    const int k = k0 + i, n = n0 + tx;
-    if (n < N && k < K) rt[(int64_t)k * N + n] = tile[tx][i];
+  const int nc = (tid & 7) * 8;  // 8 consecutive n
+  for (int kr = tid >> 3; kr < 64; kr += 32) {
+    const int n = n0 + nc;
+    if (n + 8 <= N) {
+      *reinterpret_cast<uint4*>(rt + (int64_t)(k0 + kr) * N + n) =
+          *reinterpret_cast<const uint4*>(tile + kr * kPitch + nc);
+    } else {
+      for (int i = 0; i < 8 && n + i < N; ++i) rt[(int64_t)(k0 + kr) * N + n + i] = tile[kr * kPitch + nc + i];
+    }
   }
 }
 
@@ -176,7 +195,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
 wq_status launch_residual(wq_format fmt, const float* W, int64_t N, int64_t K, int32_t G,
                           const void* qweight, const void* scales, const void* zeros, void* rt,
                           cudaStream_t st) {
-  const dim3 grid((unsigned)((K + 31) / 32), (unsigned)((N + 31) / 32));
+  const dim3 grid((unsigned)(K / 64), (unsigned)((N + 63) / 64));
   if (fmt == WQ_FMT_NF4)
     residual_kernel<true><<<grid, 256, 0, st>>>(
         W, (int)N, (int)K, G, nullptr, static_cast<const uint8_t*>(qweight), nullptr, nullptr,

@@ -180,7 +180,7 @@ wq_status wq_w4a16_gemv(const void* x, int64_t M, int64_t N, int64_t K,
  *   weights and parameters as for wq_w4a16_gemv. W_hat is (q - z) * s (exact
  *   in fp32) for INT4 and fp32(codebook[q] * absmax) for NF4; the subtraction
  *   rounds once in fp32, the result once to fp16. Bit-exact with the oracle.
- *   N == 0 is a no-op.
+ *   Requires K % 64 == 0 and N % 8 == 0; N == 0 is a no-op.
  *
  * wq_select_salient: the k salient channels of x bf16 [M, K] (M >= 1,
  *   0 <= k <= K <= 65536): the k largest max_m |x[m, c]|, ranked by the bf16

@@ -106,6 +106,8 @@ def test_residual_correction_validation(wq):
     assert L.wq_residual(0, A16, 64, 128, 64, A16, A16, None, A16, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_residual(0, MIS, 64, 128, 64, A16, A16, A16, A16, None) == wq.WQ_ERR_ALIGNMENT
     assert L.wq_residual(0, A16, 0, 128, 64, A16, A16, A16, A16, None) == wq.WQ_OK
+    assert L.wq_residual(0, A16, 60, 128, 64, A16, A16, A16, A16, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_residual(0, A16, 64, 96, 32, A16, A16, A16, A16, None) == wq.WQ_ERR_UNSUPPORTED
     # wq_select_salient(x, M, K, k, idx, stream)
     assert L.wq_select_salient(A16, 1, 4096, 4097, A16, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_select_salient(A16, 0, 4096, 8, A16, None) == wq.WQ_ERR_INVALID_ARG

@@ -19,6 +19,7 @@
 // The host-memory placement of the residuals on the page's laptop GPU is not
 // reproduced: R^T lives in device memory and only the k selected rows are read.
 #include "common.cuh"
+#include "salient.cuh"
 
 namespace wq {
 namespace {
@@ -82,112 +83,12 @@ __global__ void __launch_bounds__(256) residual_kernel(
 
 constexpr int kSelThreads = 1024;
 
-// Exclusive prefix sum over the CTA's threads; *total gets the sum.
-__device__ __forceinline__ unsigned block_exclusive_scan(unsigned v, unsigned* warp_sums,
-                                                         unsigned* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned t = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += t;
-  }
-  if (lane == 31) warp_sums[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    unsigned w = warp_sums[lane];
-    unsigned wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned t = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += t;
-    }
-    warp_sums[lane] = wi - w;  // exclusive over warps
-    if (lane == 31) *total = wi;
-  }
-  __syncthreads();
-  const unsigned r = warp_sums[warp] + inc - v;
-  __syncthreads();
-  return r;
-}
-
-// The histogram bin holding the want-th largest key, and how many keys lie in
-// higher bins: thread t takes bin nbins - 1 - t, an exclusive scan over the
-// threads counts the keys above it, and the one thread whose bin contains
-// the want-th key writes the answer. All threads call it.
-__device__ __forceinline__ void find_bin(const unsigned* hist, int nbins, unsigned want,
-                                         unsigned* warp_sums, unsigned* total, unsigned* bin,
-                                         unsigned* above) {
-  const int t = threadIdx.x;
-  const unsigned h = t < nbins ? hist[nbins - 1 - t] : 0u;
-  const unsigned before = block_exclusive_scan(h, warp_sums, total);
-  if (t < nbins && h > 0 && before < want && want <= before + h) {
-    *bin = (unsigned)(nbins - 1 - t);
-    *above = before;
-  }
-  __syncthreads();
-}
-
-// hist[bin] += 1 for every calling lane, one shared-memory atomic per
-// distinct bin among the warp's active lanes.
-__device__ __forceinline__ void hist_add(unsigned* hist, unsigned bin) {
-  const unsigned peers = __match_any_sync(__activemask(), bin);
-  if ((__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&hist[bin], __popc(peers));
-}
-
-// The k salient channels of x [M, K] (1 <= k <= K), one CTA: 15-bit keys in
-// shared memory, a two-pass radix select of the k-th largest key T (high 8
-// bits, then low 7), then an order-preserving compaction that takes every key
-// above T and the lowest-index keys equal to T.
+// One CTA selects for the whole step.
 __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __restrict__ x, int M,
                                                              int K, int k, int* __restrict__ idx) {
   extern __shared__ uint16_t keys[];
-  __shared__ unsigned hist[256];
-  __shared__ unsigned warp_sums[32];
-  __shared__ unsigned s_bin, s_above, s_T, s_need, s_total;
-  const int tid = threadIdx.x;
-  for (int c = tid; c < K; c += kSelThreads) {
-    unsigned best = 0;
-    for (int m = 0; m < M; ++m) best = max(best, (unsigned)(x[(size_t)m * K + c] & 0x7FFFu));
-    keys[c] = (uint16_t)best;
-  }
-  if (tid < 256) hist[tid] = 0;
-  __syncthreads();
-  for (int c = tid; c < K; c += kSelThreads) hist_add(hist, keys[c] >> 7);
-  __syncthreads();
-  find_bin(hist, 256, (unsigned)k, warp_sums, &s_total, &s_bin, &s_above);
-  const unsigned hi = s_bin, above_hi = s_above;
-  if (tid < 256) hist[tid] = 0;
-  __syncthreads();
-  for (int c = tid; c < K; c += kSelThreads)
-    if ((unsigned)(keys[c] >> 7) == hi) hist_add(hist, keys[c] & 0x7Fu);
-  __syncthreads();
-  find_bin(hist, 128, (unsigned)k - above_hi, warp_sums, &s_total, &s_bin, &s_above);
-  if (tid == 0) {
-    s_T = (hi << 7) | s_bin;
-    s_need = (unsigned)k - above_hi - s_above;  // keys equal to T to take, >= 1
-  }
-  __syncthreads();
-  const unsigned T = s_T, need = s_need;
-  // this thread's contiguous range of channels
-  const int per = (K + kSelThreads - 1) / kSelThreads;
-  const int c0 = min(K, tid * per), c1 = min(K, c0 + per);
-  unsigned n_gt = 0, n_eq = 0;
-  for (int c = c0; c < c1; ++c) {
-    n_gt += keys[c] > T;
-    n_eq += keys[c] == T;
-  }
-  const unsigned eq_before = block_exclusive_scan(n_eq, warp_sums, &s_total);
-  const unsigned take_eq = eq_before >= need ? 0u : min(n_eq, need - eq_before);
-  unsigned pos = block_exclusive_scan(n_gt + take_eq, warp_sums, &s_total);
-  unsigned taken = 0;
-  for (int c = c0; c < c1; ++c) {
-    const unsigned key = keys[c];
-    if (key > T || (key == T && taken < take_eq)) {
-      idx[pos++] = c;
-      if (key == T) ++taken;
-    }
-  }
+  __shared__ salient::Scratch sc;
+  salient::select_block(x, M, K, k, keys, sc, idx);
 }
 
 }  // namespace

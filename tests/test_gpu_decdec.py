@@ -97,20 +97,20 @@ def test_select_salient_ties_nan_inf(wq):
         assert np.array_equal(got, ref), nsel
 
 
-def _corrected_case(wq, fmt, m, n, k, nsel, seed):
+def _corrected_case(wq, fmt, m, n, k, nsel, seed, group=128):
     x = _x(m, k, seed)
     xd = x.cuda()
     xf = helpers.x_f32(x)
     if fmt == "int4":
-        w, q, s, z, qweight = _int4(n, k, 128, seed)
+        w, q, s, z, qweight = _int4(n, k, group, seed)
         qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
-        rt = wq.wq_residual(wq.WQ_FMT_INT4_ASYM, torch.from_numpy(w).cuda(), 128, qw, sc, zr)
+        rt = wq.wq_residual(wq.WQ_FMT_INT4_ASYM, torch.from_numpy(w).cuda(), group, qw, sc, zr)
         idx = wq.wq_select_salient(xd, nsel)
-        y = wq.wq_w4a16_gemv_corrected(xd, n, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr, rt, idx)
-        ref_rt = decdec.int4_residual_t(w, q, s, z, 128)
+        y = wq.wq_w4a16_gemv_corrected(xd, n, wq.WQ_FMT_INT4_ASYM, group, qw, sc, zr, rt, idx)
+        ref_rt = decdec.int4_residual_t(w, q, s, z, group)
         ref_idx = decdec.select_salient(xf, nsel)
-        y_ref = decdec.int4_corrected(xf, q, s, z, 128, ref_rt, ref_idx)
-        y_base = decdec.int4_corrected(xf, q, s, z, 128, ref_rt, ref_idx[:0])
+        y_ref = decdec.int4_corrected(xf, q, s, z, group, ref_rt, ref_idx)
+        y_base = decdec.int4_corrected(xf, q, s, z, group, ref_rt, ref_idx[:0])
         slack = 1e-4
     else:
         w, codes, absmax, packed = _nf4(n, k, seed)
@@ -138,6 +138,12 @@ def _corrected_case(wq, fmt, m, n, k, nsel, seed):
                                         (2, 1040, 640, 0)])
 def test_corrected_gemv_matches_oracle(wq, fmt, m, n, k, nsel):
     _corrected_case(wq, fmt, m, n, k, nsel, seed=m + nsel)
+
+
+@pytest.mark.parametrize("m,n,k,nsel", [(3, 1040, 640, 40), (16, 2064, 1152, 100)])
+def test_corrected_gemv_int4_g64(wq, m, n, k, nsel):
+    """The 8-byte-load GEMV (INT4 groups of 64) with the correction."""
+    _corrected_case(wq, "int4", m, n, k, nsel, seed=m, group=64)
 
 
 @pytest.mark.parametrize("fmt", ["int4", "nf4"])

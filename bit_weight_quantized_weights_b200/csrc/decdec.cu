@@ -66,7 +66,8 @@ __global__ void __launch_bounds__(256) residual_kernel(
     }
     const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tile[(kq + i) * kPitch + r] = __float2half_rn(__fsub_rn(wv[i], wh[i]));
+    for (int i = 0; i < 4; ++i)
+      tile[(kq + i) * kPitch + r] = __float2half_rn(__fsub_rn(wv[i], wh[i]));
   }
   __syncthreads();
   const int nc = (tid & 7) * 8;  // 8 consecutive n
@@ -76,7 +77,8 @@ __global__ void __launch_bounds__(256) residual_kernel(
       *reinterpret_cast<uint4*>(rt + (int64_t)(k0 + kr) * N + n) =
           *reinterpret_cast<const uint4*>(tile + kr * kPitch + nc);
     } else {
-      for (int i = 0; i < 8 && n + i < N; ++i) rt[(int64_t)(k0 + kr) * N + n + i] = tile[kr * kPitch + nc + i];
+      for (int i = 0; i < 8 && n + i < N; ++i)
+        rt[(int64_t)(k0 + kr) * N + n + i] = tile[kr * kPitch + nc + i];
     }
   }
 }

@@ -37,9 +37,13 @@
 //   64-element absmax block, so one fp16x2 multiply per register applies the
 //   block's absmax to the A operand before the MMA (code, absmax and product
 //   each rounded once to fp16, as in the fused GEMM), which lets NF4 use the
-//   16-byte layout. The NF4 product runs in fp16: the staged x chunk is converted to fp16 scaled per token by a power
-//   of two that puts its largest magnitude in [2^14, 2^15) (exact for bf16
-//   values down to 2^-28 of it); the power is divided back out of the partial.
+//   16-byte layout. The NF4 product runs in fp16: the staged x chunk is
+//   converted to fp16 scaled per token by a power of two that puts its largest
+//   magnitude in [2^14, 2^15) (exact for bf16 values down to 2^-28 of it); the
+//   power is divided back out of the partial.
+// * Optional salient-channel residual correction (kRes, "DecDEC: A Systems
+//   Approach to Advancing Low-Bit LLM Quantization", Abstract): the owners add
+//   sum_j x[m, c_j] R^T[c_j, n] to each output in fp32 before its rounding.
 // * Split-K across a thread-block cluster: the S CTAs of a cluster share one
 //   128-row tile and split K. Each CTA pushes its fp32 partials into the
 //   shared memory of the rank that owns those rows (remote stores, no round
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   __syncthreads();
 
   if (!kNF4) {
-    // In place, chunk by chunk: sums of x per 64- (narrow) or 128-wide (wide)
+    // In place, chunk by chunk: sums of x per 64- (8-byte layout) or 128-wide (16-byte layout)
     // sub-group, and the (k, k + 4) pairing of the INT4 nibbles. The chunks of
     // one sub-group sit in 8 or 16 consecutive lanes; the loop runs whole
     // warps (bound rounded up to 32) for the shuffles.
@@ -534,7 +538,8 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   }
   const bool res = k > 0;
   if (fmt == WQ_FMT_NF4) {
-    if (res) return NT == 1 ? launch_t<1, true, true, true>(a, st) : launch_t<2, true, true, true>(a, st);
+    if (res)
+      return NT == 1 ? launch_t<1, true, true, true>(a, st) : launch_t<2, true, true, true>(a, st);
     return NT == 1 ? launch_t<1, true, true, false>(a, st) : launch_t<2, true, true, false>(a, st);
   }
   if (group % 128 == 0) {

@@ -283,9 +283,33 @@ def dequant_then_cublas(wq, step, fused_ms, warmup):
         if i >= max(warmup, 1):
             t_deq += ev[0].elapsed_time(ev[1]) / reps
             t_mm += ev[1].elapsed_time(ev[2]) / reps
+    # the same comparison at smaller prefill sizes (the first rows of the step's
+    # x): the dequantization is a fixed cost per call, so its share grows as M
+    # shrinks
+    sweep = []
+    for ms in (512, 2048, 4096):
+        xs = step.px[:ms]
+        ys = torch.empty(ms, n, dtype=torch.bfloat16, device=step.px.device)
+        ws = wq.gemm_workspace(ms, n, k, 128, step.px.device)
+        t_f = t_c = 0.0
+        for i in range(max(warmup, 1) + reps):
+            ev[0].record()
+            wq.wq_w4a16_gemm(xs, n, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr, workspace=ws, out=ys)
+            ev[1].record()
+            wq.wq_int4_dequant(qw, sc, zr, n, k, 128, out=wd)
+            torch.matmul(xs, wd.t(), out=ys)
+            ev[2].record()
+            torch.cuda.synchronize()
+            if i >= max(warmup, 1):
+                t_f += ev[0].elapsed_time(ev[1]) / reps
+                t_c += ev[1].elapsed_time(ev[2]) / reps
+        sweep.append({"m": ms, "fused_ms": round(t_f, 4), "dequant_then_cublas_ms": round(t_c, 4),
+                      "fused_speedup": round(t_c / t_f, 3)})
+        del ys, ws
     del wd, y
     flops = 2.0 * m * n * k
     return {"workload": "gemm int4-g128 %dx%dx%d" % (m, n, k),
+            "sweep_smaller_m": sweep,
             "dequant_then_cublas_ms": round(t_deq + t_mm, 4), "dequant_ms": round(t_deq, 4),
             "cublas_bf16_ms": round(t_mm, 4),
             "dequant_then_cublas_tflops": round(flops / ((t_deq + t_mm) * 1e-3) / 1e12, 1),

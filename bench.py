@@ -385,12 +385,17 @@ def measure_decdec(wq, peaks, device, with_oracle):
         corr = _graph_us([lambda t=t: wq.wq_w4a16_gemv_corrected(
             x, n, wq.WQ_FMT_INT4_ASYM, 128, t[1], t[2], t[3], t[4], idx, out=y)
             for t in sets], 32)
+        step_us = _graph_us([lambda t=t: wq.wq_w4a16_gemv_salient(
+            x, n, wq.WQ_FMT_INT4_ASYM, 128, t[1], t[2], t[3], t[4], DECDEC_K, idx=idx, out=y)
+            for t in sets], 32)
         gemv_bytes = n * k * 0.5 + n * (k // 128) * 4 + 2 * m * k + 2 * m * n
         corr_bytes = DECDEC_K * n * 2
         out["m%d" % m] = {
             "gemv_us": round(plain, 2), "select_us": round(sel, 2),
             "corrected_gemv_us": round(corr, 2),
             "overhead_pct": round(100.0 * (corr + sel - plain) / plain, 1),
+            "salient_step_us": round(step_us, 2),
+            "salient_step_overhead_pct": round(100.0 * (step_us - plain) / plain, 1),
             "correction_bytes": corr_bytes,
             "corrected_gemv_gbs": round((gemv_bytes + corr_bytes) / (corr * 1e-6) / 1e9, 1)}
     if with_oracle:

@@ -38,7 +38,7 @@ EXPORTED = [
     "wq_quantize_pack", "wq_unpack", "wq_nf4_dequant", "wq_int4_dequant",
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
-    "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected",
+    "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
 ]
 
 
@@ -79,6 +79,8 @@ def _load():
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
         "wq_w4a16_gemv_corrected": ([P, I64, I64, I64, ctypes.c_int, I32, P, P, P, P, P, I32, P,
                                      P], ctypes.c_int),
+        "wq_w4a16_gemv_salient": ([P, I64, I64, I64, ctypes.c_int, I32, P, P, P, P, I32, P, P,
+                                   P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -265,6 +267,25 @@ def wq_w4a16_gemv_corrected(x, n, fmt, group, qweight, scales, zeros, residual_t
     _check(lib.wq_w4a16_gemv_corrected(_ptr(x), m, n, k, fmt, group, _ptr(qweight), _ptr(scales),
                                        _ptr(zeros), _ptr(residual_t), _ptr(idx), nsel, _ptr(out),
                                        _stream(stream)), "wq_w4a16_gemv_corrected")
+    return out
+
+
+def wq_w4a16_gemv_salient(x, n, fmt, group, qweight, scales, zeros, residual_t, nsel, idx=None,
+                          out=None, stream=None):
+    """One corrected decode step: select the nsel salient channels into idx
+    (int32 scratch, allocated if None), then the corrected GEMV, launched to
+    overlap the selection. Returns y."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _cuda(out, torch.bfloat16, "y")
+    if idx is None:
+        idx = torch.empty(max(nsel, 1), dtype=torch.int32, device=x.device)
+    _cuda(idx, torch.int32, "idx")
+    _check(lib.wq_w4a16_gemv_salient(_ptr(x), m, n, k, fmt, group, _ptr(qweight), _ptr(scales),
+                                     _ptr(zeros), _ptr(residual_t), nsel, _ptr(idx), _ptr(out),
+                                     _stream(stream)), "wq_w4a16_gemv_salient")
     return out
 
 

@@ -15,7 +15,7 @@ wq_status launch_int4_dequant(const uint32_t*, const void*, const void*, int64_t
 wq_status launch_gemv(const void*, int64_t, int64_t, int64_t, wq_format, int32_t, const void*,
                       const void*, const void*, void*, cudaStream_t,
                       const void* residual_t = nullptr, const int32_t* idx = nullptr,
-                      int32_t k = 0);
+                      int32_t k = 0, bool early = false);
 wq_status launch_residual(wq_format, const float*, int64_t, int64_t, int32_t, const void*,
                           const void*, const void*, void*, cudaStream_t);
 wq_status launch_select_salient(const void*, int64_t, int64_t, int32_t, int32_t*, cudaStream_t);
@@ -237,6 +237,31 @@ wq_status wq_w4a16_gemv_corrected(const void* x, int64_t M, int64_t N, int64_t K
   return guarded([&] {
     return launch_gemv(x, M, N, K, fmt, group, qweight, scales, zeros, y, as_stream(stream),
                        residual_t, idx, k);
+  });
+}
+
+wq_status wq_w4a16_gemv_salient(const void* x, int64_t M, int64_t N, int64_t K, wq_format fmt,
+                                int32_t group, const void* qweight, const void* scales,
+                                const void* zeros, const void* residual_t, int32_t k,
+                                int32_t* idx, void* y, void* stream) {
+  wq_status s = check_product(x, M, N, K, fmt, group, qweight, scales, zeros, y);
+  if (s != WQ_OK) return s;
+  if (k < 0 || k > K) return WQ_ERR_INVALID_ARG;
+  if (M > 16) return WQ_ERR_UNSUPPORTED;
+  if (N % 16 != 0) return WQ_ERR_UNSUPPORTED;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (k > 0) {
+    if (!residual_t || !idx) return WQ_ERR_INVALID_ARG;
+    if (!all_aligned({residual_t, idx})) return WQ_ERR_ALIGNMENT;
+    if (K > 65536) return WQ_ERR_UNSUPPORTED;
+  }
+  return guarded([&] {
+    if (k > 0) {
+      const wq_status r = launch_select_salient(x, M, K, k, idx, as_stream(stream));
+      if (r != WQ_OK) return r;
+    }
+    return launch_gemv(x, M, N, K, fmt, group, qweight, scales, zeros, y, as_stream(stream),
+                       residual_t, idx, k, /*early=*/true);
   });
 }
 

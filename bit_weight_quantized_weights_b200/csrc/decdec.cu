@@ -90,6 +90,9 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const uint16_t* __r
                                                              int K, int k, int* __restrict__ idx) {
   extern __shared__ uint16_t keys[];
   __shared__ salient::Scratch sc;
+  // a GEMV launched after this one with programmatic stream serialization
+  // may start now; it waits (griddepcontrol.wait) before it reads idx
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   salient::select_block(x, M, K, k, keys, sc, idx);
 }
 

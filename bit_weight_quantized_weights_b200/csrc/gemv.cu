@@ -495,7 +495,7 @@ size_t gemv_smem(int kc, int S) {
 }
 
 template <int NT, bool kNF4, bool kWide, bool kRes>
-wq_status launch_t(GemvArgs a, cudaStream_t st) {
+wq_status launch_t(GemvArgs a, cudaStream_t st, bool early = false) {
   auto kern = gemv_kernel<NT, kNF4, kWide, kRes>;
   const int M = a.M;
   const Plan pl = cached_plan(reinterpret_cast<const void*>(kern), M, a.N, a.K, 0, [&] {
@@ -506,14 +506,15 @@ wq_status launch_t(GemvArgs a, cudaStream_t st) {
   if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
   a.S = pl.S;
   a.kc = pl.kc;
-  return launch_split(kern, pl, 256, a.N, st, a, nf4_table());
+  return launch_split(kern, pl, 256, a.N, st, a, nf4_table(), false, early && kRes);
 }
 
 }  // namespace
 
 wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format fmt, int32_t group,
                       const void* qweight, const void* scales, const void* zeros, void* y,
-                      cudaStream_t st, const void* residual_t, const int32_t* idx, int32_t k) {
+                      cudaStream_t st, const void* residual_t, const int32_t* idx, int32_t k,
+                      bool early) {
   const int NT = M <= 8 ? 1 : 2;
   GemvArgs a;
   a.x = static_cast<const uint16_t*>(x);
@@ -539,16 +540,19 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   const bool res = k > 0;
   if (fmt == WQ_FMT_NF4) {
     if (res)
-      return NT == 1 ? launch_t<1, true, true, true>(a, st) : launch_t<2, true, true, true>(a, st);
+      return NT == 1 ? launch_t<1, true, true, true>(a, st, early)
+                     : launch_t<2, true, true, true>(a, st, early);
     return NT == 1 ? launch_t<1, true, true, false>(a, st) : launch_t<2, true, true, false>(a, st);
   }
   if (group % 128 == 0) {
     if (res)
-      return NT == 1 ? launch_t<1, false, true, true>(a, st) : launch_t<2, false, true, true>(a, st);
+      return NT == 1 ? launch_t<1, false, true, true>(a, st, early)
+                     : launch_t<2, false, true, true>(a, st, early);
     return NT == 1 ? launch_t<1, false, true, false>(a, st) : launch_t<2, false, true, false>(a, st);
   }
   if (res)
-    return NT == 1 ? launch_t<1, false, false, true>(a, st) : launch_t<2, false, false, true>(a, st);
+    return NT == 1 ? launch_t<1, false, false, true>(a, st, early)
+                   : launch_t<2, false, false, true>(a, st, early);
   return NT == 1 ? launch_t<1, false, false, false>(a, st) : launch_t<2, false, false, false>(a, st);
 }
 

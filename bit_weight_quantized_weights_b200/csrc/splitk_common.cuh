@@ -172,6 +172,10 @@ __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], cons
       if (n < N) y[(int64_t)tok * N + n] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xFFFFu);
     }
   } else {
+    // When this grid was launched early after the channel selection
+    // (programmatic dependent launch), wait for it before reading idx; a no-op
+    // otherwise.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // Item (token, owned row) i is handled by the L consecutive lanes of slot
     // i mod slots: with fewer items than threads, each item's k channels are
     // split over L lanes (a power of two up to 32) and summed by shuffles.
@@ -333,7 +337,8 @@ Plan cached_plan(const void* kern, int M, int64_t N, int64_t K, int extra, MakeF
 // over the row tiles y, y + gridDim.y, ...
 template <class Kern, class Args>
 wq_status launch_split(Kern kern, const Plan& pl, int threads, int64_t N, cudaStream_t st,
-                       const Args& args, const Nf4Table& tab, bool persistent = false) {
+                       const Args& args, const Nf4Table& tab, bool persistent = false,
+                       bool early = false) {
   // the attribute is a per-function maximum; plans of other shapes may have
   // set a smaller one since
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
@@ -346,13 +351,17 @@ wq_status launch_split(Kern kern, const Plan& pl, int threads, int64_t N, cudaSt
   cfg.blockDim = dim3((unsigned)threads, 1, 1);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)pl.S;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // early: programmatic dependent launch after the preceding kernel, which
+  // must only read what this kernel reads before its griddepcontrol.wait
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = early ? 2 : 1;
   if (cudaLaunchKernelEx(&cfg, kern, args, tab) != cudaSuccess) return WQ_ERR_CUDA;
   return launch_status();
 }

@@ -208,6 +208,20 @@ wq_status wq_w4a16_gemv_corrected(const void* x, int64_t M, int64_t N, int64_t K
                                   void* stream);
 
 /*
+ * wq_w4a16_gemv_salient: one decode step of the correction, selection
+ * included: wq_select_salient into idx (caller-owned int32 [k] scratch,
+ * written), then wq_w4a16_gemv_corrected. The GEMV is launched as a
+ * programmatic dependent of the selection: it starts while the selection
+ * runs and waits for it only before its epilogue reads idx. Requires
+ * K <= 65536 when k > 0; k == 0 is wq_w4a16_gemv.
+ */
+wq_status wq_w4a16_gemv_salient(const void* x, int64_t M, int64_t N, int64_t K,
+                                wq_format fmt, int32_t group,
+                                const void* qweight, const void* scales,
+                                const void* zeros, const void* residual_t,
+                                int32_t k, int32_t* idx, void* y, void* stream);
+
+/*
  * Prefill W4A16 GEMM with fused dequantization on the tensor cores ([MSD]:
  * the dequantize-then-multiply product; here the dequantized tile is written
  * straight into tensor memory and never leaves the SM). Same arguments and

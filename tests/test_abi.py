@@ -126,6 +126,15 @@ def test_residual_correction_validation(wq):
     assert cg(A16, 17, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 8, A16,
               None) == wq.WQ_ERR_UNSUPPORTED
     assert cg(A16, 0, 4096, 4096, 0, 128, A16, A16, A16, A16, A16, 8, A16, None) == wq.WQ_OK
+    # wq_w4a16_gemv_salient(x, M, N, K, fmt, G, q, s, z, residual_t, k, idx, y, stream)
+    sg = L.wq_w4a16_gemv_salient
+    assert sg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, A16, 8, None, A16,
+              None) == wq.WQ_ERR_INVALID_ARG                        # idx scratch needed
+    assert sg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, A16, 8, MIS, A16,
+              None) == wq.WQ_ERR_ALIGNMENT
+    assert sg(A16, 1, 4096, 4096, 0, 128, A16, A16, A16, A16, 4097, A16, A16,
+              None) == wq.WQ_ERR_INVALID_ARG
+    assert sg(A16, 0, 4096, 4096, 0, 128, A16, A16, A16, A16, 8, A16, A16, None) == wq.WQ_OK
 
 
 def test_gemm_and_msd_validation(wq):

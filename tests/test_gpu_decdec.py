@@ -140,6 +140,46 @@ def test_corrected_gemv_matches_oracle(wq, fmt, m, n, k, nsel):
     _corrected_case(wq, fmt, m, n, k, nsel, seed=m + nsel)
 
 
+@pytest.mark.parametrize("fmt", ["int4", "nf4"])
+@pytest.mark.parametrize("m,n,k,nsel", [(1, 11008, 4096, 64), (16, 11008, 4096, 64),
+                                        (4, 4096, 11008, 110), (3, 1040, 640, 640)])
+def test_salient_step_matches_oracle(wq, fmt, m, n, k, nsel):
+    """Selection and corrected GEMV in one call, the GEMV launched to overlap
+    the selection: same result as the oracle's corrected product, and the
+    channel set written to the scratch equals the oracle's."""
+    seed = m + nsel + 5
+    x = _x(m, k, seed)
+    xd = x.cuda()
+    xf = helpers.x_f32(x)
+    if fmt == "int4":
+        w, q, s, z, qweight = _int4(n, k, 128, seed)
+        pk = helpers.to_dev_int4(s, z, qweight)
+        f, g = wq.WQ_FMT_INT4_ASYM, 128
+        ref_rt = decdec.int4_residual_t(w, q, s, z, 128)
+        ref_idx = decdec.select_salient(xf, nsel)
+        y_ref = decdec.int4_corrected(xf, q, s, z, 128, ref_rt, ref_idx)
+        slack = 1e-4
+    else:
+        w, codes, absmax, packed = _nf4(n, k, seed)
+        cw, am = helpers.to_dev_nf4(absmax, packed)
+        pk = (cw, am, None)
+        f, g = wq.WQ_FMT_NF4, 64
+        ref_rt = decdec.nf4_residual_t(w, codes, absmax)
+        ref_idx = decdec.select_salient(xf, nsel)
+        y_ref = decdec.nf4_corrected(xf, codes, absmax, k, ref_rt, ref_idx)
+        slack = 3e-3
+    rt = wq.wq_residual(f, torch.from_numpy(w).cuda(), g, *pk)
+    idx = torch.full((nsel,), -1, dtype=torch.int32, device="cuda")
+    y = wq.wq_w4a16_gemv_salient(xd, n, f, g, *pk, rt, nsel, idx=idx)
+    torch.cuda.synchronize()
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    what = "%s salient step M=%d %dx%d k=%d" % (fmt, m, n, k, nsel)
+    helpers.check_product(y, y_ref, what)
+    helpers.check_within_bf16_rounding(y, y_ref, what, slack=slack)
+
+
 @pytest.mark.parametrize("m,n,k,nsel", [(3, 1040, 640, 40), (16, 2064, 1152, 100)])
 def test_corrected_gemv_int4_g64(wq, m, n, k, nsel):
     """The 8-byte-load GEMV (INT4 groups of 64) with the correction."""

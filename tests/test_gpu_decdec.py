@@ -14,7 +14,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import decdec, formats, numerics
+from oracle import decdec, formats
 from tests import helpers
 
 pytestmark = pytest.mark.gpu

@@ -10,11 +10,10 @@ round once to fp16, as in the fused GEMM, so its element bound carries the
 same 3e-3 RMS slack as the GEMM's NF4 cases.
 """
 
-import numpy as np
 import pytest
 import torch
 
-from oracle import formats, products
+from oracle import products
 from tests import helpers
 
 pytestmark = pytest.mark.gpu

@@ -56,8 +56,14 @@ def compare(y, y_ref):
 
 
 def bf16_ulp(v):
-    """Spacing of bf16 numbers at |v| (for element-wise one-ulp checks)."""
+    """Spacing of bf16 numbers at |v| (for element-wise one-ulp checks).
+
+    bf16 keeps 8 significant bits, so in the binade [2^e, 2^(e+1)) its numbers
+    are 2^(e-7) apart; below 2^-126 (subnormals) they are 2^-133 apart. The
+    binade comes from frexp (|v| = m 2^f with m in [0.5, 1), so e = f - 1),
+    which is exact; a floating log2 can round up into the next binade for
+    values just below a power of two."""
     a = np.abs(np.asarray(v, dtype=np.float64))
     a = np.maximum(a, np.finfo(np.float32).tiny)
-    e = np.floor(np.log2(a))
-    return np.exp2(e - 7)
+    _, f = np.frexp(a)
+    return np.ldexp(1.0, f - 1 - 7)

@@ -37,6 +37,45 @@ def test_bf16_round_keeps_nan():
     assert np.isnan(out).all()
 
 
+def _bf16_spacing_torch(v):
+    """Gap between consecutive bf16 numbers in the binade of |v|, from the
+    bf16 type itself: the largest bf16 value not above |v| (b), then
+    nextafter(b, +inf) - b. Independent of numerics.bf16_ulp."""
+    a = torch.from_numpy(np.abs(np.asarray(v, dtype=np.float64)))
+    b = a.to(torch.bfloat16)                      # round to nearest even ...
+    over = b.double() > a
+    b = torch.where(over, torch.nextafter(b, torch.zeros_like(b)), b)   # ... then down
+    up = torch.nextafter(b, torch.full_like(b, float("inf")))
+    return (up.double() - b.double()).numpy()
+
+
+def test_bf16_ulp_matches_bf16_type():
+    """bf16 keeps 8 significant bits: in the binade [2^e, 2^(e+1)) its numbers
+    are 2^(e-7) apart, and below 2^-126 (subnormal) 2^-133 apart. Checked
+    against torch.nextafter on bf16 values over every normal binade, on exact
+    powers of two and on the fp64 values just below them (where a floating
+    log2 can round up into the next binade), negatives and subnormals."""
+    rng = np.random.default_rng(7)
+    e = np.arange(-140, 127)
+    pow2 = np.ldexp(1.0, e)
+    vals = np.concatenate([
+        pow2, -pow2,
+        np.nextafter(pow2, 0.0), -np.nextafter(pow2, 0.0),
+        np.nextafter(pow2, np.inf),
+        rng.uniform(1.0, 2.0, 4000) * np.ldexp(1.0, rng.integers(-140, 127, 4000)),
+        -rng.uniform(1.0, 2.0, 1000) * np.ldexp(1.0, rng.integers(-30, 30, 1000)),
+        rng.standard_normal(2000) * 5.6,
+        np.array([1e-45, 3.0e-39, 1.1754942e-38, 0.0]),
+    ])
+    got = numerics.bf16_ulp(vals)
+    ref = _bf16_spacing_torch(vals)
+    bad = got != ref
+    assert not bad.any(), list(zip(vals[bad][:5], got[bad][:5], ref[bad][:5]))
+    # spot values by hand: 1 -> 2^-7, 3 -> 2^-6, just below 1 -> 2^-8
+    assert numerics.bf16_ulp(np.array([1.0, 3.0, np.nextafter(1.0, 0.0), -0.75])).tolist() == [
+        2.0 ** -7, 2.0 ** -6, 2.0 ** -8, 2.0 ** -8]
+
+
 def test_compare_metrics_closed_form():
     ref = np.array([3.0, 4.0])
     rel, mx = numerics.compare(ref + np.array([0.3, -0.4]), ref)

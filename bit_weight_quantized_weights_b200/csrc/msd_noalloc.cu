@@ -55,11 +55,14 @@ extern "C" {
 wq_status wq_msd_gemm_noalloc(const void* x, int64_t M, int64_t N, int64_t K,
                               int32_t n_components, int32_t group, const void* qweight,
                               const void* scales, const void* zeros, void* y, void* stream) {
-  // Same argument rules as wq_msd_gemm; the scratch it would take from the
-  // caller must fit the fixed array.
-  if (M < 0 || N < 0 || K <= 0) return WQ_ERR_INVALID_ARG;
-  if (n_components < 1 || n_components > 3) return WQ_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return WQ_OK;
+  // Same argument rules as wq_msd_gemm, checked first and by wq_msd_gemm
+  // itself: with no workspace it validates every argument and returns
+  // WQ_ERR_WORKSPACE only when they are all valid (WQ_OK for the empty
+  // problems it leaves untouched), so a bad argument gets the status it
+  // would get there. Only then is the scratch size compared with the array.
+  const wq_status v = wq_msd_gemm(x, M, N, K, n_components, group, qweight, scales, zeros, y,
+                                  nullptr, 0, stream);
+  if (v != WQ_ERR_WORKSPACE) return v;
   const size_t need = wq::msd_workspace_bytes(M, K, n_components);
   if (need > kScratchBytes) return WQ_ERR_UNSUPPORTED;
   void* scratch = nullptr;
@@ -69,9 +72,8 @@ wq_status wq_msd_gemm_noalloc(const void* x, int64_t M, int64_t N, int64_t K,
   } catch (...) {
     return WQ_ERR_CUDA;
   }
-  // wq_msd_gemm does all remaining validation (formats, shapes, alignment)
-  // before it launches anything; the digit planes and scales are rewritten by
-  // every call before they are read, so nothing has to start at zero.
+  // The digit planes and scales are rewritten by every call before they are
+  // read, so nothing in the array has to start at zero.
   return wq_msd_gemm(x, M, N, K, n_components, group, qweight, scales, zeros, y, scratch,
                      kScratchBytes, stream);
 }

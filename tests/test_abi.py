@@ -163,6 +163,29 @@ def test_gemm_and_msd_validation(wq):
     assert L.wq_msd_decompose(A16, 0, 128, 2, A16, A16, None) == wq.WQ_OK
 
 
+def test_noalloc_validates_like_msd_gemm(wq):
+    """wq_msd_gemm_noalloc checks its arguments exactly as wq_msd_gemm does
+    before it compares the problem's scratch with its fixed array, so an
+    oversized problem with a bad argument reports the bad argument."""
+    L = wq.lib
+    big = (A16, 4096, 5120, 5120, 2, 128, A16, A16, A16, A16)      # ~40 MiB of scratch
+    assert L.wq_msd_gemm_noalloc(*big, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_msd_gemm_noalloc(A16, 4096, 5120, 5000, 2, 125, A16, A16, A16, A16,
+                                 None) == wq.WQ_ERR_INVALID_ARG       # group % 8
+    assert L.wq_msd_gemm_noalloc(None, 4096, 5120, 5120, 2, 128, A16, A16, A16, A16,
+                                 None) == wq.WQ_ERR_INVALID_ARG       # x NULL
+    assert L.wq_msd_gemm_noalloc(A16, 4096, 5120, 5120, 2, 128, A16, A16, None, A16,
+                                 None) == wq.WQ_ERR_INVALID_ARG       # zeros NULL
+    assert L.wq_msd_gemm_noalloc(A16, 4096, 5120, 5120, 2, 128, A16, A16, A16, MIS,
+                                 None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_msd_gemm_noalloc(A16, 4096, 5120, 5120, 4, 128, A16, A16, A16, A16,
+                                 None) == wq.WQ_ERR_INVALID_ARG       # C in 1..3
+    assert L.wq_msd_gemm_noalloc(A16, 4096, 5120, 5120, 2, 64, A16, A16, A16, A16,
+                                 None) == wq.WQ_ERR_UNSUPPORTED       # G % 128
+    assert L.wq_msd_gemm_noalloc(A16, 0, 5120, 5120, 2, 128, A16, A16, A16, A16,
+                                 None) == wq.WQ_OK                    # empty: no-op
+
+
 def test_pack_and_dequant_validation(wq):
     L = wq.lib
     assert L.wq_quantize_pack(0, A16, 16, 100, 64, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG

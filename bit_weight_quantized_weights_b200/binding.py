@@ -39,6 +39,7 @@ EXPORTED = [
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
+    "wq_test_set_wait",
 ]
 
 
@@ -74,6 +75,7 @@ def _load():
         "wq_workspace_bytes": ([ctypes.c_int, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
                                ctypes.c_int),
         "wq_device_error": ([P, ctypes.c_int, ctypes.POINTER(U32)], ctypes.c_int),
+        "wq_test_set_wait": ([ctypes.c_uint64, ctypes.c_int], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -357,3 +359,10 @@ def wq_device_error(clear=True, stream=None):
     d = ctypes.c_uint32()
     st = lib.wq_device_error(_stream(stream), 1 if clear else 0, ctypes.byref(d))
     return st, d.value
+
+
+def wq_test_set_wait(limit_ns=0, stall=0):
+    """Test hook of the bounded device waits (see include/wq.h): the wait
+    limit in ns (0 = the default 2 s) and whether the loader withholds the
+    first k-tile of the tensor-core kernels."""
+    _check(lib.wq_test_set_wait(int(limit_ns), int(stall)), "wq_test_set_wait")

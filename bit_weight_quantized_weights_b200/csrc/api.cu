@@ -1,5 +1,6 @@
 // C ABI of the library: argument validation and dispatch to the kernels.
 // Every check happens before any launch; no C++ exception crosses the ABI.
+#include <atomic>
 #include <cstring>
 #include <exception>
 
@@ -30,6 +31,18 @@ size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C);
 wq_status read_gemm_error(bool clear, uint32_t* v);
 wq_status read_msd_error(bool clear, uint32_t* v);
 wq_status read_gemv_error(bool clear, uint32_t* v);
+}  // namespace wq
+
+namespace wq {
+namespace {
+std::atomic<uint64_t> g_wait_limit_ns{0};  // 0: the default
+std::atomic<int> g_wait_stall{0};
+}  // namespace
+
+WaitCtl wait_ctl() {
+  const uint64_t l = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return WaitCtl{l ? l : sm100_default_wait_ns(), g_wait_stall.load(std::memory_order_relaxed)};
+}
 }  // namespace wq
 
 using namespace wq;
@@ -328,6 +341,13 @@ wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K, int32_t 
       return WQ_OK;
   }
   return WQ_ERR_INVALID_ARG;
+}
+
+wq_status wq_test_set_wait(uint64_t limit_ns, int stall) {
+  if (stall != 0 && stall != 1) return WQ_ERR_INVALID_ARG;
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+  g_wait_stall.store(stall, std::memory_order_relaxed);
+  return WQ_OK;
 }
 
 wq_status wq_device_error(void* stream, int clear, uint32_t* detail) {

@@ -23,6 +23,21 @@ struct Nf4Table {
 // Host: the table computed once per process from the QLoRA construction.
 const Nf4Table& nf4_table();
 
+// Wait control of the kernels with bounded mbarrier waits, passed by value.
+//   limit_ns  how long any one wait may last before the kernel gives up
+//   stall     test hook: when 1, the TMA producer withholds the loads of the
+//             first k-tile, so the first waits on them expire (exercises the
+//             timeout, abort and drain path without a device fault)
+struct WaitCtl {
+  uint64_t limit_ns;
+  int32_t stall;
+};
+
+// Host: the process-wide setting (set by wq_test_set_wait; 2 s, no stall by
+// default).
+WaitCtl wait_ctl();
+constexpr uint64_t sm100_default_wait_ns() { return 2000000000ull; }
+
 // Host-side helpers shared by the launch wrappers.
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

@@ -30,7 +30,10 @@
 //               into y.
 // NF4 weights (block 64 = one k-tile) take the same path: a 256-entry
 // per-lane table turns each code byte into the fp16 pair of its two codebook
-// values, and one fp16 multiply applies the block's absmax.
+// values, and one fp16 multiply applies the block's absmax, prescaled in
+// fp32 by a power of two per weight row (the row's largest absmax lands in
+// [2^14, 2^15), so the product stays in fp16's normal range for any absmax;
+// the epilogue divides it back out).
 // Operands are fp16, not bf16: the activations arrive as fp16 copies scaled
 // by a power of two per row (exact), and the dequantized weight is
 // fp16_rn((q - z) * s): the nibble becomes fp16 1024 + q or 64 + q by one
@@ -50,6 +53,7 @@ namespace {
 __device__ unsigned int g_gemm_error;
 
 constexpr int BW = 128;          // weight rows per CTA (MMA M)
+constexpr int kRowMaxBytes = 4 * BW * 4;  // NF4: per-row partial absmax maxima [4][BW]
 constexpr int BK = 64;           // k per stage
 constexpr int kDeqWarps = 8;     // per k-tile: two per TMEM lane quarter
 // Dequantization warp groups, each taking every kGroups-th k-tile: a warp
@@ -84,9 +88,10 @@ struct GemmCfg {
   static constexpr int kRingOrOut = kRing > kOutBytes ? kRing : kOutBytes;
   static constexpr int kLutBytes = 256 * 32 * 4;  // NF4: byte -> fp16 pair, one copy per lane
   // ring or staging, 2^-e per token, barriers (512 B), alignment slack; NF4
-  // adds the lookup table after the barriers
+  // adds the lookup table and the per-row partial absmax maxima after the
+  // barriers
   static constexpr int kSmem = kRingOrOut + BT * 4 + 512 + 1024;
-  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
+  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes + kRowMaxBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
   static constexpr uint32_t kTmemCols = (BT + SA * kACols <= 256) ? 256 : 512;
   static_assert(BT + SA * kACols <= 512, "A stages fit in TMEM");
@@ -121,13 +126,38 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t zb_hi, uint32_
   out[3] = f16x2_mul(f16x2_sub(lop3_and_or(w8, 0x00F000F0u, 0x54005400u), zb_lo), s2);
 }
 
+// NF4: per weight row a power of two 2^e that puts the row's largest block
+// absmax in [2^14, 2^15), so that codebook value x absmax x 2^e rounds to
+// fp16 in its normal range (never above 2^15) whatever the absmax; the
+// epilogue multiplies by 2^-e. Blocks more than 2^28 below the row's largest
+// underflow toward zero, a negligible part of the row's products. The four
+// dequantization threads of a row (two groups x two k halves) each take the
+// max over every fourth block; `part` (0..3) names this thread's share and
+// rmax[part][128] collects them. All 32 * kDeqWarps * 2 dequantization
+// threads call this; returns (2^e, 2^-e).
+__device__ __forceinline__ float2 nf4_row_pow2(const float* arow, int nblk, int part, int r,
+                                               float* rmax, int nthreads) {
+  float mx = 0.0f;
+  for (int j = part; j < nblk; j += 4) mx = fmaxf(mx, __ldg(arow + j));
+  rmax[part * BW + r] = mx;
+  sm100::named_barrier(2, (uint32_t)nthreads);
+  mx = fmaxf(fmaxf(rmax[r], rmax[BW + r]), fmaxf(rmax[2 * BW + r], rmax[3 * BW + r]));
+  int e = 0;
+  if (mx > 0.0f && mx <= 3.4028235e38f) {
+    e = 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127);
+    e = e > 126 ? 126 : (e < -126 ? -126 : e);
+  }
+  return make_float2(__uint_as_float((uint32_t)(127 + e) << 23),
+                     __uint_as_float((uint32_t)(127 - e) << 23));
+}
+
 template <int BT, bool kNF4, int KB>
 __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x,
                       const __grid_constant__ CUtensorMap tmap_w,
                       const __grid_constant__ CUtensorMap tmap_y, const void* __restrict__ scales,
                       const __half* __restrict__ zeros, const float* __restrict__ inv_scale, int M,
-                      int N, int K, int G, Nf4Table tab) {
+                      int N, int K, int G, Nf4Table tab, WaitCtl wc) {
   using C = GemmCfg<BT, kNF4, KB>;
   constexpr int ST = C::kStages;
   constexpr int kDeqGroups = Deq<kNF4>::kGroups;
@@ -147,8 +177,10 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // NF4 only: lut[byte][lane] = fp16 pair (codebook[high nibble], codebook[low
-  // nibble]) = elements (2j, 2j + 1); lane l reads column l, so bank l
+  // nibble]) = elements (2j, 2j + 1); lane l reads column l, so bank l; then
+  // the per-row partial absmax maxima
   uint32_t* lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 512);
+  float* rmax = reinterpret_cast<float*>(lut + 256 * 32);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BW;
@@ -190,14 +222,18 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  int last_issued = -1;  // producer: the last k-tile whose loads it issued
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u;
-        if (kt >= ST && !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_gemm_error, 0x101u, abort_flag))
+        if (kt >= ST && !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_gemm_error, 0x101u, abort_flag,
+                                          wc.limit_ns))
           break;
+        if (wc.stall && kt == 0) continue;  // test hook: the first k-tile never arrives
+        last_issued = kt;
         uint8_t* st = ring + s * C::kStageBytes;
         sm100::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
 #pragma unroll
@@ -214,8 +250,8 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST, a = kt % SA;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u, pa = (uint32_t)(kt / SA) & 1u;
-        if (!sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x201u, abort_flag)) break;
-        if (!sm100::mbar_wait(&aready[a], pa, &g_gemm_error, 0x202u, abort_flag)) break;
+        if (!sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x201u, abort_flag, wc.limit_ns)) break;
+        if (!sm100::mbar_wait(&aready[a], pa, &g_gemm_error, 0x202u, abort_flag, wc.limit_ns)) break;
         sm100::tc_fence_after();
         const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
 #pragma unroll
@@ -262,6 +298,10 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     auto am_block = [&](int kt) { return (kt * KB + hk * (KB / 2)) / 64; };
     float am_next = (kNF4 && any) ? arow[am_block(grp)] : 0.0f;
     const uint32_t* lut_lane = lut + lane;
+    // NF4: the row's power of two (2^e, 2^-e); 1 for INT4
+    const float2 rpow = kNF4 ? nf4_row_pow2(arow, K / 64, 2 * grp + hk, r, rmax,
+                                            32 * kDeqWarps * kDeqGroups)
+                             : make_float2(1.0f, 1.0f);
     bool ok = true;
     for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
       const int s = kt % ST, a = kt % SA;
@@ -269,9 +309,9 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       const bool more = kt + kDeqGroups < KT;
       uint32_t am2 = 0;
       if (kNF4) {
-        // fp16x2 (absmax, absmax), rounded once; this warp's next one is
-        // loaded now
-        am2 = pack_f16x2(am_next, am_next);
+        // fp16x2 (absmax 2^e, absmax 2^e), rounded once; this warp's next
+        // one is loaded now
+        am2 = pack_f16x2(am_next * rpow.x, am_next * rpow.x);
         if (more) am_next = arow[am_block(kt + kDeqGroups)];
       } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
@@ -287,9 +327,9 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         left = tiles_per_group;
       }
       if (!kNF4) --left;
-      bool got = sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x301u, abort_flag);
+      bool got = sm100::mbar_wait(&full[s], ph, &g_gemm_error, 0x301u, abort_flag, wc.limit_ns);
       if (got && kt >= SA)
-        got = sm100::mbar_wait(&afree[a], pa ^ 1u, &g_gemm_error, 0x302u, abort_flag);
+        got = sm100::mbar_wait(&afree[a], pa ^ 1u, &g_gemm_error, 0x302u, abort_flag, wc.limit_ns);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -324,7 +364,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       if (lane == 0) sm100::mbar_arrive(&aready[a]);
     }
     // ---------------- epilogue ----------------
-    if (ok) ok = sm100::mbar_wait(accf, 0, &g_gemm_error, 0x401u, abort_flag);
+    if (ok) ok = sm100::mbar_wait(accf, 0, &g_gemm_error, 0x401u, abort_flag, wc.limit_ns);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (all_ok) {
       sm100::tc_fence_after();
@@ -338,7 +378,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         sm100::tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float val = __uint_as_float(v[j]) * s_inv[c0 + j];
+          const float val = __uint_as_float(v[j]) * s_inv[c0 + j] * rpow.y;
           out_s[(c0 + j) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
         }
       }
@@ -354,6 +394,22 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
 
   sm100::tc_fence_before();
   __syncthreads();
+  // After an abort (every role has left its loop, so nothing new is issued):
+  // the producer waits until each load it issued has landed (only its last
+  // ST can be in flight: k-tile kt was issued after k-tile kt - ST had been
+  // consumed), and the MMA issuer until its final commit reports every MMA
+  // done, so that no copy or MMA touches this CTA's shared memory or TMEM
+  // after it frees them and exits.
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int kt = max(0, last_issued - ST + 1); kt <= last_issued; ++kt)
+        if (!(wc.stall && kt == 0))
+          sm100::mbar_wait_drain(&full[kt % ST], (uint32_t)(kt / ST) & 1u, wc.limit_ns);
+    } else if (warp == 1 && lane == 0) {
+      sm100::mbar_wait_drain(accf, 0, wc.limit_ns);
+    }
+    __syncthreads();
+  }
   if (warp == 1) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, C::kTmemCols);
@@ -406,15 +462,16 @@ struct Gemm2Cfg {
   static constexpr int kOutBytes = BT * BW * 2;   // epilogue staging (reuses the ring)
   static constexpr int kLutBytes = 256 * 32 * 4;
   static constexpr int kSmem = kRing + BT * 4 + 512 + 1024;
-  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes : 0); }
+  static constexpr int smem(bool nf4) { return kSmem + (nf4 ? kLutBytes + kRowMaxBytes : 0); }
   static constexpr uint32_t kAccCols = BT;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kAccCols + kStages * kACols <= kTmemCols, "A stages fit in TMEM");
   static_assert(kOutBytes <= kRing, "the staging tile fits in the ring");
   static_assert(kStages % 2 == 0, "every stage is waited on by one group (up to two)");
   static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
-  // xfull, wfull, done, aready, accf, then the TMEM slot and the abort flag
-  static_assert(8 * (4 * kStages + 1) + 8 <= 512, "barriers fit their 512 bytes");
+  // xfull, wfull, done, aready, accf, then the TMEM slot, the abort flag and
+  // the two words the other CTA writes at the end
+  static_assert(8 * (4 * kStages + 1) + 16 <= 512, "barriers fit their 512 bytes");
 };
 
 template <bool kNF4, int KB>
@@ -424,7 +481,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
                            const __grid_constant__ CUtensorMap tmap_y,
                            const void* __restrict__ scales, const __half* __restrict__ zeros,
                            const float* __restrict__ inv_scale, int M, int N, int K, int G,
-                           Nf4Table tab) {
+                           Nf4Table tab, WaitCtl wc) {
   using C = Gemm2Cfg<KB>;
   constexpr int BT = C::BT;
   constexpr int ST = C::kStages;
@@ -444,7 +501,11 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   uint64_t* accf = aready + ST;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // written by the other CTA's producer at the end: its last issued k-tile
+  // and whether it gave up
+  volatile int* peer_info = reinterpret_cast<volatile int*>(tmem_slot + 2);
   uint32_t* lut = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(bars) + 512);
+  float* rmax = reinterpret_cast<float*>(lut + 256 * 32);  // NF4 per-row partial maxima
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = sm100::cluster_ctarank();  // 0: issues the MMAs
@@ -488,14 +549,18 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  int last_issued = -1;  // producer: the last k-tile whose loads it issued
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer (both CTAs) ----------------
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u;
-        if (kt >= ST && !sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x111u, abort_flag))
+        if (kt >= ST && !sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x111u, abort_flag,
+                                          wc.limit_ns))
           break;
+        if (wc.stall && kt == 0) continue;  // test hook: the first k-tile never arrives
+        last_issued = kt;
         uint8_t* st = ring + s * C::kStageBytes;
         sm100::mbar_arrive_expect_tx(&wfull[s], C::kWBytes);
         sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &wfull[s], kt * (kNF4 ? KB / 2 : KB / 8),
@@ -515,8 +580,8 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       for (int kt = 0; kt < KT; ++kt) {
         const int s = kt % ST;
         const uint32_t ph = (uint32_t)(kt / ST) & 1u;
-        if (!sm100::mbar_wait(&xfull[s], ph, &g_gemm_error, 0x211u, abort_flag)) break;
-        if (!sm100::mbar_wait(&aready[s], ph, &g_gemm_error, 0x212u, abort_flag)) break;
+        if (!sm100::mbar_wait(&xfull[s], ph, &g_gemm_error, 0x211u, abort_flag, wc.limit_ns)) break;
+        if (!sm100::mbar_wait(&aready[s], ph, &g_gemm_error, 0x212u, abort_flag, wc.limit_ns)) break;
         sm100::tc_fence_after();
         const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
 #pragma unroll
@@ -561,6 +626,10 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
     auto am_block = [&](int kt) { return (kt * KB + hk * (KB / 2)) / 64; };
     float am_next = (kNF4 && any) ? arow[am_block(grp)] : 0.0f;
     const uint32_t* lut_lane = lut + lane;
+    // NF4: the row's power of two (2^e, 2^-e); 1 for INT4
+    const float2 rpow = kNF4 ? nf4_row_pow2(arow, K / 64, 2 * grp + hk, r, rmax,
+                                            32 * kDeqWarps * kDeqGroups)
+                             : make_float2(1.0f, 1.0f);
     bool ok = true;
     for (int kt = grp; kt < KT && ok; kt += kDeqGroups) {
       const int s = kt % ST;
@@ -568,7 +637,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       const bool more = kt + kDeqGroups < KT;
       uint32_t am2 = 0;
       if (kNF4) {
-        am2 = pack_f16x2(am_next, am_next);
+        am2 = pack_f16x2(am_next * rpow.x, am_next * rpow.x);
         if (more) am_next = arow[am_block(kt + kDeqGroups)];
       } else if (left == 0) {
         const uint32_t sb = __half_as_ushort(s_next);
@@ -586,9 +655,9 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       if (!kNF4) --left;
       // the weight tile landed; A stage s is free once the MMAs of k-tile
       // kt - ST completed (they also freed the stage this tile landed in)
-      bool got = sm100::mbar_wait(&wfull[s], ph, &g_gemm_error, 0x311u, abort_flag);
+      bool got = sm100::mbar_wait(&wfull[s], ph, &g_gemm_error, 0x311u, abort_flag, wc.limit_ns);
       if (got && kt >= ST)
-        got = sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x312u, abort_flag);
+        got = sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x312u, abort_flag, wc.limit_ns);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
@@ -626,7 +695,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
       }
     }
     // ---------------- epilogue: this CTA's 128 rows x 256 tokens ----------------
-    if (ok) ok = sm100::mbar_wait(accf, 0, &g_gemm_error, 0x411u, abort_flag);
+    if (ok) ok = sm100::mbar_wait(accf, 0, &g_gemm_error, 0x411u, abort_flag, wc.limit_ns);
     const bool all_ok = __all_sync(0xffffffffu, ok);
     if (all_ok) {
       sm100::tc_fence_after();
@@ -638,7 +707,7 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
         sm100::tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float val = __uint_as_float(v[j]) * s_inv[c0 + j];
+          const float val = __uint_as_float(v[j]) * s_inv[c0 + j] * rpow.y;
           out_s[(c0 + j) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
         }
       }
@@ -655,7 +724,53 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   // neither CTA frees its TMEM or exits while the pair may still use it
   sm100::tc_fence_before();
   __syncthreads();
+  // Every role of this CTA has left its loop. Each producer tells the other
+  // which k-tile it issued last and whether this CTA gave up (remote stores,
+  // published by the cluster barrier), so both CTAs take the same path.
+  if (warp == 0 && lane == 0) {
+    const uint32_t peer = sm100::cluster_addr((const void*)peer_info, rank ^ 1u);
+    asm volatile("st.shared::cluster.v2.s32 [%0], {%1, %2};" ::"r"(peer), "r"(last_issued),
+                 "r"(*abort_flag)
+                 : "memory");
+  }
   sm100::cluster_sync();
+  if (*abort_flag || peer_info[1]) {
+    // The drain after an abort. A CTA's x half lands on the even CTA's
+    // barrier, which completes a phase only once the even CTA armed it and
+    // both halves landed. A producer issues k-tile kt only after the MMAs of
+    // kt - ST completed, so either producer is at most ST - 1 k-tiles ahead
+    // of the other, and the stages of the k-tiles it is ahead by are free in
+    // the other CTA. The producer that is behind issues its x half of those
+    // k-tiles (the even CTA arming each first); then every x phase either
+    // producer started completes, and the even CTA waits for the last ST of
+    // them (covering both CTAs' halves), each producer for its own weight
+    // loads, and the MMA issuer for its final commit.
+    if (warp == 0 && lane == 0) {
+      const int other_last = peer_info[0];
+      for (int kt = last_issued + 1; kt <= other_last; ++kt) {
+        if (wc.stall && kt == 0) continue;
+        const int s = kt % ST;
+        uint8_t* st = ring + s * C::kStageBytes;
+        if (leader) sm100::mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kXBlocks; ++blk)
+          sm100::tma_load_2d_pair(st + blk * (128 * 64 * 2), &tmap_x,
+                                  sm100::cluster_addr(&xfull[s], 0), kt * KB + 64 * blk,
+                                  m0 + 128 * (int)rank);
+      }
+      const int last_x = max(last_issued, other_last);
+      if (leader)
+        for (int kt = max(0, last_x - ST + 1); kt <= last_x; ++kt)
+          if (!(wc.stall && kt == 0))
+            sm100::mbar_wait_drain(&xfull[kt % ST], (uint32_t)(kt / ST) & 1u, wc.limit_ns);
+      for (int kt = max(0, last_issued - ST + 1); kt <= last_issued; ++kt)
+        if (!(wc.stall && kt == 0))
+          sm100::mbar_wait_drain(&wfull[kt % ST], (uint32_t)(kt / ST) & 1u, wc.limit_ns);
+    } else if (warp == 1 && lane == 0 && leader) {
+      sm100::mbar_wait_drain(accf, 0, wc.limit_ns);
+    }
+    sm100::cluster_sync();
+  }
   if (warp == 1) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc_pair(tmem, C::kTmemCols);
@@ -701,7 +816,8 @@ wq_status launch_pair(const void* x16, const float* inv_scale, int64_t M, int64_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, scales, static_cast<const __half*>(zeros),
-                         inv_scale, (int)M, (int)N, (int)K, G, nf4_table()) != cudaSuccess)
+                         inv_scale, (int)M, (int)N, (int)K, G, nf4_table(), wait_ctl()) !=
+      cudaSuccess)
     return WQ_ERR_CUDA;
   return launch_status();
 }
@@ -732,8 +848,10 @@ wq_status launch_bt(const void* x16, const float* inv_scale, int64_t M, int64_t 
       cudaSuccess)
     return WQ_ERR_CUDA;
   dim3 grid((unsigned)(N / BW), (unsigned)((M + BT - 1) / BT));
-  kern<<<grid, Deq<kNF4>::kThreads, smem, st>>>(tx, tw, ty, scales, static_cast<const __half*>(zeros),
-                                     inv_scale, (int)M, (int)N, (int)K, G, nf4_table());
+  kern<<<grid, Deq<kNF4>::kThreads, smem, st>>>(tx, tw, ty, scales,
+                                                 static_cast<const __half*>(zeros), inv_scale,
+                                                 (int)M, (int)N, (int)K, G, nf4_table(),
+                                                 wait_ctl());
   return launch_status();
 }
 

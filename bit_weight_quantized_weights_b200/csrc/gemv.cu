@@ -11,8 +11,8 @@
 // B200 design
 // -----------
 // * The weight stream is the whole cost (0.53 byte per weight against 2*M
-//   flops). Weights are read with plain 16-byte (8-byte for INT4 groups of
-//   64) loads that do not allocate in L1, by two 256-thread CTAs per SM,
+//   flops). Weights are read with plain 16-byte (8-byte for NF4 and INT4
+//   groups of 64) loads that do not allocate in L1, by two 256-thread CTAs per SM,
 //   each warp keeping three or four 128-k units of its 16 rows (with their
 //   group parameters) in flight while it computes the oldest. Measured on
 //   B200, plain coalesced loads stream HBM far better than a TMA ring of
@@ -33,14 +33,14 @@
 // * NF4 codes go through a 256-entry table indexed by a whole packed byte that
 //   yields the two fp16 code values already paired as one A-operand register.
 //   The table is replicated per lane (lane l reads column l, so bank l): every
-//   lookup is conflict-free. Each lane's 16 bytes (32 codes) lie inside one
-//   64-element absmax block, so one fp16x2 multiply per register applies the
-//   block's absmax to the A operand before the MMA (code, absmax and product
-//   each rounded once to fp16, as in the fused GEMM), which lets NF4 use the
-//   16-byte layout. The NF4 product runs in fp16: the staged x chunk is
-//   converted to fp16 scaled per token by a power of two that puts its largest
-//   magnitude in [2^14, 2^15) (exact for bf16 values down to 2^-28 of it); the
-//   power is divided back out of the partial.
+//   lookup is conflict-free. NF4 uses the 8-byte layout: half h of a unit is
+//   one 64-element absmax block, so every MMA stays inside one block and the
+//   block's fp32 absmax multiplies the MMA's partial sum in fp32 (only the
+//   code value is rounded, once, to fp16; a block of any absmax, however
+//   small, keeps full precision). The NF4 product runs in fp16: the staged x
+//   chunk is converted to fp16 scaled per token by a power of two that puts
+//   its largest magnitude in [2^14, 2^15) (exact for bf16 values down to
+//   2^-28 of it); the power is divided back out of the partial.
 // * Optional salient-channel residual correction (kRes, "DecDEC: A Systems
 //   Approach to Advancing Low-Bit LLM Quantization", Abstract): the owners add
 //   sum_j x[m, c_j] R^T[c_j, n] to each output in fp32 before its rounding.
@@ -56,9 +56,9 @@
 //   xs   [8*NT tokens][Kc] bf16 (fp16 for NF4), the CTA's K-chunk of x, in
 //        16-byte chunks. Only the M real tokens are written: a padding
 //        token's MMA column never reaches an output. Chunk c of token m sits
-//        at chunk c ^ (m & 1), and for the 16-byte layout (NF4, INT4 groups
-//        that are multiples of 128) also ^ (bit 3 of c moved to bit 1), so that the
-//        fragment loads of a warp hit distinct banks. For INT4 each chunk
+//        at chunk c ^ (m & 1), and for the 16-byte layout (INT4 groups that
+//        are multiples of 128) also ^ (bit 3 of c moved to bit 1), so that
+//        the fragment loads of a warp hit distinct banks. For INT4 each chunk
 //        holds the pairs (x0,x4)(x1,x5)(x2,x6)(x3,x7), the nibble pairing.
 //   xsum [Kc/64 or Kc/128][8*NT tokens] fp32, sums of x per group part (INT4)
 //   lut  [256 entries][32 lanes] u32 (NF4 only)
@@ -105,12 +105,6 @@ __device__ __forceinline__ void mma16816_f16(float (&d)[4], uint32_t a0, uint32_
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t f16x2_mul(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
 // (128 + nibble) as bf16 for nibbles e and e + 4 of w -> one bf16x2 register.
 __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
   return lop3_and_or(w >> (4 * e), 0x000F000Fu, 0x43004300u);
@@ -126,8 +120,8 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
 //           32 + 8t), w[4..7] the same of row g + 8; prm[2h + i] = the scale
 //           bits of half h for row g (i = 0) or g + 8 (i = 1), zz[2h + i] the
 //           zero bits.
-// NF4 (wide): prm[i] = the fp32 absmax bits of the lane's block (2u + t / 2)
-// of row g (i = 0) or g + 8 (i = 1).
+// NF4 (narrow): prm[2h + i] = the fp32 absmax bits of block 2u + h of row g
+// (i = 0) or g + 8 (i = 1).
 // The fp16 parameters stay as loaded (zero-extended 16-bit loads, no
 // arithmetic on them) until the unit is computed, so the loads never stall a
 // warp that is still issuing its first units and staging x.
@@ -140,7 +134,7 @@ struct Unit {
 template <bool kNF4, bool kWide>
 __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint8_t* wB, int u,
                                           int nA, int nB, const GemvArgs& p, int ng, int t) {
-  static_assert(kWide || !kNF4, "NF4 uses the 16-byte layout");
+  static_assert(!(kWide && kNF4), "NF4 uses the 8-byte layout");
   const int64_t off = (int64_t)u * 64;
   if (kWide) {
     const uint4 a = ld_stream_u4(wA + off), b = ld_stream_u4(wB + off);
@@ -153,12 +147,13 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
   }
   if (kNF4) {
-    // the lane's 32 codes (bytes 16t .. 16t + 15 of the unit) lie in block
-    // 2u + t / 2 of rows g and g + 8
+    // half h of the unit (bytes 32h + 8t .. + 7 of each row) is block 2u + h
     const float* am = static_cast<const float*>(p.scales);
-    const int blk = 2 * u + (t >> 1);
-    U.prm[0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + blk));
-    U.prm[1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + blk));
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      U.prm[2 * h + 0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + 2 * u + h));
+      U.prm[2 * h + 1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + 2 * u + h));
+    }
   } else {
     const unsigned short* s16 = reinterpret_cast<const unsigned short*>(p.scales);
     const unsigned short* z16 = reinterpret_cast<const unsigned short*>(p.zeros);
@@ -203,47 +198,57 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
                                              const float* xsum, const uint32_t* lut_lane, int g,
                                              int t, float (&acc)[NT][4], int mlast = 15) {
   constexpr int kTok = 8 * NT;
-  if (kNF4 && kWide) {
-    // The lane's 16 bytes of rows g and g + 8 hold codes k = 32t .. 32t + 31,
-    // all in one absmax block, applied to the A operand before the MMA (one
-    // fp16 multiply per code pair). Step (w, hh) uses bytes 4w + 2hh and
-    // 4w + 2hh + 1: codes 32t + 8w + 4hh + {0..3}; x is staged in natural
-    // order, so that chunk 4t + w of each token holds exactly those x.
-    const uint32_t amA = pack_f16x2(__uint_as_float(U.prm[0]), __uint_as_float(U.prm[0]));
-    const uint32_t amB = pack_f16x2(__uint_as_float(U.prm[1]), __uint_as_float(U.prm[1]));
-    float cp[2][NT][4];
+  if (kNF4) {
+    // Narrow layout: half h of the unit is one 64-element absmax block, so
+    // every MMA below stays inside one block. The table gives the fp16 code
+    // values (each rounded once); the MMA sums them against the fp16 x
+    // (exact) in fp32, and the block's fp32 absmax multiplies that partial
+    // sum in fp32. Step ks = (jw, hh) of half h uses bytes 4jw + 2hh and
+    // 4jw + 2hh + 1 of word 2h + jw: codes 64h + 16t + 8jw + 4hh + {0..3};
+    // x is staged in natural order, so chunk 8h + 2t + jw holds them.
 #pragma unroll
-    for (int c = 0; c < 2; ++c)
+    for (int h = 0; h < 2; ++h) {
+      float cp[2][NT][4];
 #pragma unroll
-      for (int a = 0; a < NT; ++a)
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) cp[c][a][r] = 0.0f;
+        for (int a = 0; a < NT; ++a)
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      uint4 X[NT];
+          for (int r = 0; r < 4; ++r) cp[c][a][r] = 0.0f;
+      uint4 X[NT][2];
 #pragma unroll
       for (int a = 0; a < NT; ++a) {
         const int tok = min(g + 8 * a, mlast);
-        const int pc = (16 * lu + 4 * t + w) ^ (t & 2) ^ (tok & 1);
-        X[a] = *reinterpret_cast<const uint4*>(xs + (size_t)tok * kc + pc * 8);
+        const int c0 = 16 * lu + 8 * h + 2 * t;
+        const uint16_t* base = xs + (size_t)tok * kc;
+        X[a][0] = *reinterpret_cast<const uint4*>(base + (c0 ^ (tok & 1)) * 8);
+        X[a][1] = *reinterpret_cast<const uint4*>(base + ((c0 + 1) ^ (tok & 1)) * 8);
       }
-      const uint32_t WA = U.w[w], WB = U.w[4 + w];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+      for (int ks = 0; ks < 4; ++ks) {
+        const int jw = ks >> 1, hh = ks & 1;
+        const uint32_t WA = U.w[2 * h + jw], WB = U.w[4 + 2 * h + jw];
         const int sh0 = 16 * hh, sh1 = sh0 + 8;
-        const uint32_t a0 = f16x2_mul(lut_lane[((WA >> sh0) & 0xFFu) * 32], amA);
-        const uint32_t a1 = f16x2_mul(lut_lane[((WB >> sh0) & 0xFFu) * 32], amB);
-        const uint32_t a2 = f16x2_mul(lut_lane[((WA >> sh1) & 0xFFu) * 32], amA);
-        const uint32_t a3 = f16x2_mul(lut_lane[((WB >> sh1) & 0xFFu) * 32], amB);
+        const uint32_t a0 = lut_lane[((WA >> sh0) & 0xFFu) * 32];
+        const uint32_t a1 = lut_lane[((WB >> sh0) & 0xFFu) * 32];
+        const uint32_t a2 = lut_lane[((WA >> sh1) & 0xFFu) * 32];
+        const uint32_t a3 = lut_lane[((WB >> sh1) & 0xFFu) * 32];
 #pragma unroll
-        for (int a = 0; a < NT; ++a)
-          mma16816_f16(cp[hh][a], a0, a1, a2, a3, hh ? X[a].z : X[a].x, hh ? X[a].w : X[a].y);
+        for (int a = 0; a < NT; ++a) {
+          const uint32_t b0 = hh ? X[a][jw].z : X[a][jw].x;
+          const uint32_t b1 = hh ? X[a][jw].w : X[a][jw].y;
+          mma16816_f16(cp[hh][a], a0, a1, a2, a3, b0, b1);
+        }
+      }
+      const float amA = __uint_as_float(U.prm[2 * h]), amB = __uint_as_float(U.prm[2 * h + 1]);
+#pragma unroll
+      for (int a = 0; a < NT; ++a) {
+        acc[a][0] = fmaf(amA, cp[0][a][0] + cp[1][a][0], acc[a][0]);
+        acc[a][1] = fmaf(amA, cp[0][a][1] + cp[1][a][1], acc[a][1]);
+        acc[a][2] = fmaf(amB, cp[0][a][2] + cp[1][a][2], acc[a][2]);
+        acc[a][3] = fmaf(amB, cp[0][a][3] + cp[1][a][3], acc[a][3]);
       }
     }
-#pragma unroll
-    for (int a = 0; a < NT; ++a)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) acc[a][r] += cp[0][a][r] + cp[1][a][r];
   } else if (kWide) {
     // two accumulator chains (even and odd k-steps) halve the MMA dependency chain
     float cp[2][NT][4];
@@ -540,9 +545,10 @@ wq_status launch_gemv(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
   const bool res = k > 0;
   if (fmt == WQ_FMT_NF4) {
     if (res)
-      return NT == 1 ? launch_t<1, true, true, true>(a, st, early)
-                     : launch_t<2, true, true, true>(a, st, early);
-    return NT == 1 ? launch_t<1, true, true, false>(a, st) : launch_t<2, true, true, false>(a, st);
+      return NT == 1 ? launch_t<1, true, false, true>(a, st, early)
+                     : launch_t<2, true, false, true>(a, st, early);
+    return NT == 1 ? launch_t<1, true, false, false>(a, st)
+                   : launch_t<2, true, false, false>(a, st);
   }
   if (group % 128 == 0) {
     if (res)

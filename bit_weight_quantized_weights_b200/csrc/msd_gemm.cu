@@ -81,7 +81,7 @@ struct MsdCfg {
   static constexpr int kStages = (4 * kStageBytes + 256 + 1024 <= 232448) ? 4 : 3;
   static constexpr int kSmem = kStages * kStageBytes + 256 + 1024;
   // the transpose tile and the split-K partials reuse the stage ring
-  static_assert(kStages >= 2 && 3 * kStages + 2 * kNB <= 31, "stages and barriers");
+  static_assert(kStages >= 2 && 3 * kStages + 2 * kNB + 1 <= 31, "stages and barriers");
   static_assert(kStages * kStageBytes >= BM * kOutPitch * 2, "transpose tile");
   // S ranks of ceil(128 / S) rows, S <= 8
   static_assert(kStages * kStageBytes >= (BN + 7) * kRedPitch * 4, "split-K partials");
@@ -136,7 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     msd_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const __grid_constant__ CUtensorMap tmap_w, const __half* __restrict__ scales,
                     const __half* __restrict__ zeros, const float* __restrict__ comp_scales,
-                    uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad, int S) {
+                    uint16_t* __restrict__ y, int M, int N, int K, int G, int m_pad, int S,
+                    WaitCtl wc) {
   using Cfg = MsdCfg<C>;
   constexpr int NB = Cfg::kNB;
   constexpr int kStages = Cfg::kStages;
@@ -152,7 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = bars + 2 * kStages;
   uint64_t* acc_full = bars + 3 * kStages;
   uint64_t* acc_empty = acc_full + NB;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + NB);
+  uint64_t* mma_done = acc_empty + NB;  // the MMA issuer's final commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,6 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm100::mbar_init(&acc_full[b], 1);
       sm100::mbar_init(&acc_empty[b], kEpiWarps);
     }
+    sm100::mbar_init(mma_done, 1);
     *abort_flag = 0;
     sm100::fence_mbar_init();
   }
@@ -198,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm100::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  int last_issued = -1;  // producer: the last k-tile (of this rank) whose loads it issued
   if (warp == 0) {
     if (lane == 0) {
       for (int i = 0; i < KT; ++i) {
@@ -205,8 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % kStages;
         const uint32_t ph = (uint32_t)(i / kStages) & 1u;
         if (i >= kStages &&
-            !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_msd_error, 0x1101u, abort_flag))
+            !sm100::mbar_wait(&empty[s], ph ^ 1u, &g_msd_error, 0x1101u, abort_flag, wc.limit_ns))
           break;
+        if (wc.stall && i == 0) continue;  // test hook: the first k-tile never arrives
+        last_issued = i;
         sm100::mbar_arrive_expect_tx(&full[s], C * kPlaneBytes + kWBytes);
 #pragma unroll
         for (int c = 0; c < C; ++c)
@@ -229,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = gi % NB;
         if (gi >= NB) {
           if (!sm100::mbar_wait(&acc_empty[b], (uint32_t)((gi / NB) - 1) & 1u, &g_msd_error,
-                                0x1201u, abort_flag)) {
+                                0x1201u, abort_flag, wc.limit_ns)) {
             ok = false;
             break;
           }
@@ -241,8 +247,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < sg1 - sg0; ++t, ++i) {
           const int s = i % kStages;
           const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-          if (!sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1202u, abort_flag) ||
-              !sm100::mbar_wait(&deq[s], ph, &g_msd_error, 0x1203u, abort_flag)) {
+          if (!sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1202u, abort_flag, wc.limit_ns) ||
+              !sm100::mbar_wait(&deq[s], ph, &g_msd_error, 0x1203u, abort_flag, wc.limit_ns)) {
             ok = false;
             break;
           }
@@ -269,6 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) sm100::mma_commit(&acc_full[b]);
       }
+      sm100::mma_commit(mma_done);
     }
   } else if (warp < 2 + kUnpackWarps) {
     // ---------------- unpack: B row r = feature n0 + r ----------------
@@ -288,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         zrep = (uint32_t)__half2float(z_next) * 0x01010101u;
         z_next = zrow[min(kt / TPG + 1, NG - 1)];
       }
-      bool got = sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1301u, abort_flag);
+      bool got = sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1301u, abort_flag, wc.limit_ns);
       if (!__all_sync(0xffffffffu, got)) break;
       const uint4* wsrc = reinterpret_cast<const uint4*>(sW + s * kWBytes + r * 64);
       uint8_t* bdst = sB + s * kBBytes + r * 128;
@@ -329,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float scl_next = gi + 1 < NSG ? __half2float(srow[gi + 1]) : 0.0f;
       if (ok) {
         bool got = sm100::mbar_wait(&acc_full[b], (uint32_t)(gi / NB) & 1u, &g_msd_error,
-                                    0x1401u, abort_flag);
+                                    0x1401u, abort_flag, wc.limit_ns);
         ok = __all_sync(0xffffffffu, got);
       }
       if (!ok) break;
@@ -449,6 +456,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   sm100::tc_fence_before();
   __syncthreads();
+  // After an abort (every role has left its loop): the producer waits until
+  // each load it issued has landed (only its last kStages can be in flight:
+  // k-tile i was issued after k-tile i - kStages had been consumed), and the
+  // MMA issuer until its final commit reports every MMA done, before TMEM is
+  // freed and the CTA exits.
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int i = max(0, last_issued - kStages + 1); i <= last_issued; ++i)
+        if (!(wc.stall && i == 0))
+          sm100::mbar_wait_drain(&full[i % kStages], (uint32_t)(i / kStages) & 1u, wc.limit_ns);
+    } else if (warp == 1 && lane == 0) {
+      sm100::mbar_wait_drain(mma_done, 0, wc.limit_ns);
+    }
+    __syncthreads();
+  }
   if (warp == 1) {
     sm100::tc_fence_after();
     sm100::tmem_dealloc(tmem, Cfg::kTmemCols);
@@ -542,7 +564,7 @@ wq_status launch_c(const CUtensorMap& ta, const CUtensorMap& tw, const void* sca
   cfg.numAttrs = S > 1 ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, kern, ta, tw, static_cast<const __half*>(scales),
                          static_cast<const __half*>(zeros), cs, static_cast<uint16_t*>(y), (int)M,
-                         (int)N, (int)K, G, (int)mp, S) != cudaSuccess)
+                         (int)N, (int)K, G, (int)mp, S, wait_ctl()) != cudaSuccess)
     return WQ_ERR_CUDA;
   return launch_status();
 }

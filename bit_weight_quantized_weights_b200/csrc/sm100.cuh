@@ -10,12 +10,14 @@ namespace wq {
 namespace sm100 {
 
 // ---------------------------------------------------------------------------
-// Bounded waits. Every wait gives up after kWaitLimitNs of wall time, records
+// Bounded waits. Every wait gives up after a limit of wall time (WaitCtl,
+// chosen by the host: 2 s by default, sm100_default_wait_ns(); real waits
+// take microseconds), records
 // `site` in the kernel's error word and returns false. Callers then skip the
-// rest of their role and fall through to the common exit (which frees TMEM).
+// rest of their role and fall through to the common exit, which first drains
+// what is still in flight (the producer waits for its issued TMA loads, the
+// MMA issuer for its last commit) and then frees TMEM.
 // ---------------------------------------------------------------------------
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s; real waits take microseconds
-
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -56,19 +58,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase of `bar` with the given parity to complete. `abort` is a
 // shared flag any role sets when it gives up, so the others stop waiting too.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned int* err,
-                                          uint32_t site, volatile int* abort) {
+                                          uint32_t site, volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         atomicCAS(err, 0u, site);
         *abort = 1;
         return false;
       }
     }
+  }
+}
+
+// The drain after an abort: wait for the phase regardless of the abort flag,
+// still bounded by the limit (false if it expired).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 0 && globaltimer() - t0 > limit_ns) return false;
   }
 }
 

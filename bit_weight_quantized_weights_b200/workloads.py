@@ -60,3 +60,26 @@ def layer(m, n, k, seed=0, outliers=None):
 def flat_weights(n, k, seed=0):
     """fp32 [N, K] weights for the standalone NF4 dequantization workload."""
     return weights(n, k, seed=seed)
+
+
+def scaled_weights(n, k, seed=0, row_exp=None, block_exp=None, factor=1.0):
+    """fp32 [N, K] ~ N(0, 0.02) x `factor`, with rows and/or 64-element blocks
+    (of the flattened row-major matrix) scaled by powers of ten, CPU:
+
+    row_exp (lo, hi): row n is multiplied by 10^(lo + n mod (hi - lo + 1));
+    block_exp (lo, hi): each block is multiplied by 10^u, u drawn uniformly
+    from [lo, hi] on the same generator after W.
+
+    Layers whose weights span many orders of magnitude, for the NF4 paths
+    whose block absmax enters a narrower floating-point type."""
+    g = generator(seed)
+    w = weights(n, k, gen=g) * factor
+    if block_exp is not None:
+        lo, hi = block_exp
+        u = torch.rand(n * k // 64, generator=g, dtype=torch.float64) * (hi - lo) + lo
+        w = (w.reshape(-1, 64).double() * torch.pow(10.0, u)[:, None]).float().reshape(n, k)
+    if row_exp is not None:
+        lo, hi = row_exp
+        e = lo + torch.arange(n) % (hi - lo + 1)
+        w = (w.double() * torch.pow(10.0, e.double())[:, None]).float()
+    return w

@@ -158,9 +158,12 @@ wq_status wq_int4_dequant(const uint32_t* qweight, const void* scales,
  *   x bf16 [M, K] row-major; y bf16 [M, N] row-major.
  *   INT4: scales/zeros fp16 [N, K/G], G % 64 == 0, K % G == 0. The group's
  *         scale and zero are applied after the group's sum ([MIXPE]).
- *   NF4 : group == 64, scales = fp32 absmax [N*K/64], zeros NULL; the code
- *         value, the block's absmax and their product are each rounded once
- *         to fp16 (absmax <= 65504), as in wq_w4a16_gemm.
+ *   NF4 : group == 64, scales = fp32 absmax [N*K/64], zeros NULL. The code
+ *         values are rounded once to fp16 and multiply an fp16 copy of x
+ *         (scaled per token by a power of two: exact for bf16 values down to
+ *         2^-28 of the token's largest) with fp32 accumulation; each 64-element
+ *         block's partial sum is then multiplied by its fp32 absmax in fp32, so
+ *         blocks of any finite absmax, however small, keep full precision.
  * Requires K % 128 == 0 and N % 16 == 0. M == 0 or N == 0 is a no-op.
  * Workspace: none needed (pass NULL, 0); split-K partials are reduced on chip
  * through thread-block-cluster shared memory.
@@ -226,10 +229,14 @@ wq_status wq_w4a16_gemv_salient(const void* x, int64_t M, int64_t N, int64_t K,
  * the dequantize-then-multiply product; here the dequantized tile is written
  * straight into tensor memory and never leaves the SM). Same arguments and
  * layouts as wq_w4a16_gemv, any
- * M >= 1, INT4 or NF4 ([NF4]: codebook value x block absmax, both rounded to
- * fp16 and multiplied in fp16). Requires K % 128 == 0, N % 128 == 0,
- * G % 64 == 0, K % G == 0, and INT4 group scales with 15 * s <= 65504 (NF4
- * absmax <= 65504).
+ * M >= 1, INT4 or NF4. Requires K % 128 == 0, N % 128 == 0, G % 64 == 0,
+ * K % G == 0, and INT4 group scales with 15 * s <= 65504.
+ * NF4 ([NF4]: codebook value x block absmax): per weight row n a power of two
+ * 2^e_n puts the row's largest absmax in [2^14, 2^15); each weight is
+ * fp16_rn(fp16(code) * fp16_rn(absmax * 2^e_n)) and the epilogue divides 2^e_n
+ * back out. Any finite absmax works; a block more than 2^28 below its row's
+ * largest absmax loses relative precision, a negligible part of that row's
+ * outputs.
  * The product runs in fp16 with fp32 accumulation: x is first copied to fp16
  * scaled per row by a power of two (exact for bf16 values down to 2^-28 of the
  * row's largest), each weight is fp16_rn((q - z) * s), and the epilogue
@@ -310,6 +317,25 @@ wq_status wq_msd_gemm_noalloc(const void* x, int64_t M, int64_t N, int64_t K,
 wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K,
                              int32_t group, int32_t n_components,
                              size_t* bytes);
+
+/*
+ * Test hook for the bounded device waits. The pages have no counterpart: it
+ * exists so that the timeout path can be exercised without a device fault.
+ * It applies to every later launch, in this process, of the kernels with
+ * bounded waits (the tensor-core kernels of wq_w4a16_gemm, and of
+ * wq_msd_gemm for M > 16):
+ *   limit_ns  how long any one device wait may last before the kernel gives
+ *             up; 0 restores the default of 2 s;
+ *   stall     1: the kernel's loader withholds the first k-tile, so the first
+ *             waits on it expire after limit_ns; 0: normal operation.
+ * A kernel that gives up records its wait site for wq_device_error
+ * (WQ_ERR_TIMEOUT), waits (bounded by limit_ns) for the copies and
+ * tensor-core operations it has in flight, frees its tensor memory and
+ * returns; its output is then unspecified. Host only; process-wide; change it
+ * only while no such kernel is being launched from another thread.
+ * Returns WQ_ERR_INVALID_ARG for a stall other than 0 or 1.
+ */
+wq_status wq_test_set_wait(uint64_t limit_ns, int stall);
 
 /*
  * Read (and, if `clear` != 0, reset) the library's sticky device error word,

@@ -51,6 +51,30 @@ def check_within_bf16_rounding(y_gpu, y_ref, what="", slack=1e-4):
         what, int(bad.sum()), float(np.max(np.abs(y - r) - bound)))
 
 
+# Unit roundoff of binary16 (half the spacing at 1): the largest relative
+# error of one round-to-nearest to fp16 in its normal range.
+FP16_U = 2.0 ** -11
+
+
+def check_within_error_bound(y_gpu, y_ref, y_abs, eps, what=""):
+    """Element-wise forward error bound of a dot product:
+    |y - y_ref| <= one bf16 ulp of y_ref + eps * sum_k |x_k| |w_k|.
+
+    y_abs is sum_k |x_k| |w_k| per output (the oracle's product of |x| and
+    |W_hat|); eps is the kernel's relative error per term (its roundings of
+    each weight or activation, plus fp32 accumulation), and the bf16 ulp
+    covers the output's own rounding. Unlike a slack in units of the output's
+    RMS, this bound holds for outputs that cancel inside rows whose terms are
+    far larger than the typical output."""
+    y = y_gpu.float().cpu().numpy().astype(np.float64) if isinstance(y_gpu, torch.Tensor) \
+        else np.asarray(y_gpu, dtype=np.float64)
+    r = np.asarray(y_ref, dtype=np.float64)
+    bound = numerics.bf16_ulp(r) + eps * np.asarray(y_abs, dtype=np.float64)
+    bad = np.abs(y - r) > bound
+    assert not bad.any(), "%s: %d elements beyond the error bound (worst %.3e)" % (
+        what, int(bad.sum()), float(np.max(np.abs(y - r) - bound)))
+
+
 @functools.lru_cache(maxsize=16)
 def int4_packed(n, k, group, seed=0):
     """Oracle-quantized INT4 weights of the seeded W [N, K]: (q, s, z, qweight)."""

@@ -157,3 +157,73 @@ def test_gemm_nf4_full_size_sampled(wq, m, n, k):
     rows = np.sort(rng.choice(m, 48, replace=False))
     cols = np.sort(rng.choice(n, 192, replace=False))
     _run_nf4_gemm(wq, m, n, k, seed=1, rows=rows, cols=cols)
+
+
+# NF4 layers whose block absmax spans many orders of magnitude (see the GEMV
+# test of the same name): the per-row power of two must keep every row's
+# products in fp16's normal range. Rows are checked class by class, every
+# output against the dot product's forward error bound.
+NF4_RANGE_CASES = {
+    "layer_1e-6": dict(factor=1e-6),
+    "layer_1e-9": dict(factor=1e-9),
+    "layer_1e4": dict(factor=1e4),
+    "blocks_1e-8_1e3": dict(block_exp=(-8, 3)),
+    "rows_1e-9_1e2": dict(row_exp=(-9, 2)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(NF4_RANGE_CASES))
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (520, 9472, 1024)])
+def test_gemm_nf4_absmax_range(wq, case, m, n, k):
+    from bit_weight_quantized_weights_b200 import workloads
+    from oracle import formats
+    w = workloads.scaled_weights(n, k, seed=12, **NF4_RANGE_CASES[case]).numpy()
+    codes, absmax = formats.nf4_quantize(w)
+    cw, am = helpers.to_dev_nf4(absmax, formats.nf4_pack(codes))
+    x = _x(m, k, 12)
+    ws = wq.gemm_workspace(m, n, k, 64)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None, workspace=ws)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    xf = helpers.x_f32(x)
+    y_ref = products.w4a16_nf4(xf, codes, absmax, k)
+    w_abs = np.abs(formats.nf4_dequant_exact(codes, absmax).reshape(n, k))
+    y_abs = products.matmul_exact(np.abs(xf), w_abs)
+    # per weight: the code value, absmax x 2^e and their product each round
+    # once to fp16 (x is exact in fp16); fp32 accumulation adds at most
+    # K x 2^-23 relative of the sum of |terms|
+    eps = 3 * helpers.FP16_U + k * 2.0 ** -23
+    yc = y.cpu()
+    classes = [np.arange(n)]
+    if "row_exp" in NF4_RANGE_CASES[case]:
+        lo, hi = NF4_RANGE_CASES[case]["row_exp"]
+        classes = [np.arange(c, n, hi - lo + 1) for c in range(hi - lo + 1)]
+    for cols in classes:
+        what = "nf4 gemm %s %dx%dx%d rows %d.." % (case, m, n, k, cols[0])
+        helpers.check_product(yc[:, cols], y_ref[:, cols], what)
+        helpers.check_within_error_bound(yc[:, cols], y_ref[:, cols], y_abs[:, cols], eps, what)
+
+
+def test_gemm_tiny_activations_beside_large(wq):
+    """The fp16 copy of x scales each row so its largest value lands in
+    [2^14, 2^15): bf16 values more than 2^28 below it become 0. A row with one
+    large value and the rest 2^-29 .. 2^-31 of it (all flushed), a row with
+    values spread over 2^-20 .. 1 of its largest, and plain rows all stay
+    within the product tolerance and one bf16 rounding."""
+    m, n, k, group = 130, 256, 512, 128
+    q, s, z, qweight = helpers.int4_packed(n, k, group, seed=21)
+    qw, sc, zr = helpers.to_dev_int4(s, z, qweight)
+    x = _x(m, k, 21).float()
+    g = torch.Generator().manual_seed(21)
+    x[0] = 1000.0 * torch.randn(k, generator=g) * 2.0 ** -30
+    x[0, 7] = 1000.0
+    x[1] = torch.randn(k, generator=g) * torch.pow(2.0, -20.0 * torch.rand(k, generator=g))
+    x = x.to(torch.bfloat16)
+    y = wq.wq_w4a16_gemm(x.cuda(), n, wq.WQ_FMT_INT4_ASYM, group, qw, sc, zr)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    y_ref = products.w4a16_int4(helpers.x_f32(x), q, s, z, group)
+    for rows in (np.array([0]), np.array([1]), np.arange(2, m)):
+        what = "gemm tiny-x rows %d.." % rows[0]
+        helpers.check_product(y[rows], y_ref[rows], what)
+        helpers.check_within_bf16_rounding(y[rows], y_ref[rows], what, slack=EVERY_ELEMENT_SLACK)

@@ -5,11 +5,13 @@ NF4 b64, 1% outlier channels x20) and the tiny INT4 g64 case are run at full
 size, every output compared. INT4 dequantizes exactly inside the kernel, so
 besides the product tolerance every INT4 output must lie within one bf16
 rounding of the exact product. NF4 multiplies exactly scaled fp16 activations
-by fp16 weights: the code value, the block's absmax and their product each
-round once to fp16, as in the fused GEMM, so its element bound carries the
-same 3e-3 RMS slack as the GEMM's NF4 cases.
+by the fp16 code values (each rounded once) and applies each block's absmax in
+fp32 to the block's partial sum; its element bound keeps the 3e-3 RMS slack of
+the GEMM's NF4 cases (the code rounding alone, at most 2^-11 relative per
+weight, stays well inside it).
 """
 
+import numpy as np
 import pytest
 import torch
 
@@ -50,8 +52,8 @@ def _run_nf4(wq, m, n, k, outliers=(0.01, 20.0), seed=0):
     y = wq.wq_w4a16_gemv(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None)
     torch.cuda.synchronize()
     y_ref = products.w4a16_nf4(helpers.x_f32(x), codes, absmax, k)
-    # three fp16 roundings per weight (code, absmax, product; 2^-11 relative
-    # each, about 2^-10.2 together) spread over the K-term sum
+    # one fp16 rounding per weight (the code value, 2^-11 relative at most),
+    # spread over the K-term sum
     helpers.check_within_bf16_rounding(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k), slack=3e-3)
     return helpers.check_product(y, y_ref, "nf4 gemv M=%d %dx%d" % (m, n, k))
 
@@ -160,3 +162,47 @@ def test_gemv_nan_propagates(wq):
     x[1, 7] = float("nan")
     y = wq.wq_w4a16_gemv(x.cuda(), 128, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, zr).cpu()
     assert torch.isfinite(y[0].float()).all() and torch.isnan(y[1].float()).all()
+
+
+# NF4 layers whose block absmax spans many orders of magnitude: the whole
+# layer tiny (absmax ~5e-8 and ~5e-11, below fp16's normal range), blocks
+# spread over 1e-8 .. 1e3 within every row, and rows of 1e-9 .. 1e2, checked
+# class by class so that the tiny rows are held to their own scale, every
+# output against the dot product's forward error bound.
+NF4_RANGE_CASES = {
+    "layer_1e-6": dict(factor=1e-6),
+    "layer_1e-9": dict(factor=1e-9),
+    "blocks_1e-8_1e3": dict(block_exp=(-8, 3)),
+    "rows_1e-9_1e2": dict(row_exp=(-9, 2)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(NF4_RANGE_CASES))
+@pytest.mark.parametrize("m", [1, 16])
+def test_gemv_nf4_absmax_range(wq, case, m):
+    from bit_weight_quantized_weights_b200 import workloads
+    from oracle import formats
+    n, k = 1024, 4096
+    w = workloads.scaled_weights(n, k, seed=11, **NF4_RANGE_CASES[case]).numpy()
+    codes, absmax = formats.nf4_quantize(w)
+    cw, am = helpers.to_dev_nf4(absmax, formats.nf4_pack(codes))
+    x = _x(m, k, 11, (0.01, 20.0))
+    y = wq.wq_w4a16_gemv(x.cuda(), n, wq.WQ_FMT_NF4, 64, cw, am, None)
+    torch.cuda.synchronize()
+    xf = helpers.x_f32(x)
+    y_ref = products.w4a16_nf4(xf, codes, absmax, k)
+    w_abs = np.abs(formats.nf4_dequant_exact(codes, absmax).reshape(n, k))
+    y_abs = products.matmul_exact(np.abs(xf), w_abs)
+    # per weight: the code value rounds once to fp16 (x is exact in fp16, the
+    # absmax is applied in fp32: one more rounding of a partial sum); fp32
+    # accumulation adds at most K x 2^-23 relative of the sum of |terms|
+    eps = helpers.FP16_U + k * 2.0 ** -23
+    yc = y.cpu()
+    classes = [np.arange(n)]
+    if "row_exp" in NF4_RANGE_CASES[case]:
+        lo, hi = NF4_RANGE_CASES[case]["row_exp"]
+        classes = [np.arange(c, n, hi - lo + 1) for c in range(hi - lo + 1)]
+    for cols in classes:
+        what = "nf4 gemv %s M=%d rows %d.." % (case, m, cols[0])
+        helpers.check_product(yc[:, cols], y_ref[:, cols], what)
+        helpers.check_within_error_bound(yc[:, cols], y_ref[:, cols], y_abs[:, cols], eps, what)

@@ -13,16 +13,26 @@ with outlier channels):
 
 Metric: "% of B200 roofline" of the whole step, work-weighted: for every op
 its roofline time max(algorithmic bytes / HBM peak, algorithmic ops / tensor
-peak) is summed, and divided by the measured step time. With N GPUs each rank
-runs its own replica (no data-path collective) and the value is the sum over
-ranks (weak scaling; 100 per GPU is the ceiling).
+peak) is summed, and divided by the measured step time. The tensor peak is the
+measured bf16 burst figure, or the sustained one if this run's own clock
+record shows the power cap (or clocks well below maximum); int8 is twice
+bf16. With N GPUs each rank runs its own replica (no data-path collective)
+and the value is the sum over ranks (weak scaling; 100 per GPU is the
+ceiling).
 
 Timing: W untimed warm-up steps, then exactly K steps between a barrier +
 synchronize on both sides, CUDA events on the launching stream, max over
-ranks. L2: every op's inputs were last touched one step earlier and the 600 MB
-NF4 dequantization stream (> 4x the 126 MB L2) runs in between, so every op
-starts L2-cold. `--impl reference` times the CPU oracle on a bounded sample of
-the same step instead (rank 0 only).
+ranks. L2: every op's weights were last touched one step earlier and the
+600 MB NF4 dequantization stream (> 4x the 126 MB L2) runs in between (each op
+has its own weights), so every op's weights start L2-cold. `--impl reference`
+times the CPU oracle on a bounded sample of the same step instead (rank 0
+only).
+
+After the step (outside its value): the dequantize-then-cuBLAS comparator,
+the salient-channel correction rows, and `per_config`, the throughput and
+roofline fraction of every workload of the five configurations, each
+graph-timed over rotating weight copies larger than 4x L2 with its own clock
+median.
 """
 
 import argparse
@@ -61,18 +71,28 @@ def load_peaks():
     return d
 
 
-def op_table(peaks):
+def tensor_peak(peaks, clocks):
+    """The bf16 tensor peak (TFLOP/s) that matches the clocks recorded while
+    the timed work ran: the burst figure (measured for a kernel timed alone at
+    full clock) unless the power cap was active or the SM clock sat well below
+    its maximum, in which case the sustained figure (measured back to back for
+    seconds, under the cap). Returns (TFLOP/s, "burst" | "sustained")."""
+    mhz, mx = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    if capped or (mhz and mx and mhz < 0.9 * mx):
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
+def op_table(peaks, tf16_tflops):
     """Algorithmic bytes and ops of each op of the step, with its roofline time.
 
     Bytes: packed weights (0.5 B/weight) + scales/zeros or absmax + activations
     read + outputs written; ops: 2*M*N*K multiply-adds (x2 components for MSD).
-    The tensor peak is the measured SUSTAINED bf16 rate: every op here is
-    timed inside a long run of back-to-back steps, which is the regime that
-    figure was measured in (the burst figure applies to a kernel timed
-    alone). The int8 peak is that bf16 peak x 2 (dense int8 runs at twice the
-    bf16 rate on B200)."""
+    tf16_tflops is the bf16 tensor peak chosen by tensor_peak(); the int8 peak
+    is twice it (dense int8 runs at twice the bf16 rate on B200)."""
     bw = peaks["hbm_gbs"] * 1e9
-    tf16 = peaks["bf16_tflops_sustained"] * 1e12
+    tf16 = tf16_tflops * 1e12
     ti8 = 2.0 * tf16
     n, k = NF4_SHAPE
     gn, gk = GEMV_SHAPE
@@ -101,13 +121,15 @@ def op_table(peaks):
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML every 50 ms."""
+    """Samples SM clock and throttle reasons through NVML every `period` s,
+    with wall-clock stamps, so that any window of the run (one case) can be
+    summarised on its own."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
 
-    def __init__(self, index):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
+    def __init__(self, index, period=0.05):
+        self.samples, self.max_mhz, self.period = [], None, period  # (t, mhz, reasons)
         self._stop = threading.Event()
         self._ok = False
         try:
@@ -124,14 +146,14 @@ class ClockSampler:
         nv = self._nv
         while not self._stop.is_set():
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
                 mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit and name != "gpu_idle":
-                        self.reasons.add(name)
+                names = {name for bit, name in self.REASONS.items()
+                         if mask & bit and name != "gpu_idle"}
+                self.samples.append((time.time(), mhz, names))
             except Exception:
                 pass
-            time.sleep(0.05)
+            time.sleep(self.period)
 
     def __enter__(self):
         if self._ok:
@@ -144,11 +166,17 @@ class ClockSampler:
             self._stop.set()
             self._t.join()
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons)}
+    def summary(self, t0=None, t1=None):
+        sel = [(m, r) for t, m, r in self.samples
+               if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": ["unavailable" if not self._ok else "no sample in window"]}
+        reasons = set()
+        for _, r in sel:
+            reasons |= r
+        return {"sm_mhz": statistics.median(m for m, _ in sel), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(sel)}
 
 
 # ---------------------------------------------------------------------------
@@ -199,6 +227,9 @@ class Step:
         sn, sk = MSD_SHAPE
         w = normal(sn, sk, std=0.02)
         self.sw = wq.wq_quantize_pack(F, w, 128)
+        # the decode MSD op has its own copy of the layer: the prefill MSD op's
+        # weights are read only the two GEMVs (~50 MB, under L2) before it
+        self.sw16 = wq.wq_quantize_pack(F, w, 128)
         del w
         self.sx16 = acts(16, sk, 0.005, 50.0)
         self.sx1024 = acts(1024, sk, 0.005, 50.0)
@@ -226,7 +257,7 @@ class Step:
                                                    *self.gi, out=self.gy_i)),
             ("gemv_nf4", lambda: wq.wq_w4a16_gemv(self.gx, gn, wq.WQ_FMT_NF4, 64, *self.gn,
                                                   out=self.gy_n)),
-            ("msd_m16", lambda: wq.wq_msd_gemm(self.sx16, sn, 2, 128, *self.sw,
+            ("msd_m16", lambda: wq.wq_msd_gemm(self.sx16, sn, 2, 128, *self.sw16,
                                                workspace=self.sws16, out=self.sy16)),
             ("nf4_dequant", lambda: wq.wq_nf4_dequant(self.nf4_codes, self.nf4_absmax, n * k,
                                                       out=self.nf4_out)),
@@ -405,10 +436,245 @@ def measure_decdec(wq, peaks, device, with_oracle):
     return out
 
 
+# ---------------------------------------------------------------------------
+# per-config throughput: every workload of the five configurations
+# ---------------------------------------------------------------------------
+
+L2_BYTES = 126 * 2 ** 20
+
+
+def _copies_for(nbytes):
+    """Weight copies whose total exceeds 4x L2 (at least 1, at most 1024)."""
+    return int(max(1, min(1024, -(-4 * L2_BYTES // max(1, int(nbytes))))))
+
+
+def _timed_launches(fns, sampler, min_ms=60.0):
+    """Mean device time (us) of one call of fns[i] in a stream of back-to-back
+    calls: the calls are captured as one CUDA graph, cycling over fns (each
+    call on its own copy of the weights, so a copy is read again only after
+    > 4x L2 of other copies), and the graph is replayed between two CUDA
+    events until at least min_ms of device time is averaged; time / calls.
+    (Events around every call inside the graph would add ~4 us each, measured
+    on B200, which swamps decode-size kernels.) Returns (us, clocks of the
+    replays)."""
+    n = len(fns)
+    reps = max(n, 16)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for f in fns[:2]:
+            f()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(reps):
+            fns[i % n]()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    total, cnt = 0.0, 0
+    t0 = time.time()
+    while True:
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+        cnt += reps
+        if total >= min_ms and cnt >= 2 * reps:
+            break
+    t1 = time.time()
+    del g
+    return 1e3 * total / cnt, sampler.summary(t0, t1)
+
+
+def measure_per_config(wq, peaks, device):
+    """Absolute throughput and roofline fraction of every workload of the
+    five configurations (timed after the step, not part of its value):
+
+      1  decode GEMV, INT4 g64, M = 1, 1024 x 1024
+      2  NF4 dequantization, 28672 x 8192, 8192 x 8192, 5120 x 25600
+      3  decode GEMV, M = 1, 4, 8, 16 x (4096 x 4096, 11008 x 4096,
+         4096 x 11008), INT4 g128 and NF4 b64, 1 % outlier channels x 20
+      4  prefill fused GEMM, M = 512, 2048, 8192 x (4096 x 4096,
+         14336 x 4096, 4096 x 14336), INT4 g128, beside dequantize-then-cuBLAS
+      5  MSD GEMM, C = 2, M = 1, 16, 128, 1024 x (5120 x 5120, 25600 x 5120,
+         5120 x 25600), per-channel and g128, 0.5 % outlier channels x 50;
+         at M = 128 and 1024 (g128) beside the fused GEMM on the same layer,
+         and the relative L2 errors of MSD and of the bf16
+         dequantize-then-cuBLAS product against the exact product
+
+    Each workload is graph-timed as a stream of back-to-back calls over
+    rotating copies of its weights (> 4x L2 in total), with its own SM clock
+    median. Bytes and ops are the
+    algorithmic ones: packed weights, scales/zeros or absmax, activations
+    read and outputs written; 2MNK flops (x C for MSD). Peaks: measured HBM
+    copy; bf16 and int8 (2x bf16) tensor peaks, burst or sustained by each
+    case's own clocks."""
+    g = torch.Generator(device=device)
+    g.manual_seed(1234)
+    F, NF = wq.WQ_FMT_INT4_ASYM, wq.WQ_FMT_NF4
+    bw = peaks["hbm_gbs"] * 1e9
+    out = {"config1_gemv_tiny": [], "config2_nf4_dequant": [], "config3_gemv": [],
+           "config4_gemm": [], "config5_msd": [], "msd_vs_fused_gemm": [], "msd_accuracy": []}
+
+    def normal(*shape, std=1.0):
+        return torch.randn(*shape, generator=g, device=device) * std
+
+    def acts(m, k, frac, scale):
+        x = normal(m, k)
+        if frac:
+            idx = torch.randperm(k, generator=g, device=device)[:max(1, round(frac * k))]
+            x[:, idx] *= scale
+        return x.to(torch.bfloat16)
+
+    def packed_bytes(fmt, n, k, group):
+        return n * k // 2 + (n * k // 64 * 4 if fmt == NF else n * (k // group) * 4)
+
+    def weight_copies(fmt, n, k, group):
+        one = wq.wq_quantize_pack(fmt, normal(n, k, std=0.02), group)
+        r = _copies_for(packed_bytes(fmt, n, k, group))
+        return [one] + [tuple(t.clone() if t is not None else None for t in one)
+                        for _ in range(r - 1)]
+
+    def entry(name, us, clk, nbytes, flops, int8=False, extra=None):
+        tf16_kind = tensor_peak(peaks, clk)
+        tpk = (2.0 if int8 else 1.0) * tf16_kind[0] * 1e12
+        t_roof = max(nbytes / bw, flops / tpk if flops else 0.0)
+        e = {"case": name, "us": round(us, 2), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
+             "tflops": round(flops / (us * 1e-6) / 1e12, 1),
+             "bound": "hbm" if nbytes / bw >= (flops / tpk if flops else 0.0) else "tensor",
+             "roofline_frac": round(t_roof / (us * 1e-6), 4),
+             "peak": "hbm %.0f GB/s, %s %s %.0f TFLOP/s" % (
+                 peaks["hbm_gbs"], tf16_kind[1], "int8" if int8 else "bf16", tpk / 1e12),
+             "sm_mhz": clk.get("sm_mhz"), "clock_reasons": clk.get("reasons")}
+        if extra:
+            e.update(extra)
+        return e
+
+    def gemv_case(key, m, n, k, fmt, group, outliers):
+        ws = weight_copies(fmt, n, k, group)
+        x = acts(m, k, *(outliers or (0, 0)))
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        fns = [lambda c=c: wq.wq_w4a16_gemv(x, n, fmt, group, *c, out=y) for c in ws]
+        us, clk = _timed_launches(fns, sampler)
+        nb = packed_bytes(fmt, n, k, group) + 2 * m * k + 2 * m * n
+        out[key].append(entry("%s M=%d %dx%d" % ("nf4-b64" if fmt == NF else "int4-g%d" % group,
+                                                 m, n, k), us, clk, nb, 2 * m * n * k,
+                              extra={"weight_copies": len(ws)}))
+        del ws, fns
+
+    with ClockSampler(torch.cuda.current_device(), period=0.01) as sampler:
+        # 1: the tiny GEMV
+        gemv_case("config1_gemv_tiny", 1, 1024, 1024, F, 64, None)
+        # 2: NF4 dequantization
+        for n, k in [(28672, 8192), (8192, 8192), (5120, 25600)]:
+            cw, am, _ = wq.wq_quantize_pack(NF, normal(n, k, std=0.02), 64)
+            r = _copies_for(n * k // 2 + n * k // 16)
+            sets = [(cw, am)] + [(cw.clone(), am.clone()) for _ in range(r - 1)]
+            o = torch.empty(n * k, dtype=torch.bfloat16, device=device)
+            fns = [lambda c=c: wq.wq_nf4_dequant(c[0], c[1], n * k, out=o) for c in sets]
+            us, clk = _timed_launches(fns, sampler)
+            out["config2_nf4_dequant"].append(entry("%dx%d" % (n, k), us, clk,
+                                                    n * k * (0.5 + 4 / 64 + 2), 0))
+            del sets, fns, o, cw, am
+            torch.cuda.empty_cache()
+        # 3: decode GEMV
+        for n, k in [(4096, 4096), (11008, 4096), (4096, 11008)]:
+            for fmt, group in ((F, 128), (NF, 64)):
+                for m in (1, 4, 8, 16):
+                    gemv_case("config3_gemv", m, n, k, fmt, group, (0.01, 20.0))
+            torch.cuda.empty_cache()
+        # 4: prefill GEMM beside dequantize-then-cuBLAS
+        for n, k in [(4096, 4096), (14336, 4096), (4096, 14336)]:
+            ws = weight_copies(F, n, k, 128)
+            wd = torch.empty(n, k, dtype=torch.bfloat16, device=device)
+            for m in (512, 2048, 8192):
+                x = acts(m, k, 0, 0)
+                y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+                wsp = wq.gemm_workspace(m, n, k, 128, device)
+                fused = [lambda c=c: wq.wq_w4a16_gemm(x, n, F, 128, *c, workspace=wsp, out=y)
+                         for c in ws]
+                us, clk = _timed_launches(fused, sampler)
+
+                def deq_mm(c):
+                    wq.wq_int4_dequant(c[0], c[1], c[2], n, k, 128, out=wd)
+                    torch.matmul(x, wd.t(), out=y)
+                us_c, _ = _timed_launches([lambda c=c: deq_mm(c) for c in ws], sampler)
+                nb = packed_bytes(F, n, k, 128) + 2 * m * k + 2 * m * n
+                out["config4_gemm"].append(entry(
+                    "int4-g128 M=%d %dx%d" % (m, n, k), us, clk, nb, 2 * m * n * k,
+                    extra={"dequant_then_cublas_us": round(us_c, 2),
+                           "fused_speedup": round(us_c / us, 3), "weight_copies": len(ws)}))
+                del x, y, wsp, fused
+            del ws, wd
+            torch.cuda.empty_cache()
+        # 5: MSD GEMM (and the fused GEMM on the same g128 layer at M >= 128)
+        for n, k in [(5120, 5120), (25600, 5120), (5120, 25600)]:
+            for group in (k, 128):
+                ws = weight_copies(F, n, k, group)
+                for m in (1, 16, 128, 1024):
+                    x = acts(m, k, 0.005, 50.0)
+                    y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+                    wsp = wq.msd_workspace(m, n, k, group, 2, device)
+                    fns = [lambda c=c: wq.wq_msd_gemm(x, n, 2, group, *c, workspace=wsp, out=y)
+                           for c in ws]
+                    us, clk = _timed_launches(fns, sampler)
+                    nb = packed_bytes(F, n, k, group) + 2 * m * k + 2 * m * n
+                    tag = "per-channel" if group == k else "g128"
+                    out["config5_msd"].append(entry("C=2 %s M=%d %dx%d" % (tag, m, n, k), us, clk,
+                                                    nb, 2 * 2 * m * n * k, int8=True,
+                                                    extra={"weight_copies": len(ws)}))
+                    if group == 128 and m >= 128:
+                        gws = wq.gemm_workspace(m, n, k, 128, device)
+                        fused = [lambda c=c: wq.wq_w4a16_gemm(x, n, F, 128, *c, workspace=gws,
+                                                              out=y) for c in ws]
+                        us_f, _ = _timed_launches(fused, sampler)
+                        out["msd_vs_fused_gemm"].append({
+                            "case": "g128 M=%d %dx%d" % (m, n, k), "msd_us": round(us, 2),
+                            "fused_gemm_us": round(us_f, 2), "msd_over_fused": round(us / us_f, 3)})
+                        del gws, fused
+                    if m == 128:
+                        out["msd_accuracy"].append(dict(
+                            case="%s M=128 %dx%d" % (tag, n, k),
+                            **msd_accuracy(wq, x, n, k, group, ws[0], y, device)))
+                    del x, y, wsp, fns
+                del ws
+                torch.cuda.empty_cache()
+    return out
+
+
+def msd_accuracy(wq, x, n, k, group, w, y, device, rows=64, cols=512):
+    """Relative L2 errors, on sampled outputs, of the MSD product (C = 2) and
+    of the bf16 dequantize-then-cuBLAS product against the exact product
+    x . ((q - z) s)^T in fp64 (the codes from wq_unpack, the fp16 scales and
+    zeros widened exactly; fp64 cuBLAS on the GPU). "Multi-Scale Dequant...",
+    Abstract, reports lower L2 error than dequantization baselines in many
+    settings but prints no numbers: this is a measurement, not a parity
+    check."""
+    qw, sc, zr = w
+    m = x.shape[0]
+    gen = torch.Generator(device="cpu").manual_seed(n + k + group)
+    ri = torch.randperm(m, generator=gen)[:rows].to(device)
+    ci = torch.randperm(n, generator=gen)[:cols].to(device)
+    codes = wq.wq_unpack(wq.WQ_FMT_INT4_ASYM, qw, n, k).view(n, k)[ci].double()  # [cols, k]
+    s64 = sc[ci].double().repeat_interleave(group, dim=1)
+    z64 = zr[ci].double().repeat_interleave(group, dim=1)
+    exact = x[ri].double() @ ((codes - z64) * s64).t()
+    ws = wq.msd_workspace(m, n, k, group, 2, device)
+    y_msd = wq.wq_msd_gemm(x, n, 2, group, qw, sc, zr, workspace=ws, out=y)[ri][:, ci].double()
+    wd = wq.wq_int4_dequant(qw, sc, zr, n, k, group)
+    y_deq = torch.matmul(x, wd.t())[ri][:, ci].double()
+    nrm = exact.norm()
+    return {"rel_l2_msd_c2": float((y_msd - exact).norm() / nrm),
+            "rel_l2_bf16_dequant_cublas": float((y_deq - exact).norm() / nrm),
+            "sample": "%d rows x %d cols" % (rows, cols)}
+
+
 def run_gpu(args, rank, world, device):
     from bit_weight_quantized_weights_b200 import binding as wq
     peaks = load_peaks()
-    table = op_table(peaks)
     step = Step(wq, device)
     ops = step.ops()
 
@@ -446,7 +712,7 @@ def run_gpu(args, rank, world, device):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clocks:
+    with ClockSampler(torch.cuda.current_device(), period=0.005) as clocks:
         t0.record()
         if graph is not None:
             graph.replay()
@@ -462,11 +728,18 @@ def run_gpu(args, rank, world, device):
     if st != wq.WQ_OK:
         raise RuntimeError("device error word set during timing: 0x%x" % detail)
 
+    # the tensor peak that matches this run's clocks (the same on every rank:
+    # each rank's own record decides, and the value is summed over ranks)
+    clk = clocks.summary()
+    tf16, peak_kind = tensor_peak(peaks, clk)
+    table = op_table(peaks, tf16)
+
     comparator = dequant_then_cublas(wq, step, per_op_ms["gemm"], args.warmup) if rank == 0 else None
     next_rows = None
     if rank == 0 and args.next_rows:
         next_rows = {"decdec": measure_decdec(
             wq, peaks, device, with_oracle=world == 1 and not args.no_cpu_baseline)}
+    per_config = measure_per_config(wq, peaks, device) if rank == 0 and args.per_config else None
 
     ms_per_step = elapsed_ms / args.steps
     value = job_value(table, ms_per_step, world)
@@ -475,10 +748,14 @@ def run_gpu(args, rank, world, device):
     dom = max(per_op_ms, key=per_op_ms.get)
     d = table[dom]
     dur_s = per_op_ms[dom] * 1e-3
+    other = {}
     if d["bound"] == "tensor":
         achieved = d["flops"] / dur_s / 1e12
         peak = d["peak_flops"] / 1e12
         unit = "TFLOP/s" if dom == "gemm" else "TOP/s"
+        mult = 1.0 if dom == "gemm" else 2.0
+        other = {"frac_burst": round(achieved / (mult * peaks["bf16_tflops"]), 4),
+                 "frac_sustained": round(achieved / (mult * peaks["bf16_tflops_sustained"]), 4)}
     else:
         achieved = d["bytes"] / dur_s / 1e9
         peak = peaks["hbm_gbs"]
@@ -502,25 +779,35 @@ def run_gpu(args, rank, world, device):
                                "11008x4096; msd C=2 g128 M=16 25600x5120; nf4_dequant "
                                "28672x8192; gemm int4-g128 8192x14336x4096; msd C=2 g128 "
                                "M=1024 25600x5120",
-                   "l2": "cold: each op's inputs were last touched a step earlier, with the "
-                         "600 MB NF4 stream (>4x L2) in between",
+                   "l2": "weights cold: each op has its own weights, last touched a step "
+                         "earlier with the 600 MB NF4 stream (>4x L2) in between; activations "
+                         "of the decode ops (<= 164 KB) may be L2-warm",
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "timing": ("eager launches" if args.eager else
                               "the K timed steps replayed as one captured CUDA graph") +
                              ", per-op CUDA events inside, device time"},
-        "roofline": {"bound": d["bound"], "kernel": dom, "achieved": round(achieved, 2),
-                     "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "peak_source": peaks["source"] + (" (HBM copy)" if d["bound"] == "hbm" else " (sustained bf16" + (")" if dom == "gemm" else " x 2 for int8)"))},
+        "roofline": dict({"bound": d["bound"], "kernel": dom, "achieved": round(achieved, 2),
+                          "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+                          "traffic": traffic,
+                          "peak_source": peaks["source"] + (
+                              " (HBM copy)" if d["bound"] == "hbm" else
+                              " (%s bf16, chosen by this run's clocks%s)"
+                              % (peak_kind, "" if dom == "gemm" else "; x 2 for int8"))},
+                         **other),
         "per_op": {k: {a: round(b, 4) for a, b in v.items()} for k, v in details.items()},
         "comparator": comparator,
         "next_rows": next_rows,
         "gpu_launches": Step.LAUNCHES_PER_STEP * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clk,
+        "tensor_peak": {"kind": peak_kind, "bf16_tflops": tf16,
+                        "rule": "burst unless the timed region saw sw_power_cap or a median SM "
+                                "clock below 0.9 x max"},
+        "per_config": per_config,
     }
     if e2e is not None:
         line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(peaks)
+        line["cpu_baseline"] = cpu_baseline(peaks, tf16=tf16)
     return line
 
 
@@ -603,8 +890,8 @@ class OracleSample:
     only the oracle's arithmetic and returns (cpu seconds, roofline seconds of
     the sampled work). `scale` shrinks every sample proportionally."""
 
-    def __init__(self, peaks, scale=1.0):
-        self.table = op_table(peaks)
+    def __init__(self, peaks, scale=1.0, tf16=None):
+        self.table = op_table(peaks, tf16 if tf16 is not None else peaks["bf16_tflops"])
         self.scale = scale
         self.frac = {"nf4_dequant": scale / 256, "gemv_int4": scale / 16,
                      "gemv_nf4": scale / 16, "gemm": max(1, round(16 * scale)) / 8192,
@@ -689,9 +976,9 @@ def oracle_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(peaks, scale=1.0):
+def cpu_baseline(peaks, scale=1.0, tf16=None):
     """The oracle as it stands, timed once on a bounded sample of the step."""
-    sample = OracleSample(peaks, scale).prepare()
+    sample = OracleSample(peaks, scale, tf16).prepare()
     t_cpu, roof = sample.run()
     return {"value": round(100.0 * roof / t_cpu, 6), "unit": UNIT, "cores": oracle_cores(),
             "kind": "oracle", "sample": sample.describe(), "cpu_seconds": round(t_cpu, 2)}
@@ -790,6 +1077,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", dest="next_rows", action="store_false",
                     help="skip the widening measurements timed after the step")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the per-config throughput of every workload, timed after the step")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as a "
                          "captured CUDA graph")

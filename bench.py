@@ -1001,7 +1001,8 @@ def max_over_ranks(v, world, device):
     return float(t.item())
 
 
-PROFILE_CASES = ("nf4", "gemv_int4", "gemv_nf4", "gemm", "msd", "msd_m16", "decdec")
+PROFILE_CASES = ("nf4", "gemv_int4", "gemv_int4_m1", "gemv_nf4", "gemm", "msd", "msd_m16",
+                 "decdec")
 
 
 def profile_case(case, device):
@@ -1020,9 +1021,9 @@ def profile_case(case, device):
         cw, am, _ = wq.wq_quantize_pack(wq.WQ_FMT_NF4, normal(n, k, std=0.02), 64)
         out = torch.empty(n * k, dtype=torch.bfloat16, device=device)
         fn = lambda: wq.wq_nf4_dequant(cw, am, n * k, out=out)  # noqa: E731
-    elif case in ("gemv_int4", "gemv_nf4"):
-        (n, k), m = GEMV_SHAPE, 16
-        fmt = wq.WQ_FMT_INT4_ASYM if case == "gemv_int4" else wq.WQ_FMT_NF4
+    elif case in ("gemv_int4", "gemv_int4_m1", "gemv_nf4"):
+        (n, k), m = GEMV_SHAPE, (1 if case == "gemv_int4_m1" else 16)
+        fmt = wq.WQ_FMT_NF4 if case == "gemv_nf4" else wq.WQ_FMT_INT4_ASYM
         grp = 128 if fmt == wq.WQ_FMT_INT4_ASYM else 64
         pw = wq.wq_quantize_pack(fmt, normal(n, k, std=0.02), grp)
         x = normal(m, k).to(torch.bfloat16)

@@ -73,7 +73,7 @@ __device__ unsigned int g_gemv_error;  // this kernel has no waits; kept for the
 
 using namespace splitk;
 
-constexpr int kMaxXChunkBytes = 64 * 1024;
+constexpr size_t kMaxSmemBytes = 227 * 1024;  // dynamic shared memory of one CTA
 
 struct GemvArgs {
   const uint16_t* x;
@@ -111,7 +111,7 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
 }
 
 // One 128-k unit of this lane's two weight rows (g and g + 8), with its
-// group parameters.
+// group parameters, as the MMA loop takes it.
 //   wide  : w[0..3] = 16 bytes of row g at byte 16t, w[4..7] the same of row
 //           g + 8 (k = 32t .. 32t + 31); INT4: prm[0..1] = the scale bits of
 //           rows g, g + 8 and prm[2..3] their zero bits (one group spans the
@@ -122,37 +122,61 @@ __device__ __forceinline__ uint32_t int4_pair(uint32_t w, int e) {
 //           zero bits.
 // NF4 (narrow): prm[2h + i] = the fp32 absmax bits of block 2u + h of row g
 // (i = 0) or g + 8 (i = 1).
-// The fp16 parameters stay as loaded (zero-extended 16-bit loads, no
-// arithmetic on them) until the unit is computed, so the loads never stall a
-// warp that is still issuing its first units and staging x.
 struct Unit {
   uint32_t w[8];
   uint32_t prm[4];
   uint32_t zz[4];  // narrow INT4 only
 };
 
-template <bool kNF4, bool kWide>
-__device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint8_t* wB, int u,
-                                          int nA, int nB, const GemvArgs& p, int ng, int t) {
-  static_assert(!(kWide && kNF4), "NF4 uses the 8-byte layout");
-  const int64_t off = (int64_t)u * 64;
-  if (kWide) {
-    const uint4 a = ld_stream_u4(wA + off), b = ld_stream_u4(wB + off);
-    U.w[0] = a.x; U.w[1] = a.y; U.w[2] = a.z; U.w[3] = a.w;
-    U.w[4] = b.x; U.w[5] = b.y; U.w[6] = b.z; U.w[7] = b.w;
-  } else {
-    const uint2 a0 = ld_stream_u2(wA + off), a1 = ld_stream_u2(wA + off + 32);
-    const uint2 b0 = ld_stream_u2(wB + off), b1 = ld_stream_u2(wB + off + 32);
-    U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
-    U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
+// ---------------------------------------------------------------------------
+// The weight stream. Each warp owns 16 rows and streams them through a ring
+// of kStages shared-memory stages of 256 k: 16 rows x 128 contiguous bytes
+// (two 128-k units). Measured on B200, 128 or more contiguous bytes per row
+// and request stream a row-strided matrix at 6 TB/s, where 64-byte pieces
+// (one unit per request) reach far less. A stage is copied by 16-byte
+// cp.async (one warp instruction covers 4 rows x 128 bytes), issued
+// kStages - 1 stages ahead of the one computed and awaited with
+// cp.async.wait_group, so the copies of later stages stay in flight while a
+// stage is computed whatever the compute costs. Chunk c (16 bytes) of row r
+// is stored at chunk c ^ swz(r): the fragment reads of a warp then hit
+// distinct banks (wide: each 8-lane phase reads two rows of different parity;
+// narrow: each 16-lane phase reads four rows 0..3 mod 4).
+// The group parameters of a stage (fp16 scale and zero, or fp32 absmax) are
+// loaded into registers when its copies are issued.
+// ---------------------------------------------------------------------------
+constexpr int kStageRowBytes = 128;            // per row per stage (256 k)
+constexpr int kStageBytes = 16 * kStageRowBytes;  // per warp per stage
+
+template <bool kWide>
+__device__ __forceinline__ int swz(int r) {
+  return kWide ? 4 * (r & 1) : 2 * (r & 3);
+}
+
+// Copies of stage (units ub, ub + 1; only ub when one = true) of the warp's
+// 16 rows starting at wtile into slot.
+template <bool kWide>
+__device__ __forceinline__ void issue_stage(uint8_t* slot, const uint8_t* wtile,
+                                            int64_t row_bytes, int ub, bool one, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int q = 32 * i + lane, r = q >> 3, c = q & 7;
+    if (!one || c < 4)
+      cp_async16(slot + r * kStageRowBytes + ((c ^ swz<kWide>(r)) << 4),
+                 wtile + (int64_t)r * row_bytes + (int64_t)ub * 64 + 16 * c);
   }
+}
+
+// Group parameters of unit u (see Unit) into prm[0..3], zz[0..3].
+template <bool kNF4, bool kWide>
+__device__ __forceinline__ void load_unit_prm(uint32_t* prm, uint32_t* zz, int u, int nA, int nB,
+                                              const GemvArgs& p, int ng) {
   if (kNF4) {
-    // half h of the unit (bytes 32h + 8t .. + 7 of each row) is block 2u + h
+    // half h of the unit (bytes 32h .. 32h + 31 of each row) is block 2u + h
     const float* am = static_cast<const float*>(p.scales);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      U.prm[2 * h + 0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + 2 * u + h));
-      U.prm[2 * h + 1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + 2 * u + h));
+      prm[2 * h + 0] = __float_as_uint(__ldg(am + (int64_t)nA * (p.K / 64) + 2 * u + h));
+      prm[2 * h + 1] = __float_as_uint(__ldg(am + (int64_t)nB * (p.K / 64) + 2 * u + h));
     }
   } else {
     const unsigned short* s16 = reinterpret_cast<const unsigned short*>(p.scales);
@@ -161,16 +185,46 @@ __device__ __forceinline__ void load_unit(Unit& U, const uint8_t* wA, const uint
     for (int h = 0; h < (kWide ? 1 : 2); ++h) {
       const int gi = div_by_magic(2 * u + h, p.gmagic);
       const int64_t iA = (int64_t)nA * ng + gi, iB = (int64_t)nB * ng + gi;
-      U.prm[2 * h + 0] = __ldg(s16 + iA);
-      U.prm[2 * h + 1] = __ldg(s16 + iB);
+      prm[2 * h + 0] = __ldg(s16 + iA);
+      prm[2 * h + 1] = __ldg(s16 + iB);
       if (kWide) {
-        U.prm[2] = __ldg(z16 + iA);
-        U.prm[3] = __ldg(z16 + iB);
+        prm[2] = __ldg(z16 + iA);
+        prm[3] = __ldg(z16 + iB);
       } else {
-        U.zz[2 * h + 0] = __ldg(z16 + iA);
-        U.zz[2 * h + 1] = __ldg(z16 + iB);
+        zz[2 * h + 0] = __ldg(z16 + iA);
+        zz[2 * h + 1] = __ldg(z16 + iB);
       }
     }
+  }
+}
+
+// The parameters of the two units of one stage.
+struct StagePrm {
+  uint32_t prm[2][4];
+  uint32_t zz[2][4];
+};
+
+// Unit h of a stage slot: this lane's bytes of rows g and g + 8 (see Unit).
+template <bool kWide>
+__device__ __forceinline__ void read_unit(Unit& U, const uint8_t* slot, int h, int g, int t) {
+  const uint8_t* ra = slot + g * kStageRowBytes;
+  const uint8_t* rb = slot + (g + 8) * kStageRowBytes;
+  const int sw = swz<kWide>(g);  // rows g and g + 8 share it
+  if (kWide) {
+    const int c = ((4 * h + t) ^ sw) << 4;
+    const uint4 a = *reinterpret_cast<const uint4*>(ra + c);
+    const uint4 b = *reinterpret_cast<const uint4*>(rb + c);
+    U.w[0] = a.x; U.w[1] = a.y; U.w[2] = a.z; U.w[3] = a.w;
+    U.w[4] = b.x; U.w[5] = b.y; U.w[6] = b.z; U.w[7] = b.w;
+  } else {
+    const int c0 = (((4 * h + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
+    const int c1 = (((4 * h + 2 + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
+    const uint2 a0 = *reinterpret_cast<const uint2*>(ra + c0);
+    const uint2 a1 = *reinterpret_cast<const uint2*>(ra + c1);
+    const uint2 b0 = *reinterpret_cast<const uint2*>(rb + c0);
+    const uint2 b1 = *reinterpret_cast<const uint2*>(rb + c1);
+    U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
+    U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
   }
 }
 
@@ -329,26 +383,35 @@ __device__ __forceinline__ void compute_unit(const Unit& U, int lu, const uint16
   }
 }
 
-// Units of weights each warp keeps in flight ahead of the one it computes.
-template <int NT>
-struct PrefetchDepth {
-  static constexpr int value = NT == 1 ? 4 : 3;
-};
+// The CTA: 16 warps of 16 rows (a 256-row tile), one CTA per SM, each warp
+// with its own ring of kStages stages.
+constexpr int kGemvRows = 256;
+constexpr int kGemvThreads = 2 * kGemvRows;
+constexpr int kStages = 3;
+
+template <int NT, bool kNF4>
+__host__ __device__ constexpr size_t gemv_fixed_smem() {
+  return (size_t)(kGemvThreads / 32) * kStages * kStageBytes + (kNF4 ? 256 * 32 * 4 : 0);
+}
 
 template <int NT, bool kNF4, bool kWide, bool kRes>
-__global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) {
+__global__ void __launch_bounds__(kGemvThreads, 1) gemv_kernel(GemvArgs p, Nf4Table tab) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int kTok = 8 * NT;
-  constexpr int D = PrefetchDepth<NT>::value;
   const int kc = p.kc;
-  uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* cursor = smem + (size_t)kTok * kc * 2;
+  // weight rings first (16-byte copies need 16-byte slots), then the
+  // lookup table (NF4), x, its group sums (INT4), the reduction buffer
+  uint8_t* rings = smem;
+  uint8_t* cursor = smem + (size_t)(kGemvThreads / 32) * kStages * kStageBytes;
   uint32_t* lut = nullptr;
-  float* xsum = nullptr;
   if (kNF4) {
     lut = reinterpret_cast<uint32_t*>(cursor);
     cursor += 256 * 32 * 4;
-  } else {
+  }
+  uint16_t* xs = reinterpret_cast<uint16_t*>(cursor);
+  cursor += (size_t)kTok * kc * 2;
+  float* xsum = nullptr;
+  if (!kNF4) {
     xsum = reinterpret_cast<float*>(cursor);
     cursor += (size_t)kTok * (kc / 64) * 4;
   }
@@ -361,16 +424,48 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   const int u1 = (int)((int64_t)(rank + 1) * p.units / p.S);
   const int k0 = u0 * 128;
   const int klen = (u1 - u0) * 128;
-  const int row_tile = (int)blockIdx.y * kRowsPerCta;
+  const int row_tile = (int)blockIdx.y * kGemvRows;
   const int g = lane >> 2, t = lane & 3;
   const int n0 = row_tile + warp * 16;
   const bool active = n0 < p.N;
   const int nA = n0 + g, nB = n0 + g + 8;
   const int ng = p.K / p.G;
 
+  // Programmatic dependent launch: a following kernel launched with the
+  // attribute may start its own weight stream while this one finishes (it
+  // waits for this grid before it reads x); this grid in turn starts its
+  // weight stream before waiting for the preceding kernel, whose output may
+  // be x. (The correction variants keep their own order: they may run as the
+  // dependent of the channel selection, which only reads x, and wait before
+  // their epilogue reads the selected channels.)
+  if constexpr (!kRes) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---- the first kStages - 1 weight stages of this warp (and their
+  // parameters): one copy group per stage, committed by every thread (empty
+  // for inactive warps and beyond the last stage) so that group counts agree
+  const int64_t row_bytes = (int64_t)p.K / 2;
+  const int nunits = u1 - u0;
+  const int nst = (nunits + 1) / 2;
+  uint8_t* wring = rings + (size_t)warp * kStages * kStageBytes;
+  const uint8_t* wtile = p.qw + (int64_t)(active ? n0 : 0) * row_bytes;
+  StagePrm sp[kStages];
+  auto issue = [&](int j, StagePrm& prm, uint8_t* slot) {
+    const bool one = 2 * j + 1 >= nunits;
+    issue_stage<kWide>(slot, wtile, row_bytes, u0 + 2 * j, one, lane);
+    load_unit_prm<kNF4, kWide>(prm.prm[0], prm.zz[0], u0 + 2 * j, nA, nB, p, ng);
+    if (!one) load_unit_prm<kNF4, kWide>(prm.prm[1], prm.zz[1], u0 + 2 * j + 1, nA, nB, p, ng);
+  };
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) {
+    if (active && i < nst) issue(i, sp[i], wring + i * kStageBytes);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+
   // ---- x[:, k0 : k0+klen) -> shared memory, as 16-byte asynchronous copies
-  // issued before the weight loads (every MMA waits on x). Only the M real
-  // tokens are copied: a padding token's MMA column never reaches an output.
+  // (after the preceding grid, which may have written x, has completed). Only
+  // the M real tokens are copied: a padding token's MMA column never reaches
+  // an output.
+  if constexpr (!kRes) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int kchunks = klen / 8;  // a multiple of 16
   const uint32_t cmagic = div_magic((uint32_t)kchunks);
   for (int c = tid; c < p.M * kchunks; c += blockDim.x) {
@@ -379,18 +474,8 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
     if (kWide) pc ^= (cl >> 2) & 2;
     cp_async16(xs + (size_t)gt * kc + pc * 8, p.x + (size_t)gt * p.K + k0 + cl * 8);
   }
-
-  // then the first D units of weights of this warp
-  const int64_t row_bytes = (int64_t)p.K / 2;
-  const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + (kWide ? 16 : 8) * t;
-  const uint8_t* wrowB = wrowA + 8 * row_bytes;
-  Unit ring[D];
-  if (active) {
-#pragma unroll
-    for (int i = 0; i < D; ++i)
-      if (u0 + i < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng, t);
-  }
-  cp_async_wait_all();
+  // every copy issued so far (x and the first weight stages) has landed
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
   if (!kNF4) {
@@ -435,34 +520,36 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
   }
   __syncthreads();
   if (kNF4) {
-    // per token: x chunk -> fp16 * 2^e in place (the swizzle moves whole chunks)
-    constexpr int tpt = 256 / kTok;  // threads per token: 32 or 16
-    const int gt = tid / tpt, j = tid % tpt;
-    uint16_t* row = xs + (size_t)gt * kc;
-    float mx = 0.0f;
-    for (int c = j; c < kchunks; c += tpt) {
-      const uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // per token: x chunk -> fp16 * 2^e in place (the swizzle moves whole
+    // chunks); warp gt converts token gt (the max is a warp reduction)
+    if (warp < kTok) {
+      const int gt = warp, j = lane;
+      uint16_t* row = xs + (size_t)gt * kc;
+      float mx = 0.0f;
+      for (int c = j; c < kchunks; c += 32) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        mx = fmaxf(mx, fmaxf(fabsf(bf16_lo_to_f32(w[i])), fabsf(bf16_hi_to_f32(w[i]))));
-    }
+        for (int i = 0; i < 4; ++i)
+          mx = fmaxf(mx, fmaxf(fabsf(bf16_lo_to_f32(w[i])), fabsf(bf16_hi_to_f32(w[i]))));
+      }
 #pragma unroll
-    for (int o = tpt / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    int e = 0;
-    if (mx > 0.0f && mx <= 3.0e38f) {
-      e = 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127);
-      e = e > 100 ? 100 : (e < -100 ? -100 : e);
-    }
-    const float sc = __uint_as_float((uint32_t)(127 + e) << 23);
-    if (j == 0) tok_inv[gt] = __uint_as_float((uint32_t)(127 - e) << 23);
-    for (int c = j; c < kchunks; c += tpt) {
-      uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
-      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int e = 0;
+      if (mx > 0.0f && mx <= 3.0e38f) {
+        e = 14 - ((int)((__float_as_uint(mx) >> 23) & 0xFF) - 127);
+        e = e > 100 ? 100 : (e < -100 ? -100 : e);
+      }
+      const float sc = __uint_as_float((uint32_t)(127 + e) << 23);
+      if (j == 0) tok_inv[gt] = __uint_as_float((uint32_t)(127 - e) << 23);
+      for (int c = j; c < kchunks; c += 32) {
+        uint4 v = *reinterpret_cast<const uint4*>(row + c * 8);
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-        w[i] = pack_f16x2(bf16_lo_to_f32(w[i]) * sc, bf16_hi_to_f32(w[i]) * sc);
-      *reinterpret_cast<uint4*>(row + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int i = 0; i < 4; ++i)
+          w[i] = pack_f16x2(bf16_lo_to_f32(w[i]) * sc, bf16_hi_to_f32(w[i]) * sc);
+        *reinterpret_cast<uint4*>(row + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
     }
     __syncthreads();
   }
@@ -474,29 +561,49 @@ __global__ void __launch_bounds__(256, 2) gemv_kernel(GemvArgs p, Nf4Table tab) 
 #pragma unroll
     for (int r = 0; r < 4; ++r) acc[a][r] = 0.0f;
 
-  if (active) {
-    const uint32_t* lut_lane = kNF4 ? lut + lane : nullptr;
-    for (int ub = u0; ub < u1; ub += D) {
+  const uint32_t* lut_lane = kNF4 ? lut + lane : nullptr;
+  for (int jb = 0; jb < nst; jb += kStages) {
 #pragma unroll
-      for (int i = 0; i < D; ++i) {
-        const int u = ub + i;
-        if (u < u1) {
-          compute_unit<NT, kNF4, kWide>(ring[i], u - u0, xs, kc, xsum, lut_lane, g, t, acc);
-          if (u + D < u1) load_unit<kNF4, kWide>(ring[i], wrowA, wrowB, u + D, nA, nB, p, ng, t);
+    for (int i = 0; i < kStages; ++i) {
+      const int j = jb + i;
+      if (j < nst) {
+        // stage j + kStages - 1 goes into the slot stage j - 1 left
+        const int kNext = (i + kStages - 1) % kStages;  // a constant once unrolled
+        if (active && j + kStages - 1 < nst)
+          issue(j + kStages - 1, sp[kNext], wring + kNext * kStageBytes);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
+        __syncwarp();  // every lane's copies of stage j are visible to the warp
+        if (active) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int lu = 2 * j + h;
+            if (lu < nunits) {
+              Unit U;
+              read_unit<kWide>(U, wring + i * kStageBytes, h, g, t);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                U.prm[q] = sp[i].prm[h][q];
+                U.zz[q] = sp[i].zz[h][q];
+              }
+              compute_unit<NT, kNF4, kWide>(U, lu, xs, kc, xsum, lut_lane, g, t, acc);
+            }
+          }
         }
+        __syncwarp();  // stage j's slot is refilled in the next iteration
       }
     }
   }
 
   // ---- cluster split-K reduction (through distributed shared memory) -----
-  reduce_and_store<NT, kRes>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile, p.M, p.N,
-                             p.y, p.rc);
+  reduce_and_store<NT, kRes, kGemvRows>(acc, kNF4 ? tok_inv : nullptr, red, p.S, rank, row_tile,
+                                        p.M, p.N, p.y, p.rc);
 }
 
 template <int NT, bool kNF4>
 size_t gemv_smem(int kc, int S) {
-  return (size_t)8 * NT * kc * 2 + red_bytes(S) +
-         (kNF4 ? 256 * 32 * 4 : (size_t)8 * NT * (kc / 64) * 4);
+  return gemv_fixed_smem<NT, kNF4>() + (size_t)8 * NT * kc * 2 + red_bytes<kGemvRows>(S) +
+         (kNF4 ? 0 : (size_t)8 * NT * (kc / 64) * 4);
 }
 
 template <int NT, bool kNF4, bool kWide, bool kRes>
@@ -505,13 +612,17 @@ wq_status launch_t(GemvArgs a, cudaStream_t st, bool early = false) {
   const int M = a.M;
   const Plan pl = cached_plan(reinterpret_cast<const void*>(kern), M, a.N, a.K, 0, [&] {
     return make_plan(
-        kern, 256, a.N, a.K, [&](int kc) { return (int64_t)8 * NT * kc * 2 <= kMaxXChunkBytes; },
-        [&](int kc, int S) { return gemv_smem<NT, kNF4>(kc, S); });
+        kern, kGemvThreads, a.N, a.K,
+        [&](int kc) { return gemv_smem<NT, kNF4>(kc, kMaxSplit) <= kMaxSmemBytes; },
+        [&](int kc, int S) { return gemv_smem<NT, kNF4>(kc, S); }, false, kGemvRows);
   });
   if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
   a.S = pl.S;
   a.kc = pl.kc;
-  return launch_split(kern, pl, 256, a.N, st, a, nf4_table(), false, early && kRes);
+  // the plain GEMV is always launched as a programmatic dependent (see the
+  // kernel); the correction variants only when asked (after the selection)
+  return launch_split(kern, pl, kGemvThreads, a.N, st, a, nf4_table(), false, kRes ? early : true,
+                      kGemvRows);
 }
 
 }  // namespace

@@ -1,7 +1,8 @@
 // Shared pieces of the decode (M <= 16) kernels: the W4A16 GEMV and the
-// Multi-Scale Dequant GEMV. Both give every CTA one 128-row weight tile over
-// one K-chunk, split K across a thread-block cluster, and reduce the fp32
-// partials through distributed shared memory.
+// Multi-Scale Dequant GEMV. Both give every CTA one weight tile of ROWS rows
+// (16 per warp: 256 for the GEMV, 128 for the MSD GEMV) over one K-chunk,
+// split K across a thread-block cluster, and reduce the fp32 partials through
+// distributed shared memory.
 #pragma once
 
 #include <mutex>
@@ -11,7 +12,7 @@
 namespace wq {
 namespace splitk {
 
-constexpr int kRowsPerCta = 128;
+constexpr int kRowsPerCta = 128;  // default tile: 8 warps x 16 rows
 constexpr int kMaxSplit = 16;  // cluster size limit (non-portable above 8)
 
 // n / d without a divide: umulhi(n, floor(2^32 / d) + 1) is exact whenever
@@ -46,15 +47,20 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
-// Rows of a 128-row tile are split over the S ranks of a cluster as
-// [b(r), b(r + 1)) with b(r) = floor(128 r / S); the owner of row is the r
+// Rows of a ROWS-row tile are split over the S ranks of a cluster as
+// [b(r), b(r + 1)) with b(r) = floor(ROWS r / S); the owner of row is the r
 // with b(r) <= row < b(r + 1).
-__host__ __device__ __forceinline__ int rank_row_begin(int r, int S) { return r * 128 / S; }
-__device__ __forceinline__ int row_owner(int row, int S) { return ((row + 1) * S + 127) / 128 - 1; }
+template <int ROWS = kRowsPerCta>
+__host__ __device__ __forceinline__ int rank_row_begin(int r, int S) { return r * ROWS / S; }
+template <int ROWS = kRowsPerCta>
+__device__ __forceinline__ int row_owner(int row, int S) {
+  return ((row + 1) * S + ROWS - 1) / ROWS - 1;
+}
 
-// Shared-memory bytes of the reduction buffer red[S ranks][ceil(128/S)][16].
+// Shared-memory bytes of the reduction buffer red[S ranks][ceil(ROWS/S)][16].
+template <int ROWS = kRowsPerCta>
 __host__ __device__ __forceinline__ size_t red_bytes(int S) {
-  return (size_t)S * ((kRowsPerCta + S - 1) / S) * 16 * 4;
+  return (size_t)S * ((ROWS + S - 1) / S) * 16 * 4;
 }
 
 // Optional salient-channel residual correction ("DecDEC: A Systems Approach
@@ -71,9 +77,8 @@ struct Residual {
 };
 
 // Items (token, owned row) per thread in the owners' epilogue: nrows * M is
-// at most 128 * 16 = 2048 over 256 threads.
+// at most ROWS * 16 over 2 * ROWS threads (8 warps per 128 rows).
 constexpr int kMaxItemsPerThread = 8;
-static_assert(kRowsPerCta * 16 <= 256 * kMaxItemsPerThread, "items of a 256-thread CTA");
 
 // This thread's part of the correction of its items (token tok[it], row
 // n[it]; n < 0 for none): channels j = j0, j0 + L, j0 + 2L, ... in batches
@@ -125,21 +130,22 @@ __device__ __forceinline__ void residual_parts(const Residual& rc, const int (&t
 // stores need no round trip, and no CTA touches another's shared memory after
 // the barrier. With kRes the owners add the residual correction rc (k >= 1)
 // before the rounding. All threads of the CTA must call this.
-template <int NT, bool kRes = false>
+template <int NT, bool kRes = false, int ROWS = kRowsPerCta>
 __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], const float* tok_scale,
                                                  float* red, int S, int rank, int row_tile, int M,
                                                  int N, uint16_t* y,
                                                  const Residual& rc = Residual()) {
+  static_assert(ROWS * 16 <= 2 * ROWS * kMaxItemsPerThread, "items per thread");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const int rows_max = (kRowsPerCta + S - 1) / S;
+  const int rows_max = (ROWS + S - 1) / S;
 #pragma unroll
   for (int a = 0; a < NT; ++a)
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
       const int row = warp * 16 + g + 8 * hr;
-      const int owner = row_owner(row, S);
-      const int lr = row - rank_row_begin(owner, S);
+      const int owner = row_owner<ROWS>(row, S);
+      const int lr = row - rank_row_begin<ROWS>(owner, S);
       const int tok = 8 * a + 2 * t;
       float v0 = acc[a][2 * hr], v1 = acc[a][2 * hr + 1];
       if (tok_scale) {
@@ -154,8 +160,8 @@ __device__ __forceinline__ void reduce_and_store(const float (&acc)[NT][4], cons
         dst[1] = v1;
       }
     }
-  const int r_begin = rank_row_begin(rank, S);
-  const int nrows = rank_row_begin(rank + 1, S) - r_begin;
+  const int r_begin = rank_row_begin<ROWS>(rank, S);
+  const int nrows = rank_row_begin<ROWS>(rank + 1, S) - r_begin;
   const int items = nrows * M;
   if constexpr (!kRes) {
     if (S > 1) {
@@ -244,8 +250,8 @@ struct Plan {
 // CTA's dynamic shared memory.
 template <class Kern, class Fits, class SmemOf>
 Plan make_plan(Kern kern, int threads, int64_t N, int64_t K, Fits fits, SmemOf smem_of,
-               bool persistent = false) {
-  const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
+               bool persistent = false, int rows = kRowsPerCta) {
+  const int64_t tiles = (N + rows - 1) / rows;
   const int64_t units = K / 128;
   cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   cudaGetLastError();
@@ -338,14 +344,14 @@ Plan cached_plan(const void* kern, int M, int64_t N, int64_t K, int extra, MakeF
 template <class Kern, class Args>
 wq_status launch_split(Kern kern, const Plan& pl, int threads, int64_t N, cudaStream_t st,
                        const Args& args, const Nf4Table& tab, bool persistent = false,
-                       bool early = false) {
+                       bool early = false, int rows = kRowsPerCta) {
   // the attribute is a per-function maximum; plans of other shapes may have
   // set a smaller one since
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  const int64_t tiles = (N + kRowsPerCta - 1) / kRowsPerCta;
+  const int64_t tiles = (N + rows - 1) / rows;
   const int64_t gy = persistent && pl.resident > 0 && pl.resident < tiles ? pl.resident : tiles;
   cfg.gridDim = dim3((unsigned)pl.S, (unsigned)gy, 1);
   cfg.blockDim = dim3((unsigned)threads, 1, 1);

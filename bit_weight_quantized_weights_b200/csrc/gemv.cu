@@ -128,44 +128,6 @@ struct Unit {
   uint32_t zz[4];  // narrow INT4 only
 };
 
-// ---------------------------------------------------------------------------
-// The weight stream. Each warp owns 16 rows and streams them through a ring
-// of kStages shared-memory stages of 256 k: 16 rows x 128 contiguous bytes
-// (two 128-k units). Measured on B200, 128 or more contiguous bytes per row
-// and request stream a row-strided matrix at 6 TB/s, where 64-byte pieces
-// (one unit per request) reach far less. A stage is copied by 16-byte
-// cp.async (one warp instruction covers 4 rows x 128 bytes), issued
-// kStages - 1 stages ahead of the one computed and awaited with
-// cp.async.wait_group, so the copies of later stages stay in flight while a
-// stage is computed whatever the compute costs. Chunk c (16 bytes) of row r
-// is stored at chunk c ^ swz(r): the fragment reads of a warp then hit
-// distinct banks (wide: each 8-lane phase reads two rows of different parity;
-// narrow: each 16-lane phase reads four rows 0..3 mod 4).
-// The group parameters of a stage (fp16 scale and zero, or fp32 absmax) are
-// loaded into registers when its copies are issued.
-// ---------------------------------------------------------------------------
-constexpr int kStageRowBytes = 128;            // per row per stage (256 k)
-constexpr int kStageBytes = 16 * kStageRowBytes;  // per warp per stage
-
-template <bool kWide>
-__device__ __forceinline__ int swz(int r) {
-  return kWide ? 4 * (r & 1) : 2 * (r & 3);
-}
-
-// Copies of stage (units ub, ub + 1; only ub when one = true) of the warp's
-// 16 rows starting at wtile into slot.
-template <bool kWide>
-__device__ __forceinline__ void issue_stage(uint8_t* slot, const uint8_t* wtile,
-                                            int64_t row_bytes, int ub, bool one, int lane) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int q = 32 * i + lane, r = q >> 3, c = q & 7;
-    if (!one || c < 4)
-      cp_async16(slot + r * kStageRowBytes + ((c ^ swz<kWide>(r)) << 4),
-                 wtile + (int64_t)r * row_bytes + (int64_t)ub * 64 + 16 * c);
-  }
-}
-
 // Group parameters of unit u (see Unit) into prm[0..3], zz[0..3].
 template <bool kNF4, bool kWide>
 __device__ __forceinline__ void load_unit_prm(uint32_t* prm, uint32_t* zz, int u, int nA, int nB,
@@ -204,28 +166,10 @@ struct StagePrm {
   uint32_t zz[2][4];
 };
 
-// Unit h of a stage slot: this lane's bytes of rows g and g + 8 (see Unit).
+// Unit h of a stage slot into U.w (see Unit).
 template <bool kWide>
 __device__ __forceinline__ void read_unit(Unit& U, const uint8_t* slot, int h, int g, int t) {
-  const uint8_t* ra = slot + g * kStageRowBytes;
-  const uint8_t* rb = slot + (g + 8) * kStageRowBytes;
-  const int sw = swz<kWide>(g);  // rows g and g + 8 share it
-  if (kWide) {
-    const int c = ((4 * h + t) ^ sw) << 4;
-    const uint4 a = *reinterpret_cast<const uint4*>(ra + c);
-    const uint4 b = *reinterpret_cast<const uint4*>(rb + c);
-    U.w[0] = a.x; U.w[1] = a.y; U.w[2] = a.z; U.w[3] = a.w;
-    U.w[4] = b.x; U.w[5] = b.y; U.w[6] = b.z; U.w[7] = b.w;
-  } else {
-    const int c0 = (((4 * h + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
-    const int c1 = (((4 * h + 2 + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
-    const uint2 a0 = *reinterpret_cast<const uint2*>(ra + c0);
-    const uint2 a1 = *reinterpret_cast<const uint2*>(ra + c1);
-    const uint2 b0 = *reinterpret_cast<const uint2*>(rb + c0);
-    const uint2 b1 = *reinterpret_cast<const uint2*>(rb + c1);
-    U.w[0] = a0.x; U.w[1] = a0.y; U.w[2] = a1.x; U.w[3] = a1.y;
-    U.w[4] = b0.x; U.w[5] = b0.y; U.w[6] = b1.x; U.w[7] = b1.y;
-  }
+  read_stage_unit<kWide>(U.w, slot, h, g, t);
 }
 
 // acc += s * (P - (128 + z) * sum(x)) for the four accumulator slots of one

@@ -21,6 +21,10 @@ __global__ void __launch_bounds__(256) msd_decompose_kernel(const uint16_t* __re
                                                             int8_t* __restrict__ digits,
                                                             float* __restrict__ comp_scales) {
   __shared__ float red[8];
+  // a grid launched after this one as a programmatic dependent (the decode
+  // GEMV) may start at once: it waits for this grid before it reads the
+  // planes and scales
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int m = blockIdx.x;
   const uint16_t* row = x + (int64_t)m * K;
   const int chunks = K / 16;

@@ -26,6 +26,10 @@
 // 8-element group, so the planes are staged with the even-k bytes of each
 // group first, then the odd-k bytes.
 //
+// It is launched as a programmatic dependent of the decomposition kernel: its
+// first weight loads overlap the decomposition, and it waits for it only
+// before it reads the digit planes.
+//
 // Data placement per CTA (dynamic shared memory):
 //   pl   [C][M][Kc] int8, the CTA's K-chunk of the digit planes; 16-byte chunk
 //        c of token m at chunk c ^ (m & 1) (conflict-free fragment loads)
@@ -129,19 +133,14 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
   bool active = n0 < p.N;
   int nA = n0 + g, nB = n0 + g + 8;
 
-  // ---- digit planes [C][M][k0 : k0+klen) -> shared memory (16-byte copies),
-  // issued before the weight loads
-  const int kchunks = klen / 16;  // a multiple of 8
-  const int per_plane = M * kchunks;
-  const uint32_t mag_plane = div_magic((uint32_t)per_plane), mag_row = div_magic((uint32_t)kchunks);
-  for (int i = tid; i < C * per_plane; i += blockDim.x) {
-    const int c = div_by_magic(i, mag_plane), rem = i - c * per_plane;
-    const int gt = div_by_magic(rem, mag_row), cl = rem - gt * kchunks;
-    cp_async16(pl + ((size_t)c * M + gt) * kc + (cl ^ (gt & 1)) * 16,
-               p.planes + ((int64_t)c * p.plane_rows + gt) * p.K + k0 + cl * 16);
-  }
+  // Programmatic dependent launch: this grid starts while the decomposition
+  // that writes the digit planes and their scales may still run (its CTAs
+  // release this grid at once); it issues its first weight units, then waits
+  // for that grid before it reads the planes. It releases its own dependents
+  // at once in turn.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // then the first D units of weights of this warp
+  // ---- the first D units of weights of this warp
   const int64_t row_bytes = (int64_t)p.K / 2;
   const uint8_t* wrowA = p.qw + (int64_t)(active ? nA : 0) * row_bytes + 16 * t;
   const uint8_t* wrowB = wrowA + 8 * row_bytes;
@@ -151,6 +150,19 @@ __global__ void __launch_bounds__(256, 2) msd_gemv_kernel(MsdArgs p, Nf4Table) {
 #pragma unroll
     for (int i = 0; i < D; ++i)
       if (u0 + i < u1) msd_load_unit(ring[i], wrowA, wrowB, u0 + i, nA, nB, p, ng);
+  }
+
+  // ---- then the digit planes [C][M][k0 : k0+klen) -> shared memory
+  // (16-byte copies), once the decomposition has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int kchunks = klen / 16;  // a multiple of 8
+  const int per_plane = M * kchunks;
+  const uint32_t mag_plane = div_magic((uint32_t)per_plane), mag_row = div_magic((uint32_t)kchunks);
+  for (int i = tid; i < C * per_plane; i += blockDim.x) {
+    const int c = div_by_magic(i, mag_plane), rem = i - c * per_plane;
+    const int gt = div_by_magic(rem, mag_row), cl = rem - gt * kchunks;
+    cp_async16(pl + ((size_t)c * M + gt) * kc + (cl ^ (gt & 1)) * 16,
+               p.planes + ((int64_t)c * p.plane_rows + gt) * p.K + k0 + cl * 16);
   }
   cp_async_wait_all();
   __syncthreads();
@@ -323,7 +335,9 @@ wq_status launch_msd_t(MsdArgs a, cudaStream_t st) {
   if (pl.S < 1) return WQ_ERR_UNSUPPORTED;
   a.S = pl.S;
   a.kc = pl.kc;
-  return launch_split(kern, pl, 256, a.N, st, a, nf4_table(), /*persistent=*/true);
+  // a programmatic dependent of the decomposition (see the kernel)
+  return launch_split(kern, pl, 256, a.N, st, a, nf4_table(), /*persistent=*/true,
+                      /*early=*/true);
 }
 
 template <int NT>

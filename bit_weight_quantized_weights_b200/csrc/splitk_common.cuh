@@ -47,6 +47,73 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------
+// The weight stream. Each warp owns 16 rows and streams them through a ring
+// of kStages shared-memory stages of 256 k: 16 rows x 128 contiguous bytes
+// (two 128-k units). Measured on B200, 128 or more contiguous bytes per row
+// and request stream a row-strided matrix at 6 TB/s, where 64-byte pieces
+// (one unit per request) reach far less. A stage is copied by 16-byte
+// cp.async (one warp instruction covers 4 rows x 128 bytes), issued
+// kStages - 1 stages ahead of the one computed and awaited with
+// cp.async.wait_group, so the copies of later stages stay in flight while a
+// stage is computed whatever the compute costs. Chunk c (16 bytes) of row r
+// is stored at chunk c ^ swz(r): the fragment reads of a warp then hit
+// distinct banks (wide: each 8-lane phase reads two rows of different parity;
+// narrow: each 16-lane phase reads four rows 0..3 mod 4).
+// The group parameters of a stage are loaded into registers when its copies
+// are issued.
+// ---------------------------------------------------------------------------
+constexpr int kStageRowBytes = 128;            // per row per stage (256 k)
+constexpr int kStageBytes = 16 * kStageRowBytes;  // per warp per stage
+
+template <bool kWide>
+__device__ __forceinline__ int swz(int r) {
+  return kWide ? 4 * (r & 1) : 2 * (r & 3);
+}
+
+// Copies of stage (units ub, ub + 1; only ub when one = true) of the warp's
+// 16 rows starting at wtile into slot.
+template <bool kWide>
+__device__ __forceinline__ void issue_stage(uint8_t* slot, const uint8_t* wtile,
+                                            int64_t row_bytes, int ub, bool one, int lane) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int q = 32 * i + lane, r = q >> 3, c = q & 7;
+    if (!one || c < 4)
+      cp_async16(slot + r * kStageRowBytes + ((c ^ swz<kWide>(r)) << 4),
+                 wtile + (int64_t)r * row_bytes + (int64_t)ub * 64 + 16 * c);
+  }
+}
+
+// Unit h (128 k) of a stage slot: this lane's bytes of rows g and g + 8.
+//   wide  : w[0..3] = 16 bytes of row g at byte 16t of the unit, w[4..7] the
+//           same of row g + 8;
+//   narrow: w[0..1] row g, bytes 8t .. 8t + 7, w[2..3] row g, bytes
+//           32 + 8t .., w[4..7] the same of row g + 8.
+template <bool kWide>
+__device__ __forceinline__ void read_stage_unit(uint32_t (&w)[8], const uint8_t* slot, int h, int g,
+                                                int t) {
+  const uint8_t* ra = slot + g * kStageRowBytes;
+  const uint8_t* rb = slot + (g + 8) * kStageRowBytes;
+  const int sw = swz<kWide>(g);  // rows g and g + 8 share it
+  if (kWide) {
+    const int c = ((4 * h + t) ^ sw) << 4;
+    const uint4 a = *reinterpret_cast<const uint4*>(ra + c);
+    const uint4 b = *reinterpret_cast<const uint4*>(rb + c);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  } else {
+    const int c0 = (((4 * h + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
+    const int c1 = (((4 * h + 2 + (t >> 1)) ^ sw) << 4) + 8 * (t & 1);
+    const uint2 a0 = *reinterpret_cast<const uint2*>(ra + c0);
+    const uint2 a1 = *reinterpret_cast<const uint2*>(ra + c1);
+    const uint2 b0 = *reinterpret_cast<const uint2*>(rb + c0);
+    const uint2 b1 = *reinterpret_cast<const uint2*>(rb + c1);
+    w[0] = a0.x; w[1] = a0.y; w[2] = a1.x; w[3] = a1.y;
+    w[4] = b0.x; w[5] = b0.y; w[6] = b1.x; w[7] = b1.y;
+  }
+}
+
 // Rows of a ROWS-row tile are split over the S ranks of a cluster as
 // [b(r), b(r + 1)) with b(r) = floor(ROWS r / S); the owner of row is the r
 // with b(r) <= row < b(r + 1).

@@ -24,14 +24,21 @@ Modules
                decomposed integer product.
 ``decdec``     salient-channel residual correction: the residual matrix,
                the per-step channel selection and the corrected product.
+``mx``         MX block formats (MXFP4 E2M1, MXFP8 E4M3, power-of-two block
+               scales), the two-pass MXFP4 activation decomposition, the
+               single-pass MXFP8 comparator, and their product with MXFP4
+               weights.
 
 Parity pins: every function is pinned by ``tests/test_oracle_*.py`` against
 facts that do not come from the oracle itself (hand-computed golden groups,
 closed forms, exact rational brute force, library routines, and the
-construction's own defining property). One claim is *parity unpinned*: the
+construction's own defining property). Claims that are *parity unpinned*: the
 pages' statement that the decomposed product is no less accurate than the
-dequantize-then-multiply baseline prints no numbers; it is measured and
-reported, never asserted.
+dequantize-then-multiply baseline prints no numbers (it is measured and
+reported, never asserted); and the two-pass MXFP4 figures (near 6.6 effective
+bits, 1/64 per block), which the plainest MX readings do not reproduce (they
+measure 6.15 bits, worst block amax/37, derived bound amax/12; the page's
+single-pass MXFP8 figure, 5.24 bits, does reproduce and is pinned).
 """
 
-from . import numerics, formats, products, msd, decdec  # noqa: F401
+from . import numerics, formats, products, msd, decdec, mx  # noqa: F401

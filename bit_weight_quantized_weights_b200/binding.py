@@ -31,6 +31,7 @@ WQ_FP32 = 2
 WQ_OP_GEMV = 0
 WQ_OP_GEMM = 1
 WQ_OP_MSD_GEMM = 2
+WQ_OP_MX_GEMV = 3
 
 # every symbol include/wq.h declares
 EXPORTED = [
@@ -39,7 +40,7 @@ EXPORTED = [
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
-    "wq_test_set_wait",
+    "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv",
 ]
 
 
@@ -76,6 +77,9 @@ def _load():
                                ctypes.c_int),
         "wq_device_error": ([P, ctypes.c_int, ctypes.POINTER(U32)], ctypes.c_int),
         "wq_test_set_wait": ([ctypes.c_uint64, ctypes.c_int], ctypes.c_int),
+        "wq_mx_quantize": ([P, I64, I64, P, P, P], ctypes.c_int),
+        "wq_mx_decompose": ([P, I64, I64, I32, P, P, P], ctypes.c_int),
+        "wq_mx_gemv": ([P, I64, I64, I64, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -366,3 +370,47 @@ def wq_test_set_wait(limit_ns=0, stall=0):
     limit in ns (0 = the default 2 s) and whether the loader withholds the
     first k-tile of the tensor-core kernels."""
     _check(lib.wq_test_set_wait(int(limit_ns), int(stall)), "wq_test_set_wait")
+
+
+def wq_mx_quantize(w, codes=None, scales=None, stream=None):
+    """MXFP4 weights: w fp32 [N, K] -> (codes uint8 [N, K/2], scale bytes uint8 [N, K/32])."""
+    _cuda(w, torch.float32, "w")
+    n, k = w.shape
+    if codes is None:
+        codes = torch.empty(n, k // 2, dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty(n, k // 32, dtype=torch.uint8, device=w.device)
+    _check(lib.wq_mx_quantize(_ptr(w), n, k, _ptr(codes), _ptr(scales), _stream(stream)),
+           "wq_mx_quantize")
+    return codes, scales
+
+
+def wq_mx_decompose(x, n_passes=2, planes=None, scales=None, stream=None):
+    """x bf16 [M, K] -> (planes uint8 [P, M, K] E4M3 bytes, scale bytes uint8 [P, M, K/32])."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if planes is None:
+        planes = torch.empty(n_passes, m, k, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(n_passes, m, k // 32, dtype=torch.uint8, device=x.device)
+    _check(lib.wq_mx_decompose(_ptr(x), m, k, n_passes, _ptr(planes), _ptr(scales),
+                               _stream(stream)), "wq_mx_decompose")
+    return planes, scales
+
+
+def mx_workspace(m, n, k, n_passes=2, device="cuda"):
+    nbytes = wq_workspace_bytes(WQ_OP_MX_GEMV, m, n, k, 0, n_passes)
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def wq_mx_gemv(x, n, n_passes, codes, scales, workspace=None, out=None, stream=None):
+    """y bf16 [M, N] = x_hat . w_hat^T (MXFP4 weights; two MXFP4 passes or one MXFP8 pass)."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if workspace is None:
+        workspace = mx_workspace(m, n, k, n_passes, x.device)
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib.wq_mx_gemv(_ptr(x), m, n, k, n_passes, _ptr(codes), _ptr(scales), _ptr(out),
+                          _ptr(workspace), workspace.numel(), _stream(stream)), "wq_mx_gemv")
+    return out

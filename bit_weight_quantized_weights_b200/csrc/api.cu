@@ -28,6 +28,12 @@ wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, 
 wq_status launch_msd_gemm(const void*, int64_t, int64_t, int64_t, int32_t, int32_t, const void*,
                           const void*, const void*, void*, void*, cudaStream_t);
 size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C);
+wq_status launch_mx_quantize(const float*, int64_t, int64_t, uint8_t*, uint8_t*, cudaStream_t);
+wq_status launch_mx_decompose(const void*, int64_t, int64_t, int32_t, uint8_t*, uint8_t*,
+                              cudaStream_t);
+wq_status launch_mx_gemv(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
+                         const uint8_t*, void*, void*, cudaStream_t);
+size_t mx_workspace_bytes(int64_t M, int64_t K, int32_t P);
 wq_status read_gemm_error(bool clear, uint32_t* v);
 wq_status read_msd_error(bool clear, uint32_t* v);
 wq_status read_gemv_error(bool clear, uint32_t* v);
@@ -323,6 +329,44 @@ wq_status wq_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_
   });
 }
 
+wq_status wq_mx_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales,
+                         void* stream) {
+  if (N < 0 || K <= 0 || K % 32 != 0) return WQ_ERR_INVALID_ARG;
+  if (N == 0) return WQ_OK;
+  if (!W || !codes || !scales) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({W, codes, scales})) return WQ_ERR_ALIGNMENT;
+  return guarded([&] { return launch_mx_quantize(W, N, K, codes, scales, as_stream(stream)); });
+}
+
+wq_status wq_mx_decompose(const void* x, int64_t M, int64_t K, int32_t n_passes, uint8_t* planes,
+                          uint8_t* scales, void* stream) {
+  if (M < 0 || K <= 0 || K % 32 != 0) return WQ_ERR_INVALID_ARG;
+  if (n_passes != 1 && n_passes != 2) return WQ_ERR_INVALID_ARG;
+  if (M == 0) return WQ_OK;
+  if (!x || !planes || !scales) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({x, planes, scales})) return WQ_ERR_ALIGNMENT;
+  if (M > INT32_MAX || K > INT32_MAX) return WQ_ERR_UNSUPPORTED;
+  return guarded(
+      [&] { return launch_mx_decompose(x, M, K, n_passes, planes, scales, as_stream(stream)); });
+}
+
+wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_passes,
+                     const uint8_t* codes, const uint8_t* scales, void* y, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % 32 != 0) return WQ_ERR_INVALID_ARG;
+  if (n_passes != 1 && n_passes != 2) return WQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (!x || !codes || !scales || !y) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({x, codes, scales, y})) return WQ_ERR_ALIGNMENT;
+  if (M > 16 || K % 256 != 0 || N % 16 != 0) return WQ_ERR_UNSUPPORTED;
+  if (N > INT32_MAX || K > INT32_MAX) return WQ_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < mx_workspace_bytes(M, K, n_passes)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return WQ_ERR_ALIGNMENT;
+  return guarded([&] {
+    return launch_mx_gemv(x, M, N, K, n_passes, codes, scales, y, workspace, as_stream(stream));
+  });
+}
+
 wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K, int32_t group,
                              int32_t n_components, size_t* bytes) {
   (void)N;
@@ -338,6 +382,10 @@ wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K, int32_t 
     case WQ_OP_MSD_GEMM:
       if (n_components < 1 || n_components > 3) return WQ_ERR_INVALID_ARG;
       *bytes = M == 0 ? 0 : msd_workspace_bytes(M, K, n_components);
+      return WQ_OK;
+    case WQ_OP_MX_GEMV:
+      if (n_components != 1 && n_components != 2) return WQ_ERR_INVALID_ARG;
+      *bytes = M == 0 ? 0 : mx_workspace_bytes(M, K, n_components);
       return WQ_OK;
   }
   return WQ_ERR_INVALID_ARG;

@@ -82,7 +82,7 @@ typedef enum {
 
 typedef enum { WQ_FMT_INT4_ASYM = 0, WQ_FMT_NF4 = 1 } wq_format;
 typedef enum { WQ_BF16 = 0, WQ_FP16 = 1, WQ_FP32 = 2 } wq_dtype;
-typedef enum { WQ_OP_GEMV = 0, WQ_OP_GEMM = 1, WQ_OP_MSD_GEMM = 2 } wq_op;
+typedef enum { WQ_OP_GEMV = 0, WQ_OP_GEMM = 1, WQ_OP_MSD_GEMM = 2, WQ_OP_MX_GEMV = 3 } wq_op;
 
 /* Human-readable name of a status. Never NULL. Host only. */
 const char* wq_status_string(wq_status status);
@@ -311,7 +311,47 @@ wq_status wq_msd_gemm_noalloc(const void* x, int64_t M, int64_t N, int64_t K,
                               const void* scales, const void* zeros, void* y, void* stream);
 
 /*
- * Workspace bytes an entry point needs for the given problem (0 if none).
+ * MX path of Multi-Scale Dequant ([MSD]: for MXFP4 weights, two MXFP4 passes
+ * over the bf16 activations multiply the weights directly, against one MXFP8
+ * pass). The page names the formats without defining them; the library reads
+ * them as microscaling blocks:
+ *   - 32 consecutive elements along K share one power-of-two scale 2^e, stored
+ *     as the byte e + 127 (e in -127..127): the smallest e such that no
+ *     element saturates (amax <= 6 * 2^e for E2M1, 448 * 2^e for E4M3);
+ *   - MXFP4 elements are FP4 E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4,
+ *     6; bit 3 = sign), MXFP8 elements FP8 E4M3 bytes; both round to nearest
+ *     with ties to the even code, and a value that rounds to zero is +0.
+ *
+ * wq_mx_quantize: MXFP4 weights W fp32 [N, K] (device) -> codes uint8
+ *   [N, K/2] (element 2j in the low nibble of byte j) and scale bytes uint8
+ *   [N, K/32]. K % 32 == 0. Bit-exact with the oracle.
+ * wq_mx_decompose: activations x bf16 [M, K] -> n_passes planes uint8
+ *   [n_passes][M][K] and scale bytes uint8 [n_passes][M][K/32].
+ *   n_passes == 2: x1 = MXFP4(x), r = x - x1 (exact), x2 = MXFP4(r) with its
+ *     own block scales; the planes hold the MXFP4 values as E4M3 bytes (every
+ *     E2M1 value is exact in E4M3).
+ *   n_passes == 1: one MXFP8 pass (the comparator).
+ *   K % 32 == 0. Bit-exact with the oracle.
+ * wq_mx_gemv: decode product y bf16 [M, N] = x_hat . w_hat^T for 1 <= M <= 16
+ *   (M == 0 or N == 0: no-op), with x_hat the n_passes decomposition of x and
+ *   w_hat the MXFP4 weights; every MMA covers one 32-element block of both
+ *   operands exactly and its partial sum takes the two block scales in fp32.
+ *   Requires K % 256 == 0 and N % 16 == 0. Workspace: at least
+ *   wq_workspace_bytes(WQ_OP_MX_GEMV, M, N, K, 0, n_passes) bytes (it holds
+ *   the decomposition); contents on entry do not matter.
+ * All are asynchronous on `stream`; every buffer is caller-owned.
+ */
+wq_status wq_mx_quantize(const float* W, int64_t N, int64_t K, uint8_t* codes, uint8_t* scales,
+                         void* stream);
+wq_status wq_mx_decompose(const void* x, int64_t M, int64_t K, int32_t n_passes, uint8_t* planes,
+                          uint8_t* scales, void* stream);
+wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_passes,
+                     const uint8_t* codes, const uint8_t* scales, void* y, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes an entry point needs for the given problem (0 if none);
+ * for WQ_OP_MX_GEMV, n_components is the number of passes (1 or 2).
  * Host only; `bytes` is a host pointer.
  */
 wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K,

@@ -186,6 +186,26 @@ def test_noalloc_validates_like_msd_gemm(wq):
                                  None) == wq.WQ_OK                    # empty: no-op
 
 
+def test_mx_validation(wq):
+    L = wq.lib
+    assert L.wq_mx_quantize(A16, 16, 100, A16, A16, None) == wq.WQ_ERR_INVALID_ARG   # K % 32
+    assert L.wq_mx_quantize(MIS, 16, 128, A16, A16, None) == wq.WQ_ERR_ALIGNMENT
+    assert L.wq_mx_quantize(A16, 0, 128, A16, A16, None) == wq.WQ_OK
+    assert L.wq_mx_decompose(A16, 4, 128, 3, A16, A16, None) == wq.WQ_ERR_INVALID_ARG  # passes
+    assert L.wq_mx_decompose(A16, 4, 100, 2, A16, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert L.wq_mx_decompose(A16, 0, 128, 2, A16, A16, None) == wq.WQ_OK
+    # wq_mx_gemv(x, M, N, K, passes, codes, scales, y, ws, ws_bytes, stream)
+    g = L.wq_mx_gemv
+    assert g(A16, 17, 256, 512, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 256, 480, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 250, 512, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 256, 512, 0, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 256, 512, 2, A16, A16, A16, None, 0, None) == wq.WQ_ERR_WORKSPACE
+    assert g(A16, 4, 256, 512, 2, A16, A16, MIS, A16, 1 << 20, None) == wq.WQ_ERR_ALIGNMENT
+    assert g(A16, 0, 256, 512, 2, A16, A16, A16, None, 0, None) == wq.WQ_OK
+    assert wq.wq_workspace_bytes(wq.WQ_OP_MX_GEMV, 16, 256, 512, 0, 2) == 2 * 16 * 512 + 2 * 16 * 16
+
+
 def test_pack_and_dequant_validation(wq):
     L = wq.lib
     assert L.wq_quantize_pack(0, A16, 16, 100, 64, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG

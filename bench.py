@@ -504,6 +504,8 @@ def measure_per_config(wq, peaks, device):
          at M = 128 and 1024 (g128) beside the fused GEMM on the same layer,
          and the relative L2 errors of MSD and of the bf16
          dequantize-then-cuBLAS product against the exact product
+      MX  the MX path of MSD on the same shapes at M = 1 and 16: MXFP4
+         weights with two MXFP4 activation passes, and one MXFP8 pass
 
     Each workload is graph-timed as a stream of back-to-back calls over
     rotating copies of its weights (> 4x L2 in total), with its own SM clock
@@ -517,7 +519,8 @@ def measure_per_config(wq, peaks, device):
     F, NF = wq.WQ_FMT_INT4_ASYM, wq.WQ_FMT_NF4
     bw = peaks["hbm_gbs"] * 1e9
     out = {"config1_gemv_tiny": [], "config2_nf4_dequant": [], "config3_gemv": [],
-           "config4_gemm": [], "config5_msd": [], "msd_vs_fused_gemm": [], "msd_accuracy": []}
+           "config4_gemm": [], "config5_msd": [], "msd_vs_fused_gemm": [], "msd_accuracy": [],
+           "mx_msd_decode": []}
 
     def normal(*shape, std=1.0):
         return torch.randn(*shape, generator=g, device=device) * std
@@ -538,16 +541,17 @@ def measure_per_config(wq, peaks, device):
         return [one] + [tuple(t.clone() if t is not None else None for t in one)
                         for _ in range(r - 1)]
 
-    def entry(name, us, clk, nbytes, flops, int8=False, extra=None):
+    def entry(name, us, clk, nbytes, flops, int8=False, extra=None, fp8=False):
         tf16_kind = tensor_peak(peaks, clk)
-        tpk = (2.0 if int8 else 1.0) * tf16_kind[0] * 1e12
+        tpk = (2.0 if (int8 or fp8) else 1.0) * tf16_kind[0] * 1e12
         t_roof = max(nbytes / bw, flops / tpk if flops else 0.0)
         e = {"case": name, "us": round(us, 2), "gbs": round(nbytes / (us * 1e-6) / 1e9, 1),
              "tflops": round(flops / (us * 1e-6) / 1e12, 1),
              "bound": "hbm" if nbytes / bw >= (flops / tpk if flops else 0.0) else "tensor",
              "roofline_frac": round(t_roof / (us * 1e-6), 4),
              "peak": "hbm %.0f GB/s, %s %s %.0f TFLOP/s" % (
-                 peaks["hbm_gbs"], tf16_kind[1], "int8" if int8 else "bf16", tpk / 1e12),
+                 peaks["hbm_gbs"], tf16_kind[1], "fp8" if fp8 else ("int8" if int8 else "bf16"),
+                 tpk / 1e12),
              "sm_mhz": clk.get("sm_mhz"), "clock_reasons": clk.get("reasons")}
         if extra:
             e.update(extra)
@@ -642,6 +646,29 @@ def measure_per_config(wq, peaks, device):
                     del x, y, wsp, fns
                 del ws
                 torch.cuda.empty_cache()
+        # the MX path ("Multi-Scale Dequant...", Abstract): MXFP4 weights with
+        # two MXFP4 activation passes, and one MXFP8 pass as the comparator,
+        # decode sizes on the same Qwen3-32B shapes
+        for n, k in [(5120, 5120), (25600, 5120), (5120, 25600)]:
+            one = wq.wq_mx_quantize(normal(n, k, std=0.02))
+            nb = n * k // 2 + n * k // 32
+            ws = [one] + [tuple(t.clone() for t in one) for _ in range(_copies_for(nb) - 1)]
+            for m in (1, 16):
+                x = acts(m, k, 0.005, 50.0)
+                y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+                for passes in (2, 1):
+                    wsp = wq.mx_workspace(m, n, k, passes, device)
+                    fns = [lambda c=c: wq.wq_mx_gemv(x, n, passes, *c, workspace=wsp, out=y)
+                           for c in ws]
+                    us, clk = _timed_launches(fns, sampler)
+                    out["mx_msd_decode"].append(entry(
+                        "%s M=%d %dx%d" % ("two MXFP4 passes" if passes == 2 else "one MXFP8 pass",
+                                           m, n, k),
+                        us, clk, nb + 2 * m * k + 2 * m * n, 2 * passes * m * n * k, fp8=True,
+                        extra={"weight_copies": len(ws)}))
+                del x, y
+            del ws
+            torch.cuda.empty_cache()
     return out
 
 
@@ -1002,7 +1029,7 @@ def max_over_ranks(v, world, device):
 
 
 PROFILE_CASES = ("nf4", "gemv_int4", "gemv_int4_m1", "gemv_nf4", "gemm", "msd", "msd_m16",
-                 "decdec")
+                 "decdec", "mx_m16")
 
 
 def profile_case(case, device):
@@ -1044,6 +1071,13 @@ def profile_case(case, device):
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
         ws = wq.msd_workspace(m, n, k, 128, 2, device)
         fn = lambda: wq.wq_msd_gemm(x, n, 2, 128, *pw, workspace=ws, out=y)  # noqa: E731
+    elif case == "mx_m16":
+        m, (n, k) = 16, MSD_SHAPE
+        codes, scales = wq.wq_mx_quantize(normal(n, k, std=0.02))
+        x = normal(m, k).to(torch.bfloat16)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        ws = wq.mx_workspace(m, n, k, 2, device)
+        fn = lambda: wq.wq_mx_gemv(x, n, 2, codes, scales, workspace=ws, out=y)  # noqa: E731
     elif case == "decdec":
         # select, then the corrected GEMV (ncu -k regex:gemv_kernel captures it)
         (n, k), m = DECDEC_SHAPE, 1

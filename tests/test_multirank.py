@@ -54,6 +54,21 @@ def test_job_value_is_summed_over_replicas(world):
     import bench
     peaks = {"hbm_gbs": 6456.5, "bf16_tflops": 1698.5, "bf16_tflops_sustained": 1422.0,
              "source": "test"}
-    table = bench.op_table(peaks)
+    table = bench.op_table(peaks, peaks["bf16_tflops"])
     roof_ms = sum(v["t_roof"] for v in table.values()) * 1e3
     assert bench.job_value(table, 2 * roof_ms, world) == pytest.approx(50.0 * world)
+
+
+def test_tensor_peak_follows_the_recorded_clocks():
+    """The bf16 denominator is the burst figure unless the timed region's own
+    clock record shows the power cap or clocks well below maximum."""
+    import bench
+    peaks = {"hbm_gbs": 6456.5, "bf16_tflops": 1698.5, "bf16_tflops_sustained": 1422.0}
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": []}) == (
+        1698.5, "burst")
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1965, "sm_max_mhz": 1965,
+                                     "reasons": ["sw_power_cap"]}) == (1422.0, "sustained")
+    assert bench.tensor_peak(peaks, {"sm_mhz": 1372, "sm_max_mhz": 1965, "reasons": []}) == (
+        1422.0, "sustained")
+    assert bench.tensor_peak(peaks, {"sm_mhz": None, "sm_max_mhz": None,
+                                     "reasons": ["unavailable"]}) == (1698.5, "burst")

@@ -194,7 +194,7 @@ __device__ __forceinline__ void mx_issue_stage(uint8_t* slot, const uint8_t* wti
 // Data placement per CTA (dynamic shared memory):
 //   ring [8 warps][kMxStages][16 rows][128 B]  weight stages
 //   xp   [P][M][Kc] E4M3 bytes, 16-byte chunk c of token m at c ^ 2(m & 3)
-//   xsc  [P][M][Kc/32] activation scale bytes
+//   xsc  [P][M][Kc/32] activation block scales as fp32 powers of two
 //   red  [S ranks][ceil(128/S)][16] fp32
 template <int NT, int P>
 __global__ void __launch_bounds__(256, 2) mx_gemv_kernel(MxArgs p, Nf4Table) {
@@ -202,8 +202,8 @@ __global__ void __launch_bounds__(256, 2) mx_gemv_kernel(MxArgs p, Nf4Table) {
   const int kc = p.kc, M = p.M;
   uint8_t* rings = smem;
   uint8_t* xp = smem + (size_t)8 * kMxStages * kStageBytes;
-  uint8_t* xsc = xp + (size_t)P * M * kc;
-  float* red = reinterpret_cast<float*>(xsc + ((size_t)P * M * (kc / 32) + 15) / 16 * 16);
+  float* xsc = reinterpret_cast<float*>(xp + (size_t)P * M * kc);
+  float* red = xsc + (size_t)P * M * (kc / 32);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = (int)blockIdx.x;
@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(256, 2) mx_gemv_kernel(MxArgs p, Nf4Table) {
   }
   for (int c = tid; c < P * M * (klen / 32); c += blockDim.x) {
     const int pm = c / (klen / 32), b = c - pm * (klen / 32);
-    xsc[(size_t)pm * (kc / 32) + b] = p.xs[(int64_t)pm * nblk + k0 / 32 + b];
+    xsc[(size_t)pm * (kc / 32) + b] = pow2f((int)p.xs[(int64_t)pm * nblk + k0 / 32 + b] - 127);
   }
   asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
   __syncthreads();
@@ -308,10 +308,8 @@ __global__ void __launch_bounds__(256, 2) mx_gemv_kernel(MxArgs p, Nf4Table) {
                     8 * (t & 1));
                 float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 mma_e4m3(d, a0, a1, a2, a3, xv.x, xv.y);
-                const float fx0 =
-                    pow2f((int)xsc[((size_t)pp * M + tokc[a][0]) * (kc / 32) + lb] - 127);
-                const float fx1 =
-                    pow2f((int)xsc[((size_t)pp * M + tokc[a][1]) * (kc / 32) + lb] - 127);
+                const float fx0 = xsc[((size_t)pp * M + tokc[a][0]) * (kc / 32) + lb];
+                const float fx1 = xsc[((size_t)pp * M + tokc[a][1]) * (kc / 32) + lb];
                 acc[a][0] = fmaf(d[0] * fwA, fx0, acc[a][0]);
                 acc[a][1] = fmaf(d[1] * fwA, fx1, acc[a][1]);
                 acc[a][2] = fmaf(d[2] * fwB, fx0, acc[a][2]);
@@ -330,7 +328,7 @@ __global__ void __launch_bounds__(256, 2) mx_gemv_kernel(MxArgs p, Nf4Table) {
 template <int NT, int P>
 size_t mx_smem(int kc, int S, int M) {
   return (size_t)8 * kMxStages * kStageBytes + (size_t)P * M * kc +
-         ((size_t)P * M * (kc / 32) + 15) / 16 * 16 + red_bytes(S);
+         (size_t)P * M * (kc / 32) * 4 + red_bytes(S);
 }
 
 template <int NT, int P>

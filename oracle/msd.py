@@ -131,3 +131,57 @@ def effective_bits(x, a, s):
     ok = amax > 0
     err = np.maximum(err[ok], np.finfo(np.float64).tiny)
     return float(np.min(np.log2(amax[ok] / err)))
+
+
+# ---------------------------------------------------------------------------
+# NF4 weights on the MSD path
+# ---------------------------------------------------------------------------
+# The pages give MSD for integer weights; NF4 codes index 16 real codebook
+# values ("Fast NF4 Dequantization Kernels for Large Language Model
+# Inference", Abstract), which no integer GEMM takes as they are. The reading
+# used here keeps MSD's point (integer activation digits times integer
+# weights, no weight converted to floating point): the codebook values become
+# integers c_int = rint(c * 2^13) in [-8192, 8192] (within 2^-14 of c), split
+# into two signed 8-bit digits c_int = 128 h + l with l in [-64, 63] and h in
+# [-64, 64]; the block's absmax is applied after the block's integer sum:
+#
+#   y[m, n] = sum_c s_c[m] sum_blk absmax[n, blk] 2^-13
+#             * sum_{k in blk} a_c[m, k] (128 h[q] + l[q])
+#
+# which equals x_hat . w_int^T exactly, with w_int = absmax * c_int * 2^-13
+# (each weight within 2^-14 absmax of the NF4 value codebook[q] * absmax).
+
+NF4_INT_SHIFT = 13
+
+
+def nf4_int_codebook(codebook):
+    """The 16 NF4 code values as integers rint(c * 2^13) (int64 [16])."""
+    cb = np.asarray(codebook, dtype=np.float64)
+    return np.rint(cb * 2.0 ** NF4_INT_SHIFT).astype(np.int64)
+
+
+def nf4_int_digits(codebook):
+    """(h, l) int64 [16]: c_int = 128 h + l with l in [-64, 63]."""
+    ci = nf4_int_codebook(codebook)
+    h = np.floor((ci + 64) / 128.0).astype(np.int64)
+    return h, ci - 128 * h
+
+
+def msd_nf4_product(a, s, codes, absmax, k, codebook):
+    """y [M, N] in fp64: sum_c s_c sum_blk absmax 2^-13 sum a_c (128 h + l),
+    integer inner sums exact. codes: NF4 codes of the row-major [N, K] weight
+    (flattened), absmax fp32 [N * K / 64]."""
+    h, l = nf4_int_digits(codebook)
+    q = np.asarray(codes, dtype=np.int64).reshape(-1, k)
+    n = q.shape[0]
+    w_int = (128 * h[q] + l[q]).astype(np.float64)          # [N, K], exact integers
+    am = np.asarray(absmax, dtype=np.float64).reshape(n, k // 64)
+    c_total, m = s.shape
+    y = np.zeros((m, n), dtype=np.float64)
+    for ci in range(c_total):
+        a64 = np.asarray(a[ci], dtype=np.float64)
+        for b in range(k // 64):
+            sl = slice(64 * b, 64 * (b + 1))
+            p = a64[:, sl] @ w_int[:, sl].T                    # exact integers in fp64
+            y += np.asarray(s[ci], dtype=np.float64)[:, None] * (am[None, :, b] * p)
+    return y * 2.0 ** -NF4_INT_SHIFT

@@ -97,3 +97,53 @@ def test_group_sums_and_partials_definition():
     assert msd.group_sums(a, 2).tolist() == [[[-1, 7]]]
     p = msd.int_partials(a, q, 2)
     assert p[0, 0].tolist() == [[-3, 25], [-30, 60]]
+
+
+# ---------------------------------------------------------------------------
+# NF4 weights on the MSD path
+# ---------------------------------------------------------------------------
+
+def test_nf4_integer_codebook_digits_and_bound():
+    from oracle import formats
+    cb = formats.nf4_codebook()
+    ci = msd.nf4_int_codebook(cb)
+    h, l = msd.nf4_int_digits(cb)
+    assert np.all(np.abs(ci / 8192.0 - cb.astype(np.float64)) <= 2.0 ** -14)
+    assert np.array_equal(128 * h + l, ci)
+    assert l.min() >= -64 and l.max() <= 63 and h.min() >= -64 and h.max() <= 64
+    assert ci[0] == -8192 and ci[15] == 8192 and ci[7] == 0      # -1, +1 and the exact zero
+
+
+def test_msd_nf4_product_is_exact_against_rationals():
+    """The product equals x_hat . w_int^T exactly (brute force in rationals on
+    a tiny problem), and lies within the weight bound of the exact NF4
+    product: |w_int - w| <= absmax 2^-14 per weight."""
+    from fractions import Fraction
+    from oracle import formats
+    rng = np.random.default_rng(11)
+    m, n, k = 2, 3, 128
+    w = (rng.standard_normal((n, k)) * 0.02).astype(np.float32)
+    codes, absmax = formats.nf4_quantize(w)
+    x = rng.standard_normal((m, k)).astype(np.float32)
+    a, s = msd.decompose(x, 2)
+    cb = formats.nf4_codebook()
+    y = msd.msd_nf4_product(a, s, codes, absmax, k, cb)
+    h, l = msd.nf4_int_digits(cb)
+    q = codes.reshape(n, k).astype(np.int64)
+    am = absmax.reshape(n, k // 64)
+    for i in range(m):
+        for j in range(n):
+            tot = Fraction(0)
+            for c in range(2):
+                for kk in range(k):
+                    wij = Fraction(float(am[j, kk // 64])) * (128 * int(h[q[j, kk]]) + int(l[q[j, kk]]))
+                    tot += Fraction(float(s[c, i])) * int(a[c, i, kk]) * wij
+            tot /= 8192
+            # the integer inner sums are exact; the scaled fp64 sums round a few times
+            assert abs(Fraction(float(y[i, j])) - tot) <= abs(tot) * Fraction(1, 2 ** 45)
+    # against the exact NF4 product of the decomposed activations
+    from oracle import products
+    x_hat = msd.reconstruct(a, s)
+    y_nf4 = products.w4a16_nf4(x_hat, codes, absmax, k)
+    bound = np.abs(x_hat) @ np.repeat(am, 64, axis=1).T * 2.0 ** -14
+    assert np.all(np.abs(y - y_nf4) <= bound * (1 + 1e-9))

@@ -40,7 +40,7 @@ EXPORTED = [
     "wq_w4a16_gemv", "wq_w4a16_gemm", "wq_msd_decompose", "wq_msd_gemm",
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
-    "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv",
+    "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv", "wq_msd_gemm_nf4",
 ]
 
 
@@ -80,6 +80,7 @@ def _load():
         "wq_mx_quantize": ([P, I64, I64, P, P, P], ctypes.c_int),
         "wq_mx_decompose": ([P, I64, I64, I32, P, P, P], ctypes.c_int),
         "wq_mx_gemv": ([P, I64, I64, I64, I32, P, P, P, P, SZ, P], ctypes.c_int),
+        "wq_msd_gemm_nf4": ([P, I64, I64, I64, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -413,4 +414,18 @@ def wq_mx_gemv(x, n, n_passes, codes, scales, workspace=None, out=None, stream=N
         out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
     _check(lib.wq_mx_gemv(_ptr(x), m, n, k, n_passes, _ptr(codes), _ptr(scales), _ptr(out),
                           _ptr(workspace), workspace.numel(), _stream(stream)), "wq_mx_gemv")
+    return out
+
+
+def wq_msd_gemm_nf4(x, n, n_components, codes, absmax, workspace=None, out=None, stream=None):
+    """Decode MSD product with NF4 weights (integer codebook digits); M <= 16."""
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    if workspace is None:
+        workspace = msd_workspace(m, n, k, 64, n_components, x.device)
+    if out is None:
+        out = torch.empty(m, n, dtype=torch.bfloat16, device=x.device)
+    _check(lib.wq_msd_gemm_nf4(_ptr(x), m, n, k, n_components, _ptr(codes), _ptr(absmax),
+                               _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "wq_msd_gemm_nf4")
     return out

@@ -34,6 +34,8 @@ wq_status launch_mx_decompose(const void*, int64_t, int64_t, int32_t, uint8_t*, 
 wq_status launch_mx_gemv(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
                          const uint8_t*, void*, void*, cudaStream_t);
 size_t mx_workspace_bytes(int64_t M, int64_t K, int32_t P);
+wq_status launch_msd_nf4(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
+                         const float*, void*, void*, cudaStream_t);
 wq_status read_gemm_error(bool clear, uint32_t* v);
 wq_status read_msd_error(bool clear, uint32_t* v);
 wq_status read_gemv_error(bool clear, uint32_t* v);
@@ -326,6 +328,22 @@ wq_status wq_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_
   return guarded([&] {
     return launch_msd_gemm(x, M, N, K, n_components, group, qweight, scales, zeros, y, workspace,
                            as_stream(stream));
+  });
+}
+
+wq_status wq_msd_gemm_nf4(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_components,
+                          const uint8_t* codes, const float* absmax, void* y, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  wq_status s = check_product(x, M, N, K, WQ_FMT_NF4, 64, codes, absmax, nullptr, y);
+  if (s != WQ_OK) return s;
+  if (n_components < 1 || n_components > 3) return WQ_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return WQ_OK;
+  if (M > 16 || K % 256 != 0 || N % 16 != 0) return WQ_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < msd_workspace_bytes(M, K, n_components)) return WQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return WQ_ERR_ALIGNMENT;
+  return guarded([&] {
+    return launch_msd_nf4(x, M, N, K, n_components, codes, absmax, y, workspace,
+                          as_stream(stream));
   });
 }
 

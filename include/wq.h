@@ -283,6 +283,25 @@ wq_status wq_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K,
                       void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Multi-Scale Dequant with NF4 weights, decode (1 <= M <= 16) ([MSD] with
+ * [NF4]). The pages give MSD for integer weights; NF4 codes index real
+ * codebook values, so the library reads NF4-MSD as: the 16 code values become
+ * integers c_int = rint(c * 2^13) (within 2^-14 of c), split into two signed
+ * 8-bit digits c_int = 128 h + l; the activation digits of wq_msd_decompose
+ * multiply them on the int8 tensor cores and each 64-element block's absmax
+ * is applied after the block's integer sum:
+ *   y[m, n] = sum_c s_c[m] sum_blk absmax[n, blk] 2^-13
+ *             sum_{k in blk} a_c[m, k] (128 h[q] + l[q])
+ * (each weight within 2^-14 absmax of codebook[q] * absmax). No weight is
+ * converted to floating point. codes/absmax: the canonical NF4 layout. M == 0
+ * or N == 0 is a no-op; requires K % 256 == 0, N % 16 == 0, 1 <= n_components
+ * <= 3. Workspace: at least wq_workspace_bytes(WQ_OP_MSD_GEMM, ...) bytes.
+ */
+wq_status wq_msd_gemm_nf4(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_components,
+                          const uint8_t* codes, const float* absmax, void* y, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/*
  * wq_msd_gemm for callers that cannot allocate device memory. The library's
  * pages have no counterpart to this call; it exists for deployment. Some
  * callers cannot hand the library a workspace: an engine that carves up all

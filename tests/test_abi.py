@@ -206,6 +206,19 @@ def test_mx_validation(wq):
     assert wq.wq_workspace_bytes(wq.WQ_OP_MX_GEMV, 16, 256, 512, 0, 2) == 2 * 16 * 512 + 2 * 16 * 16
 
 
+def test_msd_nf4_validation(wq):
+    g = wq.lib.wq_msd_gemm_nf4
+    # (x, M, N, K, C, codes, absmax, y, ws, ws_bytes, stream)
+    assert g(A16, 17, 256, 512, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 256, 640, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 250, 512, 2, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_UNSUPPORTED
+    assert g(A16, 4, 256, 512, 4, A16, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 256, 512, 2, None, A16, A16, A16, 1 << 20, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 256, 512, 2, A16, A16, A16, None, 0, None) == wq.WQ_ERR_WORKSPACE
+    assert g(A16, 4, 256, 512, 2, A16, MIS, A16, A16, 1 << 20, None) == wq.WQ_ERR_ALIGNMENT
+    assert g(A16, 0, 256, 512, 2, A16, A16, A16, None, 0, None) == wq.WQ_OK
+
+
 def test_pack_and_dequant_validation(wq):
     L = wq.lib
     assert L.wq_quantize_pack(0, A16, 16, 100, 64, A16, A16, A16, None) == wq.WQ_ERR_INVALID_ARG

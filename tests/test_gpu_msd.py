@@ -116,3 +116,44 @@ def test_msd_accuracy_not_below_dequant_baseline(wq):
     rel_deq, _ = numerics.compare(numerics.bf16_round(y_bf16w.astype(np.float32)), y_exact)
     print("relative L2 error: msd C=2 %.3e, bf16 dequantize-then-GEMM %.3e" % (rel_msd, rel_deq))
     assert rel_msd <= helpers.REL_FRO_TOL
+
+
+# ---------------------------------------------------------------------------
+# NF4 weights on the MSD path (integer codebook digits), decode sizes
+# ---------------------------------------------------------------------------
+
+def _nf4_msd_case(wq, m, n, k, c, seed, cols=None):
+    from oracle import formats, products
+    codes, absmax, packed = helpers.nf4_packed(n, k, seed)
+    cw, am = helpers.to_dev_nf4(absmax, packed)
+    x = _x(m, k, seed)
+    y = wq.wq_msd_gemm_nf4(x.cuda(), n, c, cw, am)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
+    xf = helpers.x_f32(x)
+    a, sa = msd.decompose(xf, c)
+    cols = np.arange(n) if cols is None else cols
+    q2 = codes.reshape(n, k)[cols].reshape(-1)
+    am2 = absmax.reshape(n, k // 64)[cols].reshape(-1)
+    y_dec = msd.msd_nf4_product(a, sa, q2, am2, k, formats.nf4_codebook())
+    yg = y.cpu()[:, cols]
+    what = "msd-nf4 C=%d M=%d %dx%d" % (c, m, n, k)
+    helpers.check_within_bf16_rounding(yg, y_dec, what + " vs decomposed", slack=1e-4)
+    if c >= 2:
+        helpers.check_product(yg, products.w4a16_nf4(xf, q2, am2, k), what + " vs exact NF4")
+
+
+@pytest.mark.parametrize("m,n,k,c", [
+    (1, 128, 256, 2), (5, 1040, 768, 2), (16, 256, 2560, 2), (9, 384, 512, 1), (16, 128, 1024, 3),
+    (16, 38016, 256, 2),   # more row tiles than one wave of clusters
+])
+def test_msd_nf4_every_element(wq, m, n, k, c):
+    _nf4_msd_case(wq, m, n, k, c, seed=m + n + c)
+
+
+@pytest.mark.parametrize("n,k", [(5120, 5120), (25600, 5120), (5120, 25600)])
+@pytest.mark.parametrize("m", [1, 16])
+def test_msd_nf4_qwen_shapes_sampled(wq, m, n, k):
+    rng = np.random.default_rng(m + n + k)
+    cols = np.sort(rng.choice(n, 256, replace=False))
+    _nf4_msd_case(wq, m, n, k, 2, seed=2, cols=cols)

@@ -506,6 +506,8 @@ def measure_per_config(wq, peaks, device):
          dequantize-then-cuBLAS product against the exact product
       MX  the MX path of MSD on the same shapes at M = 1 and 16: MXFP4
          weights with two MXFP4 activation passes, and one MXFP8 pass
+      NF4 MSD with NF4 weights (integer codebook digits), same shapes, M = 1
+         and 16
 
     Each workload is graph-timed as a stream of back-to-back calls over
     rotating copies of its weights (> 4x L2 in total), with its own SM clock
@@ -520,7 +522,7 @@ def measure_per_config(wq, peaks, device):
     bw = peaks["hbm_gbs"] * 1e9
     out = {"config1_gemv_tiny": [], "config2_nf4_dequant": [], "config3_gemv": [],
            "config4_gemm": [], "config5_msd": [], "msd_vs_fused_gemm": [], "msd_accuracy": [],
-           "mx_msd_decode": []}
+           "mx_msd_decode": [], "nf4_msd_decode": []}
 
     def normal(*shape, std=1.0):
         return torch.randn(*shape, generator=g, device=device) * std
@@ -667,6 +669,25 @@ def measure_per_config(wq, peaks, device):
                         us, clk, nb + 2 * m * k + 2 * m * n, 2 * passes * m * n * k, fp8=True,
                         extra={"weight_copies": len(ws)}))
                 del x, y
+            del ws
+            torch.cuda.empty_cache()
+        # NF4 weights on the MSD path (integer codebook digits), decode sizes
+        for n, k in [(5120, 5120), (25600, 5120), (5120, 25600)]:
+            one = wq.wq_quantize_pack(NF, normal(n, k, std=0.02), 64)[:2]
+            nb = n * k // 2 + n * k // 16
+            ws = [one] + [tuple(t.clone() for t in one) for _ in range(_copies_for(nb) - 1)]
+            for m in (1, 16):
+                x = acts(m, k, 0.005, 50.0)
+                y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+                wsp = wq.msd_workspace(m, n, k, 64, 2, device)
+                fns = [lambda c=c: wq.wq_msd_gemm_nf4(x, n, 2, *c, workspace=wsp, out=y)
+                       for c in ws]
+                us, clk = _timed_launches(fns, sampler)
+                out["nf4_msd_decode"].append(entry(
+                    "C=2 M=%d %dx%d" % (m, n, k), us, clk, nb + 2 * m * k + 2 * m * n,
+                    2 * 2 * 2 * m * n * k, int8=True,
+                    extra={"weight_copies": len(ws), "ops": "int8 MMAs: 2 planes x 2 weight digits"}))
+                del x, y, wsp
             del ws
             torch.cuda.empty_cache()
     return out

@@ -24,6 +24,9 @@ Modules
                decomposed integer product.
 ``decdec``     salient-channel residual correction: the residual matrix,
                the per-step channel selection and the corrected product.
+``kvmsd``      decode attention over an INT4 KV cache with MSD on both
+               products (query digits times K codes, softmax-weight digits
+               times V codes), chunked softmax with the flash-decoding merge.
 ``mx``         MX block formats (MXFP4 E2M1, MXFP8 E4M3, power-of-two block
                scales), the two-pass MXFP4 activation decomposition, the
                single-pass MXFP8 comparator, and their product with MXFP4
@@ -41,4 +44,4 @@ measure 6.15 bits, worst block amax/37, derived bound amax/12; the page's
 single-pass MXFP8 figure, 5.24 bits, does reproduce and is pinned).
 """
 
-from . import numerics, formats, products, msd, decdec, mx  # noqa: F401
+from . import numerics, formats, products, msd, decdec, mx, kvmsd  # noqa: F401

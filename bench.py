@@ -508,6 +508,10 @@ def measure_per_config(wq, peaks, device):
          weights with two MXFP4 activation passes, and one MXFP8 pass
       NF4 MSD with NF4 weights (integer codebook digits), same shapes, M = 1
          and 16
+      KV  MSD decode attention over an INT4 KV cache, C = 2, Qwen3-32B heads
+         (Hq = 64, Hkv = 8, D = 128), B x L = 32 x 8192 and 8 x 32768,
+         beside torch's scaled-dot-product attention on a bf16 cache (bytes:
+         K and V codes with their fp16 scales and zeros, q and out)
 
     Each workload is graph-timed as a stream of back-to-back calls over
     rotating copies of its weights (> 4x L2 in total), with its own SM clock
@@ -522,7 +526,7 @@ def measure_per_config(wq, peaks, device):
     bw = peaks["hbm_gbs"] * 1e9
     out = {"config1_gemv_tiny": [], "config2_nf4_dequant": [], "config3_gemv": [],
            "config4_gemm": [], "config5_msd": [], "msd_vs_fused_gemm": [], "msd_accuracy": [],
-           "mx_msd_decode": [], "nf4_msd_decode": []}
+           "mx_msd_decode": [], "nf4_msd_decode": [], "kv_msd_decode_attention": []}
 
     def normal(*shape, std=1.0):
         return torch.randn(*shape, generator=g, device=device) * std
@@ -689,6 +693,42 @@ def measure_per_config(wq, peaks, device):
                     extra={"weight_copies": len(ws), "ops": "int8 MMAs: 2 planes x 2 weight digits"}))
                 del x, y, wsp
             del ws
+            torch.cuda.empty_cache()
+        # MSD decode attention over an INT4 KV cache ("Multi-Scale Dequant...",
+        # Abstract: the cache is never dequantized), Qwen3-32B heads, beside
+        # torch's scaled-dot-product attention on a bf16 cache of the same shape
+        hq, hkv, d = 64, 8, 128
+        for b, length in ((32, 8192), (8, 32768)):
+            cache = [wq.kv_quantize(normal(b, hkv, length, d, std=0.5)),
+                     wq.kv_quantize(normal(b, hkv, length, d))]
+            nb = 2 * b * hkv * length * (d // 2 + 4)          # codes + fp16 scale and zero
+            copies = [cache] + [[tuple(t.clone() for t in kv) for kv in cache]
+                                for _ in range(_copies_for(nb) - 1)]
+            q = normal(b, hq, d).to(torch.bfloat16)
+            o = torch.empty(b, hq, d, dtype=torch.bfloat16, device=device)
+            wsp = wq.attention_workspace(b, hq, hkv, length, d, 2, device)
+            fns = [lambda c=c: wq.wq_msd_decode_attention(q, c[0], c[1], 2, workspace=wsp, out=o)
+                   for c in copies]
+            us, clk = _timed_launches(fns, sampler)
+            del copies, cache, fns
+            torch.cuda.empty_cache()
+            kb = normal(b, hkv, length, d).to(torch.bfloat16)
+            vb = normal(b, hkv, length, d).to(torch.bfloat16)
+            q4 = q.view(b, hq, 1, d)
+            sdpa = [lambda: torch.nn.functional.scaled_dot_product_attention(
+                q4, kb, vb, enable_gqa=True)]
+            us_ref, _ = _timed_launches(sdpa, sampler)
+            nb_ref = 2 * b * hkv * length * d * 2
+            del kb, vb, sdpa
+            torch.cuda.empty_cache()
+            out["kv_msd_decode_attention"].append(entry(
+                "C=2 B=%d L=%d Hq=%d Hkv=%d D=%d" % (b, length, hq, hkv, d), us, clk,
+                nb + 2 * 2 * b * hq * d, 2 * 2 * 2 * 2 * b * hq * length * d, int8=True,
+                extra={"sdpa_bf16_cache_us": round(us_ref, 2),
+                       "sdpa_bf16_cache_gbs": round(nb_ref / (us_ref * 1e-6) / 1e9, 1),
+                       "speedup_vs_sdpa_bf16": round(us_ref / us, 3),
+                       "cache_bytes_int4": nb, "cache_bytes_bf16": nb_ref}))
+            del q, o, wsp
             torch.cuda.empty_cache()
     return out
 

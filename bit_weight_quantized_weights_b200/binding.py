@@ -41,6 +41,7 @@ EXPORTED = [
     "wq_workspace_bytes", "wq_device_error", "wq_msd_gemm_noalloc",
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
     "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv", "wq_msd_gemm_nf4",
+    "wq_msd_decode_attention", "wq_msd_decode_attention_workspace",
 ]
 
 
@@ -81,6 +82,10 @@ def _load():
         "wq_mx_decompose": ([P, I64, I64, I32, P, P, P], ctypes.c_int),
         "wq_mx_gemv": ([P, I64, I64, I64, I32, P, P, P, P, SZ, P], ctypes.c_int),
         "wq_msd_gemm_nf4": ([P, I64, I64, I64, I32, P, P, P, P, SZ, P], ctypes.c_int),
+        "wq_msd_decode_attention": ([P, I64, I64, I64, I64, I32, I32, P, P, P, P, P, P, P, P, SZ,
+                                     P], ctypes.c_int),
+        "wq_msd_decode_attention_workspace": ([I64, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
+                                              ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -428,4 +433,50 @@ def wq_msd_gemm_nf4(x, n, n_components, codes, absmax, workspace=None, out=None,
     _check(lib.wq_msd_gemm_nf4(_ptr(x), m, n, k, n_components, _ptr(codes), _ptr(absmax),
                                _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "wq_msd_gemm_nf4")
+    return out
+
+
+def kv_quantize(kv, stream=None):
+    """INT4-quantize a KV cache fp32 [B, Hkv, L, D] on the GPU, one group per
+    (sequence, head, token) row: returns (codes int32 [B, Hkv, L, D/8], scales
+    fp16 [B, Hkv, L], zeros fp16 [B, Hkv, L])."""
+    _cuda(kv, torch.float32, "kv")
+    b, hkv, length, d = kv.shape
+    qw, sc, zr = wq_quantize_pack(WQ_FMT_INT4_ASYM, kv.reshape(-1, d), d, stream=stream)
+    return (qw.view(b, hkv, length, d // 8), sc.view(b, hkv, length), zr.view(b, hkv, length))
+
+
+def attention_workspace(b, hq, hkv, length, d, n_components, device):
+    size = ctypes.c_size_t(0)
+    _check(lib.wq_msd_decode_attention_workspace(b, hq, hkv, length, d, n_components,
+                                                 ctypes.byref(size)),
+           "wq_msd_decode_attention_workspace")
+    return torch.empty(max(int(size.value), 1), dtype=torch.uint8, device=device)
+
+
+def wq_msd_decode_attention(q, k_cache, v_cache, n_components=2, workspace=None, out=None,
+                            stream=None):
+    """MSD decode attention: q bf16 [B, Hq, D]; k_cache / v_cache = (codes,
+    scales, zeros) as kv_quantize returns them. Returns out bf16 [B, Hq, D]."""
+    _cuda(q, torch.bfloat16, "q")
+    b, hq, d = q.shape
+    kq, ks, kz = k_cache
+    vq, vs, vz = v_cache
+    hkv, length = ks.shape[1], ks.shape[2]
+    for t, dt, name in ((kq, torch.int32, "k_codes"), (ks, torch.float16, "k_scales"),
+                        (kz, torch.float16, "k_zeros"), (vq, torch.int32, "v_codes"),
+                        (vs, torch.float16, "v_scales"), (vz, torch.float16, "v_zeros")):
+        _cuda(t, dt, name)
+    if tuple(kq.shape) != (b, hkv, length, d // 8) or tuple(vq.shape) != tuple(kq.shape) or \
+            tuple(vs.shape) != tuple(ks.shape) or tuple(kz.shape) != tuple(ks.shape) or \
+            tuple(vz.shape) != tuple(ks.shape) or ks.shape[0] != b:
+        raise ValueError("KV cache shapes do not match q")
+    if workspace is None:
+        workspace = attention_workspace(b, hq, hkv, length, d, n_components, q.device)
+    if out is None:
+        out = torch.empty(b, hq, d, dtype=torch.bfloat16, device=q.device)
+    _check(lib.wq_msd_decode_attention(_ptr(q), b, hq, hkv, length, d, n_components, _ptr(kq),
+                                       _ptr(ks), _ptr(kz), _ptr(vq), _ptr(vs), _ptr(vz), _ptr(out),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "wq_msd_decode_attention")
     return out

@@ -36,6 +36,10 @@ wq_status launch_mx_gemv(const void*, int64_t, int64_t, int64_t, int32_t, const 
 size_t mx_workspace_bytes(int64_t M, int64_t K, int32_t P);
 wq_status launch_msd_nf4(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
                          const float*, void*, void*, cudaStream_t);
+size_t kv_msd_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int32_t C);
+wq_status launch_kv_msd(const void*, int64_t, int64_t, int64_t, int64_t, int32_t, const void*,
+                        const void*, const void*, const void*, const void*, const void*, void*,
+                        void*, cudaStream_t);
 wq_status read_gemm_error(bool clear, uint32_t* v);
 wq_status read_msd_error(bool clear, uint32_t* v);
 wq_status read_gemv_error(bool clear, uint32_t* v);
@@ -103,6 +107,20 @@ wq_status check_product(const void* x, int64_t M, int64_t N, int64_t K, wq_forma
   if (K % 128 != 0) return WQ_ERR_UNSUPPORTED;
   if (fmt == WQ_FMT_INT4_ASYM && group % 64 != 0) return WQ_ERR_UNSUPPORTED;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return WQ_ERR_UNSUPPORTED;
+  return WQ_OK;
+}
+
+// Shape checks of the KV-cache attention: WQ_OK, or the status to return.
+wq_status check_attention_shape(int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int32_t D,
+                                int32_t n_components) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || D <= 0 || D % 8 != 0)
+    return WQ_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || n_components < 1 || n_components > 3) return WQ_ERR_INVALID_ARG;
+  const int64_t R = Hq / Hkv;
+  if (D != 128 || n_components == 3 || (R != 1 && R != 2 && R != 4 && R != 8))
+    return WQ_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535 || L > INT32_MAX - 256 || B * Hq > INT32_MAX)
+    return WQ_ERR_UNSUPPORTED;
   return WQ_OK;
 }
 
@@ -382,6 +400,36 @@ wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_p
   if (!aligned16(workspace)) return WQ_ERR_ALIGNMENT;
   return guarded([&] {
     return launch_mx_gemv(x, M, N, K, n_passes, codes, scales, y, workspace, as_stream(stream));
+  });
+}
+
+wq_status wq_msd_decode_attention_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t L,
+                                            int32_t D, int32_t n_components, size_t* bytes) {
+  if (!bytes) return WQ_ERR_INVALID_ARG;
+  wq_status s = check_attention_shape(B, Hq, Hkv, L, D, n_components);
+  if (s != WQ_OK) return s;
+  *bytes = B == 0 ? 0 : kv_msd_workspace_bytes(B, Hq, L, n_components);
+  return WQ_OK;
+}
+
+wq_status wq_msd_decode_attention(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64_t L,
+                                  int32_t D, int32_t n_components, const void* k_codes,
+                                  const void* k_scales, const void* k_zeros, const void* v_codes,
+                                  const void* v_scales, const void* v_zeros, void* out,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  wq_status s = check_attention_shape(B, Hq, Hkv, L, D, n_components);
+  if (s != WQ_OK) return s;
+  if (B == 0) return WQ_OK;
+  if (!q || !k_codes || !k_scales || !k_zeros || !v_codes || !v_scales || !v_zeros || !out)
+    return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({q, k_codes, k_scales, k_zeros, v_codes, v_scales, v_zeros, out}))
+    return WQ_ERR_ALIGNMENT;
+  if (!workspace || ws_bytes < kv_msd_workspace_bytes(B, Hq, L, n_components))
+    return WQ_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return WQ_ERR_ALIGNMENT;
+  return guarded([&] {
+    return launch_kv_msd(q, B, Hq, Hkv, L, n_components, k_codes, k_scales, k_zeros, v_codes,
+                         v_scales, v_zeros, out, workspace, as_stream(stream));
   });
 }
 

@@ -83,3 +83,28 @@ def scaled_weights(n, k, seed=0, row_exp=None, block_exp=None, factor=1.0):
         e = lo + torch.arange(n) % (hi - lo + 1)
         w = (w.double() * torch.pow(10.0, e.double())[:, None]).float()
     return w
+
+
+# Decode attention over a quantized KV cache: Qwen3-32B's attention heads
+# (64 query heads sharing 8 KV heads, head dimension 128).
+ATTN_HEADS = dict(Hq=64, Hkv=8, D=128)
+KV_K_OUTLIERS = (0.04, 8.0)
+
+
+def decode_attention(b, hq, hkv, length, d=128, seed=0, k_outliers=KV_K_OUTLIERS):
+    """(q bf16 [B, Hq, D], K fp32 [B, Hkv, L, D], V fp32 [B, Hkv, L, D]), CPU,
+    drawn in that order from one generator: q ~ N(0, 1) rounded once to bf16,
+    K ~ N(0, 0.5) with a few channels (the same for every token of a head,
+    chosen by randperm) scaled up, as keys carry per-channel outliers, and
+    V ~ N(0, 1)."""
+    g = generator(seed)
+    q = torch.randn(b, hq, d, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn(b, hkv, length, d, generator=g, dtype=torch.float32) * 0.5
+    if k_outliers is not None:
+        frac, scale = k_outliers
+        cnt = max(1, round(frac * d))
+        for h in range(hkv):
+            idx = torch.randperm(d, generator=g)[:cnt]
+            k[:, h, :, idx] *= scale
+    v = torch.randn(b, hkv, length, d, generator=g, dtype=torch.float32)
+    return q, k, v

@@ -369,6 +369,54 @@ wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_p
                      size_t ws_bytes, void* stream);
 
 /*
+ * Multi-Scale Dequant in decode attention over an INT4 KV cache ([MSD],
+ * Abstract: the quantized KV cache multiplies low-precision components of
+ * the other operand directly, so the cache is never dequantized and its HBM
+ * traffic in attention shrinks). One new query token per sequence:
+ *   q        bf16 [B, Hq, D] (device); Hq = R * Hkv, query head h reads KV
+ *            head h / R (grouped heads), R in {1, 2, 4, 8}; D == 128;
+ *   K and V  each INT4 asymmetric with one group per (sequence, head, token)
+ *            row, the layout of wq_quantize_pack(WQ_FMT_INT4_ASYM, group = D)
+ *            applied to the [B * Hkv * L, D] rows: codes uint32
+ *            [B, Hkv, L, D/8] (element d in nibble d % 8 of word d / 8, low
+ *            nibble first), scales fp16 [B, Hkv, L], zeros fp16 [B, Hkv, L]
+ *            holding integers 0..15;
+ *   out      bf16 [B, Hq, D] = softmax(q . k^T / sqrt(D)) . v over the L
+ *            cached tokens, computed as follows (the page gives no formulas;
+ *            this is the library's reading):
+ *   - the query row is split into n_components int8 digit planes a_c with
+ *     scales sigma_c (the rules of wq_msd_decompose); the scores are
+ *     s[l] = sk[l] sum_c sigma_c (sum_d a_c[d] qk[l][d] - zk[l] sum_d a_c[d])
+ *     / sqrt(D), with exact integer inner sums;
+ *   - per chunk j of 256 tokens: m_j = max s, e = exp(s - m_j), E_j = sum e,
+ *     and w = e * sv (fp32) split into digit planes b_c with scales tau_c by
+ *     the same rules, the chunk's tokens taken as one row; then
+ *     O_j[d] = sum_c tau_c (sum_l b_c[l] qv[l][d] - sum_l b_c[l] zv[l]), exact
+ *     integer inner sums;
+ *   - out = sum_j e^(m_j - M) O_j / sum_j e^(m_j - M) E_j, M = max_j m_j.
+ * With n_components == 2 both products carry ~16-bit operands, so out agrees
+ * with fp32 attention over the dequantized cache to bf16 rounding plus the
+ * fp32 error of the softmax. B == 0 is a no-op; L == 0, Hq % Hkv != 0, or
+ * n_components outside 1..3 return WQ_ERR_INVALID_ARG; D != 128,
+ * n_components == 3, an R outside {1, 2, 4, 8}, B or Hkv > 65535, L >
+ * 2^31 - 257 or B * Hq > 2^31 - 1 return WQ_ERR_UNSUPPORTED. Workspace: at
+ * least wq_msd_decode_attention_workspace(...) bytes; contents on entry do
+ * not matter. Asynchronous on `stream`; every buffer is caller-owned.
+ */
+wq_status wq_msd_decode_attention(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64_t L,
+                                  int32_t D, int32_t n_components, const void* k_codes,
+                                  const void* k_scales, const void* k_zeros, const void* v_codes,
+                                  const void* v_scales, const void* v_zeros, void* out,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Workspace bytes of wq_msd_decode_attention (0 for B == 0); the same shape
+ * checks and status codes. Host only; `bytes` is a host pointer.
+ */
+wq_status wq_msd_decode_attention_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t L,
+                                            int32_t D, int32_t n_components, size_t* bytes);
+
+/*
  * Workspace bytes an entry point needs for the given problem (0 if none);
  * for WQ_OP_MX_GEMV, n_components is the number of passes (1 or 2).
  * Host only; `bytes` is a host pointer.

@@ -229,3 +229,35 @@ def test_pack_and_dequant_validation(wq):
     assert L.wq_nf4_dequant(A16, A16, 128, 64, A16, 2, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_nf4_dequant(A16, A16, 0, 64, A16, 0, None) == wq.WQ_OK
     assert L.wq_int4_dequant(A16, A16, A16, 16, 128, 12, A16, 0, None) == wq.WQ_ERR_INVALID_ARG
+
+
+def test_decode_attention_validation(wq):
+    g = wq.lib.wq_msd_decode_attention
+    ws = wq.lib.wq_msd_decode_attention_workspace
+    # (q, B, Hq, Hkv, L, D, C, kq, ks, kz, vq, vs, vz, out, ws, ws_bytes, stream)
+    def call(b=2, hq=16, hkv=4, length=300, d=128, c=2, ptr=A16, kq=A16, wsp=A16,
+             ws_bytes=1 << 24):
+        return g(ptr, b, hq, hkv, length, d, c, kq, A16, A16, A16, A16, A16, A16, wsp, ws_bytes,
+                 None)
+    assert call(hq=12, hkv=8) == wq.WQ_ERR_INVALID_ARG          # Hq % Hkv
+    assert call(hq=48, hkv=16) == wq.WQ_ERR_UNSUPPORTED         # R = 3
+    assert call(hq=64, hkv=4) == wq.WQ_ERR_UNSUPPORTED          # R = 16
+    assert call(d=64) == wq.WQ_ERR_UNSUPPORTED
+    assert call(d=100) == wq.WQ_ERR_INVALID_ARG
+    assert call(c=3) == wq.WQ_ERR_UNSUPPORTED
+    assert call(c=0) == wq.WQ_ERR_INVALID_ARG
+    assert call(length=0) == wq.WQ_ERR_INVALID_ARG
+    assert call(b=-1) == wq.WQ_ERR_INVALID_ARG
+    assert call(b=70000) == wq.WQ_ERR_UNSUPPORTED
+    assert call(kq=None) == wq.WQ_ERR_INVALID_ARG
+    assert call(kq=MIS) == wq.WQ_ERR_ALIGNMENT
+    assert call(wsp=None, ws_bytes=0) == wq.WQ_ERR_WORKSPACE
+    assert call(b=0, ptr=None, kq=None, wsp=None, ws_bytes=0) == wq.WQ_OK
+    size = ctypes.c_size_t(0)
+    assert ws(2, 16, 4, 300, 128, 2, ctypes.byref(size)) == wq.WQ_OK
+    # query digits (2 x 32 rows x 128 bytes), their scales (rounded up to 256
+    # bytes), then 2 chunks x (128 + 2) floats per query head
+    assert size.value == 2 * 32 * 128 + 256 + 32 * 2 * 130 * 4
+    assert call(ws_bytes=size.value - 1) == wq.WQ_ERR_WORKSPACE
+    assert ws(2, 16, 4, 300, 128, 3, ctypes.byref(size)) == wq.WQ_ERR_UNSUPPORTED
+    assert ws(0, 16, 4, 300, 128, 2, ctypes.byref(size)) == wq.WQ_OK and size.value == 0

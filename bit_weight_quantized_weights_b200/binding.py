@@ -42,6 +42,7 @@ EXPORTED = [
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
     "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv", "wq_msd_gemm_nf4",
     "wq_msd_decode_attention", "wq_msd_decode_attention_workspace",
+    "wq_test_set_attention_split",
 ]
 
 
@@ -86,6 +87,7 @@ def _load():
                                      P], ctypes.c_int),
         "wq_msd_decode_attention_workspace": ([I64, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
                                               ctypes.c_int),
+        "wq_test_set_attention_split": ([I32], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -480,3 +482,8 @@ def wq_msd_decode_attention(q, k_cache, v_cache, n_components=2, workspace=None,
                                        _ptr(workspace), workspace.numel(), _stream(stream)),
            "wq_msd_decode_attention")
     return out
+
+
+def wq_test_set_attention_split(chunks_per_cta=0):
+    """Fix the attention kernel's chunks per CTA (0: chosen per launch)."""
+    _check(lib.wq_test_set_attention_split(chunks_per_cta), "wq_test_set_attention_split")

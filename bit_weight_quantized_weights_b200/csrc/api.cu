@@ -37,6 +37,7 @@ size_t mx_workspace_bytes(int64_t M, int64_t K, int32_t P);
 wq_status launch_msd_nf4(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
                          const float*, void*, void*, cudaStream_t);
 size_t kv_msd_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int32_t C);
+extern std::atomic<int> g_kv_chunks_per_cta;
 wq_status launch_kv_msd(const void*, int64_t, int64_t, int64_t, int64_t, int32_t, const void*,
                         const void*, const void*, const void*, const void*, const void*, void*,
                         void*, cudaStream_t);
@@ -461,6 +462,12 @@ wq_status wq_test_set_wait(uint64_t limit_ns, int stall) {
   if (stall != 0 && stall != 1) return WQ_ERR_INVALID_ARG;
   g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
   g_wait_stall.store(stall, std::memory_order_relaxed);
+  return WQ_OK;
+}
+
+wq_status wq_test_set_attention_split(int32_t chunks_per_cta) {
+  if (chunks_per_cta < 0 || chunks_per_cta > 64) return WQ_ERR_INVALID_ARG;
+  g_kv_chunks_per_cta.store(chunks_per_cta, std::memory_order_relaxed);
   return WQ_OK;
 }
 

@@ -21,23 +21,29 @@
 // scales and integer zeros [B, Hkv, L].
 //
 // B200 design. Decode attention reads the cache once, so the kernel is bound
-// by HBM and the products only have to keep up: both are integer tensor-core
-// products (mma.m16n8k32, s8 digits x u8 codes). One CTA per (256-key chunk,
-// KV head, sequence) copies its K and V code rows into shared memory with
-// 16-byte cp.async, issued before it waits for the query decomposition (a
-// programmatic dependent launch). The R x C digit rows of the query are the
-// A operand (M = 16 rows, the unused ones zero):
+// by HBM when its per-key work keeps up. Both products are integer
+// tensor-core MMAs (mma.m16n8k32, s8 digits x u8 codes) with the R x C query
+// digit rows as the A operand (M = 16, unused rows zero):
 //   scores: N = keys, K = d. A K code word unpacks to two u8 words (even d,
-//           odd d); the query digits are stored in that order, so the
-//           contraction order matches without moving the codes;
+//           odd d); the query digits are stored in that order. Column n of
+//           n-tile t of warp w is key 32 w + (n >> 1) + 4 t + 16 (n & 1), so
+//           the accumulator fragment gives each lane 8 keys whose value digits
+//           pack into two 32-bit words per digit row;
 //   values: N = d, K = keys. The B fragment wants four keys of one d in a
 //           register: three byte permutes gather them from four code rows.
-//           The keys of a 32-key step are taken in the order that makes those
-//           row reads conflict-free, and the value digits are stored in the
-//           same order.
-// Each warp owns 16 output elements over all 256 keys, so no cross-warp
-// reduction is needed; the chunk's partial O_j and (m_j, E_j) go to the
-// workspace and a second kernel merges the chunks.
+//           The zero terms sum_l b_c[l] zv[l] are one more MMA per step, with
+//           the zero bytes as every column of B.
+// The chunk softmax runs on the score fragments: the lanes holding the two
+// components of a head swap halves (one shuffle), each lane takes one head
+// for its 8 keys, and the chunk statistics need one warp reduction and one
+// cross-warp step through shared memory. A CTA streams ns consecutive chunks
+// of one (sequence, KV head): the next chunk's K codes are copied (cp.async)
+// once the scores are done, its V codes once the values are done, and the
+// chunks merge in registers (flash-decoding rescaling); a second kernel
+// merges the CTAs' partials.
+#include <algorithm>
+#include <atomic>
+
 #include "splitk_common.cuh"
 
 namespace wq {
@@ -52,25 +58,29 @@ constexpr int kQwStride = kD / 4 + 4;    // words per query digit row (padded)
 constexpr int kBdStride = kT + 16;       // bytes per value digit row (padded)
 
 // shared memory carve-up (bytes)
-constexpr int kOffK = 0;                                  // K codes, later P
+constexpr int kOffK = 0;                                  // K codes of one chunk
 constexpr int kOffV = kOffK + kT * kRowBytes;             // V codes
 constexpr int kOffBd = kOffV + kT * kRowBytes;            // value digits [16][kBdStride]
-constexpr int kOffSc = kOffBd + 16 * kBdStride;           // sk, sv (fp32), zk, zv (int)
-constexpr int kOffQw = kOffSc + 4 * kT * 4;               // query digits [16][kQwStride]
-constexpr int kOffQm = kOffQw + 16 * kQwStride * 4;       // qsig, qsum, tau, zt: [16] each
-constexpr int kOffRed = kOffQm + 4 * 16 * 4;              // [8 warps][16]
-constexpr int kSmemBytes = kOffRed + 8 * 16 * 4;
+constexpr int kOffKi = kOffBd + 16 * kBdStride;           // per key: sk, zk, sv (float4)
+constexpr int kOffZv = kOffKi + kT * 16;                  // zv bytes in digit-slot order
+constexpr int kOffQw = kOffZv + kT;                       // query digits [16][kQwStride]
+constexpr int kOffQm = kOffQw + 16 * kQwStride * 4;       // qsig[16], qsum[16]
+constexpr int kOffCo = kOffQm + 2 * 16 * 4;               // coefA[16], coefB[16] per digit row
+constexpr int kOffRun = kOffCo + 2 * 16 * 4;              // running M[8], E[8] per head
+constexpr int kOffRed = kOffRun + 2 * 8 * 4;              // [3][8 warps][8 heads]
+constexpr int kSmemBytes = kOffRed + 3 * 8 * 8 * 4;
 static_assert(kSmemBytes <= 48 * 1024, "static shared memory");
-static_assert(16 * kT * 4 <= kT * kRowBytes, "P fits the K buffer");
 
-// 16-byte chunk c (0..3) of key row l is stored at chunk c ^ ((l >> 1) & 3).
+// 16-byte chunk c (0..3) of key row l is stored at chunk c ^ sw(l), with
+// sw(l) = bit 1 of l in bit 0 and bit 4 of l in bit 1: the score B loads
+// (rows a + 16 b + 4 t, a in 0..3, b in 0..1) and the value B loads (rows
+// t + 4 i, t in 0..3) then hit distinct banks.
 __device__ __forceinline__ int kv_off(int l, int c) {
-  return l * kRowBytes + ((c ^ ((l >> 1) & 3)) << 4);
+  const int sw = ((l >> 1) & 1) | ((l >> 3) & 2);
+  return l * kRowBytes + ((c ^ sw) << 4);
 }
-// P[hc][l] (int) at word hc * kT + (l ^ ((hc & 3) << 3)).
-__device__ __forceinline__ int p_idx(int hc, int l) { return hc * kT + (l ^ ((hc & 3) << 3)); }
-// Column of key kk (0..255) in the value digit rows: within each 16-key half
-// of a 32-key step, key t + 4 i sits at slot 4 t + i (t, i in 0..3).
+// Slot of key kk (0..255) in the value digit rows: within each 16-key half of
+// a 32-key step, key t + 4 i sits at slot 4 t + i (t, i in 0..3).
 __device__ __forceinline__ int bd_col(int kk) {
   return (kk & ~15) + 4 * (kk & 3) + ((kk >> 2) & 3);
 }
@@ -84,6 +94,16 @@ __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// a / b rounded to nearest from y = RN(1 / b): one correction step on the
+// product a y (Markstein's theorem: with y the correctly rounded reciprocal
+// and the residual a - b q formed exactly by a fused multiply-add, the
+// corrected quotient is the correctly rounded a / b, barring overflow and
+// underflow).
+__device__ __forceinline__ float div_by(float a, float b, float y) {
+  const float q = a * y;
+  return __fmaf_rn(__fmaf_rn(-q, b, a), y, q);
+}
+
 struct KvArgs {
   const int8_t* qd;       // [C][B*Hq][D] query digits
   const float* qs;        // [C][B*Hq] their scales
@@ -93,117 +113,145 @@ struct KvArgs {
   const uint8_t* vq;      // V codes
   const __half* vs;
   const __half* vz;
-  float* part;            // [B, Hkv, nch, R, D] chunk outputs O_j
-  float* stat;            // [B, Hkv, nch, R, 2] (m_j, E_j)
-  int B, Hq, Hkv, L, nch;
+  float* part;            // [B, Hkv, nsplit, R, D] partial outputs
+  float* stat;            // [B, Hkv, nsplit, R, 2] (M, E) of each partial
+  int B, Hq, Hkv, L, nch, ns, nsplit;
   float inv_sqrt_d;
 };
 
-// v[i] combined over the CTA (256 threads); red holds [8][N] values; every
-// thread receives the result.
-template <int N, typename T, typename Op>
-__device__ __forceinline__ void block_all(T (&v)[N], T* red, Op op) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int i = 0; i < N; ++i)
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v[i] = op(v[i], __shfl_xor_sync(0xffffffffu, v[i], o));
-  __syncthreads();
-  if (lane == 0)
-#pragma unroll
-    for (int i = 0; i < N; ++i) red[warp * N + i] = v[i];
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < N; ++i) {
-    T a = red[i];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) a = op(a, red[w * N + i]);
-    v[i] = a;
-  }
-}
-
 template <int R, int C>
-__global__ void __launch_bounds__(256, 3) kv_msd_chunk_kernel(KvArgs p) {
+__global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
   constexpr int RC = R * C;
-  static_assert(RC <= 16, "at most 16 digit rows");
+  static_assert(RC <= 16 && (C == 1 || C == 2), "digit rows");
   __shared__ __align__(16) uint8_t sm[kSmemBytes];
   uint8_t* kc = sm + kOffK;
   uint8_t* vc = sm + kOffV;
-  int* P = reinterpret_cast<int*>(sm + kOffK);
   int8_t* bd = reinterpret_cast<int8_t*>(sm + kOffBd);
-  float* skf = reinterpret_cast<float*>(sm + kOffSc);
-  float* svf = skf + kT;
-  int* zki = reinterpret_cast<int*>(svf + kT);
-  int* zvi = zki + kT;
+  float4* ki = reinterpret_cast<float4*>(sm + kOffKi);
+  uint8_t* zvb = sm + kOffZv;
   uint32_t* qw = reinterpret_cast<uint32_t*>(sm + kOffQw);
   float* qsig = reinterpret_cast<float*>(sm + kOffQm);
   int* qsum = reinterpret_cast<int*>(qsig + 16);
-  float* tau = reinterpret_cast<float*>(qsum + 16);
-  int* zt = reinterpret_cast<int*>(tau + 16);
-  float* redf = reinterpret_cast<float*>(sm + kOffRed);
+  float* coefA = reinterpret_cast<float*>(sm + kOffCo);
+  float* coefB = coefA + 16;
+  float* Mrun = reinterpret_cast<float*>(sm + kOffRun);
+  float* Erun = Mrun + 8;
+  float* redm = reinterpret_cast<float*>(sm + kOffRed);
+  float* rede = redm + 64;
+  float* reda = rede + 64;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
-  const int j = blockIdx.x, kh = blockIdx.y, b = blockIdx.z;
-  const int l0 = j * kT;
-  const int nk = min(kT, p.L - l0);
-  const int64_t row0 = ((int64_t)b * p.Hkv + kh) * p.L + l0;  // first cache row of the chunk
+  const int split = blockIdx.x, kh = blockIdx.y, b = blockIdx.z;
+  const int j0 = split * p.ns;
+  const int nsub = min(p.ns, p.nch - j0);
+  const int64_t seq0 = ((int64_t)b * p.Hkv + kh) * p.L;  // cache row of token 0
+  // the head this lane takes in the softmax: rows (2h, 2h + 1) are held by
+  // lanes g = 2h (h < 4, as row g and, after the swap, g + 1) and g = 2h - 7
+  // (h >= 4, as rows g + 7 and g + 8)
+  const int hl = C == 2 ? ((g & 1) ? (g + 7) >> 1 : g >> 1) : g;
+  const bool hv = hl < R;
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // ---- the chunk's K and V code rows; the cache is not written by the grid
-  // this one may overlap, so the copies go before the wait
-  for (int i = tid; i < nk * 4; i += 256) {
-    const int l = i >> 2, c = i & 3;
-    cp_async16(kc + kv_off(l, c), p.kq + (row0 + l) * kRowBytes + 16 * c);
-    cp_async16(vc + kv_off(l, c), p.vq + (row0 + l) * kRowBytes + 16 * c);
-  }
+
+  auto issue_codes = [&](const uint8_t* src, uint8_t* dst, int jc) {
+    const int l0 = jc * kT, nk = min(kT, p.L - l0);
+    const uint8_t* s = src + (seq0 + l0) * kRowBytes;
+    for (int i = tid; i < nk * 4; i += 256)
+      cp_async16(dst + kv_off(i >> 2, i & 3), s + (i >> 2) * kRowBytes + 16 * (i & 3));
+  };
+  // key tid's (sk, zk, sv, zv) of chunk jc, zeros past the end of the cache
+  auto load_info = [&](int jc, __half (&h)[4]) {
+    const int l = jc * kT + tid;
+    const __half z = __float2half(0.0f);
+    h[0] = h[1] = h[2] = h[3] = z;
+    if (l < p.L) {
+      h[0] = p.ks[seq0 + l];
+      h[1] = p.kz[seq0 + l];
+      h[2] = p.vs[seq0 + l];
+      h[3] = p.vz[seq0 + l];
+    }
+  };
+  auto store_info = [&](const __half (&h)[4]) {
+    ki[tid] = make_float4(__half2float(h[0]), __half2float(h[1]), __half2float(h[2]), 0.0f);
+    zvb[bd_col(tid)] = (uint8_t)__half2float(h[3]);
+  };
+
+  // ---- prologue: the first chunk's codes and key data; the cache is not
+  // written by the grid this one may overlap, so they go before the wait
+  issue_codes(p.kq, kc, j0);
   asm volatile("cp.async.commit_group;" ::: "memory");
-  if (tid < nk) {
-    skf[tid] = __half2float(p.ks[row0 + tid]);
-    svf[tid] = __half2float(p.vs[row0 + tid]);
-    zki[tid] = (int)__half2float(p.kz[row0 + tid]);
-    zvi[tid] = (int)__half2float(p.vz[row0 + tid]);
+  issue_codes(p.vq, vc, j0);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  {
+    __half h[4];
+    load_info(j0, h);
+    store_info(h);
   }
-  // ---- the query digits of this KV head's R query heads (rows hc = h C + c)
+  if (tid < R) {
+    Mrun[tid] = -INFINITY;
+    Erun[tid] = 0.0f;
+  }
+  // the query digits of this KV head's R query heads (rows hc = h C + c), in
+  // the even-d / odd-d order of the unpacked K code words, and their sums
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int qrow0 = b * p.Hq + kh * R;
   const int64_t plane = (int64_t)p.B * p.Hq;
-  if (tid < RC * (kD / 8)) {
-    const int hc = tid >> 4, g8 = tid & 15;
-    const int h = hc / C, c = hc - h * C;
-    const uint2 v =
-        *reinterpret_cast<const uint2*>(p.qd + ((int64_t)c * plane + qrow0 + h) * kD + 8 * g8);
-    qw[hc * kQwStride + 2 * g8] = prmt(v.x, v.y, 0x6420u);      // d = 8 g8 + 0, 2, 4, 6
-    qw[hc * kQwStride + 2 * g8 + 1] = prmt(v.x, v.y, 0x7531u);  // d = 8 g8 + 1, 3, 5, 7
-  }
-  if (tid < RC) {
-    const int h = tid / C, c = tid - h * C;
-    qsig[tid] = p.qs[(int64_t)c * plane + qrow0 + h];
-  }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-  if (tid < RC) {
-    int s = 0;
-    for (int i = 0; i < kD / 4; ++i) s = __dp4a((int)qw[tid * kQwStride + i], 0x01010101, s);
-    qsum[tid] = s;
-  }
-
-  // ---- scores: warp w takes keys 32 w .. 32 w + 31 (four n-tiles of 8 keys)
-  int sacc[4][4];
   {
-    uint32_t a[4][4];  // [k-step][fragment register]
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      a[s][0] = g < RC ? qw[g * kQwStride + 8 * s + t4] : 0u;
-      a[s][1] = g + 8 < RC ? qw[(g + 8) * kQwStride + 8 * s + t4] : 0u;
-      a[s][2] = g < RC ? qw[g * kQwStride + 8 * s + 4 + t4] : 0u;
-      a[s][3] = g + 8 < RC ? qw[(g + 8) * kQwStride + 8 * s + 4 + t4] : 0u;
+    int part = 0;
+    if (tid < RC * (kD / 8)) {
+      const int hc = tid >> 4, g8 = tid & 15;
+      const int h = hc / C, c = hc - h * C;
+      const uint2 v = *reinterpret_cast<const uint2*>(
+          p.qd + ((int64_t)c * plane + qrow0 + h) * kD + 8 * g8);
+      const uint32_t ev = prmt(v.x, v.y, 0x6420u), od = prmt(v.x, v.y, 0x7531u);
+      qw[hc * kQwStride + 2 * g8] = ev;       // d = 8 g8 + 0, 2, 4, 6
+      qw[hc * kQwStride + 2 * g8 + 1] = od;   // d = 8 g8 + 1, 3, 5, 7
+      part = __dp4a((int)ev, 0x01010101, __dp4a((int)od, 0x01010101, 0));
     }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (tid < RC * (kD / 8) && (tid & 15) == 0) qsum[tid >> 4] = part;
+    if (tid < RC) {
+      const int h = tid / C, c = tid - h * C;
+      qsig[tid] = p.qs[(int64_t)c * plane + qrow0 + h];
+    }
+  }
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+  __syncthreads();
+  uint32_t a[4][4];  // score A fragments, [k-step][register]
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    a[s][0] = g < RC ? qw[g * kQwStride + 8 * s + t4] : 0u;
+    a[s][1] = g + 8 < RC ? qw[(g + 8) * kQwStride + 8 * s + t4] : 0u;
+    a[s][2] = g < RC ? qw[g * kQwStride + 8 * s + 4 + t4] : 0u;
+    a[s][3] = g + 8 < RC ? qw[(g + 8) * kQwStride + 8 * s + 4 + t4] : 0u;
+  }
+  const int r0 = hv ? hl * C : 0;
+  const float sig0 = qsig[r0], sig1 = C == 2 ? qsig[r0 + 1] : 0.0f;
+  const int qs0 = qsum[r0], qs1 = C == 2 ? qsum[r0 + 1] : 0;
+
+  float O[2][4];
+#pragma unroll
+  for (int jm = 0; jm < 2; ++jm)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) O[jm][i] = 0.0f;
+
+  for (int i = 0; i < nsub; ++i) {
+    const int jc = j0 + i;
+    const int nk = min(kT, p.L - jc * kT);
+    const bool more = i + 1 < nsub;
+    if (i > 0) {
+      asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's K codes
+      __syncthreads();
+    }
+    // ---- scores: warp w takes keys 32 w .. 32 w + 31
+    int sacc[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) sacc[nt][i] = 0;
-      const int l = 32 * warp + 8 * nt + g;
+      for (int r = 0; r < 4; ++r) sacc[nt][r] = 0;
+      const int l = 32 * warp + (g >> 1) + 4 * nt + 16 * (g & 1);
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
         const uint32_t* ch = reinterpret_cast<const uint32_t*>(kc + kv_off(l, s));
@@ -213,165 +261,204 @@ __global__ void __launch_bounds__(256, 3) kv_msd_chunk_kernel(KvArgs p) {
                  (w1 >> sh) & 0x0F0F0F0Fu);
       }
     }
-  }
-  __syncthreads();  // every warp is done with the K codes: P takes their place
+    // the lane's head for its keys 32 w + t4 + 4 nt + 16 e
+    float sc[4][2];
+    float mx = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    const int l = 32 * warp + 8 * nt + 2 * t4;
-    *reinterpret_cast<int2*>(P + p_idx(g, l)) = make_int2(sacc[nt][0], sacc[nt][1]);
-    *reinterpret_cast<int2*>(P + p_idx(g + 8, l)) = make_int2(sacc[nt][2], sacc[nt][3]);
-  }
-  __syncthreads();
-
-  // ---- softmax statistics of the chunk; thread tid takes key tid
-  const bool valid = tid < nk;
-  float m[R], es[R], am[R], w[R];
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-  for (int h = 0; h < R; ++h) {
-    float s = 0.0f;
+      for (int e = 0; e < 2; ++e) {
+        int p0 = sacc[nt][e], p1 = 0;
+        if (C == 2) {
+          const int send = (g & 1) ? sacc[nt][e] : sacc[nt][2 + e];
+          const int recv = __shfl_xor_sync(0xffffffffu, send, 4);
+          p0 = (g & 1) ? recv : sacc[nt][e];
+          p1 = (g & 1) ? sacc[nt][2 + e] : recv;
+        }
+        const int kk = 32 * warp + t4 + 4 * nt + 16 * e;
+        const float4 inf = ki[kk];
+        const int zk = (int)inf.y;
+        float s = sig0 * (float)(p0 - zk * qs0);  // |.| < 2^24: exact
+        if (C == 2) s = fmaf(sig1, (float)(p1 - zk * qs1), s);
+        s = (hv && kk < nk) ? s * inf.x * p.inv_sqrt_d : -INFINITY;
+        sc[nt][e] = s;
+        mx = fmaxf(mx, s);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    if (t4 == 0 && hv) redm[warp * 8 + hl] = mx;
+    __syncthreads();  // every warp is done with the K codes
+    // the next chunk's K codes and key data
+    if (more) issue_codes(p.kq, kc, jc + 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    __half nxt[4];
+    if (more) load_info(jc + 1, nxt);
+    float m = -INFINITY;
+    if (hv)
 #pragma unroll
-    for (int c = 0; c < C; ++c) {
-      const int hc = h * C + c;
-      const int dint = P[p_idx(hc, tid)] - (valid ? zki[tid] : 0) * qsum[hc];  // |.| < 2^24
-      s = fmaf(qsig[hc], (float)dint, s);
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, redm[w * 8 + hl]);
+    float wv[4][2], es = 0.0f, am = 0.0f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int kk = 32 * warp + t4 + 4 * nt + 16 * e;
+        const float ex = sc[nt][e] == -INFINITY ? 0.0f : expf(sc[nt][e] - m);
+        es += ex;
+        wv[nt][e] = ex * ki[kk].z;
+        am = fmaxf(am, fabsf(wv[nt][e]));
+      }
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      es += __shfl_xor_sync(0xffffffffu, es, o);
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     }
-    m[h] = valid ? s * skf[tid] * p.inv_sqrt_d : -INFINITY;
-    w[h] = m[h];
-  }
-  block_all<R>(m, redf, [](float x, float y) { return fmaxf(x, y); });
-#pragma unroll
-  for (int h = 0; h < R; ++h) {
-    const float e = valid ? expf(w[h] - m[h]) : 0.0f;
-    es[h] = e;
-    w[h] = e * (valid ? svf[tid] : 0.0f);
-    am[h] = fabsf(w[h]);
-  }
-  block_all<R>(es, redf, [](float x, float y) { return x + y; });
-  const int64_t base = (((int64_t)b * p.Hkv + kh) * p.nch + j) * R;
-#pragma unroll
-  for (int h = 0; h < R; ++h)
-    if (tid == h) *reinterpret_cast<float2*>(p.stat + (base + h) * 2) = make_float2(m[h], es[h]);
-  block_all<R>(am, redf, [](float x, float y) { return fmaxf(x, y); });
-  // the decomposition of w over the chunk's keys, as for an activation row:
-  // s_1 = amax / 127, s_{c+1} = s_c / 256, digit rint(r / s_c) (the first
-  // clamped to +-127), residual r - s_c a_c rounded once, and a digit of +128
-  // becomes -128 with a carry into the digit before it. Thread h computes
-  // head h's scales once.
-#pragma unroll
-  for (int h = 0; h < R; ++h)
-    if (tid == h) {
-      float sc = am[h] > 0.0f ? __fdiv_rn(am[h], 127.0f) : 1.0f;
-#pragma unroll
-      for (int c = 0; c < C; ++c, sc *= (1.0f / 256.0f)) tau[h * C + c] = sc;
+    if (t4 == 0 && hv) {
+      rede[warp * 8 + hl] = es;
+      reda[warp * 8 + hl] = am;
     }
-  __syncthreads();
-  {
-    const int col = bd_col(tid);
+    __syncthreads();
+    float E = 0.0f, A = 0.0f;
+    if (hv)
 #pragma unroll
-    for (int h = 0; h < R; ++h) {
-      int dg[C];
-      float r = w[h];
+      for (int w = 0; w < 8; ++w) {
+        E += rede[w * 8 + hl];
+        A = fmaxf(A, reda[w * 8 + hl]);
+      }
+    // the decomposition of w over the chunk's keys, as for an activation row:
+    // s_1 = amax / 127, s_{c+1} = s_c / 256, digit rint(r / s_c) (the first
+    // clamped to +-127), residual r - s_c a_c rounded once, and a digit of
+    // +128 becomes -128 with a carry into the digit before it
+    const float tau0 = A > 0.0f ? __fdiv_rn(A, 127.0f) : 1.0f;
+    const float y0 = __frcp_rn(tau0);
+    const float tau1 = tau0 * (1.0f / 256.0f), y1 = y0 * 256.0f;
+    uint32_t word[C][2];
+#pragma unroll
+    for (int c = 0; c < C; ++c) word[c][0] = word[c][1] = 0u;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float r = wv[nt][e];
+        const float q0 = fminf(fmaxf(rintf(div_by(r, tau0, y0)), -127.0f), 127.0f);
+        int d0 = (int)q0;
+        if (C == 2) {
+          r = __fmaf_rn(-tau0, q0, r);
+          int d1 = (int)rintf(div_by(r, tau1, y1));
+          if (d1 == 128) {
+            d1 = -128;
+            d0 += 1;
+          }
+          word[C - 1][e] |= (uint32_t)(d1 & 0xFF) << (8 * nt);
+        }
+        word[0][e] |= (uint32_t)(d0 & 0xFF) << (8 * nt);
+      }
+    if (hv)
+#pragma unroll
+      for (int c = 0; c < C; ++c)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          *reinterpret_cast<uint32_t*>(bd + (hl * C + c) * kBdStride + 32 * warp + 16 * e +
+                                       4 * t4) = word[c][e];
+    // merge weights of this chunk into the CTA's running sums
+    if (warp == 0 && t4 == 0 && hv) {
+      const float M0 = Mrun[hl], Mn = fmaxf(M0, m);
+      const float al = expf(M0 - Mn), be = expf(m - Mn);  // M0 = -inf: al = 0
+      Erun[hl] = fmaf(Erun[hl], al, E * be);
+      Mrun[hl] = Mn;
 #pragma unroll
       for (int c = 0; c < C; ++c) {
-        const float sc = tau[h * C + c];
-        float q = rintf(__fdiv_rn(r, sc));
-        if (c == 0) q = fminf(fmaxf(q, -127.0f), 127.0f);
-        dg[c] = (int)q;
-        r = __fmaf_rn(-sc, q, r);
+        coefA[hl * C + c] = al;
+        coefB[hl * C + c] = be * (c == 0 ? tau0 : tau1);
       }
-#pragma unroll
-      for (int c = C - 1; c > 0; --c)
-        if (dg[c] == 128) {
-          dg[c] = -128;
-          dg[c - 1] += 1;
-        }
-#pragma unroll
-      for (int c = 0; c < C; ++c) bd[(h * C + c) * kBdStride + col] = (int8_t)dg[c];
     }
-  }
-  __syncthreads();
-  // the zero terms zt[hc] = sum_l b_c[l] zv[l]: warp w takes digit rows 2 w, 2 w + 1
-#pragma unroll
-  for (int r2 = 0; r2 < 2; ++r2) {
-    const int hc = 2 * warp + r2;
-    if (hc < RC) {
-      int acc = 0;
-#pragma unroll
-      for (int i = 0; i < kT / 32; ++i) {
-        const int l = lane + 32 * i;
-        acc += (int)bd[hc * kBdStride + bd_col(l)] * (l < nk ? zvi[l] : 0);
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (lane == 0) zt[hc] = acc;
-    }
-  }
-  __syncthreads();
+    asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's V codes
+    __syncthreads();
 
-  // ---- values: warp w owns d in [16 w, 16 w + 16), words wi = 2 w, 2 w + 1
-  // of each code row. MMA jm, column n: d = 8 (2 w + (n >> 2)) + (n & 3) + 4 jm.
-  int vacc[2][4];
+    // ---- values: warp w owns d in [16 w, 16 w + 16), words wi = 2 w, 2 w + 1
+    // of each code row. MMA jm, column n: d = 8 (2 w + (n >> 2)) + (n & 3) + 4 jm.
+    int vacc[2][4], zacc[4];
 #pragma unroll
-  for (int jm = 0; jm < 2; ++jm)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) vacc[jm][i] = 0;
-  {
-    const int wi = 2 * warp + (g >> 2);
-    const int q = g & 3;
-    const int sh = 4 * (q & 1);
-    // byte (q >> 1) of two rows into bytes 0, 1 (jm = 0); byte 2 + (q >> 1) (jm = 1)
-    const uint32_t sel0 = (uint32_t)((q >> 1) | ((4 + (q >> 1)) << 4));
-    const uint32_t sel1 = sel0 + 0x22u;
-    const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride);
-    const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride);
+    for (int r = 0; r < 4; ++r) vacc[0][r] = vacc[1][r] = zacc[r] = 0;
+    {
+      const int wi = 2 * warp + (g >> 2);
+      const int q = g & 3;
+      const int sh = 4 * (q & 1);
+      // byte (q >> 1) of two rows into bytes 0, 1 (jm = 0); byte 2 + (q >> 1) (jm = 1)
+      const uint32_t sel0 = (uint32_t)((q >> 1) | ((4 + (q >> 1)) << 4));
+      const uint32_t sel1 = sel0 + 0x22u;
+      const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride);
+      const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride);
+      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb);
 #pragma unroll 2
-    for (int ks = 0; ks < kT / 32; ++ks) {
-      const int k0 = 32 * ks;
-      const uint32_t a0 = g < RC ? arow0[(k0 >> 2) + t4] : 0u;
-      const uint32_t a1 = g + 8 < RC ? arow1[(k0 >> 2) + t4] : 0u;
-      const uint32_t a2 = g < RC ? arow0[(k0 >> 2) + 4 + t4] : 0u;
-      const uint32_t a3 = g + 8 < RC ? arow1[(k0 >> 2) + 4 + t4] : 0u;
-      uint32_t bb[2][2];  // [jm][key half]
+      for (int ks = 0; ks < kT / 32; ++ks) {
+        const int k0 = 32 * ks;
+        const uint32_t a0 = g < RC ? arow0[(k0 >> 2) + t4] : 0u;
+        const uint32_t a1 = g + 8 < RC ? arow1[(k0 >> 2) + t4] : 0u;
+        const uint32_t a2 = g < RC ? arow0[(k0 >> 2) + 4 + t4] : 0u;
+        const uint32_t a3 = g + 8 < RC ? arow1[(k0 >> 2) + 4 + t4] : 0u;
+        uint32_t bb[2][2];  // [jm][key half]
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        uint32_t rw[4];
+        for (int hb = 0; hb < 2; ++hb) {
+          uint32_t rw[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int l = k0 + 16 * hb + t4 + 4 * i;
-          rw[i] = *reinterpret_cast<const uint32_t*>(vc + kv_off(l, wi >> 2) + 4 * (wi & 3));
+          for (int ii = 0; ii < 4; ++ii) {
+            const int l = k0 + 16 * hb + t4 + 4 * ii;
+            rw[ii] = *reinterpret_cast<const uint32_t*>(vc + kv_off(l, wi >> 2) + 4 * (wi & 3));
+          }
+          const uint32_t x0 = prmt(rw[0], rw[1], sel0), y0v = prmt(rw[2], rw[3], sel0);
+          const uint32_t x1 = prmt(rw[0], rw[1], sel1), y1v = prmt(rw[2], rw[3], sel1);
+          bb[0][hb] = (prmt(x0, y0v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
+          bb[1][hb] = (prmt(x1, y1v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
         }
-        const uint32_t x0 = prmt(rw[0], rw[1], sel0), y0 = prmt(rw[2], rw[3], sel0);
-        const uint32_t x1 = prmt(rw[0], rw[1], sel1), y1 = prmt(rw[2], rw[3], sel1);
-        bb[0][hb] = (prmt(x0, y0, 0x5410u) >> sh) & 0x0F0F0F0Fu;
-        bb[1][hb] = (prmt(x1, y1, 0x5410u) >> sh) & 0x0F0F0F0Fu;
+        mma_s8u8(vacc[0], a0, a1, a2, a3, bb[0][0], bb[0][1]);
+        mma_s8u8(vacc[1], a0, a1, a2, a3, bb[1][0], bb[1][1]);
+        mma_s8u8(zacc, a0, a1, a2, a3, zw[(k0 >> 2) + t4], zw[(k0 >> 2) + 4 + t4]);
       }
-      mma_s8u8(vacc[0], a0, a1, a2, a3, bb[0][0], bb[0][1]);
-      mma_s8u8(vacc[1], a0, a1, a2, a3, bb[1][0], bb[1][1]);
     }
+    // O = O alpha + beta tau_c (acc - zt) for the lane's rows g and g + 8
+#pragma unroll
+    for (int rh = 0; rh < 2; ++rh) {
+      const int row = g + 8 * rh;
+      const float cA = row < RC ? coefA[row] : 0.0f, cB = row < RC ? coefB[row] : 0.0f;
+#pragma unroll
+      for (int jm = 0; jm < 2; ++jm)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          O[jm][2 * rh + e] =
+              fmaf(O[jm][2 * rh + e], cA, cB * (float)(vacc[jm][2 * rh + e] - zacc[2 * rh]));
+    }
+    __syncthreads();  // the V codes, digits, key data and weights of this chunk are consumed
+    if (more) issue_codes(p.vq, vc, jc + 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (more) store_info(nxt);
   }
-  // ---- epilogue: O_j[h][d] = sum_c tau_c (acc - zt); the components of a
-  // head sit in C consecutive rows, held by lanes 4 apart
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+
+  // ---- the CTA's partial: the components of a head sit in C consecutive
+  // rows, held by lanes 4 apart
+  const int64_t base = (((int64_t)b * p.Hkv + kh) * p.nsplit + split) * R;
 #pragma unroll
   for (int jm = 0; jm < 2; ++jm) {
     const int d = 8 * (2 * warp + (t4 >> 1)) + 2 * (t4 & 1) + 4 * jm;  // columns 2 t4, 2 t4 + 1
 #pragma unroll
     for (int rh = 0; rh < 2; ++rh) {
-      const int hc = g + 8 * rh;
-      const int hcs = hc < RC ? hc : 0;
-      float o0 = tau[hcs] * (float)(vacc[jm][2 * rh] - zt[hcs]);
-      float o1 = tau[hcs] * (float)(vacc[jm][2 * rh + 1] - zt[hcs]);
+      const int row = g + 8 * rh;
+      float o0 = O[jm][2 * rh], o1 = O[jm][2 * rh + 1];
       if (C == 2) {
         o0 += __shfl_xor_sync(0xffffffffu, o0, 4);
         o1 += __shfl_xor_sync(0xffffffffu, o1, 4);
       }
-      if (hc < RC && hc % C == 0)
-        *reinterpret_cast<float2*>(p.part + (base + hc / C) * kD + d) = make_float2(o0, o1);
+      if (row < RC && row % C == 0)
+        *reinterpret_cast<float2*>(p.part + (base + row / C) * kD + d) = make_float2(o0, o1);
     }
   }
+  if (tid < R)
+    *reinterpret_cast<float2*>(p.stat + (base + tid) * 2) = make_float2(Mrun[tid], Erun[tid]);
 }
 
-// Merge the chunks of each (sequence, query head): out = sum_j e^(m_j - M)
-// O_j / sum_j e^(m_j - M) E_j, one CTA of 128 threads (one per element).
+// Merge the CTAs' partials of each (sequence, query head): out = sum_j
+// e^(M_j - M) O_j / sum_j e^(M_j - M) E_j, one CTA of 128 threads (one per element).
 template <int R>
 __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __restrict__ out) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -379,11 +466,11 @@ __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __
   const int b = bh / p.Hq, hq = bh - b * p.Hq;
   const int kh = hq / R, h = hq - kh * R;
   const int d = threadIdx.x;
-  const int64_t base = ((int64_t)b * p.Hkv + kh) * p.nch;
+  const int64_t base = ((int64_t)b * p.Hkv + kh) * p.nsplit;
   float big = -INFINITY;
-  for (int j = 0; j < p.nch; ++j) big = fmaxf(big, p.stat[((base + j) * R + h) * 2]);
+  for (int j = 0; j < p.nsplit; ++j) big = fmaxf(big, p.stat[((base + j) * R + h) * 2]);
   float num = 0.0f, den = 0.0f;
-  for (int j = 0; j < p.nch; ++j) {
+  for (int j = 0; j < p.nsplit; ++j) {
     const int64_t ri = (base + j) * R + h;
     const float f = expf(p.stat[ri * 2] - big);
     num = fmaf(f, p.part[ri * kD + d], num);
@@ -401,9 +488,9 @@ wq_status launch_kv_rc(const KvArgs& a, void* out, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cfg.stream = st;
-  cfg.gridDim = dim3((unsigned)a.nch, (unsigned)a.Hkv, (unsigned)a.B);
+  cfg.gridDim = dim3((unsigned)a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
   cfg.blockDim = dim3(256, 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kv_msd_chunk_kernel<R, C>, a) != cudaSuccess) return WQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kv_msd_split_kernel<R, C>, a) != cudaSuccess) return WQ_ERR_CUDA;
   cfg.gridDim = dim3((unsigned)(a.B * a.Hq), 1, 1);
   cfg.blockDim = dim3(kD, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kv_msd_merge_kernel<R>, a, static_cast<uint16_t*>(out)) !=
@@ -427,9 +514,12 @@ wq_status launch_kv_c(const KvArgs& a, int R, void* out, cudaStream_t st) {
 wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, int8_t*, float*,
                                cudaStream_t);
 
+std::atomic<int> g_kv_chunks_per_cta{0};  // 0: chosen per launch
+
 // Workspace: query digits [C][B*Hq][D] and their scales [C][B*Hq] fp32 (each
-// rounded up to 256 bytes), then the chunk outputs [B, Hkv, nch, R, D] and
-// statistics [B, Hkv, nch, R, 2] fp32.
+// rounded up to 256 bytes), then the partial outputs [B, Hkv, nsplit, R, D]
+// and statistics [B, Hkv, nsplit, R, 2] fp32, sized for nsplit = nch (one
+// chunk per CTA, the most partials any launch writes).
 size_t kv_msd_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int32_t C) {
   const int64_t nch = (L + kT - 1) / kT;
   const size_t dig = ((size_t)C * B * Hq * kD + 255) / 256 * 256;
@@ -467,6 +557,14 @@ wq_status launch_kv_msd(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64
   a.Hkv = (int)Hkv;
   a.L = (int)L;
   a.nch = (int)nch;
+  // chunks per CTA: enough CTAs for about four waves of three per SM, at most
+  // 8 (or the count the test hook fixed)
+  const int64_t total = B * Hkv * nch;
+  const int forced = g_kv_chunks_per_cta.load(std::memory_order_relaxed);
+  a.ns = forced > 0 ? forced
+                    : (int)std::max<int64_t>(
+                          1, std::min<int64_t>(8, total / ((int64_t)num_sms() * 12)));
+  a.nsplit = (int)((nch + a.ns - 1) / a.ns);
   a.inv_sqrt_d = 1.0f / sqrtf((float)kD);
   const int R = (int)(Hq / Hkv);
   return C == 1 ? launch_kv_c<1>(a, R, out, st) : launch_kv_c<2>(a, R, out, st);

@@ -445,6 +445,19 @@ wq_status wq_workspace_bytes(wq_op op, int64_t M, int64_t N, int64_t K,
 wq_status wq_test_set_wait(uint64_t limit_ns, int stall);
 
 /*
+ * Test hook for wq_msd_decode_attention. The pages have no counterpart: it
+ * exists so that tests can reach, at small sizes, the chunk-streaming path
+ * that large problems take. Each CTA of the attention kernel streams
+ * chunks_per_cta consecutive 256-token chunks of one (sequence, KV head) and
+ * merges them in registers; by default (0) the count is chosen per launch
+ * (1..8, from the problem size and the SM count). 1..64 fixes it for every
+ * later launch in this process; the result differs only by fp32 rounding.
+ * Host only; process-wide; change it only while no attention call is being
+ * made from another thread. Returns WQ_ERR_INVALID_ARG outside 0..64.
+ */
+wq_status wq_test_set_attention_split(int32_t chunks_per_cta);
+
+/*
  * Read (and, if `clear` != 0, reset) the library's sticky device error word,
  * which kernels with bounded waits set when a wait expires. SYNCHRONISES
  * `stream` first. Returns WQ_ERR_TIMEOUT if the word was set, WQ_OK if not.

@@ -261,3 +261,10 @@ def test_decode_attention_validation(wq):
     assert call(ws_bytes=size.value - 1) == wq.WQ_ERR_WORKSPACE
     assert ws(2, 16, 4, 300, 128, 3, ctypes.byref(size)) == wq.WQ_ERR_UNSUPPORTED
     assert ws(0, 16, 4, 300, 128, 2, ctypes.byref(size)) == wq.WQ_OK and size.value == 0
+
+
+def test_attention_split_hook_validation(wq):
+    assert wq.lib.wq_test_set_attention_split(-1) == wq.WQ_ERR_INVALID_ARG
+    assert wq.lib.wq_test_set_attention_split(65) == wq.WQ_ERR_INVALID_ARG
+    assert wq.lib.wq_test_set_attention_split(3) == wq.WQ_OK
+    assert wq.lib.wq_test_set_attention_split(0) == wq.WQ_OK

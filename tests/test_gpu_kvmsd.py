@@ -102,6 +102,24 @@ def test_attention_every_element(wq, b, hq, hkv, length, c):
     assert st == wq.WQ_OK, hex(detail)
 
 
+@pytest.mark.parametrize("b,hq,hkv,length", [(2, 4, 2, 1100), (1, 64, 8, 700),
+                                             (3, 8, 1, 2049)])
+@pytest.mark.parametrize("ns", [2, 3, 8])
+def test_attention_chunks_per_cta(wq, b, hq, hkv, length, ns):
+    """Each CTA streaming ns chunks of 256 keys (merged in registers), with a
+    ragged last CTA; the same bound against the oracle."""
+    q, k, v = _inputs(b, hq, hkv, length, seed=b * 7 + length + ns)
+    wq.wq_test_set_attention_split(ns)
+    try:
+        out, _, _ = _run(wq, q, k, v, 2)
+    finally:
+        wq.wq_test_set_attention_split(0)
+    kc, vc = _oracle_cache(k), _oracle_cache(v)
+    ref = kvmsd.msd_decode_attention(q.float().numpy(), kc, vc, n_components=2)
+    _check(out, ref, kvmsd.dequant_cache(*vc), 2.0 ** -12,
+           "ns=%d B=%d Hq=%d Hkv=%d L=%d" % (ns, b, hq, hkv, length))
+
+
 def test_one_key_returns_its_value(wq):
     q, k, v = _inputs(2, 4, 2, 1, seed=5)
     out, _, _ = _run(wq, q, k, v, 2)

@@ -43,6 +43,7 @@
 // merges the CTAs' partials.
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 
 #include "splitk_common.cuh"
 
@@ -104,6 +105,13 @@ __device__ __forceinline__ float div_by(float a, float b, float y) {
   return __fmaf_rn(__fmaf_rn(-q, b, a), y, q);
 }
 
+// 2^x (ex2.approx: relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct KvArgs {
   const int8_t* qd;       // [C][B*Hq][D] query digits
   const float* qs;        // [C][B*Hq] their scales
@@ -116,13 +124,14 @@ struct KvArgs {
   float* part;            // [B, Hkv, nsplit, R, D] partial outputs
   float* stat;            // [B, Hkv, nsplit, R, 2] (M, E) of each partial
   int B, Hq, Hkv, L, nch, ns, nsplit;
-  float inv_sqrt_d;
+  float score_scale;      // log2(e) / sqrt(D): scores in log2 units
 };
 
 template <int R, int C>
 __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
   constexpr int RC = R * C;
   static_assert(RC <= 16 && (C == 1 || C == 2), "digit rows");
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23 (see below)
   __shared__ __align__(16) uint8_t sm[kSmemBytes];
   uint8_t* kc = sm + kOffK;
   uint8_t* vc = sm + kOffV;
@@ -173,7 +182,8 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     }
   };
   auto store_info = [&](const __half (&h)[4]) {
-    ki[tid] = make_float4(__half2float(h[0]), __half2float(h[1]), __half2float(h[2]), 0.0f);
+    ki[tid] = make_float4(__half2float(h[0]), __int_as_float((int)__half2float(h[1])),
+                          __half2float(h[2]), 0.0f);
     zvb[bd_col(tid)] = (uint8_t)__half2float(h[3]);
   };
 
@@ -227,9 +237,33 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     a[s][2] = g < RC ? qw[g * kQwStride + 8 * s + 4 + t4] : 0u;
     a[s][3] = g + 8 < RC ? qw[(g + 8) * kQwStride + 8 * s + 4 + t4] : 0u;
   }
+  // Scores in log2 units. With C = 2 the component scales satisfy
+  // sig_1 = 256 sig_2 exactly (a power-of-two ratio), so the two integer
+  // partial sums combine exactly as 256 (P_1 - zk R_1) + (P_2 - zk R_2)
+  // = 256 P_1 + P_2 - zk (256 R_1 + R_2) (|.| < 2^31) before one conversion.
   const int r0 = hv ? hl * C : 0;
-  const float sig0 = qsig[r0], sig1 = C == 2 ? qsig[r0 + 1] : 0.0f;
-  const int qs0 = qsum[r0], qs1 = C == 2 ? qsum[r0 + 1] : 0;
+  const float cs = qsig[r0 + C - 1] * p.score_scale;
+  const int qsc = C == 2 ? 256 * qsum[r0] + qsum[r0 + 1] : qsum[r0];
+
+  // lane-constant parts of the shared-memory addresses (the swizzle of every
+  // row a lane reads depends on the lane only):
+  //   score B rows 32 w + (g >> 1) + 4 nt + 16 (g & 1): bit 1 = bit 2 of g, bit 4 = bit 0 of g;
+  //   value B rows 32 ks + 16 hb + t4 + 4 i: bit 1 = bit 1 of t4, bit 4 = hb.
+  const uint8_t* kaddr[4];
+  {
+    const int sw = ((g >> 2) & 1) | ((g & 1) << 1);
+    const uint8_t* base = kc + (32 * warp + (g >> 1) + 16 * (g & 1)) * kRowBytes + 4 * (t4 >> 1);
+#pragma unroll
+    for (int s = 0; s < 4; ++s) kaddr[s] = base + ((s ^ sw) << 4);
+  }
+  const int wi = 2 * warp + (g >> 2);  // the code word of each V row this lane reads
+  const uint8_t* vaddr[2];
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+    const int sw = ((t4 >> 1) & 1) | (hb << 1);
+    vaddr[hb] = vc + t4 * kRowBytes + (((wi >> 2) ^ sw) << 4) + 4 * (wi & 3);
+  }
+  const float4* kinf = ki + 32 * warp + t4;  // the lane's keys: + 4 nt + 16 e
 
   float O[2][4];
 #pragma unroll
@@ -245,17 +279,17 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's K codes
       __syncthreads();
     }
-    // ---- scores: warp w takes keys 32 w .. 32 w + 31
+    // ---- scores: warp w takes keys 32 w .. 32 w + 31; column n of n-tile nt
+    // is key 32 w + (n >> 1) + 4 nt + 16 (n & 1)
     int sacc[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) sacc[nt][r] = 0;
-      const int l = 32 * warp + (g >> 1) + 4 * nt + 16 * (g & 1);
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        const uint32_t* ch = reinterpret_cast<const uint32_t*>(kc + kv_off(l, s));
-        const uint32_t w0 = ch[t4 >> 1], w1 = ch[2 + (t4 >> 1)];
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kaddr[s] + nt * 4 * kRowBytes);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kaddr[s] + nt * 4 * kRowBytes + 8);
         const int sh = 4 * (t4 & 1);
         mma_s8u8(sacc[nt], a[s][0], a[s][1], a[s][2], a[s][3], (w0 >> sh) & 0x0F0F0F0Fu,
                  (w1 >> sh) & 0x0F0F0F0Fu);
@@ -268,19 +302,20 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        int p0 = sacc[nt][e], p1 = 0;
+        int dint;
         if (C == 2) {
           const int send = (g & 1) ? sacc[nt][e] : sacc[nt][2 + e];
           const int recv = __shfl_xor_sync(0xffffffffu, send, 4);
-          p0 = (g & 1) ? recv : sacc[nt][e];
-          p1 = (g & 1) ? sacc[nt][2 + e] : recv;
+          const int p0 = (g & 1) ? recv : sacc[nt][e];
+          const int p1 = (g & 1) ? sacc[nt][2 + e] : recv;
+          dint = 256 * p0 + p1;
+        } else {
+          dint = sacc[nt][e];
         }
-        const int kk = 32 * warp + t4 + 4 * nt + 16 * e;
-        const float4 inf = ki[kk];
-        const int zk = (int)inf.y;
-        float s = sig0 * (float)(p0 - zk * qs0);  // |.| < 2^24: exact
-        if (C == 2) s = fmaf(sig1, (float)(p1 - zk * qs1), s);
-        s = (hv && kk < nk) ? s * inf.x * p.inv_sqrt_d : -INFINITY;
+        const float4 inf = kinf[4 * nt + 16 * e];
+        dint -= __float_as_int(inf.y) * qsc;
+        const bool ok = hv && 32 * warp + t4 + 4 * nt + 16 * e < nk;
+        const float s = ok ? (float)dint * (inf.x * cs) : -INFINITY;
         sc[nt][e] = s;
         mx = fmaxf(mx, s);
       }
@@ -302,11 +337,10 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int kk = 32 * warp + t4 + 4 * nt + 16 * e;
-        const float ex = sc[nt][e] == -INFINITY ? 0.0f : expf(sc[nt][e] - m);
+        const float ex = hv ? exp2_approx(sc[nt][e] - m) : 0.0f;  // sc = -inf: 0
         es += ex;
-        wv[nt][e] = ex * ki[kk].z;
-        am = fmaxf(am, fabsf(wv[nt][e]));
+        wv[nt][e] = ex * kinf[4 * nt + 16 * e].z;  // >= 0: sv > 0
+        am = fmaxf(am, wv[nt][e]);
       }
 #pragma unroll
     for (int o = 1; o <= 2; o <<= 1) {
@@ -325,45 +359,45 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
         E += rede[w * 8 + hl];
         A = fmaxf(A, reda[w * 8 + hl]);
       }
-    // the decomposition of w over the chunk's keys, as for an activation row:
+    // The decomposition of w over the chunk's keys, as for an activation row:
     // s_1 = amax / 127, s_{c+1} = s_c / 256, digit rint(r / s_c) (the first
     // clamped to +-127), residual r - s_c a_c rounded once, and a digit of
-    // +128 becomes -128 with a carry into the digit before it
+    // +128 becomes -128 with a carry into the digit before it. Rounding to an
+    // integer: t = x + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing is
+    // 1, so the add rounds x to nearest-even and t's low mantissa byte is the
+    // digit's two's-complement byte (|x| <= 128.5).
     const float tau0 = A > 0.0f ? __fdiv_rn(A, 127.0f) : 1.0f;
     const float y0 = __frcp_rn(tau0);
     const float tau1 = tau0 * (1.0f / 256.0f), y1 = y0 * 256.0f;
-    uint32_t word[C][2];
-#pragma unroll
-    for (int c = 0; c < C; ++c) word[c][0] = word[c][1] = 0u;
+    uint32_t tb[C][4][2];  // the digits' float bit patterns
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float r = wv[nt][e];
-        const float q0 = fminf(fmaxf(rintf(div_by(r, tau0, y0)), -127.0f), 127.0f);
-        int d0 = (int)q0;
+        const float r = wv[nt][e];
+        float t0 = fminf(fmaxf(div_by(r, tau0, y0), -127.0f), 127.0f) + kRound;
         if (C == 2) {
-          r = __fmaf_rn(-tau0, q0, r);
-          int d1 = (int)rintf(div_by(r, tau1, y1));
-          if (d1 == 128) {
-            d1 = -128;
-            d0 += 1;
-          }
-          word[C - 1][e] |= (uint32_t)(d1 & 0xFF) << (8 * nt);
+          const float r1 = __fmaf_rn(-tau0, t0 - kRound, r);
+          const float t1 = div_by(r1, tau1, y1) + kRound;
+          if (t1 == kRound + 128.0f) t0 += 1.0f;  // the byte of +128 already reads -128
+          tb[C - 1][nt][e] = __float_as_uint(t1);
         }
-        word[0][e] |= (uint32_t)(d0 & 0xFF) << (8 * nt);
+        tb[0][nt][e] = __float_as_uint(t0);
       }
     if (hv)
 #pragma unroll
       for (int c = 0; c < C; ++c)
 #pragma unroll
-        for (int e = 0; e < 2; ++e)
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t lo = prmt(tb[c][0][e], tb[c][1][e], 0x0040u);
+          const uint32_t hi = prmt(tb[c][2][e], tb[c][3][e], 0x0040u);
           *reinterpret_cast<uint32_t*>(bd + (hl * C + c) * kBdStride + 32 * warp + 16 * e +
-                                       4 * t4) = word[c][e];
-    // merge weights of this chunk into the CTA's running sums
+                                       4 * t4) = prmt(lo, hi, 0x5410u);
+        }
+    // merge weights of this chunk into the CTA's running sums (log2 units)
     if (warp == 0 && t4 == 0 && hv) {
       const float M0 = Mrun[hl], Mn = fmaxf(M0, m);
-      const float al = expf(M0 - Mn), be = expf(m - Mn);  // M0 = -inf: al = 0
+      const float al = exp2_approx(M0 - Mn), be = exp2_approx(m - Mn);  // M0 = -inf: al = 0
       Erun[hl] = fmaf(Erun[hl], al, E * be);
       Mrun[hl] = Mn;
 #pragma unroll
@@ -381,31 +415,28 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) vacc[0][r] = vacc[1][r] = zacc[r] = 0;
     {
-      const int wi = 2 * warp + (g >> 2);
       const int q = g & 3;
       const int sh = 4 * (q & 1);
       // byte (q >> 1) of two rows into bytes 0, 1 (jm = 0); byte 2 + (q >> 1) (jm = 1)
       const uint32_t sel0 = (uint32_t)((q >> 1) | ((4 + (q >> 1)) << 4));
       const uint32_t sel1 = sel0 + 0x22u;
-      const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride);
-      const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride);
-      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb);
-#pragma unroll 2
+      const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride + 4 * t4);
+      const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride + 4 * t4);
+      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb + 4 * t4);
+#pragma unroll
       for (int ks = 0; ks < kT / 32; ++ks) {
-        const int k0 = 32 * ks;
-        const uint32_t a0 = g < RC ? arow0[(k0 >> 2) + t4] : 0u;
-        const uint32_t a1 = g + 8 < RC ? arow1[(k0 >> 2) + t4] : 0u;
-        const uint32_t a2 = g < RC ? arow0[(k0 >> 2) + 4 + t4] : 0u;
-        const uint32_t a3 = g + 8 < RC ? arow1[(k0 >> 2) + 4 + t4] : 0u;
+        const uint32_t a0 = g < RC ? arow0[8 * ks] : 0u;
+        const uint32_t a1 = g + 8 < RC ? arow1[8 * ks] : 0u;
+        const uint32_t a2 = g < RC ? arow0[8 * ks + 4] : 0u;
+        const uint32_t a3 = g + 8 < RC ? arow1[8 * ks + 4] : 0u;
         uint32_t bb[2][2];  // [jm][key half]
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           uint32_t rw[4];
 #pragma unroll
-          for (int ii = 0; ii < 4; ++ii) {
-            const int l = k0 + 16 * hb + t4 + 4 * ii;
-            rw[ii] = *reinterpret_cast<const uint32_t*>(vc + kv_off(l, wi >> 2) + 4 * (wi & 3));
-          }
+          for (int ii = 0; ii < 4; ++ii)
+            rw[ii] = *reinterpret_cast<const uint32_t*>(vaddr[hb] +
+                                                        (32 * ks + 16 * hb + 4 * ii) * kRowBytes);
           const uint32_t x0 = prmt(rw[0], rw[1], sel0), y0v = prmt(rw[2], rw[3], sel0);
           const uint32_t x1 = prmt(rw[0], rw[1], sel1), y1v = prmt(rw[2], rw[3], sel1);
           bb[0][hb] = (prmt(x0, y0v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
@@ -413,7 +444,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
         }
         mma_s8u8(vacc[0], a0, a1, a2, a3, bb[0][0], bb[0][1]);
         mma_s8u8(vacc[1], a0, a1, a2, a3, bb[1][0], bb[1][1]);
-        mma_s8u8(zacc, a0, a1, a2, a3, zw[(k0 >> 2) + t4], zw[(k0 >> 2) + 4 + t4]);
+        mma_s8u8(zacc, a0, a1, a2, a3, zw[8 * ks], zw[8 * ks + 4]);
       }
     }
     // O = O alpha + beta tau_c (acc - zt) for the lane's rows g and g + 8
@@ -472,7 +503,7 @@ __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __
   float num = 0.0f, den = 0.0f;
   for (int j = 0; j < p.nsplit; ++j) {
     const int64_t ri = (base + j) * R + h;
-    const float f = expf(p.stat[ri * 2] - big);
+    const float f = exp2_approx(p.stat[ri * 2] - big);  // M in log2 units
     num = fmaf(f, p.part[ri * kD + d], num);
     den = fmaf(f, p.stat[ri * 2 + 1], den);
   }
@@ -565,7 +596,7 @@ wq_status launch_kv_msd(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64
                     : (int)std::max<int64_t>(
                           1, std::min<int64_t>(8, total / ((int64_t)num_sms() * 12)));
   a.nsplit = (int)((nch + a.ns - 1) / a.ns);
-  a.inv_sqrt_d = 1.0f / sqrtf((float)kD);
+  a.score_scale = (float)(1.4426950408889634 / std::sqrt((double)kD));
   const int R = (int)(Hq / Hkv);
   return C == 1 ? launch_kv_c<1>(a, R, out, st) : launch_kv_c<2>(a, R, out, st);
 }

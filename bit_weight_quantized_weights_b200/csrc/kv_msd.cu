@@ -37,10 +37,13 @@
 // components of a head swap halves (one shuffle), each lane takes one head
 // for its 8 keys, and the chunk statistics need one warp reduction and one
 // cross-warp step through shared memory. A CTA streams ns consecutive chunks
-// of one (sequence, KV head): the next chunk's K codes are copied (cp.async)
-// once the scores are done, its V codes once the values are done, and the
-// chunks merge in registers (flash-decoding rescaling); a second kernel
-// merges the CTAs' partials.
+// of one (sequence, KV head) through a two-stage ring: every thread copies
+// its share of a chunk's K and V code rows (2 x 16 KB) with 16-byte cp.async
+// into the stage freed by the chunk two back, so a chunk is in flight while
+// the one before is computed. (Measured on B200: 256-row TMA tiles of these
+// 64-byte rows streamed slower than the cp.async copies.) The chunks merge in
+// registers (flash-decoding rescaling); a second kernel merges the CTAs'
+// partials.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -48,6 +51,7 @@
 #include "splitk_common.cuh"
 
 namespace wq {
+
 namespace {
 
 using namespace splitk;
@@ -57,33 +61,31 @@ constexpr int kT = 256;                  // keys per chunk
 constexpr int kRowBytes = kD / 2;        // 64 bytes of codes per key
 constexpr int kQwStride = kD / 4 + 4;    // words per query digit row (padded)
 constexpr int kBdStride = kT + 16;       // bytes per value digit row (padded)
+constexpr int kStages = 2;               // chunks of K and V codes in the ring
+constexpr int kMinBlocks = 3;            // CTAs per SM the kernel is sized for
+constexpr uint32_t kStageBytes = 2 * kT * kRowBytes;  // K codes, then V codes
 
-// shared memory carve-up (bytes)
-constexpr int kOffK = 0;                                  // K codes of one chunk
-constexpr int kOffV = kOffK + kT * kRowBytes;             // V codes
-constexpr int kOffBd = kOffV + kT * kRowBytes;            // value digits [16][kBdStride]
+// dynamic shared memory carve-up (bytes)
+constexpr int kOffBd = kStages * kStageBytes;             // value digits [16][kBdStride]
+constexpr int kOffQw = kOffBd;                            // query digits (prologue only)
 constexpr int kOffKi = kOffBd + 16 * kBdStride;           // per key: sk, zk, sv (float4)
-constexpr int kOffZv = kOffKi + kT * 16;                  // zv bytes in digit-slot order
-constexpr int kOffQw = kOffZv + kT;                       // query digits [16][kQwStride]
-constexpr int kOffQm = kOffQw + 16 * kQwStride * 4;       // qsig[16], qsum[16]
+constexpr int kOffZv = kOffKi + kT * 16;                  // zv bytes in digit-slot order, x2
+constexpr int kOffQm = kOffZv + 2 * kT;                   // qsig[16], qsum[16]
 constexpr int kOffCo = kOffQm + 2 * 16 * 4;               // coefA[16], coefB[16] per digit row
 constexpr int kOffRun = kOffCo + 2 * 16 * 4;              // running M[8], E[8] per head
 constexpr int kOffRed = kOffRun + 2 * 8 * 4;              // [3][8 warps][8 heads]
 constexpr int kSmemBytes = kOffRed + 3 * 8 * 8 * 4;
-static_assert(kSmemBytes <= 48 * 1024, "static shared memory");
+static_assert(16 * kQwStride * 4 <= 16 * kBdStride, "query digits fit the digit rows");
+// kMinBlocks CTAs per SM (228 KB, 1 KB reserved per CTA)
+static_assert(kMinBlocks * (kSmemBytes + 1024) <= 228 * 1024, "CTAs per SM");
 
-// 16-byte chunk c (0..3) of key row l is stored at chunk c ^ sw(l), with
-// sw(l) = bit 1 of l in bit 0 and bit 4 of l in bit 1: the score B loads
-// (rows a + 16 b + 4 t, a in 0..3, b in 0..1) and the value B loads (rows
-// t + 4 i, t in 0..3) then hit distinct banks.
-__device__ __forceinline__ int kv_off(int l, int c) {
-  const int sw = ((l >> 1) & 1) | ((l >> 3) & 2);
-  return l * kRowBytes + ((c ^ sw) << 4);
-}
-// Slot of key kk (0..255) in the value digit rows: within each 16-key half of
-// a 32-key step, key t + 4 i sits at slot 4 t + i (t, i in 0..3).
+// 16-byte chunk c of key row l sits at byte l * 64 + ((c ^ ((l >> 1) & 3)) << 4)
+// of its tile: the score B reads (rows 8 t + g) and the value B reads (rows
+// 8 i + 2 t4 + hb) then hit distinct banks.
+// Slot of key kk (0..255) in the value digit rows: within each 32-key step,
+// key 8 i + 2 t + h sits at slot 16 h + 4 t + i (i, t in 0..3, h in 0..1).
 __device__ __forceinline__ int bd_col(int kk) {
-  return (kk & ~15) + 4 * (kk & 3) + ((kk >> 2) & 3);
+  return (kk & ~31) + 16 * (kk & 1) + 4 * ((kk >> 1) & 3) + ((kk >> 3) & 3);
 }
 
 __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -115,30 +117,29 @@ __device__ __forceinline__ float exp2_approx(float x) {
 struct KvArgs {
   const int8_t* qd;       // [C][B*Hq][D] query digits
   const float* qs;        // [C][B*Hq] their scales
-  const uint8_t* kq;      // K codes [B, Hkv, L, D/2]
   const __half* ks;       // [B, Hkv, L]
   const __half* kz;
-  const uint8_t* vq;      // V codes
   const __half* vs;
   const __half* vz;
   float* part;            // [B, Hkv, nsplit, R, D] partial outputs
-  float* stat;            // [B, Hkv, nsplit, R, 2] (M, E) of each partial
+  float* stat;            // [B, Hkv, nsplit, R, 2] (M, E) of each partial, M in log2 units
   int B, Hq, Hkv, L, nch, ns, nsplit;
+  const uint8_t* kq;      // K codes [B, Hkv, L, D/2]
+  const uint8_t* vq;      // V codes
   float score_scale;      // log2(e) / sqrt(D): scores in log2 units
 };
 
 template <int R, int C>
-__global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
+__global__ void __launch_bounds__(256, kMinBlocks)
+    kv_msd_split_kernel(KvArgs p) {
   constexpr int RC = R * C;
   static_assert(RC <= 16 && (C == 1 || C == 2), "digit rows");
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23 (see below)
-  __shared__ __align__(16) uint8_t sm[kSmemBytes];
-  uint8_t* kc = sm + kOffK;
-  uint8_t* vc = sm + kOffV;
+  extern __shared__ __align__(16) uint8_t sm[];
   int8_t* bd = reinterpret_cast<int8_t*>(sm + kOffBd);
+  uint32_t* qw = reinterpret_cast<uint32_t*>(sm + kOffQw);
   float4* ki = reinterpret_cast<float4*>(sm + kOffKi);
   uint8_t* zvb = sm + kOffZv;
-  uint32_t* qw = reinterpret_cast<uint32_t*>(sm + kOffQw);
   float* qsig = reinterpret_cast<float*>(sm + kOffQm);
   int* qsum = reinterpret_cast<int*>(qsig + 16);
   float* coefA = reinterpret_cast<float*>(sm + kOffCo);
@@ -163,11 +164,22 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  auto issue_codes = [&](const uint8_t* src, uint8_t* dst, int jc) {
-    const int l0 = jc * kT, nk = min(kT, p.L - l0);
-    const uint8_t* s = src + (seq0 + l0) * kRowBytes;
-    for (int i = tid; i < nk * 4; i += 256)
-      cp_async16(dst + kv_off(i >> 2, i & 3), s + (i >> 2) * kRowBytes + 16 * (i & 3));
+  // chunk jc's K and V code rows into stage st, then one cp.async group:
+  // thread tid copies 16-byte piece tid & 3 of rows tid / 4 + 64 r (r < 4)
+  // of both tiles, so its swizzle ((row >> 1) & 3 = (tid >> 3) & 3) and its
+  // offsets are fixed
+  const int cp_dst = (tid >> 2) * kRowBytes + (((tid & 3) ^ ((tid >> 3) & 3)) << 4);
+  const int cp_src = (tid >> 2) * kRowBytes + 16 * (tid & 3);
+  auto issue = [&](int st, int jc) {
+    uint8_t* dst = sm + st * kStageBytes + cp_dst;
+    const int64_t off = (seq0 + (int64_t)jc * kT) * kRowBytes + cp_src;
+    const int nk = min(kT, p.L - jc * kT);
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      if ((tid >> 2) + 64 * r < nk) {
+        cp_async16(dst + r * 64 * kRowBytes, p.kq + off + r * 64 * kRowBytes);
+        cp_async16(dst + kT * kRowBytes + r * 64 * kRowBytes, p.vq + off + r * 64 * kRowBytes);
+      }
   };
   // key tid's (sk, zk, sv, zv) of chunk jc, zeros past the end of the cache
   auto load_info = [&](int jc, __half (&h)[4]) {
@@ -181,26 +193,28 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       h[3] = p.vz[seq0 + l];
     }
   };
-  auto store_info = [&](const __half (&h)[4]) {
+  auto store_info = [&](const __half (&h)[4], int buf) {
     ki[tid] = make_float4(__half2float(h[0]), __int_as_float((int)__half2float(h[1])),
                           __half2float(h[2]), 0.0f);
-    zvb[bd_col(tid)] = (uint8_t)__half2float(h[3]);
+    zvb[buf * kT + bd_col(tid)] = (uint8_t)__half2float(h[3]);
   };
 
-  // ---- prologue: the first chunk's codes and key data; the cache is not
-  // written by the grid this one may overlap, so they go before the wait
-  issue_codes(p.kq, kc, j0);
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  issue_codes(p.vq, vc, j0);
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  {
-    __half h[4];
-    load_info(j0, h);
-    store_info(h);
+  // ---- prologue: the first two chunks' codes and the first key data (the
+  // cache is not written by the grid this one may overlap, so they go before
+  // the wait)
+#pragma unroll
+  for (int st = 0; st < kStages; ++st) {
+    if (st < nsub) issue(st, j0 + st);
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
   if (tid < R) {
     Mrun[tid] = -INFINITY;
     Erun[tid] = 0.0f;
+  }
+  {
+    __half h[4];
+    load_info(j0, h);
+    store_info(h, 0);
   }
   // the query digits of this KV head's R query heads (rows hc = h C + c), in
   // the even-d / odd-d order of the unpacked K code words, and their sums
@@ -227,7 +241,6 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       qsig[tid] = p.qs[(int64_t)c * plane + qrow0 + h];
     }
   }
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
   __syncthreads();
   uint32_t a[4][4];  // score A fragments, [k-step][register]
 #pragma unroll
@@ -244,26 +257,22 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
   const int r0 = hv ? hl * C : 0;
   const float cs = qsig[r0 + C - 1] * p.score_scale;
   const int qsc = C == 2 ? 256 * qsum[r0] + qsum[r0 + 1] : qsum[r0];
+  __syncthreads();  // the query digits' space becomes the value digit rows
 
-  // lane-constant parts of the shared-memory addresses (the swizzle of every
-  // row a lane reads depends on the lane only):
-  //   score B rows 32 w + (g >> 1) + 4 nt + 16 (g & 1): bit 1 = bit 2 of g, bit 4 = bit 0 of g;
-  //   value B rows 32 ks + 16 hb + t4 + 4 i: bit 1 = bit 1 of t4, bit 4 = hb.
-  const uint8_t* kaddr[4];
+  // lane-constant parts of the shared-memory offsets within a stage (the
+  // swizzle of every row a lane reads depends on the lane only):
+  //   score B rows 32 w + 8 nt + g: (row >> 1) & 3 = (g >> 1) & 3;
+  //   value B rows 32 ks + 8 i + 2 t4 + hb: (row >> 1) & 3 = t4.
+  int koff[4];
   {
-    const int sw = ((g >> 2) & 1) | ((g & 1) << 1);
-    const uint8_t* base = kc + (32 * warp + (g >> 1) + 16 * (g & 1)) * kRowBytes + 4 * (t4 >> 1);
+    const int sw = (g >> 1) & 3;
 #pragma unroll
-    for (int s = 0; s < 4; ++s) kaddr[s] = base + ((s ^ sw) << 4);
+    for (int s = 0; s < 4; ++s)
+      koff[s] = (32 * warp + g) * kRowBytes + ((s ^ sw) << 4) + 4 * (t4 >> 1);
   }
   const int wi = 2 * warp + (g >> 2);  // the code word of each V row this lane reads
-  const uint8_t* vaddr[2];
-#pragma unroll
-  for (int hb = 0; hb < 2; ++hb) {
-    const int sw = ((t4 >> 1) & 1) | (hb << 1);
-    vaddr[hb] = vc + t4 * kRowBytes + (((wi >> 2) ^ sw) << 4) + 4 * (wi & 3);
-  }
-  const float4* kinf = ki + 32 * warp + t4;  // the lane's keys: + 4 nt + 16 e
+  const int voff = kT * kRowBytes + 2 * t4 * kRowBytes + (((wi >> 2) ^ t4) << 4) + 4 * (wi & 3);
+  const float4* kinf = ki + 32 * warp + 2 * t4;  // the lane's keys: + 8 nt + e
 
   float O[2][4];
 #pragma unroll
@@ -275,12 +284,15 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     const int jc = j0 + i;
     const int nk = min(kT, p.L - jc * kT);
     const bool more = i + 1 < nsub;
-    if (i > 0) {
-      asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's K codes
-      __syncthreads();
-    }
+    const int st = i % kStages;
+    // this chunk's group (the next chunk's may still be in flight)
+    asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
+    __syncthreads();
+    const uint8_t* kc = sm + st * kStageBytes;
+    __half nxt[4];
+    if (more) load_info(jc + 1, nxt);
     // ---- scores: warp w takes keys 32 w .. 32 w + 31; column n of n-tile nt
-    // is key 32 w + (n >> 1) + 4 nt + 16 (n & 1)
+    // is key 32 w + 8 nt + n
     int sacc[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
@@ -288,14 +300,15 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       for (int r = 0; r < 4; ++r) sacc[nt][r] = 0;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(kaddr[s] + nt * 4 * kRowBytes);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(kaddr[s] + nt * 4 * kRowBytes + 8);
+        const uint8_t* ad = kc + koff[s] + nt * 8 * kRowBytes;
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ad);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ad + 8);
         const int sh = 4 * (t4 & 1);
         mma_s8u8(sacc[nt], a[s][0], a[s][1], a[s][2], a[s][3], (w0 >> sh) & 0x0F0F0F0Fu,
                  (w1 >> sh) & 0x0F0F0F0Fu);
       }
     }
-    // the lane's head for its keys 32 w + t4 + 4 nt + 16 e
+    // the lane's head for its keys 32 w + 8 nt + 2 t4 + e
     float sc[4][2];
     float mx = -INFINITY;
 #pragma unroll
@@ -312,22 +325,23 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
         } else {
           dint = sacc[nt][e];
         }
-        const float4 inf = kinf[4 * nt + 16 * e];
+        const float4 inf = kinf[8 * nt + e];
         dint -= __float_as_int(inf.y) * qsc;
-        const bool ok = hv && 32 * warp + t4 + 4 * nt + 16 * e < nk;
-        const float s = ok ? (float)dint * (inf.x * cs) : -INFINITY;
-        sc[nt][e] = s;
-        mx = fmaxf(mx, s);
+        const float s = (float)dint * (inf.x * cs);
+        sc[nt][e] = hv ? s : -INFINITY;
       }
+    if (nk < kT)  // the cache's last chunk: keys past its end do not count
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (32 * warp + 8 * nt + 2 * t4 + e >= nk) sc[nt][e] = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][0], sc[nt][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
     if (t4 == 0 && hv) redm[warp * 8 + hl] = mx;
-    __syncthreads();  // every warp is done with the K codes
-    // the next chunk's K codes and key data
-    if (more) issue_codes(p.kq, kc, jc + 1);
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    __half nxt[4];
-    if (more) load_info(jc + 1, nxt);
+    __syncthreads();
     float m = -INFINITY;
     if (hv)
 #pragma unroll
@@ -339,7 +353,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       for (int e = 0; e < 2; ++e) {
         const float ex = hv ? exp2_approx(sc[nt][e] - m) : 0.0f;  // sc = -inf: 0
         es += ex;
-        wv[nt][e] = ex * kinf[4 * nt + 16 * e].z;  // >= 0: sv > 0
+        wv[nt][e] = ex * kinf[8 * nt + e].z;  // >= 0: sv > 0
         am = fmaxf(am, wv[nt][e]);
       }
 #pragma unroll
@@ -362,38 +376,37 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
     // The decomposition of w over the chunk's keys, as for an activation row:
     // s_1 = amax / 127, s_{c+1} = s_c / 256, digit rint(r / s_c) (the first
     // clamped to +-127), residual r - s_c a_c rounded once, and a digit of
-    // +128 becomes -128 with a carry into the digit before it. Rounding to an
-    // integer: t = x + 1.5 * 2^23 lies in [2^23, 2^24), where the spacing is
-    // 1, so the add rounds x to nearest-even and t's low mantissa byte is the
-    // digit's two's-complement byte (|x| <= 128.5).
+    // +128 becomes -128 with a carry into the digit before it. Here
+    // 0 <= w <= amax, and RN(w / s_1) <= RN(127 (1 + 2^-24)) < 127.5, so the
+    // first digit needs no clamp. Rounding to an integer: t = x + 1.5 * 2^23
+    // lies in [2^23, 2^24), where the spacing is 1, so the add rounds x to
+    // nearest-even and t's low mantissa byte is the digit's two's-complement
+    // byte (|x| <= 128.5).
     const float tau0 = A > 0.0f ? __fdiv_rn(A, 127.0f) : 1.0f;
     const float y0 = __frcp_rn(tau0);
     const float tau1 = tau0 * (1.0f / 256.0f), y1 = y0 * 256.0f;
-    uint32_t tb[C][4][2];  // the digits' float bit patterns
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int e = 0; e < 2; ++e) {
+      uint32_t tb[C][4];  // the digits' float bit patterns, keys nt = 0..3
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
+      for (int nt = 0; nt < 4; ++nt) {
         const float r = wv[nt][e];
-        float t0 = fminf(fmaxf(div_by(r, tau0, y0), -127.0f), 127.0f) + kRound;
+        float t0 = div_by(r, tau0, y0) + kRound;
         if (C == 2) {
           const float r1 = __fmaf_rn(-tau0, t0 - kRound, r);
           const float t1 = div_by(r1, tau1, y1) + kRound;
           if (t1 == kRound + 128.0f) t0 += 1.0f;  // the byte of +128 already reads -128
-          tb[C - 1][nt][e] = __float_as_uint(t1);
+          tb[C - 1][nt] = __float_as_uint(t1);
         }
-        tb[0][nt][e] = __float_as_uint(t0);
+        tb[0][nt] = __float_as_uint(t0);
       }
-    if (hv)
+      if (hv)
 #pragma unroll
-      for (int c = 0; c < C; ++c)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const uint32_t lo = prmt(tb[c][0][e], tb[c][1][e], 0x0040u);
-          const uint32_t hi = prmt(tb[c][2][e], tb[c][3][e], 0x0040u);
+        for (int c = 0; c < C; ++c)
           *reinterpret_cast<uint32_t*>(bd + (hl * C + c) * kBdStride + 32 * warp + 16 * e +
-                                       4 * t4) = prmt(lo, hi, 0x5410u);
-        }
+                                       4 * t4) =
+              prmt(prmt(tb[c][0], tb[c][1], 0x0040u), prmt(tb[c][2], tb[c][3], 0x0040u), 0x5410u);
+    }
     // merge weights of this chunk into the CTA's running sums (log2 units)
     if (warp == 0 && t4 == 0 && hv) {
       const float M0 = Mrun[hl], Mn = fmaxf(M0, m);
@@ -406,8 +419,10 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
         coefB[hl * C + c] = be * (c == 0 ? tau0 : tau1);
       }
     }
-    asm volatile("cp.async.wait_group 1;" ::: "memory");  // this chunk's V codes
     __syncthreads();
+    // the next chunk's key data (this chunk's is no longer read; its zero
+    // bytes go to the other buffer)
+    if (more) store_info(nxt, (i + 1) & 1);
 
     // ---- values: warp w owns d in [16 w, 16 w + 16), words wi = 2 w, 2 w + 1
     // of each code row. MMA jm, column n: d = 8 (2 w + (n >> 2)) + (n & 3) + 4 jm.
@@ -415,6 +430,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) vacc[0][r] = vacc[1][r] = zacc[r] = 0;
     {
+      const uint8_t* vc = kc + voff;
       const int q = g & 3;
       const int sh = 4 * (q & 1);
       // byte (q >> 1) of two rows into bytes 0, 1 (jm = 0); byte 2 + (q >> 1) (jm = 1)
@@ -422,7 +438,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
       const uint32_t sel1 = sel0 + 0x22u;
       const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride + 4 * t4);
       const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride + 4 * t4);
-      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb + 4 * t4);
+      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb + (i & 1) * kT + 4 * t4);
 #pragma unroll
       for (int ks = 0; ks < kT / 32; ++ks) {
         const uint32_t a0 = g < RC ? arow0[8 * ks] : 0u;
@@ -435,8 +451,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
           uint32_t rw[4];
 #pragma unroll
           for (int ii = 0; ii < 4; ++ii)
-            rw[ii] = *reinterpret_cast<const uint32_t*>(vaddr[hb] +
-                                                        (32 * ks + 16 * hb + 4 * ii) * kRowBytes);
+            rw[ii] = *reinterpret_cast<const uint32_t*>(vc + (32 * ks + 8 * ii + hb) * kRowBytes);
           const uint32_t x0 = prmt(rw[0], rw[1], sel0), y0v = prmt(rw[2], rw[3], sel0);
           const uint32_t x1 = prmt(rw[0], rw[1], sel1), y1v = prmt(rw[2], rw[3], sel1);
           bb[0][hb] = (prmt(x0, y0v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
@@ -459,12 +474,10 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
           O[jm][2 * rh + e] =
               fmaf(O[jm][2 * rh + e], cA, cB * (float)(vacc[jm][2 * rh + e] - zacc[2 * rh]));
     }
-    __syncthreads();  // the V codes, digits, key data and weights of this chunk are consumed
-    if (more) issue_codes(p.vq, vc, jc + 1);
+    __syncthreads();  // the stage, the digits and the weights of this chunk are consumed
+    if (i + kStages < nsub) issue(st, jc + kStages);
     asm volatile("cp.async.commit_group;" ::: "memory");
-    if (more) store_info(nxt);
   }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
 
   // ---- the CTA's partial: the components of a head sit in C consecutive
   // rows, held by lanes 4 apart
@@ -489,7 +502,7 @@ __global__ void __launch_bounds__(256, 3) kv_msd_split_kernel(KvArgs p) {
 }
 
 // Merge the CTAs' partials of each (sequence, query head): out = sum_j
-// e^(M_j - M) O_j / sum_j e^(M_j - M) E_j, one CTA of 128 threads (one per element).
+// 2^(M_j - M) O_j / sum_j 2^(M_j - M) E_j, one CTA of 128 threads (one per element).
 template <int R>
 __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __restrict__ out) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -503,7 +516,7 @@ __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __
   float num = 0.0f, den = 0.0f;
   for (int j = 0; j < p.nsplit; ++j) {
     const int64_t ri = (base + j) * R + h;
-    const float f = exp2_approx(p.stat[ri * 2] - big);  // M in log2 units
+    const float f = exp2_approx(p.stat[ri * 2] - big);
     num = fmaf(f, p.part[ri * kD + d], num);
     den = fmaf(f, p.stat[ri * 2 + 1], den);
   }
@@ -512,6 +525,12 @@ __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __
 
 template <int R, int C>
 wq_status launch_kv_rc(const KvArgs& a, void* out, cudaStream_t st) {
+  static bool attr_set = [] {
+    return cudaFuncSetAttribute(kv_msd_split_kernel<R, C>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kSmemBytes) == cudaSuccess;
+  }();
+  if (!attr_set) return WQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -521,9 +540,12 @@ wq_status launch_kv_rc(const KvArgs& a, void* out, cudaStream_t st) {
   cfg.stream = st;
   cfg.gridDim = dim3((unsigned)a.nsplit, (unsigned)a.Hkv, (unsigned)a.B);
   cfg.blockDim = dim3(256, 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kv_msd_split_kernel<R, C>, a) != cudaSuccess) return WQ_ERR_CUDA;
+  cfg.dynamicSmemBytes = kSmemBytes;
+  if (cudaLaunchKernelEx(&cfg, kv_msd_split_kernel<R, C>, a) != cudaSuccess)
+    return WQ_ERR_CUDA;
   cfg.gridDim = dim3((unsigned)(a.B * a.Hq), 1, 1);
   cfg.blockDim = dim3(kD, 1, 1);
+  cfg.dynamicSmemBytes = 0;
   if (cudaLaunchKernelEx(&cfg, kv_msd_merge_kernel<R>, a, static_cast<uint16_t*>(out)) !=
       cudaSuccess)
     return WQ_ERR_CUDA;
@@ -569,33 +591,32 @@ wq_status launch_kv_msd(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64
   int8_t* qd = reinterpret_cast<int8_t*>(w);
   float* qs = reinterpret_cast<float*>(w + dig);
   float* part = reinterpret_cast<float*>(w + dig + sc);
-  float* stat = part + (size_t)B * Hq * nch * kD;
   wq_status s = launch_msd_decompose(q, B * Hq, kD, C, B * Hq, qd, qs, st);
   if (s != WQ_OK) return s;
   KvArgs a;
   a.qd = qd;
   a.qs = qs;
   a.kq = static_cast<const uint8_t*>(kq);
+  a.vq = static_cast<const uint8_t*>(vq);
   a.ks = static_cast<const __half*>(ks);
   a.kz = static_cast<const __half*>(kz);
-  a.vq = static_cast<const uint8_t*>(vq);
   a.vs = static_cast<const __half*>(vs);
   a.vz = static_cast<const __half*>(vz);
   a.part = part;
-  a.stat = stat;
   a.B = (int)B;
   a.Hq = (int)Hq;
   a.Hkv = (int)Hkv;
   a.L = (int)L;
   a.nch = (int)nch;
-  // chunks per CTA: enough CTAs for about four waves of three per SM, at most
-  // 8 (or the count the test hook fixed)
+  // chunks per CTA: enough CTAs for about four waves of kMinBlocks per SM, at
+  // most 8 (or the count the test hook fixed)
   const int64_t total = B * Hkv * nch;
   const int forced = g_kv_chunks_per_cta.load(std::memory_order_relaxed);
   a.ns = forced > 0 ? forced
                     : (int)std::max<int64_t>(
-                          1, std::min<int64_t>(8, total / ((int64_t)num_sms() * 12)));
+                          1, std::min<int64_t>(8, total / ((int64_t)num_sms() * kMinBlocks * 4)));
   a.nsplit = (int)((nch + a.ns - 1) / a.ns);
+  a.stat = part + (size_t)B * Hkv * a.nsplit * (Hq / Hkv) * kD;
   a.score_scale = (float)(1.4426950408889634 / std::sqrt((double)kD));
   const int R = (int)(Hq / Hkv);
   return C == 1 ? launch_kv_c<1>(a, R, out, st) : launch_kv_c<2>(a, R, out, st);

@@ -699,8 +699,8 @@ def measure_per_config(wq, peaks, device):
         # torch's scaled-dot-product attention on a bf16 cache of the same shape
         hq, hkv, d = 64, 8, 128
         for b, length in ((32, 8192), (8, 32768)):
-            cache = [wq.kv_quantize(normal(b, hkv, length, d, std=0.5)),
-                     wq.kv_quantize(normal(b, hkv, length, d))]
+            cache = [wq.kv_quantize_keys(normal(b, hkv, length, d, std=0.5)),
+                     wq.kv_quantize_values(normal(b, hkv, length, d))]
             nb = 2 * b * hkv * length * (d // 2 + 4)          # codes + fp16 scale and zero
             copies = [cache] + [[tuple(t.clone() for t in kv) for kv in cache]
                                 for _ in range(_copies_for(nb) - 1)]

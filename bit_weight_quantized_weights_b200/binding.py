@@ -42,7 +42,7 @@ EXPORTED = [
     "wq_residual", "wq_select_salient", "wq_w4a16_gemv_corrected", "wq_w4a16_gemv_salient",
     "wq_test_set_wait", "wq_mx_quantize", "wq_mx_decompose", "wq_mx_gemv", "wq_msd_gemm_nf4",
     "wq_msd_decode_attention", "wq_msd_decode_attention_workspace",
-    "wq_test_set_attention_split",
+    "wq_test_set_attention_split", "wq_kv_block_values",
 ]
 
 
@@ -88,6 +88,7 @@ def _load():
         "wq_msd_decode_attention_workspace": ([I64, I64, I64, I64, I32, I32, ctypes.POINTER(SZ)],
                                               ctypes.c_int),
         "wq_test_set_attention_split": ([I32], ctypes.c_int),
+        "wq_kv_block_values": ([P, I64, I64, I32, P, P], ctypes.c_int),
         "wq_msd_gemm_noalloc": ([P, I64, I64, I64, I32, I32, P, P, P, P, P], ctypes.c_int),
         "wq_residual": ([ctypes.c_int, P, I64, I64, I32, P, P, P, P, P], ctypes.c_int),
         "wq_select_salient": ([P, I64, I64, I32, P, P], ctypes.c_int),
@@ -438,14 +439,38 @@ def wq_msd_gemm_nf4(x, n, n_components, codes, absmax, workspace=None, out=None,
     return out
 
 
-def kv_quantize(kv, stream=None):
-    """INT4-quantize a KV cache fp32 [B, Hkv, L, D] on the GPU, one group per
+def kv_quantize_keys(k, stream=None):
+    """INT4-quantize a key cache fp32 [B, Hkv, L, D] on the GPU, one group per
     (sequence, head, token) row: returns (codes int32 [B, Hkv, L, D/8], scales
     fp16 [B, Hkv, L], zeros fp16 [B, Hkv, L])."""
-    _cuda(kv, torch.float32, "kv")
-    b, hkv, length, d = kv.shape
-    qw, sc, zr = wq_quantize_pack(WQ_FMT_INT4_ASYM, kv.reshape(-1, d), d, stream=stream)
+    _cuda(k, torch.float32, "k")
+    b, hkv, length, d = k.shape
+    qw, sc, zr = wq_quantize_pack(WQ_FMT_INT4_ASYM, k.reshape(-1, d), d, stream=stream)
     return (qw.view(b, hkv, length, d // 8), sc.view(b, hkv, length), zr.view(b, hkv, length))
+
+
+def wq_kv_block_values(codes, rows, length, d, out=None, stream=None):
+    """V codes from the token layout (int32 [rows * L, D/8]) to blocks of 8
+    tokens: int32 [rows, ceil(L/8), D]."""
+    _cuda(codes, torch.int32, "codes")
+    nblk = (length + 7) // 8
+    if out is None:
+        out = torch.empty(rows, nblk, d, dtype=torch.int32, device=codes.device)
+    _check(lib.wq_kv_block_values(_ptr(codes), rows, length, d, _ptr(out), _stream(stream)),
+           "wq_kv_block_values")
+    return out
+
+
+def kv_quantize_values(v, stream=None):
+    """INT4-quantize a value cache fp32 [B, Hkv, L, D] on the GPU, one group per
+    (sequence, head, token) row: returns (codes int32 [B, Hkv, ceil(L/8), D] in
+    blocks of 8 tokens, scales fp16 [B, Hkv, L], zeros fp16 [B, Hkv, L])."""
+    _cuda(v, torch.float32, "v")
+    b, hkv, length, d = v.shape
+    qw, sc, zr = wq_quantize_pack(WQ_FMT_INT4_ASYM, v.reshape(-1, d), d, stream=stream)
+    blocked = wq_kv_block_values(qw, b * hkv, length, d, stream=stream)
+    return (blocked.view(b, hkv, (length + 7) // 8, d), sc.view(b, hkv, length),
+            zr.view(b, hkv, length))
 
 
 def attention_workspace(b, hq, hkv, length, d, n_components, device):
@@ -458,8 +483,9 @@ def attention_workspace(b, hq, hkv, length, d, n_components, device):
 
 def wq_msd_decode_attention(q, k_cache, v_cache, n_components=2, workspace=None, out=None,
                             stream=None):
-    """MSD decode attention: q bf16 [B, Hq, D]; k_cache / v_cache = (codes,
-    scales, zeros) as kv_quantize returns them. Returns out bf16 [B, Hq, D]."""
+    """MSD decode attention: q bf16 [B, Hq, D]; k_cache and v_cache = (codes,
+    scales, zeros) as kv_quantize_keys and kv_quantize_values return them.
+    Returns out bf16 [B, Hq, D]."""
     _cuda(q, torch.bfloat16, "q")
     b, hq, d = q.shape
     kq, ks, kz = k_cache
@@ -469,7 +495,8 @@ def wq_msd_decode_attention(q, k_cache, v_cache, n_components=2, workspace=None,
                         (kz, torch.float16, "k_zeros"), (vq, torch.int32, "v_codes"),
                         (vs, torch.float16, "v_scales"), (vz, torch.float16, "v_zeros")):
         _cuda(t, dt, name)
-    if tuple(kq.shape) != (b, hkv, length, d // 8) or tuple(vq.shape) != tuple(kq.shape) or \
+    if tuple(kq.shape) != (b, hkv, length, d // 8) or \
+            tuple(vq.shape) != (b, hkv, (length + 7) // 8, d) or \
             tuple(vs.shape) != tuple(ks.shape) or tuple(kz.shape) != tuple(ks.shape) or \
             tuple(vz.shape) != tuple(ks.shape) or ks.shape[0] != b:
         raise ValueError("KV cache shapes do not match q")

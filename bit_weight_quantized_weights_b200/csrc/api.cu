@@ -37,6 +37,8 @@ size_t mx_workspace_bytes(int64_t M, int64_t K, int32_t P);
 wq_status launch_msd_nf4(const void*, int64_t, int64_t, int64_t, int32_t, const uint8_t*,
                          const float*, void*, void*, cudaStream_t);
 size_t kv_msd_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int32_t C);
+wq_status launch_kv_block_values(const uint32_t*, int64_t, int64_t, int32_t, uint32_t*,
+                                 cudaStream_t);
 extern std::atomic<int> g_kv_chunks_per_cta;
 wq_status launch_kv_msd(const void*, int64_t, int64_t, int64_t, int64_t, int32_t, const void*,
                         const void*, const void*, const void*, const void*, const void*, void*,
@@ -402,6 +404,16 @@ wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_p
   return guarded([&] {
     return launch_mx_gemv(x, M, N, K, n_passes, codes, scales, y, workspace, as_stream(stream));
   });
+}
+
+wq_status wq_kv_block_values(const uint32_t* codes, int64_t rows, int64_t L, int32_t D,
+                             uint32_t* out, void* stream) {
+  if (rows < 0 || L <= 0 || D <= 0 || D % 8 != 0) return WQ_ERR_INVALID_ARG;
+  if (rows == 0) return WQ_OK;
+  if (!codes || !out) return WQ_ERR_INVALID_ARG;
+  if (!all_aligned({codes, out})) return WQ_ERR_ALIGNMENT;
+  if (L > INT32_MAX - 8 || D > 65536) return WQ_ERR_UNSUPPORTED;
+  return guarded([&] { return launch_kv_block_values(codes, rows, L, D, out, as_stream(stream)); });
 }
 
 wq_status wq_msd_decode_attention_workspace(int64_t B, int64_t Hq, int64_t Hkv, int64_t L,

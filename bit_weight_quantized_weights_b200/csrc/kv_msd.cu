@@ -17,22 +17,29 @@
 //           exact integer sums;
 //   merge   out = sum_j e^(m_j - M) O_j / sum_j e^(m_j - M) E_j.
 // The cache rows use the INT4 asymmetric quantizer with one group per row
-// (group = D = 128): codes uint32 [B, Hkv, L, 16] (low nibble first), fp16
-// scales and integer zeros [B, Hkv, L].
+// (group = D = 128), fp16 scales and integer zeros [B, Hkv, L]. K codes are
+// stored by token: uint32 [B, Hkv, L, 16], element d in nibble d % 8 of word
+// d / 8. V codes are stored in blocks of 8 tokens: uint32 [B, Hkv, ceil(L/8),
+// 128], token 8 j + t of dimension d in nibble t of word (j, d) (tokens past
+// L zero), so that one word holds 4 keys of one d in its low nibbles and 4 in
+// its high nibbles: the operand layout of the value product.
 //
 // B200 design. Decode attention reads the cache once, so the kernel is bound
 // by HBM when its per-key work keeps up. Both products are integer
 // tensor-core MMAs (mma.m16n8k32, s8 digits x u8 codes) with the R x C query
 // digit rows as the A operand (M = 16, unused rows zero):
-//   scores: N = keys, K = d. A K code word unpacks to two u8 words (even d,
-//           odd d); the query digits are stored in that order. Column n of
-//           n-tile t of warp w is key 32 w + (n >> 1) + 4 t + 16 (n & 1), so
-//           the accumulator fragment gives each lane 8 keys whose value digits
-//           pack into two 32-bit words per digit row;
-//   values: N = d, K = keys. The B fragment wants four keys of one d in a
-//           register: three byte permutes gather them from four code rows.
-//           The zero terms sum_l b_c[l] zv[l] are one more MMA per step, with
-//           the zero bytes as every column of B.
+//   scores: N = keys, K = d. One K code word (8 d of one key) gives both B
+//           registers of a lane: its low nibbles (even d) and high nibbles
+//           (odd d); the query digits are stored in that k order. Column n of
+//           n-tile t of warp w is key 32 w + 8 (n >> 1) + 2 t + (n & 1), so
+//           the accumulator fragment gives each lane the 8 keys of one V
+//           block, whose value digits pack into two 32-bit words per digit
+//           row;
+//   values: N = d, K = keys. One V code word (8 keys of one d) gives both B
+//           registers of a lane, low and high nibbles, and the value digits
+//           are stored in that k order; the digit rows (A) come in by
+//           ldmatrix. The zero terms sum_l b_c[l] zv[l] are one more MMA per
+//           step, with the zero bytes as every column of B.
 // The chunk softmax runs on the score fragments: the lanes holding the two
 // components of a head swap halves (one shuffle), each lane takes one head
 // for its 8 keys, and the chunk statistics need one warp reduction and one
@@ -68,6 +75,7 @@ constexpr uint32_t kStageBytes = 2 * kT * kRowBytes;  // K codes, then V codes
 // dynamic shared memory carve-up (bytes)
 constexpr int kOffBd = kStages * kStageBytes;             // value digits [16][kBdStride]
 constexpr int kOffQw = kOffBd;                            // query digits (prologue only)
+constexpr int kVRowWords = kD;                            // V tile: 32 rows of 8-token blocks
 constexpr int kOffKi = kOffBd + 16 * kBdStride;           // per key: sk, zk, sv (float4)
 constexpr int kOffZv = kOffKi + kT * 16;                  // zv bytes in digit-slot order, x2
 constexpr int kOffQm = kOffZv + 2 * kT;                   // qsig[16], qsum[16]
@@ -79,13 +87,23 @@ static_assert(16 * kQwStride * 4 <= 16 * kBdStride, "query digits fit the digit 
 // kMinBlocks CTAs per SM (228 KB, 1 KB reserved per CTA)
 static_assert(kMinBlocks * (kSmemBytes + 1024) <= 228 * 1024, "CTAs per SM");
 
-// 16-byte chunk c of key row l sits at byte l * 64 + ((c ^ ((l >> 1) & 3)) << 4)
-// of its tile: the score B reads (rows 8 t + g) and the value B reads (rows
-// 8 i + 2 t4 + hb) then hit distinct banks.
-// Slot of key kk (0..255) in the value digit rows: within each 32-key step,
-// key 8 i + 2 t + h sits at slot 16 h + 4 t + i (i, t in 0..3, h in 0..1).
-__device__ __forceinline__ int bd_col(int kk) {
-  return (kk & ~31) + 16 * (kk & 1) + 4 * ((kk >> 1) & 3) + ((kk >> 3) & 3);
+// Shared-memory tiles. K: 16-byte piece c of key row l at byte
+// l * 64 + ((c ^ ((l >> 3) & 3)) << 4); the score B reads (rows 8 (g >> 1) +
+// 2 t + (g & 1), one word of one piece each) then hit distinct banks. V: word
+// (block j, d) at word j * 128 + (d ^ 8 (j & 3)); the value B reads (blocks
+// 4 s + t4, 8 consecutive d) then hit distinct banks.
+// Value digits: within each 32-key step, key 8 b + 2 j + p (b, j in 0..3, p
+// in 0..1, the low (p = 0) or high nibble j of V block b) sits at k slot
+// 16 p + 4 b + j. The zero bytes are kept per step in the order 8 b + 4 p + j,
+// so one 8-byte read gives a lane both B registers of the zero-term MMA.
+__device__ __forceinline__ int zv_pos(int kk) {
+  return (kk & ~31) + 8 * ((kk >> 3) & 3) + 4 * (kk & 1) + ((kk >> 1) & 3);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
 }
 
 __device__ __forceinline__ void mma_s8u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -125,7 +143,8 @@ struct KvArgs {
   float* stat;            // [B, Hkv, nsplit, R, 2] (M, E) of each partial, M in log2 units
   int B, Hq, Hkv, L, nch, ns, nsplit;
   const uint8_t* kq;      // K codes [B, Hkv, L, D/2]
-  const uint8_t* vq;      // V codes
+  const uint8_t* vq;      // V codes [B, Hkv, nblk, D] words (8-token blocks)
+  int nblk;               // ceil(L / 8)
   float score_scale;      // log2(e) / sqrt(D): scores in log2 units
 };
 
@@ -164,22 +183,31 @@ __global__ void __launch_bounds__(256, kMinBlocks)
 
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // chunk jc's K and V code rows into stage st, then one cp.async group:
-  // thread tid copies 16-byte piece tid & 3 of rows tid / 4 + 64 r (r < 4)
-  // of both tiles, so its swizzle ((row >> 1) & 3 = (tid >> 3) & 3) and its
-  // offsets are fixed
-  const int cp_dst = (tid >> 2) * kRowBytes + (((tid & 3) ^ ((tid >> 3) & 3)) << 4);
-  const int cp_src = (tid >> 2) * kRowBytes + 16 * (tid & 3);
+  // chunk jc's K rows and V blocks into stage st (the caller commits the
+  // cp.async group). Thread tid copies 16-byte piece tid & 3 of K rows
+  // tid / 4 + 64 r and piece tid & 31 of V block rows tid / 32 + 8 r (r < 4),
+  // so its swizzles ((row >> 3) & 3 = (tid >> 5) & 3 for both) and its
+  // offsets are fixed.
+  const int sw_cp = (tid >> 5) & 3;
+  const int k_dst = (tid >> 2) * kRowBytes + (((tid & 3) ^ sw_cp) << 4);
+  const int k_src = (tid >> 2) * kRowBytes + 16 * (tid & 3);
+  const int v_dst = kT * kRowBytes + (tid >> 5) * (kVRowWords * 4) + (((tid & 31) ^ (2 * sw_cp)) << 4);
+  const int v_src = (tid >> 5) * (kVRowWords * 4) + 16 * (tid & 31);
+  const int64_t vseq = ((int64_t)b * p.Hkv + kh) * p.nblk;  // V block row of token 0
   auto issue = [&](int st, int jc) {
-    uint8_t* dst = sm + st * kStageBytes + cp_dst;
-    const int64_t off = (seq0 + (int64_t)jc * kT) * kRowBytes + cp_src;
+    uint8_t* dst = sm + st * kStageBytes;
+    const int64_t koff = (seq0 + (int64_t)jc * kT) * kRowBytes + k_src;
     const int nk = min(kT, p.L - jc * kT);
+    const int64_t voff = (vseq + (int64_t)jc * (kT / 8)) * (kVRowWords * 4) + v_src;
+    const int nb = min(kT / 8, p.nblk - jc * (kT / 8));
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-      if ((tid >> 2) + 64 * r < nk) {
-        cp_async16(dst + r * 64 * kRowBytes, p.kq + off + r * 64 * kRowBytes);
-        cp_async16(dst + kT * kRowBytes + r * 64 * kRowBytes, p.vq + off + r * 64 * kRowBytes);
-      }
+    for (int r = 0; r < 4; ++r) {
+      if ((tid >> 2) + 64 * r < nk)
+        cp_async16(dst + k_dst + r * 64 * kRowBytes, p.kq + koff + r * 64 * kRowBytes);
+      if ((tid >> 5) + 8 * r < nb)
+        cp_async16(dst + v_dst + r * 8 * kVRowWords * 4,
+                   p.vq + voff + r * 8 * kVRowWords * 4);
+    }
   };
   // key tid's (sk, zk, sv, zv) of chunk jc, zeros past the end of the cache
   auto load_info = [&](int jc, __half (&h)[4]) {
@@ -196,7 +224,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
   auto store_info = [&](const __half (&h)[4], int buf) {
     ki[tid] = make_float4(__half2float(h[0]), __int_as_float((int)__half2float(h[1])),
                           __half2float(h[2]), 0.0f);
-    zvb[buf * kT + bd_col(tid)] = (uint8_t)__half2float(h[3]);
+    zvb[buf * kT + zv_pos(tid)] = (uint8_t)__half2float(h[3]);
   };
 
   // ---- prologue: the first two chunks' codes and the first key data (the
@@ -229,8 +257,10 @@ __global__ void __launch_bounds__(256, kMinBlocks)
       const uint2 v = *reinterpret_cast<const uint2*>(
           p.qd + ((int64_t)c * plane + qrow0 + h) * kD + 8 * g8);
       const uint32_t ev = prmt(v.x, v.y, 0x6420u), od = prmt(v.x, v.y, 0x7531u);
-      qw[hc * kQwStride + 2 * g8] = ev;       // d = 8 g8 + 0, 2, 4, 6
-      qw[hc * kQwStride + 2 * g8 + 1] = od;   // d = 8 g8 + 1, 3, 5, 7
+      // k-step s = g8 / 4 holds the even-d words of its four K code words
+      // first, then the odd-d words
+      qw[hc * kQwStride + 8 * (g8 >> 2) + (g8 & 3)] = ev;      // d = 8 g8 + 0, 2, 4, 6
+      qw[hc * kQwStride + 8 * (g8 >> 2) + 4 + (g8 & 3)] = od;  // d = 8 g8 + 1, 3, 5, 7
       part = __dp4a((int)ev, 0x01010101, __dp4a((int)od, 0x01010101, 0));
     }
 #pragma unroll
@@ -258,21 +288,27 @@ __global__ void __launch_bounds__(256, kMinBlocks)
   const float cs = qsig[r0 + C - 1] * p.score_scale;
   const int qsc = C == 2 ? 256 * qsum[r0] + qsum[r0 + 1] : qsum[r0];
   __syncthreads();  // the query digits' space becomes the value digit rows
+  for (int i = RC * kBdStride / 4 + tid; i < 16 * kBdStride / 4; i += 256)
+    reinterpret_cast<uint32_t*>(bd)[i] = 0u;  // the unused A rows of the value MMA
 
   // lane-constant parts of the shared-memory offsets within a stage (the
   // swizzle of every row a lane reads depends on the lane only):
-  //   score B rows 32 w + 8 nt + g: (row >> 1) & 3 = (g >> 1) & 3;
-  //   value B rows 32 ks + 8 i + 2 t4 + hb: (row >> 1) & 3 = t4.
+  //   score B: K row 32 w + 8 (g >> 1) + 2 nt + (g & 1), word t4 of piece s;
+  //            (row >> 3) & 3 = (g >> 1) & 3;
+  //   value B: V block 4 ks + t4, word d = 16 w + 8 jm + g; (block & 3) = t4.
   int koff[4];
-  {
-    const int sw = (g >> 1) & 3;
 #pragma unroll
-    for (int s = 0; s < 4; ++s)
-      koff[s] = (32 * warp + g) * kRowBytes + ((s ^ sw) << 4) + 4 * (t4 >> 1);
-  }
-  const int wi = 2 * warp + (g >> 2);  // the code word of each V row this lane reads
-  const int voff = kT * kRowBytes + 2 * t4 * kRowBytes + (((wi >> 2) ^ t4) << 4) + 4 * (wi & 3);
-  const float4* kinf = ki + 32 * warp + 2 * t4;  // the lane's keys: + 8 nt + e
+  for (int s = 0; s < 4; ++s)
+    koff[s] = (32 * warp + 8 * (g >> 1) + (g & 1)) * kRowBytes + ((s ^ ((g >> 1) & 3)) << 4) +
+              4 * t4;
+  int voff[2];
+#pragma unroll
+  for (int jm = 0; jm < 2; ++jm)
+    voff[jm] = kT * kRowBytes + 4 * (t4 * kVRowWords + ((16 * warp + 8 * jm + g) ^ (8 * t4)));
+  const float4* kinf = ki + 32 * warp + 8 * t4;  // the lane's keys: + 2 nt + e
+  // ldmatrix row addresses of the value digit rows (A): lanes 0-7 rows 0-7,
+  // 8-15 rows 8-15, at k bytes 0-15; lanes 16-31 the same rows at 16-31
+  const int8_t* arow = bd + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kBdStride + 16 * (lane >> 4);
 
   float O[2][4];
 #pragma unroll
@@ -292,7 +328,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
     __half nxt[4];
     if (more) load_info(jc + 1, nxt);
     // ---- scores: warp w takes keys 32 w .. 32 w + 31; column n of n-tile nt
-    // is key 32 w + 8 nt + n
+    // is key 32 w + 8 (n >> 1) + 2 nt + (n & 1)
     int sacc[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
@@ -300,15 +336,12 @@ __global__ void __launch_bounds__(256, kMinBlocks)
       for (int r = 0; r < 4; ++r) sacc[nt][r] = 0;
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        const uint8_t* ad = kc + koff[s] + nt * 8 * kRowBytes;
-        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(ad);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(ad + 8);
-        const int sh = 4 * (t4 & 1);
-        mma_s8u8(sacc[nt], a[s][0], a[s][1], a[s][2], a[s][3], (w0 >> sh) & 0x0F0F0F0Fu,
-                 (w1 >> sh) & 0x0F0F0F0Fu);
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(kc + koff[s] + nt * 2 * kRowBytes);
+        mma_s8u8(sacc[nt], a[s][0], a[s][1], a[s][2], a[s][3], w & 0x0F0F0F0Fu,
+                 (w >> 4) & 0x0F0F0F0Fu);
       }
     }
-    // the lane's head for its keys 32 w + 8 nt + 2 t4 + e
+    // the lane's head for its keys 32 w + 8 t4 + 2 nt + e
     float sc[4][2];
     float mx = -INFINITY;
 #pragma unroll
@@ -325,7 +358,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
         } else {
           dint = sacc[nt][e];
         }
-        const float4 inf = kinf[8 * nt + e];
+        const float4 inf = kinf[2 * nt + e];
         dint -= __float_as_int(inf.y) * qsc;
         const float s = (float)dint * (inf.x * cs);
         sc[nt][e] = hv ? s : -INFINITY;
@@ -335,7 +368,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int e = 0; e < 2; ++e)
-          if (32 * warp + 8 * nt + 2 * t4 + e >= nk) sc[nt][e] = -INFINITY;
+          if (32 * warp + 8 * t4 + 2 * nt + e >= nk) sc[nt][e] = -INFINITY;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][0], sc[nt][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -353,7 +386,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
       for (int e = 0; e < 2; ++e) {
         const float ex = hv ? exp2_approx(sc[nt][e] - m) : 0.0f;  // sc = -inf: 0
         es += ex;
-        wv[nt][e] = ex * kinf[8 * nt + e].z;  // >= 0: sv > 0
+        wv[nt][e] = ex * kinf[2 * nt + e].z;  // >= 0: sv > 0
         am = fmaxf(am, wv[nt][e]);
       }
 #pragma unroll
@@ -424,42 +457,25 @@ __global__ void __launch_bounds__(256, kMinBlocks)
     // bytes go to the other buffer)
     if (more) store_info(nxt, (i + 1) & 1);
 
-    // ---- values: warp w owns d in [16 w, 16 w + 16), words wi = 2 w, 2 w + 1
-    // of each code row. MMA jm, column n: d = 8 (2 w + (n >> 2)) + (n & 3) + 4 jm.
+    // ---- values: warp w owns d in [16 w, 16 w + 16); MMA jm, column n:
+    // d = 16 w + 8 jm + n
     int vacc[2][4], zacc[4];
 #pragma unroll
     for (int r = 0; r < 4; ++r) vacc[0][r] = vacc[1][r] = zacc[r] = 0;
     {
-      const uint8_t* vc = kc + voff;
-      const int q = g & 3;
-      const int sh = 4 * (q & 1);
-      // byte (q >> 1) of two rows into bytes 0, 1 (jm = 0); byte 2 + (q >> 1) (jm = 1)
-      const uint32_t sel0 = (uint32_t)((q >> 1) | ((4 + (q >> 1)) << 4));
-      const uint32_t sel1 = sel0 + 0x22u;
-      const uint32_t* arow0 = reinterpret_cast<const uint32_t*>(bd + g * kBdStride + 4 * t4);
-      const uint32_t* arow1 = reinterpret_cast<const uint32_t*>(bd + (g + 8) * kBdStride + 4 * t4);
-      const uint32_t* zw = reinterpret_cast<const uint32_t*>(zvb + (i & 1) * kT + 4 * t4);
+      const uint8_t* zb = zvb + (i & 1) * kT + 8 * t4;
 #pragma unroll
       for (int ks = 0; ks < kT / 32; ++ks) {
-        const uint32_t a0 = g < RC ? arow0[8 * ks] : 0u;
-        const uint32_t a1 = g + 8 < RC ? arow1[8 * ks] : 0u;
-        const uint32_t a2 = g < RC ? arow0[8 * ks + 4] : 0u;
-        const uint32_t a3 = g + 8 < RC ? arow1[8 * ks + 4] : 0u;
-        uint32_t bb[2][2];  // [jm][key half]
+        uint32_t af[4];
+        ldsm_x4(af, arow + 32 * ks);
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          uint32_t rw[4];
-#pragma unroll
-          for (int ii = 0; ii < 4; ++ii)
-            rw[ii] = *reinterpret_cast<const uint32_t*>(vc + (32 * ks + 8 * ii + hb) * kRowBytes);
-          const uint32_t x0 = prmt(rw[0], rw[1], sel0), y0v = prmt(rw[2], rw[3], sel0);
-          const uint32_t x1 = prmt(rw[0], rw[1], sel1), y1v = prmt(rw[2], rw[3], sel1);
-          bb[0][hb] = (prmt(x0, y0v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
-          bb[1][hb] = (prmt(x1, y1v, 0x5410u) >> sh) & 0x0F0F0F0Fu;
+        for (int jm = 0; jm < 2; ++jm) {
+          const uint32_t w =
+              *reinterpret_cast<const uint32_t*>(kc + voff[jm] + 4 * (4 * ks * kVRowWords));
+          mma_s8u8(vacc[jm], af[0], af[1], af[2], af[3], w & 0x0F0F0F0Fu, (w >> 4) & 0x0F0F0F0Fu);
         }
-        mma_s8u8(vacc[0], a0, a1, a2, a3, bb[0][0], bb[0][1]);
-        mma_s8u8(vacc[1], a0, a1, a2, a3, bb[1][0], bb[1][1]);
-        mma_s8u8(zacc, a0, a1, a2, a3, zw[8 * ks], zw[8 * ks + 4]);
+        const uint2 z = *reinterpret_cast<const uint2*>(zb + 32 * ks);
+        mma_s8u8(zacc, af[0], af[1], af[2], af[3], z.x, z.y);
       }
     }
     // O = O alpha + beta tau_c (acc - zt) for the lane's rows g and g + 8
@@ -484,7 +500,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
   const int64_t base = (((int64_t)b * p.Hkv + kh) * p.nsplit + split) * R;
 #pragma unroll
   for (int jm = 0; jm < 2; ++jm) {
-    const int d = 8 * (2 * warp + (t4 >> 1)) + 2 * (t4 & 1) + 4 * jm;  // columns 2 t4, 2 t4 + 1
+    const int d = 16 * warp + 8 * jm + 2 * t4;  // columns 2 t4, 2 t4 + 1
 #pragma unroll
     for (int rh = 0; rh < 2; ++rh) {
       const int row = g + 8 * rh;
@@ -521,6 +537,31 @@ __global__ void __launch_bounds__(kD) kv_msd_merge_kernel(KvArgs p, uint16_t* __
     den = fmaf(f, p.stat[ri * 2 + 1], den);
   }
   out[(int64_t)bh * kD + d] = bf16_bits(num / den);
+}
+
+// V codes from the token layout (uint32 [rows * L, D / 8], element d in
+// nibble d % 8 of word d / 8) to blocks of 8 tokens (uint32 [rows, nblk, D],
+// token 8 j + t in nibble t of word (j, d), tokens past L zero): one thread
+// per output word.
+__global__ void __launch_bounds__(256) kv_block_values_kernel(const uint32_t* __restrict__ in,
+                                                              int64_t rows, int L, int D,
+                                                              int nblk,
+                                                              uint32_t* __restrict__ out) {
+  const int64_t total = rows * nblk * D;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int d = (int)(idx % D);
+    const int64_t rb = idx / D;  // row * nblk + block
+    const int blk = (int)(rb % nblk);
+    const int64_t row = rb / nblk;
+    uint32_t w = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int l = 8 * blk + t;
+      if (l < L) w |= ((in[(row * L + l) * (D / 8) + d / 8] >> (4 * (d % 8))) & 15u) << (4 * t);
+    }
+    out[idx] = w;
+  }
 }
 
 template <int R, int C>
@@ -580,6 +621,15 @@ size_t kv_msd_workspace_bytes(int64_t B, int64_t Hq, int64_t L, int32_t C) {
   return dig + sc + (size_t)B * Hq * nch * (kD + 2) * 4;
 }
 
+wq_status launch_kv_block_values(const uint32_t* codes, int64_t rows, int64_t L, int32_t D,
+                                 uint32_t* out, cudaStream_t st) {
+  const int nblk = (int)((L + 7) / 8);
+  const int64_t total = rows * nblk * D;
+  const int64_t grid = std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 16);
+  kv_block_values_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, rows, (int)L, D, nblk, out);
+  return launch_status();
+}
+
 wq_status launch_kv_msd(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64_t L, int32_t C,
                         const void* kq, const void* ks, const void* kz, const void* vq,
                         const void* vs, const void* vz, void* out, void* workspace,
@@ -598,6 +648,7 @@ wq_status launch_kv_msd(const void* q, int64_t B, int64_t Hq, int64_t Hkv, int64
   a.qs = qs;
   a.kq = static_cast<const uint8_t*>(kq);
   a.vq = static_cast<const uint8_t*>(vq);
+  a.nblk = (int)((L + 7) / 8);
   a.ks = static_cast<const __half*>(ks);
   a.kz = static_cast<const __half*>(kz);
   a.vs = static_cast<const __half*>(vs);

@@ -376,11 +376,14 @@ wq_status wq_mx_gemv(const void* x, int64_t M, int64_t N, int64_t K, int32_t n_p
  *   q        bf16 [B, Hq, D] (device); Hq = R * Hkv, query head h reads KV
  *            head h / R (grouped heads), R in {1, 2, 4, 8}; D == 128;
  *   K and V  each INT4 asymmetric with one group per (sequence, head, token)
- *            row, the layout of wq_quantize_pack(WQ_FMT_INT4_ASYM, group = D)
- *            applied to the [B * Hkv * L, D] rows: codes uint32
- *            [B, Hkv, L, D/8] (element d in nibble d % 8 of word d / 8, low
- *            nibble first), scales fp16 [B, Hkv, L], zeros fp16 [B, Hkv, L]
- *            holding integers 0..15;
+ *            row, as wq_quantize_pack(WQ_FMT_INT4_ASYM, group = D) computes it
+ *            for the [B * Hkv * L, D] rows: scales fp16 [B, Hkv, L], zeros
+ *            fp16 [B, Hkv, L] holding integers 0..15, and
+ *            K codes uint32 [B, Hkv, L, D/8], that call's layout (element d in
+ *            nibble d % 8 of word d / 8);
+ *            V codes uint32 [B, Hkv, ceil(L/8), D], blocks of 8 tokens (token
+ *            8 j + t of dimension d in nibble t of word (j, d), tokens past L
+ *            zero), which wq_kv_block_values makes from that call's layout;
  *   out      bf16 [B, Hq, D] = softmax(q . k^T / sqrt(D)) . v over the L
  *            cached tokens, computed as follows (the page gives no formulas;
  *            this is the library's reading):
@@ -408,6 +411,20 @@ wq_status wq_msd_decode_attention(const void* q, int64_t B, int64_t Hq, int64_t 
                                   const void* k_scales, const void* k_zeros, const void* v_codes,
                                   const void* v_scales, const void* v_zeros, void* out,
                                   void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The value-cache layout of wq_msd_decode_attention: V codes from the token
+ * layout of wq_quantize_pack (uint32 [rows * L, D / 8], element d in nibble
+ * d % 8 of word d / 8) to blocks of 8 tokens, out uint32 [rows, ceil(L/8), D]
+ * (token 8 j + t of dimension d in nibble t of word (j, d); nibbles of tokens
+ * past L are 0). rows is the number of (sequence, head) pairs. One word then
+ * holds 4 tokens of one dimension in its low nibbles and 4 in its high
+ * nibbles, the operand layout of the attention's value product. rows == 0 is
+ * a no-op; L <= 0 or D not a positive multiple of 8 return
+ * WQ_ERR_INVALID_ARG. Bit-exact rearrangement; asynchronous on `stream`.
+ */
+wq_status wq_kv_block_values(const uint32_t* codes, int64_t rows, int64_t L, int32_t D,
+                             uint32_t* out, void* stream);
 
 /*
  * Workspace bytes of wq_msd_decode_attention (0 for B == 0); the same shape

@@ -268,3 +268,14 @@ def test_attention_split_hook_validation(wq):
     assert wq.lib.wq_test_set_attention_split(65) == wq.WQ_ERR_INVALID_ARG
     assert wq.lib.wq_test_set_attention_split(3) == wq.WQ_OK
     assert wq.lib.wq_test_set_attention_split(0) == wq.WQ_OK
+
+
+def test_kv_block_values_validation(wq):
+    g = wq.lib.wq_kv_block_values
+    # (codes, rows, L, D, out, stream)
+    assert g(A16, -1, 8, 128, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 0, 128, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 8, 100, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(None, 4, 8, 128, A16, None) == wq.WQ_ERR_INVALID_ARG
+    assert g(A16, 4, 8, 128, MIS, None) == wq.WQ_ERR_ALIGNMENT
+    assert g(None, 0, 8, 128, None, None) == wq.WQ_OK

@@ -54,26 +54,49 @@ def _check(out_gpu, ref, v_deq, eps, what):
 
 
 def _run(wq, q, k, v, c):
-    kc = wq.kv_quantize(k.cuda())
-    vc = wq.kv_quantize(v.cuda())
+    kc = wq.kv_quantize_keys(k.cuda())
+    vc = wq.kv_quantize_values(v.cuda())
     out = wq.wq_msd_decode_attention(q.cuda(), kc, vc, n_components=c)
     torch.cuda.synchronize()
     return out, kc, vc
 
 
-def test_kv_quantize_bit_exact(wq):
-    q, k, v = _inputs(2, 8, 2, 300, seed=1)
-    codes, s, z = _oracle_cache(k)
-    qw, sc, zr = wq.kv_quantize(k.cuda())
-    torch.cuda.synchronize()
-    got = qw.cpu().numpy().view(np.uint32)
-    want = np.zeros(got.shape, dtype=np.uint32)
+def _pack_rows(codes):
+    """Oracle codes [..., L, D] -> uint32 words [..., L, D/8], element d in
+    nibble d % 8 of word d / 8 (a plain rearrangement)."""
     c8 = codes.reshape(*codes.shape[:-1], -1, 8).astype(np.uint32)
+    out = np.zeros(c8.shape[:-1], dtype=np.uint32)
     for i in range(8):
-        want |= c8[..., i] << (4 * i)
-    assert np.array_equal(got, want)
-    assert np.array_equal(sc.cpu().numpy().view(np.uint16), s.view(np.uint16))
-    assert np.array_equal(zr.cpu().numpy().view(np.uint16), z.view(np.uint16))
+        out |= c8[..., i] << (4 * i)
+    return out
+
+
+def _pack_blocks(codes):
+    """Oracle codes [B, H, L, D] -> uint32 words [B, H, ceil(L/8), D], token
+    8 j + t in nibble t of word (j, d), tokens past L zero."""
+    b, h, length, d = codes.shape
+    nblk = (length + 7) // 8
+    padded = np.zeros((b, h, nblk * 8, d), dtype=np.uint32)
+    padded[:, :, :length] = codes
+    blk = padded.reshape(b, h, nblk, 8, d)
+    out = np.zeros((b, h, nblk, d), dtype=np.uint32)
+    for t in range(8):
+        out |= blk[:, :, :, t, :] << (4 * t)
+    return out
+
+
+@pytest.mark.parametrize("length", [300, 17, 1, 256])
+def test_kv_quantize_bit_exact(wq, length):
+    q, k, v = _inputs(2, 8, 2, length, seed=length)
+    ck, sk, zk = _oracle_cache(k)
+    cv, sv, zv = _oracle_cache(v)
+    kq, ks, kz = wq.kv_quantize_keys(k.cuda())
+    vq, vs, vz = wq.kv_quantize_values(v.cuda())
+    torch.cuda.synchronize()
+    assert np.array_equal(kq.cpu().numpy().view(np.uint32), _pack_rows(ck))
+    assert np.array_equal(vq.cpu().numpy().view(np.uint32), _pack_blocks(cv))
+    for got, want in ((ks, sk), (kz, zk), (vs, sv), (vz, zv)):
+        assert np.array_equal(got.cpu().numpy().view(np.uint16), want.view(np.uint16))
 
 
 # (B, Hq, Hkv, L): several 256-key chunks with a ragged tail, a single partial
@@ -172,15 +195,16 @@ def test_bench_shape_sampled(wq):
 def test_rejections(wq):
     dev = "cuda"
     q = torch.zeros(1, 8, 128, dtype=torch.bfloat16, device=dev)
-    kc = wq.kv_quantize(torch.zeros(1, 2, 4, 128, device=dev))
+    kc = wq.kv_quantize_keys(torch.zeros(1, 2, 4, 128, device=dev))
+    vc = wq.kv_quantize_values(torch.zeros(1, 2, 4, 128, device=dev))
     with pytest.raises(wq.WqError) as e:      # R = 3
         wq.wq_msd_decode_attention(torch.zeros(1, 6, 128, dtype=torch.bfloat16, device=dev),
-                                   kc, kc)
+                                   kc, vc)
     assert e.value.status == wq.WQ_ERR_UNSUPPORTED
     with pytest.raises(wq.WqError) as e:      # three components
-        wq.wq_msd_decode_attention(q, kc, kc, n_components=3)
+        wq.wq_msd_decode_attention(q, kc, vc, n_components=3)
     assert e.value.status == wq.WQ_ERR_UNSUPPORTED
     ws = torch.empty(16, dtype=torch.uint8, device=dev)
     with pytest.raises(wq.WqError) as e:
-        wq.wq_msd_decode_attention(q, kc, kc, workspace=ws)
+        wq.wq_msd_decode_attention(q, kc, vc, workspace=ws)
     assert e.value.status == wq.WQ_ERR_WORKSPACE

@@ -1090,7 +1090,7 @@ def max_over_ranks(v, world, device):
 
 
 PROFILE_CASES = ("nf4", "gemv_int4", "gemv_int4_m1", "gemv_nf4", "gemm", "msd", "msd_m16",
-                 "decdec", "mx_m16")
+                 "decdec", "mx_m16", "nf4_msd_m16", "kv_attn")
 
 
 def profile_case(case, device):
@@ -1139,6 +1139,22 @@ def profile_case(case, device):
         y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
         ws = wq.mx_workspace(m, n, k, 2, device)
         fn = lambda: wq.wq_mx_gemv(x, n, 2, codes, scales, workspace=ws, out=y)  # noqa: E731
+    elif case == "nf4_msd_m16":
+        m, (n, k) = 16, MSD_SHAPE
+        codes, absmax, _ = wq.wq_quantize_pack(wq.WQ_FMT_NF4, normal(n, k, std=0.02), 64)
+        x = normal(m, k).to(torch.bfloat16)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+        ws = wq.msd_workspace(m, n, k, 64, 2, device)
+        fn = lambda: wq.wq_msd_gemm_nf4(x, n, 2, codes, absmax, workspace=ws, out=y)  # noqa
+    elif case == "kv_attn":
+        # decode attention over an INT4 KV cache, Qwen3-32B heads, B = 32 x 8192 tokens
+        b, length, hq, hkv, d = 32, 8192, 64, 8, 128
+        kc = wq.kv_quantize_keys(normal(b, hkv, length, d, std=0.5))
+        vc = wq.kv_quantize_values(normal(b, hkv, length, d))
+        q = normal(b, hq, d).to(torch.bfloat16)
+        o = torch.empty(b, hq, d, dtype=torch.bfloat16, device=device)
+        ws = wq.attention_workspace(b, hq, hkv, length, d, 2, device)
+        fn = lambda: wq.wq_msd_decode_attention(q, kc, vc, 2, workspace=ws, out=o)  # noqa
     elif case == "decdec":
         # select, then the corrected GEMV (ncu -k regex:gemv_kernel captures it)
         (n, k), m = DECDEC_SHAPE, 1

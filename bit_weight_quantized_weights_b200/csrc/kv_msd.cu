@@ -100,6 +100,11 @@ __device__ __forceinline__ int zv_pos(int kk) {
   return (kk & ~31) + 8 * ((kk >> 3) & 3) + 4 * (kk & 1) + ((kk >> 1) & 3);
 }
 
+// Slot of key kk in the per-key table (float4): bits 1-2 of kk XOR-ed with
+// bits 3-4, so the four lanes t4 of a lane group, whose keys are 8 apart,
+// read distinct banks.
+__device__ __forceinline__ int ki_pos(int kk) { return kk ^ (((kk >> 3) & 3) << 1); }
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -222,7 +227,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
     }
   };
   auto store_info = [&](const __half (&h)[4], int buf) {
-    ki[tid] = make_float4(__half2float(h[0]), __int_as_float((int)__half2float(h[1])),
+    ki[ki_pos(tid)] = make_float4(__half2float(h[0]), __int_as_float((int)__half2float(h[1])),
                           __half2float(h[2]), 0.0f);
     zvb[buf * kT + zv_pos(tid)] = (uint8_t)__half2float(h[3]);
   };
@@ -305,7 +310,9 @@ __global__ void __launch_bounds__(256, kMinBlocks)
 #pragma unroll
   for (int jm = 0; jm < 2; ++jm)
     voff[jm] = kT * kRowBytes + 4 * (t4 * kVRowWords + ((16 * warp + 8 * jm + g) ^ (8 * t4)));
-  const float4* kinf = ki + 32 * warp + 8 * t4;  // the lane's keys: + 2 nt + e
+  // the lane's keys 32 w + 8 t4 + 2 nt + e sit at slots 32 w + 8 t4 +
+  // 2 (nt ^ t4) + e
+  const float4* kinf = ki + 32 * warp + 8 * t4;
   // ldmatrix row addresses of the value digit rows (A): lanes 0-7 rows 0-7,
   // 8-15 rows 8-15, at k bytes 0-15; lanes 16-31 the same rows at 16-31
   const int8_t* arow = bd + ((lane & 7) + 8 * ((lane >> 3) & 1)) * kBdStride + 16 * (lane >> 4);
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(256, kMinBlocks)
         } else {
           dint = sacc[nt][e];
         }
-        const float4 inf = kinf[2 * nt + e];
+        const float4 inf = kinf[2 * (nt ^ t4) + e];
         dint -= __float_as_int(inf.y) * qsc;
         const float s = (float)dint * (inf.x * cs);
         sc[nt][e] = hv ? s : -INFINITY;
@@ -373,20 +380,20 @@ __global__ void __launch_bounds__(256, kMinBlocks)
     for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][0], sc[nt][1]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    if (t4 == 0 && hv) redm[warp * 8 + hl] = mx;
-    __syncthreads();
-    float m = -INFINITY;
-    if (hv)
-#pragma unroll
-      for (int w = 0; w < 8; ++w) m = fmaxf(m, redm[w * 8 + hl]);
+    // Softmax statistics in one cross-warp step: each warp exponentiates
+    // against its own maximum m_w; with M the chunk's maximum and
+    // f_w = 2^(m_w - M), E = sum_w f_w E_w, amax = max_w f_w amax_w, and a
+    // key's weight is f_own 2^(s - m_w) sv. (Rounding is monotonic, so no
+    // weight exceeds the amax computed this way.)
     float wv[4][2], es = 0.0f, am = 0.0f;
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float ex = hv ? exp2_approx(sc[nt][e] - m) : 0.0f;  // sc = -inf: 0
+        // sc = -inf: 0; a warp whose keys are all past the end (mx = -inf): 0
+        const float ex = (hv && mx != -INFINITY) ? exp2_approx(sc[nt][e] - mx) : 0.0f;
         es += ex;
-        wv[nt][e] = ex * kinf[2 * nt + e].z;  // >= 0: sv > 0
+        wv[nt][e] = ex * kinf[2 * (nt ^ t4) + e].z;  // >= 0: sv > 0
         am = fmaxf(am, wv[nt][e]);
       }
 #pragma unroll
@@ -395,17 +402,27 @@ __global__ void __launch_bounds__(256, kMinBlocks)
       am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
     }
     if (t4 == 0 && hv) {
+      redm[warp * 8 + hl] = mx;
       rede[warp * 8 + hl] = es;
       reda[warp * 8 + hl] = am;
     }
     __syncthreads();
-    float E = 0.0f, A = 0.0f;
-    if (hv)
+    float m = -INFINITY, E = 0.0f, A = 0.0f, fown = 0.0f;
+    if (hv) {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) m = fmaxf(m, redm[w * 8 + hl]);
 #pragma unroll
       for (int w = 0; w < 8; ++w) {
-        E += rede[w * 8 + hl];
-        A = fmaxf(A, reda[w * 8 + hl]);
+        const float f = exp2_approx(redm[w * 8 + hl] - m);  // a warp without keys: 0
+        E = fmaf(f, rede[w * 8 + hl], E);
+        A = fmaxf(A, f * reda[w * 8 + hl]);
       }
+      fown = exp2_approx(mx - m);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) wv[nt][e] *= fown;
     // The decomposition of w over the chunk's keys, as for an activation row:
     // s_1 = amax / 127, s_{c+1} = s_c / 256, digit rint(r / s_c) (the first
     // clamped to +-127), residual r - s_c a_c rounded once, and a digit of

@@ -41,6 +41,8 @@
 // fp16 scale rounds once (2^-12 relative, against 2^-9 for a bf16 weight).
 // Within every 8-element chunk of k both operands use the order
 // k0 k4 k1 k5 k2 k6 k3 k7 (the order one packed word dequantizes into).
+#include <algorithm>
+
 #include "sm100.cuh"
 
 namespace wq {
@@ -778,6 +780,412 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   sm100::cluster_sync();
 }
 
+// Persistent CTA-pair kernel (INT4, 128-wide k stages, G a multiple of 128).
+// The pair kernel above pays, for every 256 x 256 tile, its prologue, the
+// fill of its stage ring and its epilogue one after the other; here each pair
+// of CTAs loops over the tiles t = pair, pair + pairs, ... (features fastest),
+// and the producer, the MMA issuer and the dequantization warps run one
+// flattened sequence of (tile, k-tile) steps, so the ring's phases continue
+// from tile to tile and the next tile's loads and dequantization overlap the
+// current tile's epilogue. Sixteen epilogue warps of their own drain each tile
+// (four per TMEM lane quarter, 64 token columns each, so the accumulator is
+// free again after two TMEM loads per thread):
+//   accf       (both CTAs) the tile's MMAs completed (one phase per tile)
+//   acc_empty  (even CTA's) both CTAs' epilogue warps read the accumulator:
+//              the tile after may start its MMAs (one phase per tile)
+// The staging tile of the output has its own 64 KB (the ring is busy with the
+// next tile). The other barriers are those of the pair kernel.
+struct Gemm2PCfg {
+  static constexpr int KB = 128;
+  static constexpr int BT = 256;                  // tokens per pair tile (MMA N)
+  static constexpr int kACols = KB / 2;           // TMEM columns of one A stage
+  static constexpr int kStages = 4;
+  static constexpr int kXBytes = 128 * KB * 2;    // this CTA's x half: 32 KB
+  static constexpr int kWBytes = BW * KB / 2;     // 8 KB
+  static constexpr int kStageBytes = kXBytes + kWBytes;
+  static constexpr int kRing = kStages * kStageBytes;
+  static constexpr int kOutBytes = BT * BW * 2;   // [BT tokens][BW rows] bf16
+  static constexpr int kEpiWarps = 16;            // four per TMEM lane quarter, 64 columns each
+  static constexpr int kEpiFirst = 64 + 32 * kDeqWarps;  // first epilogue thread
+  static constexpr int kThreads = kEpiFirst + 32 * kEpiWarps;
+  static constexpr int kSmem = kRing + kOutBytes + BT * 4 + 512 + 1024;
+  static constexpr uint32_t kAccCols = BT;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kAccCols + kStages * kACols <= kTmemCols, "A stages fit in TMEM");
+  static_assert(kSmem <= 232448, "shared memory");
+  static_assert(kStageBytes % 1024 == 0, "stages stay 1024-byte aligned for the swizzle");
+};
+
+__global__ void __launch_bounds__(Gemm2PCfg::kThreads, 1)
+    w4a16_gemm_pair_persistent_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                                      const __grid_constant__ CUtensorMap tmap_w,
+                                      const __grid_constant__ CUtensorMap tmap_y,
+                                      const __half* __restrict__ scales,
+                                      const __half* __restrict__ zeros,
+                                      const float* __restrict__ inv_scale, int M, int N, int K,
+                                      int G, WaitCtl wc) {
+  using C = Gemm2PCfg;
+  constexpr int BT = C::BT, ST = C::kStages, KB = C::KB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint16_t* out_s = reinterpret_cast<uint16_t*>(smem + C::kRing);          // [BT][BW] bf16
+  float* s_inv = reinterpret_cast<float*>(smem + C::kRing + C::kOutBytes);  // [BT]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(s_inv + BT);
+  uint64_t* xfull = bars;
+  uint64_t* wfull = bars + ST;
+  uint64_t* done = bars + 2 * ST;
+  uint64_t* aready = bars + 3 * ST;
+  uint64_t* accf = bars + 4 * ST;
+  uint64_t* acc_empty = accf + 1;
+  uint64_t* mma_done = accf + 2;  // the MMA issuer's final commit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* peer_info = reinterpret_cast<volatile int*>(tmem_slot + 2);  // [2]
+  volatile int* epi_ok = reinterpret_cast<volatile int*>(tmem_slot + 4);     // [kEpiWarps]
+  static_assert(4 * (4 + Gemm2PCfg::kEpiWarps) + 8 * (4 * Gemm2PCfg::kStages + 3) <= 512,
+                "barriers and flags fit their 512 bytes");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = sm100::cluster_ctarank();  // 0: issues the MMAs
+  const bool leader = rank == 0;
+  const int npairs = (int)(gridDim.x >> 1);
+  const int pair = (int)(blockIdx.x >> 1);
+  const int ntn = N / (2 * BW);  // pair tiles along the features
+  const int ntiles = ntn * ((M + BT - 1) / BT);
+  const int nlocal = pair < ntiles ? (ntiles - pair + npairs - 1) / npairs : 0;
+  const int KT = K / KB;
+  const int total = nlocal * KT;  // this pair's (tile, k-tile) steps
+  auto tile_of = [&](int j) { return pair + j * npairs; };
+  auto n0_of = [&](int t) { return (t % ntn) * (2 * BW) + BW * (int)rank; };
+  auto m0_of = [&](int t) { return (t / ntn) * BT; };
+
+  if (threadIdx.x == 0) {
+    sm100::tma_prefetch_desc(&tmap_x);
+    sm100::tma_prefetch_desc(&tmap_w);
+    sm100::tma_prefetch_desc(&tmap_y);
+    for (int s = 0; s < ST; ++s) {
+      sm100::mbar_init(&xfull[s], 1);
+      sm100::mbar_init(&wfull[s], 1);
+      sm100::mbar_init(&done[s], 1);
+      sm100::mbar_init(&aready[s], 2 * kDeqWarps);
+    }
+    sm100::mbar_init(accf, 1);
+    sm100::mbar_init(acc_empty, 2 * C::kEpiWarps);
+    sm100::mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  if (warp == 1) {
+    sm100::tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    sm100::tmem_relinquish_pair();
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::cluster_sync();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  int last_issued = -1;  // producer: the last step whose loads it issued
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      // (k-tile, tile and its coordinates advance incrementally: no division per step)
+      int kt = 0, j = 0, n0 = n0_of(tile_of(0)), m0 = m0_of(tile_of(0));
+      for (int it = 0; it < total; ++it, ++kt) {
+        if (kt == KT) {
+          kt = 0;
+          ++j;
+          n0 = n0_of(tile_of(j));
+          m0 = m0_of(tile_of(j));
+        }
+        const int s = it % ST;
+        const uint32_t ph = (uint32_t)(it / ST) & 1u;
+        if (it >= ST && !sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x511u, abort_flag,
+                                          wc.limit_ns))
+          break;
+        if (wc.stall && it == 0) continue;  // test hook: the first step never arrives
+        last_issued = it;
+        uint8_t* st = ring + s * C::kStageBytes;
+        sm100::mbar_arrive_expect_tx(&wfull[s], C::kWBytes);
+        sm100::tma_load_2d(st + C::kXBytes, &tmap_w, &wfull[s], kt * (KB / 8), n0);
+        if (leader) sm100::mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
+#pragma unroll
+        for (int blk = 0; blk < KB / 64; ++blk)
+          sm100::tma_load_2d_pair(st + blk * (128 * 64 * 2), &tmap_x,
+                                  sm100::cluster_addr(&xfull[s], 0), kt * KB + 64 * blk,
+                                  m0 + 128 * (int)rank);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- pair MMA issuer (even CTA) ----------------
+      constexpr uint32_t idesc = sm100::idesc_f16_f32(2 * BW, BT);
+      int kt = 0, j = 0;
+      for (int it = 0; it < total; ++it, ++kt) {
+        if (kt == KT) {
+          kt = 0;
+          ++j;
+        }
+        const int s = it % ST;
+        const uint32_t ph = (uint32_t)(it / ST) & 1u;
+        if (kt == 0 && j > 0) {
+          // both CTAs' epilogues have read the previous tile's accumulator
+          if (!sm100::mbar_wait(acc_empty, (uint32_t)(j - 1) & 1u, &g_gemm_error, 0x521u,
+                                abort_flag, wc.limit_ns))
+            break;
+          sm100::tc_fence_after();
+        }
+        if (!sm100::mbar_wait(&xfull[s], ph, &g_gemm_error, 0x522u, abort_flag, wc.limit_ns)) break;
+        if (!sm100::mbar_wait(&aready[s], ph, &g_gemm_error, 0x523u, abort_flag, wc.limit_ns)) break;
+        sm100::tc_fence_after();
+        const uint32_t x_base = smem_u32(ring + s * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < KB / 16; ++kk) {
+          const uint64_t bd =
+              sm100::sdesc_sw128_kmajor(x_base + (kk / 4) * (128 * 64 * 2) + (kk % 4) * 32);
+          const uint32_t at = tmem + C::kAccCols + (uint32_t)(s * C::kACols + kk * 8);
+          sm100::mma_f16_tmem_a_pair(tmem, at, bd, idesc, (kt | kk) != 0 ? 1u : 0u);
+        }
+        sm100::mma_commit_pair(&done[s], 0x3);
+        if (kt == KT - 1) sm100::mma_commit_pair(accf, 0x3);
+      }
+      sm100::mma_commit_pair(mma_done, 0x3);
+    }
+  } else if (warp < 2 + kDeqWarps) {
+    // ---------------- dequantize (warps 2..9) ----------------
+    const int dq = warp - 2;
+    const int q = warp & 3;
+    const int hk = dq >> 2;  // which 64-k half of each k-tile
+    const int r = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int ng = K / G;
+    const int tpg = G / KB;  // k-tiles per group
+    // group parameters of row n, group g
+    auto load_prm = [&](int n, int g, __half& sv, __half& zv) {
+      const int64_t idx = (int64_t)n * ng + g;
+      sv = scales[idx];
+      zv = zeros[idx];
+    };
+    // the step's k-tile, its group and k-tile within the group, and this
+    // thread's weight row in the step's tile and in the next tile advance
+    // incrementally (no division per step); a group's parameters are loaded
+    // one group ahead
+    int kt = 0, j = 0, gi = 0, gk = 0;
+    int nrow = n0_of(tile_of(0)) + r;
+    int nrow_next = nlocal > 1 ? n0_of(tile_of(1)) + r : nrow;
+    __half s_next = __ushort_as_half(0), z_next = __ushort_as_half(0);
+    if (total > 0) load_prm(nrow, 0, s_next, z_next);
+    uint32_t zb_hi = 0, zb_lo = 0, s2 = 0;
+    for (int it = 0; it < total; ++it) {
+      const int s = it % ST;
+      const uint32_t ph = (uint32_t)(it / ST) & 1u;
+      if (gk == 0) {
+        // a group starts: its parameters were loaded a group ahead
+        const uint32_t sb = __half_as_ushort(s_next);
+        const uint32_t zq = (uint32_t)__half2float(z_next);
+        s2 = sb | (sb << 16);
+        zb_hi = (0x6400u | zq) * 0x00010001u;
+        zb_lo = (0x5400u | (zq << 4)) * 0x00010001u;
+        if (kt + tpg < KT)
+          load_prm(nrow, gi + 1, s_next, z_next);
+        else if (j + 1 < nlocal)
+          load_prm(nrow_next, 0, s_next, z_next);
+      }
+      // the weight tile landed; A stage s is free once the MMAs of step it - ST completed
+      bool got = sm100::mbar_wait(&wfull[s], ph, &g_gemm_error, 0x531u, abort_flag, wc.limit_ns);
+      if (got && it >= ST)
+        got = sm100::mbar_wait(&done[s], ph ^ 1u, &g_gemm_error, 0x532u, abort_flag, wc.limit_ns);
+      if (!__all_sync(0xffffffffu, got)) break;
+      // the packed tile arrives in the TMA 64-byte swizzle: 16-byte chunk c of
+      // row r at chunk c ^ ((r >> 1) & 3), so a warp's 16-byte reads (rows
+      // 64 bytes apart) spread over every bank
+      const uint8_t* wrow = ring + s * C::kStageBytes + C::kXBytes + r * (KB / 2);
+#pragma unroll
+      for (int h16 = 0; h16 < KB / 64; ++h16) {
+        const uint4 wv = *reinterpret_cast<const uint4*>(
+            wrow + (((2 * hk + h16) ^ ((r >> 1) & 3)) << 4));
+        uint32_t cols[16];
+        dequant_word(wv.x, zb_hi, zb_lo, s2, cols + 0);
+        dequant_word(wv.y, zb_hi, zb_lo, s2, cols + 4);
+        dequant_word(wv.z, zb_hi, zb_lo, s2, cols + 8);
+        dequant_word(wv.w, zb_hi, zb_lo, s2, cols + 12);
+        sm100::tmem_st16(tmem + lane_base + C::kAccCols +
+                             (uint32_t)(s * C::kACols + hk * (KB / 4) + h16 * 16),
+                         cols);
+      }
+      sm100::tmem_st_wait();
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          sm100::mbar_arrive(&aready[s]);
+        else
+          sm100::mbar_arrive_cluster(sm100::cluster_addr(&aready[s], 0));
+      }
+      if (++gk == tpg) {
+        gk = 0;
+        ++gi;
+      }
+      if (++kt == KT) {
+        kt = 0;
+        gi = 0;
+        gk = 0;
+        ++j;
+        nrow = nrow_next;
+        if (j + 1 < nlocal) nrow_next = n0_of(tile_of(j + 1)) + r;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 10..25): one tile at a time ----------------
+    const int eq = warp - (2 + kDeqWarps);  // 0 .. 15
+    const int q = warp & 3;                 // TMEM lane quarter
+    const int cbase = 64 * (eq >> 2);       // this warp's 64 token columns
+    const int r = 32 * q + lane;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const int e = (int)threadIdx.x - C::kEpiFirst;  // 0 .. 511
+    constexpr uint32_t kEpiThreads = 32 * C::kEpiWarps;
+    for (int j = 0; j < nlocal; ++j) {
+      const int t = tile_of(j);
+      const int m0 = m0_of(t);
+      // (a tile's mainloop is long: poll with a backoff, off the issue slots
+      // of the dequantization warps and the MMA issuer)
+      bool got = sm100::mbar_wait_sleep(accf, (uint32_t)j & 1u, &g_gemm_error, 0x541u,
+                                        abort_flag, wc.limit_ns, 256);
+      got = __all_sync(0xffffffffu, got);
+      // the epilogue warps decide together whether to go on
+      if (lane == 0) epi_ok[eq] = got ? 1 : 0;
+      sm100::named_barrier(3, kEpiThreads);
+      bool go = true;
+#pragma unroll
+      for (int w = 0; w < C::kEpiWarps; ++w) go = go && epi_ok[w] != 0;
+      // the previous tile's store has read the staging tile
+      if (e == 0) sm100::bulk_wait_read_all();
+      sm100::named_barrier(3, kEpiThreads);
+      if (!go) break;
+      sm100::tc_fence_after();
+      for (int i = e; i < BT; i += (int)kEpiThreads)
+        s_inv[i] = (m0 + i < M) ? inv_scale[m0 + i] : 0.0f;
+      sm100::named_barrier(3, kEpiThreads);
+#pragma unroll
+      for (int c0 = cbase; c0 < cbase + 64; c0 += 32) {
+        uint32_t v[32];
+        sm100::tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
+        sm100::tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const float val = __uint_as_float(v[jj]) * s_inv[c0 + jj];
+          out_s[(c0 + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
+        }
+      }
+      // the accumulator is read: the next tile's MMAs may start
+      sm100::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          sm100::mbar_arrive(acc_empty);
+        else
+          sm100::mbar_arrive_cluster(sm100::cluster_addr(acc_empty, 0));
+      }
+      sm100::fence_proxy_async_smem();
+      sm100::named_barrier(3, kEpiThreads);
+      if (e == 0) {
+        sm100::tma_store_2d(&tmap_y, out_s, n0_of(t), m0);
+        sm100::bulk_commit();
+      }
+    }
+    if (e == 0) sm100::bulk_wait_all();
+  }
+
+  // neither CTA frees its TMEM or exits while the pair may still use it
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    const uint32_t peer = sm100::cluster_addr((const void*)peer_info, rank ^ 1u);
+    asm volatile("st.shared::cluster.v2.s32 [%0], {%1, %2};" ::"r"(peer), "r"(last_issued),
+                 "r"(*abort_flag)
+                 : "memory");
+  }
+  sm100::cluster_sync();
+  if (*abort_flag || peer_info[1]) {
+    // The drain after an abort, as in the pair kernel, over the steps of the
+    // flattened sequence: the producer that is behind issues its x half of
+    // the steps the other issued (the even CTA arming each first), then the
+    // even CTA waits for the last ST x phases, each producer for its own
+    // weight loads, and the MMA issuer for its final commit.
+    if (warp == 0 && lane == 0) {
+      const int other_last = peer_info[0];
+      for (int it = last_issued + 1; it <= other_last; ++it) {
+        if (wc.stall && it == 0) continue;
+        const int j = it / KT, kt = it - j * KT;
+        const int t = tile_of(j);
+        const int s = it % ST;
+        uint8_t* st = ring + s * C::kStageBytes;
+        if (leader) sm100::mbar_arrive_expect_tx(&xfull[s], 2 * C::kXBytes);
+#pragma unroll
+        for (int blk = 0; blk < KB / 64; ++blk)
+          sm100::tma_load_2d_pair(st + blk * (128 * 64 * 2), &tmap_x,
+                                  sm100::cluster_addr(&xfull[s], 0), kt * KB + 64 * blk,
+                                  m0_of(t) + 128 * (int)rank);
+      }
+      const int last_x = max(last_issued, other_last);
+      if (leader)
+        for (int it = max(0, last_x - ST + 1); it <= last_x; ++it)
+          if (!(wc.stall && it == 0))
+            sm100::mbar_wait_drain(&xfull[it % ST], (uint32_t)(it / ST) & 1u, wc.limit_ns);
+      for (int it = max(0, last_issued - ST + 1); it <= last_issued; ++it)
+        if (!(wc.stall && it == 0))
+          sm100::mbar_wait_drain(&wfull[it % ST], (uint32_t)(it / ST) & 1u, wc.limit_ns);
+    } else if (warp == 1 && lane == 0 && leader) {
+      sm100::mbar_wait_drain(mma_done, 0, wc.limit_ns);
+    }
+    sm100::cluster_sync();
+  }
+  if (warp == 1) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc_pair(tmem, C::kTmemCols);
+  }
+  sm100::cluster_sync();
+}
+
+wq_status launch_pair_persistent(const void* x16, const float* inv_scale, int64_t M, int64_t N,
+                                 int64_t K, int32_t G, const void* qweight, const void* scales,
+                                 const void* zeros, void* y, cudaStream_t st) {
+  using C = Gemm2PCfg;
+  CUtensorMap tx, tw, ty;
+  if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x16, (uint64_t)K, (uint64_t)M,
+                    (uint64_t)K * 2, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, qweight, (uint64_t)K / 8, (uint64_t)N,
+                    (uint64_t)K / 2, C::KB / 8, BW, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                    (uint64_t)N * 2, BW, C::BT, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return WQ_ERR_CUDA;
+  auto kern = w4a16_gemm_pair_persistent_kernel;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+      cudaSuccess)
+    return WQ_ERR_CUDA;
+  const int64_t ntiles = (N / (2 * BW)) * ((M + C::BT - 1) / C::BT);
+  const int64_t pairs = std::min<int64_t>(ntiles, num_sms() / 2);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tx, tw, ty, static_cast<const __half*>(scales),
+                         static_cast<const __half*>(zeros), inv_scale, (int)M, (int)N, (int)K,
+                         G, wait_ctl()) != cudaSuccess)
+    return WQ_ERR_CUDA;
+  return launch_status();
+}
+
 template <bool kNF4, int KB>
 wq_status launch_pair(const void* x16, const float* inv_scale, int64_t M, int64_t N, int64_t K,
                       int32_t G, const void* qweight, const void* scales, const void* zeros,
@@ -868,6 +1276,17 @@ bool gemm_pairs_enabled() {
   return on;
 }
 
+// The persistent pair kernel is the default where it applies (INT4, G a
+// multiple of 128, two or more tiles per pair); WQ_GEMM_PERSIST=0 in the
+// environment selects the per-tile pair kernel instead (for comparison).
+bool gemm_persistent_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("WQ_GEMM_PERSIST");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 bool gemm_kb128_enabled() {
   static const bool on = [] {
     const char* e = getenv("WQ_GEMM_KB");
@@ -909,6 +1328,10 @@ wq_status launch_gemm(const void* x, int64_t M, int64_t N, int64_t K, wq_format 
                ? launch_bt<128, true, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)
                : launch_bt<128, true, 64>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   }
+  // persistent pairs where every pair has at least two tiles to loop over
+  if (pair && K % 128 == 0 && G % 128 == 0 && gemm_persistent_enabled() &&
+      (N / (2 * BW)) * ((M + 255) / 256) >= 2 * (int64_t)(num_sms() / 2))
+    return launch_pair_persistent(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st);
   if (pair)
     return wide_k
                ? launch_pair<false, 128>(x16, inv_scale, M, N, K, G, qweight, scales, zeros, y, st)

@@ -74,6 +74,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
 }
 
+// mbar_wait for a waiter that expects a long wait (a whole tile): between
+// polls it sleeps `sleep_ns`, so that it takes no issue slots from the warps
+// doing the work it waits for.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                                uint32_t site, volatile int* abort,
+                                                uint64_t limit_ns, uint32_t sleep_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      atomicCAS(err, 0u, site);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // The drain after an abort: wait for the phase regardless of the abort flag,
 // still bounded by the limit (false if it expired).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
@@ -259,6 +279,10 @@ __device__ __forceinline__ void bulk_commit() {
 // Wait until the shared-memory sources of this thread's bulk stores have been read.
 __device__ __forceinline__ void bulk_wait_read_all() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's bulk stores have completed (their writes are done).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

@@ -42,6 +42,9 @@ def _x(m, k, seed):
     (600, 12928, 256, 128),   # single-CTA 256-token tiles (N not a multiple of 256)
     (520, 9472, 1024, 64),    # CTA pairs, the 8-stage ring wraps twice, ragged M
     (512, 18944, 512, 512),   # CTA pairs, per-group parameters across several k-tiles
+    # the persistent pair kernel (two or more 256 x 256 tiles per pair of CTAs):
+    (1100, 8192, 512, 128),   # ragged last token tile, several tiles per pair
+    (1024, 9472, 384, 384),   # per-channel groups (three k-tiles per group)
 ])
 def test_gemm_small_every_element(wq, m, n, k, group):
     q, s, z, qweight = helpers.int4_packed(n, k, group, seed=m)

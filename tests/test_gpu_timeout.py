@@ -8,7 +8,8 @@ kernel must then record the wait site in the library's error word
 its tensor memory and return, leaving the context usable: the next normal call
 in the same process must match the oracle. Small grids of each kernel with
 bounded waits: the single-CTA fused GEMM (INT4 and NF4), the CTA-pair fused
-GEMM, and the MSD integer GEMM with and without its cluster split of K.
+GEMM (per tile and persistent), and the MSD integer GEMM with and without its
+cluster split of K.
 """
 
 import pytest
@@ -76,6 +77,7 @@ CASES = [
     ("gemm_int4_single_cta", _gemm_int4, 128, 256, 1024, range(0x100, 0x500)),
     ("gemm_nf4_single_cta", _gemm_nf4, 128, 256, 1024, range(0x100, 0x500)),
     ("gemm_int4_cta_pairs", _gemm_int4, 256, 18944, 512, range(0x100, 0x500)),
+    ("gemm_int4_persistent_pairs", _gemm_int4, 1024, 9472, 512, range(0x500, 0x600)),
     ("msd_one_rank", _msd, 128, 256, 512, range(0x1100, 0x1500)),
     ("msd_split_k", _msd, 128, 256, 2048, range(0x1100, 0x1500)),
 ]

@@ -11,11 +11,22 @@
 //
 // One CTA per activation row: a max-reduction pass, then one pass that emits
 // all C digit planes (16 elements per thread step, 16-byte stores per plane).
+// The planes are written in k order, or (for the tensor-core MSD GEMM) with
+// each run of 8 k permuted to the order of its INT4 weight nibbles after a
+// mask and a shift: k = 0, 2, 4, 6, 1, 3, 5, 7. The digits are the same; an
+// integer dot product over the permuted k is the same sum.
 #include "common.cuh"
 
 namespace wq {
 namespace {
 
+// byte position of element e (0..15) of a thread's 16-element step
+template <bool kNibbleOrder>
+__device__ __forceinline__ constexpr int digit_pos(int e) {
+  return kNibbleOrder ? (e & 8) | ((e & 1) << 2) | ((e >> 1) & 3) : e;
+}
+
+template <bool kNibbleOrder>
 __global__ void __launch_bounds__(256) msd_decompose_kernel(const uint16_t* __restrict__ x, int M,
                                                             int K, int C, int64_t plane_rows,
                                                             int8_t* __restrict__ digits,
@@ -81,7 +92,8 @@ __global__ void __launch_bounds__(256) msd_decompose_kernel(const uint16_t* __re
       if (C > 1 && d[1] == 128) { d[1] = -128; d[0] += 1; }
 #pragma unroll
       for (int p = 0; p < 3; ++p)
-        out[p][e >> 2] |= ((uint32_t)(d[p] & 0xFF)) << (8 * (e & 3));
+        out[p][digit_pos<kNibbleOrder>(e) >> 2] |= ((uint32_t)(d[p] & 0xFF))
+                                                   << (8 * (digit_pos<kNibbleOrder>(e) & 3));
     }
     for (int p = 0; p < C; ++p) {
       int8_t* dst = digits + ((int64_t)p * plane_rows + m) * K + c * 16;
@@ -94,8 +106,16 @@ __global__ void __launch_bounds__(256) msd_decompose_kernel(const uint16_t* __re
 
 wq_status launch_msd_decompose(const void* x, int64_t M, int64_t K, int32_t C, int64_t plane_rows,
                                int8_t* digits, float* comp_scales, cudaStream_t st) {
-  msd_decompose_kernel<<<(unsigned)M, 256, 0, st>>>(static_cast<const uint16_t*>(x), (int)M,
-                                                    (int)K, C, plane_rows, digits, comp_scales);
+  msd_decompose_kernel<false><<<(unsigned)M, 256, 0, st>>>(
+      static_cast<const uint16_t*>(x), (int)M, (int)K, C, plane_rows, digits, comp_scales);
+  return launch_status();
+}
+
+wq_status launch_msd_decompose_nibble_order(const void* x, int64_t M, int64_t K, int32_t C,
+                                            int64_t plane_rows, int8_t* digits,
+                                            float* comp_scales, cudaStream_t st) {
+  msd_decompose_kernel<true><<<(unsigned)M, 256, 0, st>>>(
+      static_cast<const uint16_t*>(x), (int)M, (int)K, C, plane_rows, digits, comp_scales);
   return launch_status();
 }
 

@@ -27,9 +27,12 @@
 //                weights are the MMA's A operand (M = 128 features) and a
 //                digit plane its B operand (N = 128 tokens), so a TMEM lane is
 //                one feature and a column one token.
-//   warps 2-5    unpack: nibbles -> bytes (two permutes per 8 codes), minus
-//                the group's zero point per byte, into the UMMA K-major
-//                128-byte-swizzled weight tile.
+//   warps 2-5    unpack: low and high nibbles -> bytes (a mask and a shift
+//                per 8 codes), minus the group's zero point per byte (one add
+//                and one xor per 4 codes), into the UMMA K-major
+//                128-byte-swizzled weight tile. The digit planes are written
+//                in the same permuted k order (0, 2, 4, 6, 1, 3, 5, 7 in each
+//                run of 8), so no byte permute is needed.
 //   warps 6-13   drain each finished group from TMEM: combine the components
 //                in int32, convert, scale by the group's s[n, g] (one value
 //                per thread: its feature), accumulate in fp32 registers; the
@@ -44,6 +47,8 @@ __device__ unsigned int g_msd_error;
 
 wq_status launch_msd_decompose(const void*, int64_t, int64_t, int32_t, int64_t, int8_t*, float*,
                                cudaStream_t);
+wq_status launch_msd_decompose_nibble_order(const void*, int64_t, int64_t, int32_t, int64_t,
+                                            int8_t*, float*, cudaStream_t);
 
 namespace {
 
@@ -119,16 +124,14 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   return r;
 }
 
-// 8 INT4 codes of one packed word -> 8 signed bytes q - z, in k order.
-__device__ __forceinline__ uint2 unpack_word_minus_zero(uint32_t w, uint32_t zrep) {
-  const uint32_t v = w & 0x0F0F0F0Fu;
-  const uint32_t u = (w >> 4) & 0x0F0F0F0Fu;
-  const uint32_t lo = prmt(v, u, 0x5140u);  // codes 0..3
-  const uint32_t hi = prmt(v, u, 0x7362u);  // codes 4..7
-  // per byte: (128 + q - z) ^ 128 == (q - z) as a two's-complement byte; no
-  // borrow crosses bytes because 128 + q - z >= 113
-  return make_uint2(((lo | 0x80808080u) - zrep) ^ 0x80808080u,
-                    ((hi | 0x80808080u) - zrep) ^ 0x80808080u);
+// 8 INT4 codes of one packed word -> 8 signed bytes q - z, in the order the
+// digit planes of this kernel use (codes 0, 2, 4, 6, then 1, 3, 5, 7: the low
+// and the high nibbles of each byte). zc holds 128 - z in every byte: per
+// byte 128 + q - z lies in [113, 143], so the add carries across no byte,
+// and ^ 128 turns it into q - z as a two's-complement byte.
+__device__ __forceinline__ uint2 unpack_word_minus_zero(uint32_t w, uint32_t zc) {
+  return make_uint2(((w & 0x0F0F0F0Fu) + zc) ^ 0x80808080u,
+                    (((w >> 4) & 0x0F0F0F0Fu) + zc) ^ 0x80808080u);
 }
 
 template <int C, bool kIntCombine, bool kSplit>
@@ -285,14 +288,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // and the next group's, loaded one group ahead (at 128-wide groups a
     // zero-point load at the top of each k-tile sat on the critical path)
     const int g0 = kt0 / TPG;
-    uint32_t zrep = (uint32_t)__half2float(zrow[g0]) * 0x01010101u;
+    uint32_t zc = (128u - (uint32_t)__half2float(zrow[g0])) * 0x01010101u;
     __half z_next = zrow[(kt0 % TPG == 0) ? g0 : min(g0 + 1, NG - 1)];
     for (int i = 0; i < KT; ++i) {
       const int kt = kt0 + i;
       const int s = i % kStages;
       const uint32_t ph = (uint32_t)(i / kStages) & 1u;
       if (kt % TPG == 0) {
-        zrep = (uint32_t)__half2float(z_next) * 0x01010101u;
+        zc = (128u - (uint32_t)__half2float(z_next)) * 0x01010101u;
         z_next = zrow[min(kt / TPG + 1, NG - 1)];
       }
       bool got = sm100::mbar_wait(&full[s], ph, &g_msd_error, 0x1301u, abort_flag, wc.limit_ns);
@@ -305,10 +308,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the 16-byte reads of a warp on distinct banks
         const int j4 = (jj + (r >> 1)) & 3;
         const uint4 wv = wsrc[j4];  // words 4*j4 .. 4*j4+3 -> chunks 2*j4, 2*j4+1
-        const uint2 b0 = unpack_word_minus_zero(wv.x, zrep);
-        const uint2 b1 = unpack_word_minus_zero(wv.y, zrep);
-        const uint2 b2 = unpack_word_minus_zero(wv.z, zrep);
-        const uint2 b3 = unpack_word_minus_zero(wv.w, zrep);
+        const uint2 b0 = unpack_word_minus_zero(wv.x, zc);
+        const uint2 b1 = unpack_word_minus_zero(wv.y, zc);
+        const uint2 b2 = unpack_word_minus_zero(wv.z, zc);
+        const uint2 b3 = unpack_word_minus_zero(wv.w, zc);
         const int c0 = 2 * j4, c1 = 2 * j4 + 1;
         *reinterpret_cast<uint4*>(bdst + ((c0 ^ (r & 7)) << 4)) = make_uint4(b0.x, b0.y, b1.x, b1.y);
         *reinterpret_cast<uint4*>(bdst + ((c1 ^ (r & 7)) << 4)) = make_uint4(b2.x, b2.y, b3.x, b3.y);
@@ -571,8 +574,10 @@ wq_status launch_c(const CUtensorMap& ta, const CUtensorMap& tw, const void* sca
 
 }  // namespace
 
-// Workspace: digit planes [C][M_pad][K] int8 (M_pad = M rounded up to 128),
-// then the component scales [C][M] fp32, 256-byte aligned.
+// Workspace: digit planes [C][M_pad][K] int8 (M_pad = M rounded up to 128;
+// in k order for the decode kernel, k permuted within runs of 8 for the
+// tensor-core kernel), then the component scales [C][M] fp32, 256-byte
+// aligned.
 size_t msd_workspace_bytes(int64_t M, int64_t K, int32_t C) {
   return planes_bytes(M, K, C) + (size_t)C * M * 4;
 }
@@ -588,12 +593,16 @@ wq_status launch_msd_gemm(const void* x, int64_t M, int64_t N, int64_t K, int32_
   int8_t* planes = static_cast<int8_t*>(workspace);
   float* cs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + planes_bytes(M, K, C));
   const int64_t mp = m_padded(M);
-  wq_status s = launch_msd_decompose(x, M, K, C, mp, planes, cs, st);
-  if (s != WQ_OK) return s;
   // decode sizes: the weight stream is the cost, so the split-K GEMV with
-  // integer warp MMAs replaces the 128-token tcgen05 tiles
-  if (M <= 16 && G % 128 == 0)
+  // integer warp MMAs replaces the 128-token tcgen05 tiles (it stages the
+  // planes in k order itself; the tensor-core kernel reads them permuted)
+  if (M <= 16 && G % 128 == 0) {
+    wq_status s = launch_msd_decompose(x, M, K, C, mp, planes, cs, st);
+    if (s != WQ_OK) return s;
     return launch_msd_gemv(planes, mp, cs, M, N, K, C, G, qweight, scales, zeros, y, st);
+  }
+  wq_status s = launch_msd_decompose_nibble_order(x, M, K, C, mp, planes, cs, st);
+  if (s != WQ_OK) return s;
   CUtensorMap ta, tw;
   if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, planes, (uint64_t)K, (uint64_t)(C * mp),
                     (uint64_t)K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B))

@@ -1046,40 +1046,55 @@ __global__ void __launch_bounds__(Gemm2PCfg::kThreads, 1)
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int e = (int)threadIdx.x - C::kEpiFirst;  // 0 .. 511
     constexpr uint32_t kEpiThreads = 32 * C::kEpiWarps;
+    // the token scales of the next tile travel in a register (threads e <
+    // BT hold one each) and reach shared memory before its wait, so no
+    // global load and no extra barrier sit between a finished accumulator
+    // and its release
+    float si_next = 0.0f;
+    if (nlocal > 0 && e < BT) {
+      const int m = m0_of(tile_of(0)) + e;
+      si_next = m < M ? inv_scale[m] : 0.0f;
+    }
     for (int j = 0; j < nlocal; ++j) {
       const int t = tile_of(j);
       const int m0 = m0_of(t);
-      // (a tile's mainloop is long: poll with a backoff, off the issue slots
-      // of the dequantization warps and the MMA issuer)
-      bool got = sm100::mbar_wait_sleep(accf, (uint32_t)j & 1u, &g_gemm_error, 0x541u,
-                                        abort_flag, wc.limit_ns, 256);
+      // every epilogue thread passed the previous tile's last barrier, so
+      // its conversion no longer reads s_inv
+      if (e < BT) s_inv[e] = si_next;
+      if (j + 1 < nlocal && e < BT) {
+        const int m = m0_of(tile_of(j + 1)) + e;
+        si_next = m < M ? inv_scale[m] : 0.0f;
+      }
+      // (a tile's mainloop is long: the warps wait suspended in hardware,
+      // off the issue slots of the dequantization warps and the MMA issuer,
+      // and resume as soon as the accumulator is complete)
+      bool got = sm100::mbar_wait_hint(accf, (uint32_t)j & 1u, &g_gemm_error, 0x541u,
+                                       abort_flag, wc.limit_ns, 1000000u);
       got = __all_sync(0xffffffffu, got);
-      // the epilogue warps decide together whether to go on
+      // the previous tile's store has read the staging tile (issued a whole
+      // mainloop ago)
+      if (e == 0) sm100::bulk_wait_read_all();
+      // the epilogue warps decide together whether to go on; the barrier
+      // also publishes s_inv and the staging tile's release
       if (lane == 0) epi_ok[eq] = got ? 1 : 0;
       sm100::named_barrier(3, kEpiThreads);
       bool go = true;
 #pragma unroll
       for (int w = 0; w < C::kEpiWarps; ++w) go = go && epi_ok[w] != 0;
-      // the previous tile's store has read the staging tile
-      if (e == 0) sm100::bulk_wait_read_all();
-      sm100::named_barrier(3, kEpiThreads);
       if (!go) break;
       sm100::tc_fence_after();
-      for (int i = e; i < BT; i += (int)kEpiThreads)
-        s_inv[i] = (m0 + i < M) ? inv_scale[m0 + i] : 0.0f;
-      sm100::named_barrier(3, kEpiThreads);
+      uint32_t v[32];
+      sm100::tmem_ld32(tmem + lane_base + (uint32_t)cbase, v);
+      sm100::tmem_ld_wait();
 #pragma unroll
-      for (int c0 = cbase; c0 < cbase + 64; c0 += 32) {
-        uint32_t v[32];
-        sm100::tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
-        sm100::tmem_ld_wait();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const float val = __uint_as_float(v[jj]) * s_inv[c0 + jj];
-          out_s[(c0 + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
-        }
+      for (int jj = 0; jj < 32; ++jj) {
+        const float val = __uint_as_float(v[jj]) * s_inv[cbase + jj];
+        out_s[(cbase + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
       }
-      // the accumulator is read: the next tile's MMAs may start
+      sm100::tmem_ld32(tmem + lane_base + (uint32_t)(cbase + 32), v);
+      sm100::tmem_ld_wait();
+      // the accumulator is read: the next tile's MMAs may start while this
+      // warp converts its second half
       sm100::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -1087,6 +1102,11 @@ __global__ void __launch_bounds__(Gemm2PCfg::kThreads, 1)
           sm100::mbar_arrive(acc_empty);
         else
           sm100::mbar_arrive_cluster(sm100::cluster_addr(acc_empty, 0));
+      }
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const float val = __uint_as_float(v[jj]) * s_inv[cbase + 32 + jj];
+        out_s[(cbase + 32 + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
       }
       sm100::fence_proxy_async_smem();
       sm100::named_barrier(3, kEpiThreads);

@@ -94,6 +94,39 @@ __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, 
   }
 }
 
+// mbar_wait whose polls carry a suspend-time hint: a thread whose phase is not
+// complete is suspended in hardware until the phase completes or about
+// hint_ns have passed, so a waiting warp takes no issue slots and still
+// resumes as soon as the phase completes. The limit is checked after every
+// poll.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, unsigned int* err,
+                                               uint32_t site, volatile int* abort,
+                                               uint64_t limit_ns, uint32_t hint_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      atomicCAS(err, 0u, site);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // The drain after an abort: wait for the phase regardless of the abort flag,
 // still bounded by the limit (false if it expired).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,

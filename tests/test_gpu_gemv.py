@@ -138,11 +138,21 @@ def test_gemv_operands_only_16_byte_aligned(wq, fmt):
 
 
 def test_gemv_empty_is_noop(wq):
+    """M = 0: the call succeeds, launches nothing that writes (y is an empty
+    view at the start of a sentinel buffer, which must stay untouched) and
+    leaves no device error."""
     x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
-    y = torch.full((0, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    sentinel = torch.full((4, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = sentinel[:0]
+    assert y.data_ptr() == sentinel.data_ptr()
     qw = torch.zeros(64, 32, dtype=torch.int32, device="cuda")
     sc = torch.ones(64, 2, dtype=torch.float16, device="cuda")
-    wq.wq_w4a16_gemv(x, 64, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, sc, out=y)
+    out = wq.wq_w4a16_gemv(x, 64, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, sc, out=y)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 64)
+    assert torch.all(sentinel == 7.0)
+    st, detail = wq.wq_device_error()
+    assert st == wq.WQ_OK, hex(detail)
 
 
 def test_gemv_rejects_m17(wq):

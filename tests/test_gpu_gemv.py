@@ -138,18 +138,19 @@ def test_gemv_operands_only_16_byte_aligned(wq, fmt):
 
 
 def test_gemv_empty_is_noop(wq):
-    """M = 0: the call succeeds, launches nothing that writes (y is an empty
-    view at the start of a sentinel buffer, which must stay untouched) and
-    leaves no device error."""
-    x = torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")
+    """M = 0 through the C ABI with real buffers: the call succeeds, writes
+    nothing (y points at a sentinel buffer, which must stay untouched) and
+    leaves no device error. (torch hands empty tensors a null pointer, so the
+    pointers here are those of non-empty buffers.)"""
+    xbuf = torch.zeros(1, 256, dtype=torch.bfloat16, device="cuda")
     sentinel = torch.full((4, 64), 7.0, dtype=torch.bfloat16, device="cuda")
-    y = sentinel[:0]
-    assert y.data_ptr() == sentinel.data_ptr()
     qw = torch.zeros(64, 32, dtype=torch.int32, device="cuda")
     sc = torch.ones(64, 2, dtype=torch.float16, device="cuda")
-    out = wq.wq_w4a16_gemv(x, 64, wq.WQ_FMT_INT4_ASYM, 128, qw, sc, sc, out=y)
+    st = wq.lib.wq_w4a16_gemv(xbuf.data_ptr(), 0, 64, 256, wq.WQ_FMT_INT4_ASYM, 128,
+                              qw.data_ptr(), sc.data_ptr(), sc.data_ptr(), sentinel.data_ptr(),
+                              None, 0, None)
+    assert st == wq.WQ_OK
     torch.cuda.synchronize()
-    assert out.shape == (0, 64)
     assert torch.all(sentinel == 7.0)
     st, detail = wq.wq_device_error()
     assert st == wq.WQ_OK, hex(detail)

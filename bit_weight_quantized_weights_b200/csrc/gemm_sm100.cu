@@ -780,6 +780,25 @@ __global__ void __launch_bounds__(Deq<kNF4>::kThreads, 1)
   sm100::cluster_sync();
 }
 
+// Epilogue of 32 accumulator columns of one TMEM lane (one weight row):
+// column j times the token scale si[j], rounded once to bf16, into the
+// [token][row] staging tile at dst[j * BW]. The scales are read four at a
+// time (si is 16-byte aligned) and the values converted two at a time.
+__device__ __forceinline__ void epi_store32(const uint32_t (&v)[32], const float* si,
+                                            uint16_t* dst) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 s4 = *reinterpret_cast<const float4*>(si + j);
+    const uint32_t p0 = pack_bf16x2(__uint_as_float(v[j]) * s4.x, __uint_as_float(v[j + 1]) * s4.y);
+    const uint32_t p1 =
+        pack_bf16x2(__uint_as_float(v[j + 2]) * s4.z, __uint_as_float(v[j + 3]) * s4.w);
+    dst[(j + 0) * BW] = (uint16_t)(p0 & 0xFFFFu);
+    dst[(j + 1) * BW] = (uint16_t)(p0 >> 16);
+    dst[(j + 2) * BW] = (uint16_t)(p1 & 0xFFFFu);
+    dst[(j + 3) * BW] = (uint16_t)(p1 >> 16);
+  }
+}
+
 // Persistent CTA-pair kernel (INT4, 128-wide k stages, G a multiple of 128).
 // The pair kernel above pays, for every 256 x 256 tile, its prologue, the
 // fill of its stage ring and its epilogue one after the other; here each pair
@@ -1086,11 +1105,7 @@ __global__ void __launch_bounds__(Gemm2PCfg::kThreads, 1)
       uint32_t v[32];
       sm100::tmem_ld32(tmem + lane_base + (uint32_t)cbase, v);
       sm100::tmem_ld_wait();
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const float val = __uint_as_float(v[jj]) * s_inv[cbase + jj];
-        out_s[(cbase + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
-      }
+      epi_store32(v, s_inv + cbase, out_s + cbase * BW + r);
       sm100::tmem_ld32(tmem + lane_base + (uint32_t)(cbase + 32), v);
       sm100::tmem_ld_wait();
       // the accumulator is read: the next tile's MMAs may start while this
@@ -1103,11 +1118,7 @@ __global__ void __launch_bounds__(Gemm2PCfg::kThreads, 1)
         else
           sm100::mbar_arrive_cluster(sm100::cluster_addr(acc_empty, 0));
       }
-#pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
-        const float val = __uint_as_float(v[jj]) * s_inv[cbase + 32 + jj];
-        out_s[(cbase + 32 + jj) * BW + r] = (uint16_t)(pack_bf16x2(val, 0.0f) & 0xFFFFu);
-      }
+      epi_store32(v, s_inv + cbase + 32, out_s + (cbase + 32) * BW + r);
       sm100::fence_proxy_async_smem();
       sm100::named_barrier(3, kEpiThreads);
       if (e == 0) {
